@@ -1,0 +1,371 @@
+"""Seeded synthetic workloads for the paged KV-cache decode path.
+
+This module builds the inputs that both the CUDA library and the CPU oracle
+consume, and nothing else: sequence lengths, a shuffled free list of physical
+blocks, per-sequence block tables, the values of q / K / V, and the slot of the
+one new token each sequence appends in a decode step.  It holds none of the
+method's arithmetic (no scatter, no gather, no attention); those live in the
+CUDA library and, independently, in the oracle.
+
+Structure (lengths, permutations) is drawn on the CPU from a
+``torch.Generator`` seeded with ``seed``, so it is identical on every device.
+Values are drawn i.i.d. N(0, 1) in fp32 from a generator on the target device
+seeded with ``seed + 1`` and cast to the storage dtype with round-to-nearest-
+even.  The oracle never regenerates values: it reads back these tensors.
+
+Block allocation follows the pages' description of PagedAttention: the KV cache
+is cut into fixed-size 16-token blocks that need not be contiguous, a block
+table maps a sequence's logical positions to physical blocks, blocks are handed
+out from a free list as a sequence grows (no max-length reservation), identical
+prompt prefixes point at the same physical blocks, and a shared block that a
+sequence must write into is copied first (copy-on-write).  Sources:
+"Was ändert PagedAttention an der KV-Speicherzuweisung für LLMs?"
+(slavadubrov.com), introduction and §"Gemeinsame Nutzung erfordert mehr als
+Speicherzuweisung"; "PagedAttention et vLLM" (aiunderstanding.org),
+§"Plongée profonde"; "Внутреннее устройство vLLM" (artificials.ru), paragraph
+on the KV-cache manager (16-token blocks).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+BLOCK_SIZE = 16
+PAD_BLOCK = -1  # table entries past a sequence's last block
+
+# name -> description of the five synthetic workloads
+CONFIGS = {
+    "tiny": dict(
+        desc="4 seqs, lens {35,1,16,17}, Hq=2 over Hkv=1, D=64, fp32, 16-block pool, "
+        "permuted tables, scale 1/sqrt(64)",
+    ),
+    "mha": dict(
+        desc="64 seqs, L~U{128..2048}, Hq=Hkv=32, D=128, bf16, pool 1.25x needed "
+        "(shuffled free list), cache write of 64 new tokens then one decode step",
+    ),
+    "gqa": dict(
+        desc="256 seqs, L=round(exp(N(ln 1024, 0.8^2))) clipped to [16,8192], Hq=32 over "
+        "Hkv=8, D=128, bf16, permuted blocks",
+    ),
+    "prefix": dict(
+        desc="128 seqs sharing one 4096-token prefix (256 shared blocks) plus private "
+        "suffixes L_suf~U{64..512}; Hq=32 over Hkv=8, D=128, bf16",
+    ),
+    "long": dict(
+        desc="8 seqs, L~U{32768..131072}, Hq=64 over Hkv=8, D=128, bf16, "
+        "32-block partitions + LSE reduce, permuted blocks",
+    ),
+}
+
+
+@dataclass
+class Workload:
+    name: str
+    seed: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    dtype: torch.dtype
+    scale: float  # float32 value passed to the kernel
+    num_blocks: int
+    lens_host: list  # python ints, one per sequence
+    tables_host: list  # python lists of physical block ids
+    seq_lens: torch.Tensor  # int32 [N]
+    block_tables: torch.Tensor  # int32 [N, max_blocks], padded with PAD_BLOCK
+    q: torch.Tensor  # [N, Hq, D]
+    k_cache: torch.Tensor  # [NB, Hkv, B, D]
+    v_cache: torch.Tensor  # [NB, Hkv, B, D]
+    new_k: torch.Tensor  # [T, Hkv, D]  (T = N: one new token per sequence)
+    new_v: torch.Tensor  # [T, Hkv, D]
+    slot_mapping: torch.Tensor  # int64 [T]; -1 = padding (nothing written)
+    partition_blocks: int = 0  # 0 = let the library choose
+    shared_blocks: list = field(default_factory=list)  # physical ids referenced by >1 seq
+    desc: str = ""
+
+    @property
+    def num_seqs(self) -> int:
+        return len(self.lens_host)
+
+    @property
+    def max_seq_len(self) -> int:
+        return max(self.lens_host) if self.lens_host else 0
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_tables.shape[1])
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def elem_bytes(self) -> int:
+        return torch.finfo(self.dtype).bits // 8
+
+    @property
+    def device(self) -> torch.device:
+        return self.q.device
+
+
+def scale_for(head_dim: int) -> float:
+    """1/sqrt(D) rounded to float32 (the value the kernel receives)."""
+    return float(torch.tensor(1.0 / math.sqrt(head_dim), dtype=torch.float32).item())
+
+
+def _blocks_for(n_tokens: int, block_size: int) -> int:
+    # allocation bookkeeping: how many blocks the allocator hands out
+    return -(-n_tokens // block_size)
+
+
+def _draw_lens(name: str, gen: torch.Generator) -> list:
+    if name == "tiny":
+        return [35, 1, 16, 17]
+    if name == "mha":
+        return torch.randint(128, 2048 + 1, (64,), generator=gen).tolist()
+    if name == "gqa":
+        z = torch.randn(256, generator=gen, dtype=torch.float64)
+        lens = torch.round(torch.exp(z * 0.8 + math.log(1024.0)))
+        return lens.clamp(16, 8192).to(torch.int64).tolist()
+    if name == "long":
+        return torch.randint(32768, 131072 + 1, (8,), generator=gen).tolist()
+    raise KeyError(name)
+
+
+def _randn(shape, gen: torch.Generator, device, dtype) -> torch.Tensor:
+    """N(0,1) drawn in fp32 on `device`, cast (RNE) to `dtype`; chunked so that a
+    multi-GB pool never needs a full fp32 temporary."""
+    out = torch.empty(shape, dtype=dtype, device=device)
+    flat = out.view(-1)
+    n = flat.numel()
+    chunk = 1 << 28
+    for off in range(0, n, chunk):
+        m = min(chunk, n - off)
+        flat[off : off + m] = torch.randn(m, generator=gen, device=device, dtype=torch.float32).to(dtype)
+    return out
+
+
+@dataclass
+class Plan:
+    """Structure of a workload: lengths, pool size and block tables (no values)."""
+    lens: list
+    tables: list
+    num_blocks: int
+    shared: list  # physical ids referenced by every sequence (shared prefix)
+    cow_pairs: list  # (shared source block, private copy) for a prefix ending mid-block
+    prefix_len: int = 0
+
+    @property
+    def needed_blocks(self) -> int:
+        ids = set(b for t in self.tables for b in t) | set(src for src, _ in self.cow_pairs)
+        return len(ids)
+
+
+def plan(
+    lens: Sequence[int],
+    seed: int = 0,
+    num_blocks: Optional[int] = None,
+    pool_factor: float = 1.25,
+    prefix_len: int = 0,
+) -> Plan:
+    """Allocate physical blocks for sequences of the given total lengths.
+
+    The pool holds ``ceil(pool_factor * needed)`` blocks unless ``num_blocks`` is
+    given; blocks are taken in order from a seeded random permutation of the pool
+    (a shuffled free list).  With ``prefix_len > 0`` every sequence starts with the
+    same ``prefix_len`` tokens: the full prefix blocks are allocated once and every
+    table points at them; if the prefix ends inside a block, that block is kept
+    once as a shared source and each sequence gets a private copy of it
+    (copy-on-write) into which its own suffix continues.
+    """
+    B = BLOCK_SIZE
+    lens = [int(x) for x in lens]
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    n_full_prefix = prefix_len // B
+    prefix_rem = prefix_len % B
+    if prefix_len:
+        assert all(L >= prefix_len for L in lens), "every sequence must hold the prefix"
+    # tokens of a sequence that live in its private blocks
+    private_tokens = [L - n_full_prefix * B for L in lens]
+    needed = n_full_prefix + (1 if prefix_rem else 0)
+    needed += sum(_blocks_for(n, B) for n in private_tokens)
+    if num_blocks is None:
+        num_blocks = max(1, math.ceil(pool_factor * needed))
+    assert num_blocks >= needed, (num_blocks, needed)
+
+    free = torch.randperm(num_blocks, generator=gen).tolist()
+    cursor = 0
+
+    def take() -> int:
+        nonlocal cursor
+        b = free[cursor]
+        cursor += 1
+        return b
+
+    shared = [take() for _ in range(n_full_prefix)]
+    cow_source = take() if prefix_rem else None
+    tables = []
+    cow_pairs = []
+    for rest in private_tokens:
+        t = list(shared)
+        for j in range(_blocks_for(rest, B)):
+            b = take()
+            if j == 0 and prefix_rem:
+                cow_pairs.append((cow_source, b))
+            t.append(b)
+        tables.append(t)
+    return Plan(lens, tables, num_blocks, shared, cow_pairs, prefix_len)
+
+
+def build(
+    lens: Sequence[int],
+    num_q_heads: int,
+    num_kv_heads: int,
+    head_dim: int,
+    dtype: torch.dtype,
+    seed: int = 0,
+    device="cpu",
+    num_blocks: Optional[int] = None,
+    pool_factor: float = 1.25,
+    prefix_len: int = 0,
+    poison_unused: bool = False,
+    partition_blocks: int = 0,
+    name: str = "custom",
+    desc: str = "",
+    table_width: Optional[int] = None,
+) -> Workload:
+    """Build a workload from explicit per-sequence total lengths (see ``plan``).
+
+    ``poison_unused`` fills every slot that no table reaches (unused blocks and
+    the tail of each sequence's last block) with NaN, so a kernel that reads
+    past a sequence's length produces a visibly wrong result.
+    """
+    B = BLOCK_SIZE
+    assert num_q_heads % num_kv_heads == 0
+    p = plan(lens, seed=seed, num_blocks=num_blocks, pool_factor=pool_factor, prefix_len=prefix_len)
+    lens, tables, num_blocks = p.lens, p.tables, p.num_blocks
+    prefix_rem = prefix_len % B
+
+    width = max([len(t) for t in tables] + [1])
+    if table_width is not None:
+        assert table_width >= width
+        width = table_width
+    tab = torch.full((len(lens), width), PAD_BLOCK, dtype=torch.int32)
+    for s, t in enumerate(tables):
+        if t:
+            tab[s, : len(t)] = torch.tensor(t, dtype=torch.int32)
+
+    vgen = torch.Generator(device=device)
+    vgen.manual_seed(seed + 1)
+    N = len(lens)
+    q = _randn((N, num_q_heads, head_dim), vgen, device, dtype)
+    k_cache = _randn((num_blocks, num_kv_heads, B, head_dim), vgen, device, dtype)
+    v_cache = _randn((num_blocks, num_kv_heads, B, head_dim), vgen, device, dtype)
+    new_k = _randn((N, num_kv_heads, head_dim), vgen, device, dtype)
+    new_v = _randn((N, num_kv_heads, head_dim), vgen, device, dtype)
+
+    # copy-on-write of the partial last prefix block into each private copy
+    for src, dst in p.cow_pairs:
+        k_cache[dst, :, :prefix_rem] = k_cache[src, :, :prefix_rem]
+        v_cache[dst, :, :prefix_rem] = v_cache[src, :, :prefix_rem]
+
+    slot_mapping = torch.tensor(new_token_slots(p), dtype=torch.int64)
+
+    if poison_unused:
+        used = torch.zeros((num_blocks, B), dtype=torch.bool)
+        for L, t in zip(lens, tables):
+            for j, b in enumerate(t):
+                used[b, : min(B, L - j * B)] = True
+        used = used.to(device)[:, None, :, None]
+        nan = torch.tensor(float("nan"), dtype=dtype, device=device)
+        k_cache = torch.where(used, k_cache, nan)
+        v_cache = torch.where(used, v_cache, nan)
+
+    return Workload(
+        name=name,
+        seed=seed,
+        num_q_heads=num_q_heads,
+        num_kv_heads=num_kv_heads,
+        head_dim=head_dim,
+        block_size=B,
+        dtype=dtype,
+        scale=scale_for(head_dim),
+        num_blocks=num_blocks,
+        lens_host=lens,
+        tables_host=tables,
+        seq_lens=torch.tensor(lens, dtype=torch.int32).to(device),
+        block_tables=tab.to(device),
+        q=q,
+        k_cache=k_cache,
+        v_cache=v_cache,
+        new_k=new_k,
+        new_v=new_v,
+        slot_mapping=slot_mapping.to(device),
+        partition_blocks=partition_blocks,
+        shared_blocks=sorted(p.shared + [src for src, _ in p.cow_pairs[:1]]),
+        desc=desc,
+    )
+
+
+def new_token_slots(p: Plan) -> list:
+    """Slot of each sequence's newest token (position L-1), -1 for an empty one.
+    This is the slot mapping a serving engine hands to the cache write."""
+    B = BLOCK_SIZE
+    slots = []
+    for L, t in zip(p.lens, p.tables):
+        if L == 0:
+            slots.append(-1)
+        else:
+            pos = L - 1
+            slots.append(t[pos // B] * B + pos % B)
+    return slots
+
+
+def config_lens(name: str, seed: int = 0) -> tuple:
+    """(lens, prefix_len) of a named workload, drawn from the seed."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    if name == "prefix":
+        suf = torch.randint(64, 512 + 1, (128,), generator=gen).tolist()
+        return [4096 + s for s in suf], 4096
+    return _draw_lens(name, gen), 0
+
+
+def config_plan(name: str, seed: int = 0) -> Plan:
+    lens, prefix = config_lens(name, seed)
+    return plan(lens, seed=seed, num_blocks=16 if name == "tiny" else None, prefix_len=prefix)
+
+
+def make(name: str, seed: int = 0, device="cpu", poison_unused: bool = False, **kw) -> Workload:
+    """One of the five named workloads (see CONFIGS)."""
+    desc = CONFIGS[name]["desc"]
+    lens, prefix = config_lens(name, seed)
+    common = dict(seed=seed, device=device, poison_unused=poison_unused, name=name, desc=desc)
+    if name == "tiny":
+        return build(lens, 2, 1, 64, torch.float32, num_blocks=16, **common, **kw)
+    if name == "mha":
+        return build(lens, 32, 32, 128, torch.bfloat16, **common, **kw)
+    if name == "gqa":
+        return build(lens, 32, 8, 128, torch.bfloat16, **common, **kw)
+    if name == "prefix":
+        prefix = kw.pop("prefix_len", prefix)
+        if prefix != 4096:  # variant with a different prefix length, same suffixes
+            lens = [L - 4096 + prefix for L in lens]
+        return build(lens, 32, 8, 128, torch.bfloat16, prefix_len=prefix, **common, **kw)
+    if name == "long":
+        kw.setdefault("partition_blocks", 32)
+        return build(lens, 64, 8, 128, torch.bfloat16, **common, **kw)
+    raise KeyError(name)
+
+
+def as_numpy(t: torch.Tensor) -> np.ndarray:
+    """Host copy as numpy; bf16 comes back as its raw uint16 bit patterns."""
+    t = t.detach().to("cpu").contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()

@@ -1,0 +1,80 @@
+"""The seeded generator builds the five workloads with the stated structure."""
+import math
+
+import pytest
+import torch
+
+from paged_kv_cache_432_b200 import workload as wl
+
+
+@pytest.mark.parametrize("name", ["tiny", "mha", "gqa", "prefix", "long"])
+def test_plan_structure(name):
+    p = wl.config_plan(name, seed=0)
+    nb = [len(t) for t in p.tables]
+    assert nb == [-(-L // 16) for L in p.lens]
+    ids = [b for t in p.tables for b in t]
+    assert all(0 <= b < p.num_blocks for b in ids)
+    if name == "prefix":
+        # every table starts with the same 256 shared blocks; everything else is private
+        assert all(t[:256] == p.tables[0][:256] for t in p.tables)
+        private = [b for t in p.tables for b in t[256:]]
+        assert len(set(private)) == len(private)
+        assert not set(private) & set(p.tables[0][:256])
+    else:
+        assert len(set(ids)) == len(ids), "a block is owned by one sequence"
+    if name == "tiny":
+        assert p.num_blocks == 16
+    else:
+        assert p.num_blocks == math.ceil(1.25 * p.needed_blocks)
+
+
+def test_length_distributions():
+    mha = wl.config_plan("mha").lens
+    assert len(mha) == 64 and min(mha) >= 128 and max(mha) <= 2048
+    gqa = wl.config_plan("gqa").lens
+    assert len(gqa) == 256 and min(gqa) >= 16 and max(gqa) <= 8192
+    med = sorted(gqa)[128]
+    assert 700 < med < 1500  # lognormal with median 1024
+    pre = wl.config_plan("prefix").lens
+    assert len(pre) == 128 and all(4096 + 64 <= L <= 4096 + 512 for L in pre)
+    lo = wl.config_plan("long").lens
+    assert len(lo) == 8 and all(32768 <= L <= 131072 for L in lo)
+
+
+def test_seeded_and_distinct():
+    assert wl.config_plan("gqa", 0).tables == wl.config_plan("gqa", 0).tables
+    assert wl.config_plan("gqa", 0).lens != wl.config_plan("gqa", 1).lens
+
+
+def test_new_token_slot_is_last_position():
+    w = wl.build([35, 1, 16, 17, 0], 2, 1, 16, torch.float32, seed=2)
+    for s, L in enumerate(w.lens_host):
+        slot = int(w.slot_mapping[s])
+        if L == 0:
+            assert slot == -1
+            continue
+        assert slot // 16 == w.tables_host[s][(L - 1) // 16]
+        assert slot % 16 == (L - 1) % 16
+
+
+def test_copy_on_write_of_partial_prefix_block():
+    """A prefix ending mid-block: each sequence's first private block starts with a
+    copy of the shared partial block's tokens."""
+    w = wl.build([4090 + 5, 4090 + 40], 2, 1, 16, torch.bfloat16, seed=3, prefix_len=4090)
+    p = wl.plan(w.lens_host, seed=3, prefix_len=4090)
+    assert len(p.cow_pairs) == 2
+    for src, dst in p.cow_pairs:
+        assert torch.equal(w.k_cache[dst, :, :10], w.k_cache[src, :, :10])
+        assert not torch.equal(w.k_cache[dst, :, 10:], w.k_cache[src, :, 10:])
+    # the copies are private: different tables, same logical prefix
+    assert w.tables_host[0][255] != w.tables_host[1][255]
+    assert w.tables_host[0][:255] == w.tables_host[1][:255]
+
+
+def test_poison_marks_only_unreachable_slots():
+    w = wl.build([35, 1], 2, 1, 16, torch.float32, seed=4, poison_unused=True)
+    nan = torch.isnan(w.k_cache[:, 0, :, 0])
+    for s, L in enumerate(w.lens_host):
+        for t in range(L):
+            assert not nan[w.tables_host[s][t // 16], t % 16]
+    assert int(nan.sum()) == w.num_blocks * 16 - sum(w.lens_host)
