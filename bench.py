@@ -1,0 +1,490 @@
+"""Benchmark of the paged KV-cache decode path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config mha|gqa|prefix|long|tiny]
+    python bench.py --impl reference ...      (the fp64 CPU oracle, timed on host cores)
+
+One step = one pass of the hot path over one batch: the cache write of each
+sequence's newest token (pa_cache_write), then the decode (the block-table
+walk with split-K partials, pa_decode_partitions, and the log-sum-exp merge,
+pa_decode_reduce).  Inputs are resident in HBM; L2 is flushed (512 MiB write)
+before every step, outside the timed events.  Times are CUDA events on the
+launching stream; with N > 1 (torchrun) every rank runs its own replica of the
+workload (seed + rank, no data exchange) and the step time is the max over
+ranks.  Prints one JSON line.
+
+metric: KV GB/s = algorithmic bytes of a step / step time, where the bytes are
+the KV of every token attended (each distinct physical block counted once:
+shared prefix blocks are read once), q, out, table entries and lengths, plus
+the cache write's reads and writes.  Decode tokens/s = sequences / step time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_432_b200 import workload as wl  # noqa: E402
+
+FLUSH_BYTES = 512 << 20
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "paged decode attention KV GB/s and decode tokens/s on 1 B200 vs 8 TB/s HBM roofline"
+
+
+# ---------------------------------------------------------------- bytes accounting
+def algorithmic_bytes(w: wl.Workload) -> dict:
+    """Bytes a step must move at minimum.  KV: every (distinct physical block,
+    kv head) slice attended, counted once, with the valid slots only."""
+    e = w.elem_bytes
+    D, Hkv, Hq = w.head_dim, w.num_kv_heads, w.num_q_heads
+    valid = {}
+    for L, t in zip(w.lens_host, w.tables_host):
+        for j, b in enumerate(t):
+            valid[b] = max(valid.get(b, 0), min(16, L - 16 * j))
+    kv_unique = 2 * sum(valid.values()) * Hkv * D * e
+    kv_logical = 2 * sum(w.lens_host) * Hkv * D * e
+    n_blocks_read = sum(len(t) for t in w.tables_host)
+    q_out = 2 * w.num_seqs * Hq * D * e
+    meta = 4 * n_blocks_read + 4 * w.num_seqs
+    decode = kv_unique + q_out + meta
+    T = int(w.slot_mapping.numel())
+    write = 2 * (2 * T * Hkv * D * e) + 8 * T
+    return dict(decode=decode, write=write, step=decode + write, kv_unique=kv_unique,
+                kv_logical=kv_logical, q_out=q_out, meta=meta)
+
+
+def workload_config(w: wl.Workload, pb: int) -> dict:
+    return {
+        "workload": w.name,
+        "desc": w.desc,
+        "seed": w.seed,
+        "num_seqs": w.num_seqs,
+        "tokens": sum(w.lens_host),
+        "max_seq_len": w.max_seq_len,
+        "num_q_heads": w.num_q_heads,
+        "num_kv_heads": w.num_kv_heads,
+        "head_dim": w.head_dim,
+        "block_size": w.block_size,
+        "pool_blocks": w.num_blocks,
+        "partition_blocks": pb,
+        "new_tokens": int(w.slot_mapping.numel()),
+        "slot_utilisation": round(sum(w.lens_host) / (16 * sum(len(t) for t in w.tables_host)), 5),
+        "l2": "flushed before every step (512 MiB write, outside the timed events); KV footprint "
+              "exceeds L2",
+    }
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "paged_kv_cache_432_b200", "csrc", "*"))):
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks() -> tuple:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_traffic(workload: str):
+    """dram bytes per launch of the decode kernel from a committed ncu summary,
+    if it was taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", f"decode_bf16_mma_{workload}.json")
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None
+    if d.get("source_digest") != source_digest():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks (NVML)
+_REASONS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+_BAD = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+class ClockSampler:
+    def __init__(self, device: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.err = None
+        self.h = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+            ident = vis[device].strip() if vis and vis[0] != "" and device < len(vis) else str(device)
+            if ident.startswith("GPU-") or ident.startswith("MIG-"):
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(ident)
+            else:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(int(ident))
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.err = f"nvml unavailable: {e}"
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self.h))
+            except Exception as e:  # noqa: BLE001
+                self.err = str(e)
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.h is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.h is not None:
+            self.t.join()
+
+    def summary(self) -> dict:
+        if self.h is None or not self.samples:
+            return {"error": self.err or "no samples"}
+        names = sorted(v for k, v in _REASONS.items() if self.reasons & k and v != "gpu_idle")
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples), "source": "nvml, 5 ms period"}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def oracle_step_sample(w: wl.Workload, h: dict, seqs: list) -> tuple:
+    """Runs the oracle (cache write + decode) for the given sequences; returns
+    (seconds, algorithmic bytes of that sample)."""
+    import numpy as np
+
+    import oracle
+
+    sel = np.array(seqs)
+    rows = [(s, qh) for s in seqs for qh in range(w.num_q_heads)]
+    t0 = time.perf_counter()
+    oracle.cache_write(h["nk"][sel], h["nv"][sel], h["sm"][sel], h["kc"], h["vc"], inplace=True)
+    oracle.paged_decode(h["q"], h["kc"], h["vc"], h["bt"], h["sl"], w.scale, rows=rows)
+    dt = time.perf_counter() - t0
+    e, D, Hkv, Hq = w.elem_bytes, w.head_dim, w.num_kv_heads, w.num_q_heads
+    kv = 2 * sum(w.lens_host[s] for s in seqs) * Hkv * D * e
+    by = kv + 2 * len(seqs) * Hq * D * e + 4 * sum(len(w.tables_host[s]) for s in seqs) + \
+        2 * (2 * len(seqs) * Hkv * D * e)
+    return dt, by
+
+
+def host_arrays(w: wl.Workload) -> dict:
+    return dict(q=wl.as_numpy(w.q), kc=wl.as_numpy(w.k_cache), vc=wl.as_numpy(w.v_cache),
+                bt=wl.as_numpy(w.block_tables), sl=wl.as_numpy(w.seq_lens),
+                nk=wl.as_numpy(w.new_k), nv=wl.as_numpy(w.new_v), sm=wl.as_numpy(w.slot_mapping))
+
+
+def cpu_baseline(w: wl.Workload, budget_s: float = 20.0) -> dict:
+    """The oracle as it stands, single-threaded, on a bounded sample: whole
+    sequences (all heads) in order until about budget_s of work."""
+    h = host_arrays(w)
+    total_t, total_b, seqs = 0.0, 0, []
+    s = 0
+    while s < w.num_seqs and total_t < budget_s:
+        dt, by = oracle_step_sample(w, h, [s])
+        total_t += dt
+        total_b += by
+        seqs.append(s)
+        s += 1
+    return {"value": round(total_b / total_t / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{len(seqs)} of {w.num_seqs} sequences (all {w.num_q_heads} q heads, cache "
+                      f"write + decode), {total_t:.1f} s single-threaded fp64",
+            "tokens_per_s": round(len(seqs) / total_t, 3)}
+
+
+def run_reference(args) -> None:
+    ws, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return
+    w = wl.make(args.config, seed=args.seed, device="cpu")
+    h = host_arrays(w)
+    per_step = max(1, args.ref_seqs_per_step)
+    times, nbytes, nseq = [], [], []
+    s = 0
+    for i in range(args.warmup + args.steps):
+        seqs = [(s + k) % w.num_seqs for k in range(per_step)]
+        s = (s + per_step) % w.num_seqs
+        dt, by = oracle_step_sample(w, h, seqs)
+        if i >= args.warmup:
+            times.append(dt)
+            nbytes.append(by)
+            nseq.append(len(seqs))
+    T = sum(times)
+    value = sum(nbytes) / T / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * T / len(times), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(workload_config(w, 0), l2="n/a (host)"),
+        "tokens_per_s": round(sum(nseq) / T, 3),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{per_step} whole sequence(s) per step (all {w.num_q_heads} q "
+                                   f"heads, cache write + decode), rotating over the batch"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args) -> None:
+    from paged_kv_cache_432_b200 import build as pa_build
+    from paged_kv_cache_432_b200 import pagedattn as pa
+
+    ws, rank, local = dist_setup()
+    if rank == 0:
+        pa_build.build()
+    barrier(ws)
+    dev = torch.device("cuda", local)
+    w = wl.make(args.config, seed=args.seed + rank, device=dev)
+    pb = w.partition_blocks if args.partition_blocks is None else args.partition_blocks
+    msl = w.max_seq_len
+    resolved_pb = pa.partition_blocks(w.num_seqs, w.num_kv_heads, msl, pb)
+    split = math.ceil(math.ceil(msl / 16) / resolved_pb) > 1
+    wsp = pa.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, msl, pb, device=dev)
+    out = torch.empty_like(w.q)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    by = algorithmic_bytes(w)
+    chunks = math.ceil(w.num_seqs / 2048)
+    launches_per_step = 1 + chunks + (chunks if split else 0)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        pa.cache_write(w.new_k, w.new_v, w.slot_mapping, w.k_cache, w.v_cache, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        pa.decode_partitions(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, out, msl,
+                             pb, wsp, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        if split:
+            pa.decode_reduce(w.seq_lens, out, w.num_kv_heads, w.max_blocks_per_seq, msl, pb, wsp, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if pa.device_error() != 0:
+        raise RuntimeError("device error flagged during warm-up")
+
+    def timed():
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        barrier(ws)
+        torch.cuda.synchronize(dev)
+        with ClockSampler(local) as cs:
+            for k in range(args.steps):
+                flush.zero_()
+                step(evs[k])
+            torch.cuda.synchronize(dev)
+        barrier(ws)
+        tot = sum(e[0].elapsed_time(e[3]) for e in evs)
+        dec = sum(e[1].elapsed_time(e[2]) for e in evs)
+        red = sum(e[2].elapsed_time(e[3]) for e in evs)
+        wr = sum(e[0].elapsed_time(e[1]) for e in evs)
+        return tot, dec, red, wr, cs.summary()
+
+    tot, dec, red, wr, clocks = timed()
+    if set(clocks.get("reasons", [])) & _BAD:  # re-measure once
+        tot, dec, red, wr, clocks = timed()
+        clocks["remeasured"] = True
+    K = args.steps
+    step_ms = max_over_ranks(tot / K, ws)
+    dec_ms = max_over_ranks(dec / K, ws)
+    red_ms = max_over_ranks(red / K, ws)
+    wr_ms = max_over_ranks(wr / K, ws)
+    total_bytes = sum_over_ranks(by["step"], ws)
+    total_seqs = sum_over_ranks(w.num_seqs, ws)
+    value = total_bytes / (step_ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API: inputs from pinned host memory,
+    # result read back, every step
+    e2e = None
+    if not args.no_e2e:
+        names = ["q", "new_k", "new_v", "slot_mapping", "block_tables", "seq_lens"]
+        host_in = {n: getattr(w, n).cpu().pin_memory() for n in names}
+        dev_in = {n: torch.empty_like(getattr(w, n)) for n in names}
+        host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = host_out.numel() * host_out.element_size()
+
+        def e2e_step():
+            for n in names:
+                dev_in[n].copy_(host_in[n], non_blocking=True)
+            pa.cache_write(dev_in["new_k"], dev_in["new_v"], dev_in["slot_mapping"], w.k_cache, w.v_cache, stream)
+            pa.decode(dev_in["q"], w.k_cache, w.v_cache, dev_in["block_tables"], dev_in["seq_lens"], w.scale,
+                      out=out, max_seq_len=msl, partition_blocks=pb, workspace=wsp, stream=stream)
+            host_out.copy_(out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            flush.zero_()
+            e2e_step()
+        n_e2e = max(3, min(K, 50))
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_e2e)]
+        barrier(ws)
+        torch.cuda.synchronize(dev)
+        for k in range(n_e2e):
+            flush.zero_()
+            evs[k][0].record(stream)
+            e2e_step()
+            evs[k][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(ws)
+        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / n_e2e, ws)
+        e2e = {"value": round(total_bytes / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4),
+               "steps": n_e2e}
+
+    if pa.device_error() != 0:
+        raise RuntimeError("device error flagged during timing")
+
+    peak, peak_kind = load_peaks()
+    achieved = by["decode"] / (dec_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": "decode_bf16_mma_kernel" if w.dtype == torch.bfloat16 else
+            "decode_f32_simt_kernel", "achieved": round(achieved, 1), "peak": peak,
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback 6650 GB/s", "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "frac_of_8TBs": round(achieved / 8000.0, 4),
+            "algorithmic_bytes_per_launch": by["decode"],
+            "traffic": load_traffic(w.name)}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, budget_s=args.cpu_budget_s)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic",
+        "config": workload_config(w, resolved_pb),
+        "tokens_per_s": round(total_seqs / (step_ms * 1e-3), 1),
+        "kernel_ms": {"cache_write": round(wr_ms, 5), "decode_partitions": round(dec_ms, 5),
+                      "lse_reduce": round(red_ms, 5)},
+        "bytes_per_step": by,
+        "roofline": roof,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "clocks": clocks,
+        "gpu_launches": launches_per_step * K,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="mha", choices=list(wl.CONFIGS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--partition-blocks", type=int, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    ap.add_argument("--ref-seqs-per-step", type=int, default=2)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,179 @@
+/*
+ * pagedattn.h -- C ABI of the paged KV-cache decode path (NVIDIA B200, sm_100a).
+ *
+ * PagedAttention keeps each sequence's keys and values in fixed-size physical
+ * blocks that may sit anywhere in one shared pool; a per-sequence block table
+ * maps logical token positions to those blocks, blocks are taken as a sequence
+ * grows, and several sequences may point at the same block (shared prefixes).
+ * Sources: "Was ändert PagedAttention an der KV-Speicherzuweisung für LLMs?"
+ * (slavadubrov.com), introduction, §"Ungenutzten Platz in Blöcken berechnen"
+ * (16-token blocks, only the last block partly filled) and §"Gemeinsame Nutzung
+ * erfordert mehr als Speicherzuweisung" (several requests reference one block;
+ * copy-on-write); "PagedAttention et vLLM" (aiunderstanding.org), §"Plongée
+ * profonde" (lookup table from logical positions to physical blocks);
+ * "vLLM PagedAttention: eine Revolution für den Durchsatz bei der
+ * LLM-Inferenz" (de.news.hada.io) (decoding is the memory-bandwidth-bound
+ * phase); "Внутреннее устройство vLLM" (artificials.ru), paragraphs on the
+ * KV-cache manager (16-token blocks) and on the padding-free super-batch
+ * (per-sequence lengths instead of padding).
+ *
+ * Layouts (row-major, the pages leave layout to the runtime; this is the one
+ * this library fixes):
+ *   k_cache, v_cache  [num_blocks][num_kv_heads][block_size][head_dim]
+ *   q, out            [num_seqs][num_q_heads][head_dim]
+ *   k, v (new tokens) [num_tokens][num_kv_heads][head_dim]
+ *   slot_mapping      int64  [num_tokens]; slot = block * block_size + offset
+ *   block_tables      int32  [num_seqs][max_blocks_per_seq]
+ *   seq_lens          int32  [num_seqs]   (tokens to attend, new token included)
+ * Query head i reads kv head i / (num_q_heads / num_kv_heads).
+ *
+ * Ownership and execution: every pointer argument is device memory owned by
+ * the caller (the library allocates no device memory and keeps no pointer).
+ * Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ * default stream) and return once the work is enqueued.  Host-side validation
+ * never reads device memory.  Pointers to q, k, v, caches and out must be
+ * 16-byte aligned; tables, lengths and slots naturally aligned.  The caches
+ * and tables may be shared between sequences but must not overlap `out` or the
+ * workspace.  The library never traps or aborts: bad device-side values (a
+ * slot or block id outside the pool, an impossible length) are skipped and
+ * recorded in a sticky per-device error word read by pa_get_device_error.
+ */
+#ifndef PAGEDATTN_H_
+#define PAGEDATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define PA_OK 0
+#define PA_ERR_INVALID_ARG (-1) /* null/misaligned pointer, bad sizes        */
+#define PA_ERR_UNSUPPORTED (-2) /* dtype, head_dim, block size or group size */
+#define PA_ERR_WORKSPACE (-3)   /* workspace missing or too small            */
+#define PA_ERR_CUDA (-4)        /* a CUDA call or launch failed              */
+
+/* Element types (q, caches, new k/v and out share one). */
+#define PA_DTYPE_F32 0
+#define PA_DTYPE_BF16 1
+
+/* Bits of the sticky device error word. */
+#define PA_DEVERR_SLOT_OOB 1u  /* cache write: slot >= num_blocks*block_size, token skipped */
+#define PA_DEVERR_BLOCK_OOB 2u /* decode: table entry outside [0, num_blocks), block masked */
+#define PA_DEVERR_SEQ_LEN 4u   /* decode: seq_len < 0 or beyond capacity, clamped          */
+#define PA_DEVERR_TIMEOUT 8u   /* a bounded wait on an async copy gave up                  */
+
+/*
+ * Cache write (the scatter of newly computed K/V into the paged pool).
+ * For every token t with slot s = slot_mapping[t] >= 0 and every kv head h:
+ *   k_cache[s / block_size][h][s % block_size][:] = k[t][h][:]   (same for v)
+ * Bytes are copied unchanged.  Slots < 0 are padding and write nothing; a slot
+ * beyond the pool writes nothing and sets PA_DEVERR_SLOT_OOB.  Two tokens with
+ * the same slot race (one of them wins).  block_size must be 16; head_dim 64
+ * or 128.  Source: slavadubrov.com, introduction (logical positions mapped to
+ * physical blocks); artificials.ru (16-token blocks).
+ */
+PA_API int pa_cache_write(const void* k, const void* v, const int64_t* slot_mapping,
+                   int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                   void* k_cache, void* v_cache, int32_t num_blocks,
+                   int32_t block_size, int32_t dtype, void* stream);
+
+/*
+ * Blocks per partition the decode uses: partition_blocks > 0 is taken as is,
+ * -1 means never split (one pass over the whole sequence), 0 lets the library
+ * choose from the sizes.  Returns the resolved value (a value >= the blocks of
+ * max_seq_len means no split), or a negative status on bad arguments.
+ */
+PA_API int32_t pa_decode_partition_blocks(int32_t num_seqs, int32_t num_kv_heads,
+                                   int32_t max_seq_len, int32_t block_size,
+                                   int32_t partition_blocks);
+
+/*
+ * Bytes of workspace pa_decode needs for these sizes (0 when no sequence of
+ * up to max_seq_len tokens is split).  Workspace layout, P = partitions per
+ * sequence at max_seq_len, rows r = seq * num_q_heads + q_head:
+ *   float m  [num_seqs*num_q_heads][P]     max score of the partition (natural log units)
+ *   float l  [num_seqs*num_q_heads][P]     sum of exp(score - m)
+ *   float acc[num_seqs*num_q_heads][P][D]  sum of exp(score - m) * v
+ * each array starting on a 256-byte boundary.
+ */
+PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                int32_t head_dim, int32_t max_seq_len, int32_t block_size,
+                                int32_t partition_blocks);
+
+/*
+ * Paged decode attention: for each sequence s and query head i,
+ *   out[s][i] = softmax_t(scale * q[s][i] . K_s[t]) V_s,  t < seq_lens[s],
+ * where K_s[t] = k_cache[block_tables[s][t / bs]][i / group][t % bs] (same for V).
+ * Accumulation is fp32 (bf16 inputs: scores and P.V on tensor cores with fp32
+ * accumulators); out is rounded to the input dtype (round to nearest even).  A
+ * zero-length sequence gives a zero row.  Sequences longer than
+ * partition_blocks * block_size tokens are split into partitions whose partial
+ * results are merged by a log-sum-exp reduction (pa_decode runs both steps).
+ * max_seq_len is a host-side bound on seq_lens (<= 0: max_blocks_per_seq *
+ * block_size); it sizes the workspace, and longer sequences are clamped to it
+ * with PA_DEVERR_SEQ_LEN set.  Table entries past a sequence's last block are
+ * never read.  Supported: block_size 16, head_dim 64 or 128, dtype F32 or
+ * BF16, num_q_heads / num_kv_heads <= 16.
+ * Source: slavadubrov.com, introduction and §"Ungenutzten Platz in Blöcken
+ * berechnen"; aiunderstanding.org, §"Plongée profonde"; artificials.ru,
+ * paragraph on the padding-free super-batch.
+ */
+PA_API int pa_decode(const void* q, const void* k_cache, const void* v_cache,
+              const int32_t* block_tables, int32_t max_blocks_per_seq,
+              const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+              int32_t num_blocks, int32_t block_size, float scale,
+              int32_t partition_blocks, void* workspace, size_t workspace_bytes,
+              void* out, int32_t dtype, void* stream);
+
+/*
+ * First step of pa_decode alone: walks the block tables and writes out[] for
+ * every sequence with at most one partition, and the workspace partials
+ * (layout above) for every partition of the longer ones.  Same arguments as
+ * pa_decode.
+ */
+PA_API int pa_decode_partitions(const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_tables, int32_t max_blocks_per_seq,
+                         const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                         int32_t num_blocks, int32_t block_size, float scale,
+                         int32_t partition_blocks, void* workspace, size_t workspace_bytes,
+                         void* out, int32_t dtype, void* stream);
+
+/*
+ * Second step of pa_decode alone: for every sequence with more than one
+ * partition, merges the workspace partials,
+ *   M = max_p m_p,  out = sum_p e^(m_p - M) acc_p / sum_p e^(m_p - M) l_p,
+ * and writes out[] in `dtype`.  Sequences with at most one partition are left
+ * untouched.  The sizes must be those given to pa_decode_partitions.
+ */
+PA_API int pa_decode_reduce(const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                     int32_t max_blocks_per_seq, int32_t block_size,
+                     int32_t partition_blocks, const void* workspace,
+                     size_t workspace_bytes, void* out, int32_t dtype, void* stream);
+
+/*
+ * Reads the sticky device error word of the current device (PA_DEVERR_* bits)
+ * after synchronising `stream`; clears it when `clear` is non-zero.
+ */
+PA_API int pa_get_device_error(uint32_t* bits, int32_t clear, void* stream);
+
+/* Human-readable text for a return code (for PA_ERR_CUDA: the last CUDA error
+ * seen by the calling thread). */
+PA_API const char* pa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H_ */

@@ -94,16 +94,21 @@ def slot_utilisation(lens, block_size: int = 16) -> float:
 
 
 # ---------------------------------------------------------------- cache write
-def cache_write(k, v, slot_mapping, k_cache, v_cache):
-    """Scatter new tokens into copies of the caches; returns (k_cache, v_cache, n_bad).
+def cache_write(k, v, slot_mapping, k_cache, v_cache, inplace=False):
+    """Scatter new tokens into copies of the caches (or into the given C-contiguous
+    caches when inplace=True); returns (k_cache, v_cache, n_bad).
 
     k, v: [T, Hkv, D]; caches [NB, Hkv, B, D]; slot_mapping int64 [T].
     """
     k = np.ascontiguousarray(k)
     v = np.ascontiguousarray(v)
     sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
-    kc = np.array(k_cache, copy=True, order="C")
-    vc = np.array(v_cache, copy=True, order="C")
+    if inplace:
+        assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+        kc, vc = k_cache, v_cache
+    else:
+        kc = np.array(k_cache, copy=True, order="C")
+        vc = np.array(v_cache, copy=True, order="C")
     dt = _dtype_code(k)
     assert kc.dtype == k.dtype == v.dtype == vc.dtype
     T, H, D = k.shape

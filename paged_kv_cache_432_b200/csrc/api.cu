@@ -1,0 +1,519 @@
+// api.cu -- the C ABI of the paged decode library (declared in pagedattn.h).
+//
+// Host side only: validates arguments without touching device memory, plans
+// the split of long sequences into partitions, encodes the TMA tensor maps of
+// the KV pools, sizes persistent grids from the SM count and occupancy, and
+// enqueues the kernels on the caller's stream.  All kernels live in this one
+// translation unit, so the sticky device error word is a single symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "pagedattn.h"
+
+#include "cache_write.cuh"
+#include "common.cuh"
+#include "decode_mma.cuh"
+#include "decode_simt.cuh"
+#include "items.cuh"
+#include "lse_reduce.cuh"
+
+namespace {
+
+using namespace pa;
+
+constexpr int32_t kNoSplit = 1 << 24;       // partition size meaning "never split"
+constexpr int32_t kAutoPartBlocks = 32;     // 512 tokens per partition when splitting
+constexpr int32_t kMaxSeqsPerLaunch = 2048; // sequences whose item prefix one CTA holds
+constexpr int kMaxDevices = 64;
+
+// bf16 kernel configuration: warps per CTA and ring stages per warp.
+constexpr int kMmaWarps = 4;
+constexpr int kMmaStages = 3;
+
+thread_local char g_last_cuda_error[256] = "no CUDA error recorded";
+
+int cuda_fail(cudaError_t e, const char* where) {
+    std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "CUDA error in %s: %s (%s)", where,
+                  cudaGetErrorName(e), cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct DeviceInfo {
+    int sms = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+int device_info(DeviceInfo* out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_dev[dev].sms == 0) {
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        g_dev[dev].sms = sms;
+    }
+    *out = g_dev[dev];
+    return PA_OK;
+}
+
+// Sets the dynamic shared-memory ceiling of `kernel` once per device.
+struct AttrKey {
+    const void* kernel;
+    int dev;
+};
+AttrKey g_attr_done[256];
+int g_attr_count = 0;
+
+template <typename K>
+int ensure_smem_attr(K kernel, size_t bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    const void* kp = reinterpret_cast<const void*>(kernel);
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (int i = 0; i < g_attr_count; ++i)
+        if (g_attr_done[i].kernel == kp && g_attr_done[i].dev == dev) return PA_OK;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bytes));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    if (g_attr_count < 256) g_attr_done[g_attr_count++] = AttrKey{kp, dev};
+    return PA_OK;
+}
+
+template <typename K>
+int persistent_grid(K kernel, int threads, size_t smem, int64_t max_useful_ctas, int* grid) {
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc != PA_OK) return rc;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (per_sm < 1) per_sm = 1;
+    int64_t g = static_cast<int64_t>(di.sms) * per_sm;
+    if (max_useful_ctas < g) g = max_useful_ctas;
+    *grid = static_cast<int>(g < 1 ? 1 : g);
+    return PA_OK;
+}
+
+// ------------------------------------------------------------ TMA tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+cudaError_t g_encode_err = cudaSuccess;
+
+int get_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+    std::call_once(g_encode_once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        g_encode_err = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                                        cudaEnableDefault, &q);
+        if (g_encode_err == cudaSuccess && q != cudaDriverEntryPointSuccess)
+            g_encode_err = cudaErrorSymbolNotFound;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    if (g_encode_err != cudaSuccess) return cuda_fail(g_encode_err, "cudaGetDriverEntryPoint");
+    *fn = g_encode;
+    return PA_OK;
+}
+
+// The pool seen as a 2-D bf16 tensor [num_blocks*Hkv*16 rows][head_dim],
+// loaded in 64-column x 16-row boxes with the 128-byte swizzle.
+int encode_pool_map(CUtensorMap* map, const void* base, int64_t rows, int head_dim) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    int rc = get_encoder(&enc);
+    if (rc != PA_OK) return rc;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
+    cuuint32_t box[2] = {64, 16};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
+                      "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+        return PA_ERR_CUDA;
+    }
+    return PA_OK;
+}
+
+// ------------------------------------------------------------ planning
+int32_t resolve_part_blocks(int32_t max_seq_len, int32_t partition_blocks) {
+    if (partition_blocks > 0) return partition_blocks;
+    if (partition_blocks == -1) return kNoSplit;
+    const int32_t nb = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
+    return nb <= kAutoPartBlocks ? kNoSplit : kAutoPartBlocks;
+}
+
+struct Plan {
+    int32_t part_blocks;
+    int32_t max_parts;
+    int32_t max_len;  // effective max_seq_len (the workspace is sized for it)
+    bool split;
+};
+
+Plan make_plan(int32_t max_seq_len, int32_t partition_blocks) {
+    Plan p;
+    p.max_len = max_seq_len;
+    p.part_blocks = resolve_part_blocks(max_seq_len, partition_blocks);
+    const int32_t nb = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
+    p.max_parts = nb == 0 ? 1 : 1 + (nb - 1) / p.part_blocks;
+    p.split = p.max_parts > 1;
+    return p;
+}
+
+struct WsLayout {
+    size_t off_m, off_l, off_acc, bytes;
+};
+
+WsLayout ws_layout(int64_t rows, int32_t max_parts, int32_t head_dim, bool split) {
+    WsLayout w{0, 0, 0, 0};
+    if (!split) return w;
+    const size_t ml = align256(static_cast<size_t>(rows) * max_parts * sizeof(float));
+    w.off_m = 0;
+    w.off_l = ml;
+    w.off_acc = 2 * ml;
+    w.bytes = 2 * ml + align256(static_cast<size_t>(rows) * max_parts * head_dim * sizeof(float));
+    return w;
+}
+
+struct DecodeArgs {
+    const void* q;
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    int32_t max_blocks_per_seq;
+    const int32_t* seq_lens;
+    int32_t max_seq_len;
+    int32_t num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size;
+    float scale;
+    int32_t partition_blocks;
+    void* workspace;
+    size_t workspace_bytes;
+    void* out;
+    int32_t dtype;
+    cudaStream_t stream;
+};
+
+int check_shapes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                 int32_t block_size, int32_t dtype) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (dtype != PA_DTYPE_F32 && dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (block_size != kBlockTokens) return PA_ERR_UNSUPPORTED;
+    if (num_q_heads / num_kv_heads > 16) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+// Validates and fills the kernel parameter block (workspace pointers included).
+int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan* plan) {
+    int rc = check_shapes(a.num_seqs, a.num_q_heads, a.num_kv_heads, a.head_dim, a.block_size,
+                          a.dtype);
+    if (rc != PA_OK) return rc;
+    if (a.max_blocks_per_seq <= 0 || a.partition_blocks < -1) return PA_ERR_INVALID_ARG;
+    if (!a.seq_lens || !aligned(a.seq_lens, 4) || !a.out || !aligned(a.out, 16))
+        return PA_ERR_INVALID_ARG;
+    if (need_inputs) {
+        if (!a.q || !a.k_cache || !a.v_cache || !a.block_tables) return PA_ERR_INVALID_ARG;
+        if (!aligned(a.q, 16) || !aligned(a.k_cache, 16) || !aligned(a.v_cache, 16) ||
+            !aligned(a.block_tables, 4))
+            return PA_ERR_INVALID_ARG;
+        if (a.num_blocks <= 0) return PA_ERR_INVALID_ARG;
+        // TMA row coordinates and element offsets are 32-bit
+        if (static_cast<int64_t>(a.num_blocks) * a.num_kv_heads * kBlockTokens > INT32_MAX)
+            return PA_ERR_UNSUPPORTED;
+        if (!std::isfinite(a.scale)) return PA_ERR_INVALID_ARG;
+    }
+    const int64_t table_tokens = static_cast<int64_t>(a.max_blocks_per_seq) * kBlockTokens;
+    const int32_t max_len = a.max_seq_len > 0
+                                ? a.max_seq_len
+                                : static_cast<int32_t>(table_tokens > INT32_MAX ? INT32_MAX : table_tokens);
+    *plan = make_plan(max_len, a.partition_blocks);
+    const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
+    const WsLayout ws = ws_layout(rows, plan->max_parts, a.head_dim, plan->split);
+    std::memset(P, 0, sizeof *P);
+    if (plan->split) {
+        if (!a.workspace || !aligned(a.workspace, 256)) return PA_ERR_WORKSPACE;
+        if (a.workspace_bytes < ws.bytes) return PA_ERR_WORKSPACE;
+        char* w = static_cast<char*>(a.workspace);
+        P->ws_m = reinterpret_cast<float*>(w + ws.off_m);
+        P->ws_l = reinterpret_cast<float*>(w + ws.off_l);
+        P->ws_acc = reinterpret_cast<float*>(w + ws.off_acc);
+    }
+    P->q = a.q;
+    P->k_cache = a.k_cache;
+    P->v_cache = a.v_cache;
+    P->block_tables = a.block_tables;
+    P->seq_lens = a.seq_lens;
+    P->out = a.out;
+    P->num_seqs = a.num_seqs;
+    P->num_q_heads = a.num_q_heads;
+    P->num_kv_heads = a.num_kv_heads;
+    P->head_dim = a.head_dim;
+    P->group = a.num_q_heads / a.num_kv_heads;
+    P->max_blocks_per_seq = a.max_blocks_per_seq;
+    P->num_blocks = a.num_blocks;
+    P->part_blocks = plan->part_blocks;
+    P->max_parts = plan->max_parts;
+    P->len_cap = static_cast<int32_t>(max_len < table_tokens ? max_len : table_tokens);
+    P->scale = a.scale;
+    P->scale_log2 = a.scale * 1.4426950408889634f;
+    return PA_OK;
+}
+
+template <int D, int ROWS>
+int launch_mma(const DecodeParams& base, cudaStream_t st) {
+    using Cfg = MmaCfg<D, kMmaStages, kMmaWarps>;
+    auto kernel = decode_bf16_mma_kernel<D, ROWS, kMmaStages, kMmaWarps>;
+    int rc = ensure_smem_attr(kernel, Cfg::smem_bytes(kMaxSeqsPerLaunch));
+    if (rc != PA_OK) return rc;
+    const int64_t rows = static_cast<int64_t>(base.num_blocks) * base.num_kv_heads * kBlockTokens;
+    alignas(64) CUtensorMap mk, mv;
+    if ((rc = encode_pool_map(&mk, base.k_cache, rows, D)) != PA_OK) return rc;
+    if ((rc = encode_pool_map(&mv, base.v_cache, rows, D)) != PA_OK) return rc;
+    for (int32_t b = 0; b < base.num_seqs; b += kMaxSeqsPerLaunch) {
+        DecodeParams P = base;
+        P.seq_begin = b;
+        P.seq_count = base.num_seqs - b < kMaxSeqsPerLaunch ? base.num_seqs - b : kMaxSeqsPerLaunch;
+        const size_t smem = Cfg::smem_bytes(P.seq_count);
+        const int64_t max_items = static_cast<int64_t>(P.seq_count) * P.num_kv_heads * P.max_parts;
+        int grid = 0;
+        rc = persistent_grid(kernel, Cfg::kThreads, smem, (max_items + kMmaWarps - 1) / kMmaWarps,
+                             &grid);
+        if (rc != PA_OK) return rc;
+        kernel<<<grid, Cfg::kThreads, smem, st>>>(mk, mv, P);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "decode_bf16_mma_kernel launch");
+    }
+    return PA_OK;
+}
+
+template <int D, int MAXG>
+int launch_simt(const DecodeParams& base, cudaStream_t st) {
+    auto kernel = decode_f32_simt_kernel<D, MAXG>;
+    for (int32_t b = 0; b < base.num_seqs; b += kMaxSeqsPerLaunch) {
+        DecodeParams P = base;
+        P.seq_begin = b;
+        P.seq_count = base.num_seqs - b < kMaxSeqsPerLaunch ? base.num_seqs - b : kMaxSeqsPerLaunch;
+        const size_t smem = 8 * static_cast<size_t>(P.seq_count + 1);
+        const int64_t max_items = static_cast<int64_t>(P.seq_count) * P.num_kv_heads * P.max_parts;
+        int grid = 0;
+        int rc = persistent_grid(kernel, kSimtWarps * 32, smem,
+                                 (max_items + kSimtWarps - 1) / kSimtWarps, &grid);
+        if (rc != PA_OK) return rc;
+        kernel<<<grid, kSimtWarps * 32, smem, st>>>(P);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "decode_f32_simt_kernel launch");
+    }
+    return PA_OK;
+}
+
+int run_partitions(const DecodeParams& P, int32_t dtype, cudaStream_t st) {
+    if (P.num_seqs == 0) return PA_OK;
+    if (dtype == PA_DTYPE_BF16) {
+        if (P.head_dim == 128) return P.group <= 8 ? launch_mma<128, 8>(P, st) : launch_mma<128, 16>(P, st);
+        return P.group <= 8 ? launch_mma<64, 8>(P, st) : launch_mma<64, 16>(P, st);
+    }
+    if (P.head_dim == 128) return P.group <= 4 ? launch_simt<128, 4>(P, st) : launch_simt<128, 16>(P, st);
+    return P.group <= 4 ? launch_simt<64, 4>(P, st) : launch_simt<64, 16>(P, st);
+}
+
+template <typename OutT, int D>
+int launch_reduce(const DecodeParams& base, cudaStream_t st) {
+    for (int32_t b = 0; b < base.num_seqs; b += kMaxSeqsPerLaunch) {
+        DecodeParams P = base;
+        P.seq_begin = b;
+        P.seq_count = base.num_seqs - b < kMaxSeqsPerLaunch ? base.num_seqs - b : kMaxSeqsPerLaunch;
+        const unsigned grid = static_cast<unsigned>(P.seq_count) * P.num_q_heads;
+        lse_reduce_kernel<OutT, D><<<grid, kReduceWarps * 32, 0, st>>>(P);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "lse_reduce_kernel launch");
+    }
+    return PA_OK;
+}
+
+int run_reduce(const DecodeParams& P, const Plan& plan, int32_t dtype, cudaStream_t st) {
+    if (P.num_seqs == 0 || !plan.split) return PA_OK;
+    if (dtype == PA_DTYPE_BF16)
+        return P.head_dim == 128 ? launch_reduce<__nv_bfloat16, 128>(P, st)
+                                 : launch_reduce<__nv_bfloat16, 64>(P, st);
+    return P.head_dim == 128 ? launch_reduce<float, 128>(P, st) : launch_reduce<float, 64>(P, st);
+}
+
+DecodeArgs make_args(const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                     const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                     int32_t num_blocks, int32_t block_size, float scale,
+                     int32_t partition_blocks, void* workspace, size_t workspace_bytes, void* out,
+                     int32_t dtype, void* stream) {
+    DecodeArgs a;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.seq_lens = seq_lens;
+    a.max_seq_len = max_seq_len;
+    a.num_seqs = num_seqs;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.head_dim = head_dim;
+    a.num_blocks = num_blocks;
+    a.block_size = block_size;
+    a.scale = scale;
+    a.partition_blocks = partition_blocks;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    a.out = out;
+    a.dtype = dtype;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_cache_write(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                   int32_t num_kv_heads, int32_t head_dim, void* k_cache, void* v_cache,
+                   int32_t num_blocks, int32_t block_size, int32_t dtype, void* stream) {
+    int rc = check_shapes(0, num_kv_heads, num_kv_heads, head_dim, block_size, dtype);
+    if (rc != PA_OK) return rc;
+    if (num_tokens < 0 || num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(slot_mapping, 8))
+        return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    const int32_t elem = dtype == PA_DTYPE_F32 ? 4 : 2;
+    const int32_t chunks_per_row = head_dim * elem / 16;
+    const int64_t total = static_cast<int64_t>(num_tokens) * num_kv_heads * chunks_per_row;
+    const int64_t grid = (total + 255) / 256;
+    if (grid > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    cache_write_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, total,
+        num_kv_heads, chunks_per_row, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+        static_cast<int64_t>(num_blocks) * kBlockTokens);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "cache_write_kernel launch");
+    return PA_OK;
+}
+
+int32_t pa_decode_partition_blocks(int32_t num_seqs, int32_t num_kv_heads, int32_t max_seq_len,
+                                   int32_t block_size, int32_t partition_blocks) {
+    if (num_seqs < 0 || num_kv_heads <= 0 || max_seq_len < 0 || partition_blocks < -1)
+        return PA_ERR_INVALID_ARG;
+    if (block_size != kBlockTokens) return PA_ERR_UNSUPPORTED;
+    return resolve_part_blocks(max_seq_len, partition_blocks);
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                int32_t head_dim, int32_t max_seq_len, int32_t block_size,
+                                int32_t partition_blocks) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        max_seq_len < 0 || block_size != kBlockTokens || partition_blocks < -1)
+        return 0;
+    const Plan plan = make_plan(max_seq_len, partition_blocks);
+    return ws_layout(static_cast<int64_t>(num_seqs) * num_q_heads, plan.max_parts, head_dim,
+                     plan.split)
+        .bytes;
+}
+
+int pa_decode_partitions(const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_tables, int32_t max_blocks_per_seq,
+                         const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                         int32_t num_blocks, int32_t block_size, float scale,
+                         int32_t partition_blocks, void* workspace, size_t workspace_bytes,
+                         void* out, int32_t dtype, void* stream) {
+    const DecodeArgs a = make_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                                   max_seq_len, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                   num_blocks, block_size, scale, partition_blocks, workspace,
+                                   workspace_bytes, out, dtype, stream);
+    DecodeParams P;
+    Plan plan;
+    int rc = prepare_decode(a, true, &P, &plan);
+    if (rc != PA_OK) return rc;
+    return run_partitions(P, dtype, a.stream);
+}
+
+int pa_decode_reduce(const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                     int32_t max_blocks_per_seq, int32_t block_size, int32_t partition_blocks,
+                     const void* workspace, size_t workspace_bytes, void* out, int32_t dtype,
+                     void* stream) {
+    const DecodeArgs a = make_args(nullptr, nullptr, nullptr, nullptr, max_blocks_per_seq, seq_lens,
+                                   max_seq_len, num_seqs, num_q_heads, num_kv_heads, head_dim, 1,
+                                   block_size, 1.0f, partition_blocks,
+                                   const_cast<void*>(workspace), workspace_bytes, out, dtype,
+                                   stream);
+    DecodeParams P;
+    Plan plan;
+    int rc = prepare_decode(a, false, &P, &plan);
+    if (rc != PA_OK) return rc;
+    return run_reduce(P, plan, dtype, a.stream);
+}
+
+int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+              int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t max_seq_len,
+              int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+              int32_t num_blocks, int32_t block_size, float scale, int32_t partition_blocks,
+              void* workspace, size_t workspace_bytes, void* out, int32_t dtype, void* stream) {
+    const DecodeArgs a = make_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                                   max_seq_len, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                   num_blocks, block_size, scale, partition_blocks, workspace,
+                                   workspace_bytes, out, dtype, stream);
+    DecodeParams P;
+    Plan plan;
+    int rc = prepare_decode(a, true, &P, &plan);
+    if (rc != PA_OK) return rc;
+    rc = run_partitions(P, dtype, a.stream);
+    if (rc != PA_OK) return rc;
+    return run_reduce(P, plan, dtype, a.stream);
+}
+
+int pa_get_device_error(uint32_t* bits, int32_t clear, void* stream) {
+    if (!bits) return PA_ERR_INVALID_ARG;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int v = 0;
+    e = cudaMemcpyFromSymbol(&v, pa::g_error_bits, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol");
+    if (clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(pa::g_error_bits, &zero, sizeof zero);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
+    }
+    *bits = v;
+    return PA_OK;
+}
+
+const char* pa_status_string(int status) {
+    switch (status) {
+        case PA_OK: return "ok";
+        case PA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad sizes)";
+        case PA_ERR_UNSUPPORTED: return "unsupported dtype, head_dim, block size or group size";
+        case PA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case PA_ERR_CUDA: return g_last_cuda_error;
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// cache_write.cuh -- scatter of newly computed K/V into the paged pool.
+//
+// Token t with slot s >= 0 lands in physical block s / 16 at offset s % 16 of
+// every kv head: the inverse of the block-table lookup that maps logical
+// positions to physical blocks ("Was ändert PagedAttention an der
+// KV-Speicherzuweisung für LLMs?", slavadubrov.com, introduction; 16-token
+// blocks: "Внутреннее устройство vLLM", artificials.ru).
+//
+// One thread moves one 16-byte chunk of K and the same chunk of V; a head row
+// is head_dim * elem bytes (128..512 B), so a warp covers whole rows with
+// fully coalesced 16-byte loads and stores.  Pure data movement: bytes are
+// copied unchanged.
+#pragma once
+
+#include "common.cuh"
+
+namespace pa {
+
+__global__ void __launch_bounds__(256)
+cache_write_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                   const int64_t* __restrict__ slot_mapping, int64_t total_chunks,
+                   int32_t num_kv_heads, int32_t chunks_per_row, uint4* __restrict__ k_cache,
+                   uint4* __restrict__ v_cache, int64_t num_slots) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= total_chunks) return;
+    const int64_t row = i / chunks_per_row;  // (token, head)
+    const int32_t c = static_cast<int32_t>(i - row * chunks_per_row);
+    const int64_t t = row / num_kv_heads;
+    const int32_t h = static_cast<int32_t>(row - t * num_kv_heads);
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) return;  // padding token
+    if (slot >= num_slots) {
+        if (h == 0 && c == 0) flag_error(PA_DEVERR_SLOT_OOB);
+        return;
+    }
+    const int64_t blk = slot / kBlockTokens;
+    const int64_t off = slot - blk * kBlockTokens;
+    const int64_t dst = ((blk * num_kv_heads + h) * kBlockTokens + off) * chunks_per_row + c;
+    const uint4 kv = __ldcs(k + i);
+    const uint4 vv = __ldcs(v + i);
+    k_cache[dst] = kv;
+    v_cache[dst] = vv;
+}
+
+}  // namespace pa

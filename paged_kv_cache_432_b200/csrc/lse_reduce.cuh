@@ -1,0 +1,93 @@
+// lse_reduce.cuh -- log-sum-exp merge of split-K decode partials.
+//
+// A sequence longer than one partition is processed as independent work items
+// over consecutive block ranges; each leaves (m_p, l_p, acc_p): its maximum
+// score, sum of exp(score - m_p) and the matching unnormalised sum of V rows.
+// The exact softmax over the whole sequence is recovered as
+//   M = max_p m_p,  out = sum_p e^(m_p - M) acc_p / sum_p e^(m_p - M) l_p,
+// which is the standard identity behind splitting attention over key ranges
+// (the pages do not describe the split; long sequences are where paged KV
+// matters most: "PagedAttention et vLLM", aiunderstanding.org,
+// §"L'avenir de PagedAttention et vLLM").
+//
+// One CTA (4 warps) per (sequence, query head) row: all threads find M and the
+// denominator, each warp accumulates a strided subset of the partitions'
+// acc rows with 16-byte loads, and the four warp sums are added in a fixed
+// order.  Rows of sequences with at most one partition are skipped (the decode
+// kernel wrote them).
+#pragma once
+
+#include "items.cuh"
+
+namespace pa {
+
+constexpr int kReduceWarps = 4;
+
+template <typename T>
+__device__ __forceinline__ T from_float(float x);
+template <>
+__device__ __forceinline__ float from_float<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+template <typename OutT, int D>
+__global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const DecodeParams P) {
+    constexpr int DPL = D / 32;
+    using Vec = typename std::conditional<DPL == 4, float4, float2>::type;
+    __shared__ float red[kReduceWarps][D];
+    __shared__ float wmax[kReduceWarps], wden[kReduceWarps];
+
+    const int64_t row = blockIdx.x;  // (sequence within launch) * Hq + query head
+    const int32_t s = P.seq_begin + static_cast<int32_t>(row / P.num_q_heads);
+    const int32_t qh = static_cast<int32_t>(row % P.num_q_heads);
+    const SeqGeom geo = seq_geometry(P, P.seq_lens[s]);
+    if (geo.parts <= 1) return;
+    const int parts = geo.parts;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t base = (static_cast<size_t>(s) * P.num_q_heads + qh) * P.max_parts;
+    const float* wm = P.ws_m + base;
+    const float* wl = P.ws_l + base;
+    const float* wa = P.ws_acc + base * D;
+
+    float M = -INFINITY;
+    for (int p = tid; p < parts; p += blockDim.x) M = fmaxf(M, wm[p]);
+    M = warp_max(M);
+    if (lane == 0) wmax[warp] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+
+    OutT* o = static_cast<OutT*>(P.out) + (static_cast<size_t>(s) * P.num_q_heads + qh) * D;
+    if (M == -INFINITY) {  // every partition fully masked
+        for (int d = tid; d < D; d += blockDim.x) o[d] = from_float<OutT>(0.f);
+        return;
+    }
+
+    float den = 0.f;
+    for (int p = tid; p < parts; p += blockDim.x) den += expf(wm[p] - M) * wl[p];
+    den = warp_sum(den);
+    if (lane == 0) wden[warp] = den;
+
+    float a[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) a[e] = 0.f;
+#pragma unroll 4
+    for (int p = warp; p < parts; p += kReduceWarps) {
+        const float w = expf(wm[p] - M);
+        const Vec x = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(p) * D + lane * DPL);
+        const float* f = reinterpret_cast<const float*>(&x);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) a[e] = fmaf(w, f[e], a[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) red[warp][lane * DPL + e] = a[e];
+    __syncthreads();
+    den = (wden[0] + wden[1]) + (wden[2] + wden[3]);
+    const float inv = den > 0.f ? 1.0f / den : 0.f;
+    for (int d = tid; d < D; d += blockDim.x)
+        o[d] = from_float<OutT>(((red[0][d] + red[1][d]) + (red[2][d] + red[3][d])) * inv);
+}
+
+}  // namespace pa

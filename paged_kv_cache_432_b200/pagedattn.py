@@ -1,0 +1,190 @@
+"""Python binding of libpagedattn.so (the C ABI in include/pagedattn.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the library is missing or fails, these
+functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
+
+PA_OK = 0
+PA_ERR_INVALID_ARG = -1
+PA_ERR_UNSUPPORTED = -2
+PA_ERR_WORKSPACE = -3
+PA_ERR_CUDA = -4
+
+PA_DTYPE_F32 = 0
+PA_DTYPE_BF16 = 1
+
+PA_DEVERR_SLOT_OOB = 1
+PA_DEVERR_BLOCK_OOB = 2
+PA_DEVERR_SEQ_LEN = 4
+PA_DEVERR_TIMEOUT = 8
+
+# every symbol the header declares, with (restype, argtypes)
+_P, _I32, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+_DECODE_ARGS = [_P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _F, _I32, _P, _SZ, _P, _I32, _P]
+SIGNATURES = {
+    "pa_cache_write": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _P, _P, _I32, _I32, _I32, _P]),
+    "pa_decode_partition_blocks": (_I32, [_I32, _I32, _I32, _I32, _I32]),
+    "pa_decode_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
+    "pa_decode": (ctypes.c_int, _DECODE_ARGS),
+    "pa_decode_partitions": (ctypes.c_int, _DECODE_ARGS),
+    "pa_decode_reduce": (ctypes.c_int, [_P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ, _P, _I32, _P]),
+    "pa_get_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _I32, _P]),
+    "pa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+}
+
+_lib = None
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = lib().pa_status_string(status).decode()
+        super().__init__(f"{fn} returned {status}: {msg}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing; build it with `python -m paged_kv_cache_432_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def _check(fn: str, rc: int):
+    if rc != PA_OK:
+        raise PagedAttnError(fn, rc)
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return PA_DTYPE_F32
+    if dt == torch.bfloat16:
+        return PA_DTYPE_BF16
+    raise TypeError(f"unsupported dtype {dt}")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def cache_write(k, v, slot_mapping, k_cache, v_cache, stream=None) -> None:
+    """pa_cache_write: k, v [T, Hkv, D]; caches [NB, Hkv, 16, D]; slots int64 [T]."""
+    T, H, D = k.shape
+    NB, H2, B, D2 = k_cache.shape
+    rc = lib().pa_cache_write(_ptr(k), _ptr(v), _ptr(slot_mapping), T, H, D, _ptr(k_cache),
+                              _ptr(v_cache), NB, B, dtype_code(k.dtype), _stream(stream))
+    _check("pa_cache_write", rc)
+
+
+def partition_blocks(num_seqs, num_kv_heads, max_seq_len, partition_blocks=0, block_size=16) -> int:
+    r = lib().pa_decode_partition_blocks(num_seqs, num_kv_heads, max_seq_len, block_size, partition_blocks)
+    if r < 0:
+        raise PagedAttnError("pa_decode_partition_blocks", r)
+    return r
+
+
+def workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len, partition_blocks=0,
+                   block_size=16) -> int:
+    return int(lib().pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                              max_seq_len, block_size, partition_blocks))
+
+
+def alloc_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len, partition_blocks=0,
+                    device=None) -> Optional[torch.Tensor]:
+    n = workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len, partition_blocks)
+    if n == 0:
+        return None
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _decode_call(name, q, k_cache, v_cache, block_tables, seq_lens, scale, out, max_seq_len,
+                 partition_blocks, workspace, stream):
+    N, Hq, D = q.shape
+    NB, Hkv, B, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = getattr(lib(), name)(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1],
+        _ptr(seq_lens), max_seq_len, N, Hq, Hkv, D, NB, B, float(scale), partition_blocks,
+        _ptr(workspace), ws_bytes, _ptr(out), dtype_code(q.dtype), _stream(stream))
+    _check(name, rc)
+
+
+def decode(q, k_cache, v_cache, block_tables, seq_lens, scale, out=None, max_seq_len=0,
+           partition_blocks=0, workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode: out [N, Hq, D] = paged decode attention.  Allocates `out` and the
+    workspace with PyTorch when they are not given."""
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(q.shape[0], q.shape[1], k_cache.shape[1], q.shape[2],
+                                    max_seq_len if max_seq_len > 0 else block_tables.shape[1] * 16,
+                                    partition_blocks, device=q.device)
+    _decode_call("pa_decode", q, k_cache, v_cache, block_tables, seq_lens, scale, out, max_seq_len,
+                 partition_blocks, workspace, stream)
+    return out
+
+
+def decode_partitions(q, k_cache, v_cache, block_tables, seq_lens, scale, out, max_seq_len,
+                      partition_blocks, workspace, stream=None) -> None:
+    """pa_decode_partitions: the block-table walk alone (final rows + partials)."""
+    _decode_call("pa_decode_partitions", q, k_cache, v_cache, block_tables, seq_lens, scale, out,
+                 max_seq_len, partition_blocks, workspace, stream)
+
+
+def decode_reduce(seq_lens, out, num_kv_heads, max_blocks_per_seq, max_seq_len, partition_blocks,
+                  workspace, stream=None) -> None:
+    """pa_decode_reduce: the log-sum-exp merge alone."""
+    N, Hq, D = out.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().pa_decode_reduce(_ptr(seq_lens), max_seq_len, N, Hq, num_kv_heads, D,
+                                max_blocks_per_seq, 16, partition_blocks, _ptr(workspace), ws_bytes,
+                                _ptr(out), dtype_code(out.dtype), _stream(stream))
+    _check("pa_decode_reduce", rc)
+
+
+def device_error(clear: bool = True, stream=None) -> int:
+    """Sticky device error bits (PA_DEVERR_*) of the current device."""
+    bits = ctypes.c_uint32(0)
+    rc = lib().pa_get_device_error(ctypes.byref(bits), 1 if clear else 0, _stream(stream))
+    _check("pa_get_device_error", rc)
+    return int(bits.value)
+
+
+def workspace_views(workspace: torch.Tensor, num_seqs, num_q_heads, head_dim, max_parts):
+    """(m, l, acc) float views of a workspace, following the layout the header
+    documents: arrays of [rows][P] and [rows][P][D] each on a 256-byte boundary."""
+    rows = num_seqs * num_q_heads
+    a256 = lambda x: (x + 255) // 256 * 256
+    ml = a256(rows * max_parts * 4)
+    f = workspace.view(torch.uint8)
+    m = f[:rows * max_parts * 4].view(torch.float32).view(num_seqs, num_q_heads, max_parts)
+    l = f[ml:ml + rows * max_parts * 4].view(torch.float32).view(num_seqs, num_q_heads, max_parts)
+    acc = f[2 * ml:2 * ml + rows * max_parts * head_dim * 4].view(torch.float32).view(
+        num_seqs, num_q_heads, max_parts, head_dim)
+    return m, l, acc

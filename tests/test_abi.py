@@ -1,0 +1,123 @@
+"""The C-ABI library loads, exports every symbol its header declares, and its
+host-side logic (sizing, validation) behaves as documented.  No compute calls:
+nothing here needs a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from paged_kv_cache_432_b200 import build as pa_build
+from paged_kv_cache_432_b200 import pagedattn as pa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pa_build.build()
+    return pa.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["pa_cache_write", "pa_decode", "pa_decode_partitions", "pa_decode_reduce",
+              "pa_decode_workspace_size", "pa_decode_partition_blocks", "pa_get_device_error",
+              "pa_status_string"]:
+        assert n in names
+    assert set(names) == set(pa.SIGNATURES), "binding and header disagree"
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (pa_[a-z_]+)\b", out))
+    for n in declared_functions():
+        assert n in exported, n
+        assert hasattr(lib, n)
+    # nothing else of ours leaks out of the library
+    assert exported == set(declared_functions())
+
+
+def test_status_strings(lib):
+    assert lib.pa_status_string(pa.PA_OK) == b"ok"
+    for s in (pa.PA_ERR_INVALID_ARG, pa.PA_ERR_UNSUPPORTED, pa.PA_ERR_WORKSPACE, pa.PA_ERR_CUDA):
+        assert len(lib.pa_status_string(s)) > 5
+
+
+def test_partition_policy(lib):
+    assert pa.partition_blocks(8, 8, 131072, 32) == 32
+    assert pa.partition_blocks(8, 8, 131072, -1) >= 131072 // 16
+    assert pa.partition_blocks(8, 8, 512, 0) >= 32          # short: never split
+    assert pa.partition_blocks(64, 32, 2048, 0) == 32       # long enough: 512-token partitions
+    assert lib.pa_decode_partition_blocks(8, 8, 100, 8, 0) == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_decode_partition_blocks(8, 8, 100, 16, -2) == pa.PA_ERR_INVALID_ARG
+
+
+def test_workspace_size_matches_documented_layout(lib):
+    a256 = lambda x: (x + 255) // 256 * 256
+    N, Hq, Hkv, D, L = 8, 64, 8, 128, 131072
+    P = -(-(L // 16) // 32)
+    rows = N * Hq
+    expect = 2 * a256(rows * P * 4) + a256(rows * P * D * 4)
+    assert pa.workspace_size(N, Hq, Hkv, D, L, 32) == expect
+    assert pa.workspace_size(N, Hq, Hkv, D, 512, 32) == 0        # one partition: no workspace
+    assert pa.workspace_size(N, Hq, Hkv, D, L, -1) == 0
+    assert pa.workspace_size(N, Hq, Hkv, D, 513, 32) == 2 * a256(rows * 2 * 4) + a256(rows * 2 * D * 4)
+
+
+def _decode_rc(lib, **over):
+    args = dict(q=16, k=16, v=16, bt=16, mb=4, sl=16, msl=64, N=2, Hq=4, Hkv=2, D=128, NB=8, B=16,
+                scale=0.1, pb=0, ws=None, wsb=0, out=16, dt=pa.PA_DTYPE_BF16)
+    args.update(over)
+    a = args
+    return lib.pa_decode(a["q"], a["k"], a["v"], a["bt"], a["mb"], a["sl"], a["msl"], a["N"], a["Hq"],
+                         a["Hkv"], a["D"], a["NB"], a["B"], a["scale"], a["pb"], a["ws"], a["wsb"],
+                         a["out"], a["dt"], None)
+
+
+def test_decode_rejects_bad_arguments_on_the_host(lib):
+    # (fake, never dereferenced addresses: validation happens before any CUDA call)
+    assert _decode_rc(lib, q=None) == pa.PA_ERR_INVALID_ARG
+    assert _decode_rc(lib, q=8) == pa.PA_ERR_INVALID_ARG            # misaligned
+    assert _decode_rc(lib, out=None) == pa.PA_ERR_INVALID_ARG
+    assert _decode_rc(lib, Hq=3) == pa.PA_ERR_INVALID_ARG           # not a multiple of Hkv
+    assert _decode_rc(lib, D=96) == pa.PA_ERR_UNSUPPORTED
+    assert _decode_rc(lib, B=32) == pa.PA_ERR_UNSUPPORTED
+    assert _decode_rc(lib, dt=7) == pa.PA_ERR_UNSUPPORTED
+    assert _decode_rc(lib, Hq=34, Hkv=2) == pa.PA_ERR_UNSUPPORTED   # group of 17
+    assert _decode_rc(lib, mb=0) == pa.PA_ERR_INVALID_ARG
+    assert _decode_rc(lib, pb=-5) == pa.PA_ERR_INVALID_ARG
+    assert _decode_rc(lib, scale=float("nan")) == pa.PA_ERR_INVALID_ARG
+    # split needed (1000 tokens, 32-block partitions) but no workspace
+    assert _decode_rc(lib, mb=64, msl=1000, pb=32) == pa.PA_ERR_WORKSPACE
+    assert _decode_rc(lib, mb=64, msl=1000, pb=32, ws=256, wsb=16) == pa.PA_ERR_WORKSPACE
+
+
+def test_cache_write_rejects_bad_arguments_on_the_host(lib):
+    f = lib.pa_cache_write
+    ok = dict(k=16, v=16, s=16, T=4, H=2, D=128, kc=16, vc=16, NB=8, B=16, dt=pa.PA_DTYPE_BF16)
+
+    def rc(**o):
+        a = dict(ok, **o)
+        return f(a["k"], a["v"], a["s"], a["T"], a["H"], a["D"], a["kc"], a["vc"], a["NB"], a["B"], a["dt"], None)
+
+    assert rc(k=None) == pa.PA_ERR_INVALID_ARG
+    assert rc(s=12) == pa.PA_ERR_INVALID_ARG        # slots not 8-byte aligned
+    assert rc(kc=24) == pa.PA_ERR_INVALID_ARG
+    assert rc(T=-1) == pa.PA_ERR_INVALID_ARG
+    assert rc(NB=0) == pa.PA_ERR_INVALID_ARG
+    assert rc(D=80) == pa.PA_ERR_UNSUPPORTED
+    assert rc(B=8) == pa.PA_ERR_UNSUPPORTED
+    assert rc(T=0) == pa.PA_OK                      # nothing to do, nothing launched
+
+
+def test_get_device_error_rejects_null(lib):
+    assert lib.pa_get_device_error(None, 0, None) == pa.PA_ERR_INVALID_ARG

@@ -1,0 +1,301 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle on the same
+seeded inputs.  Cache writes and block-table indexing are compared bit for bit;
+attention outputs within max-abs 2e-2 / normwise max-rel 1e-2 (bf16) or
+max-abs 1e-5 (fp32)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_close, gpu_decode, host, oracle_decode, to_f64
+from paged_kv_cache_432_b200 import pagedattn as pa
+from paged_kv_cache_432_b200 import workload as wl
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _clean_error_word():
+    if torch.cuda.is_available():
+        from paged_kv_cache_432_b200 import build
+
+        build.build()
+        pa.device_error(clear=True)
+    yield
+
+
+def _bits(a: np.ndarray) -> np.ndarray:
+    return a.view(np.uint32) if a.dtype == np.float32 else a
+
+
+# ------------------------------------------------------------------ cache write
+@pytest.mark.parametrize("name", ["tiny", "mha", "gqa"])
+def test_cache_write_bit_exact(name):
+    w = wl.make(name, device=DEV)
+    h = host(w)
+    kc, vc = w.k_cache.clone(), w.v_cache.clone()
+    pa.cache_write(w.new_k, w.new_v, w.slot_mapping, kc, vc)
+    torch.cuda.synchronize()
+    kc_o, vc_o, bad = oracle.cache_write(h["nk"], h["nv"], h["sm"], h["kc"], h["vc"])
+    assert bad == 0
+    assert np.array_equal(_bits(wl.as_numpy(kc)), _bits(kc_o))
+    assert np.array_equal(_bits(wl.as_numpy(vc)), _bits(vc_o))
+    assert pa.device_error() == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("D", [64, 128])
+def test_cache_write_padding_sentinel_and_out_of_range(dtype, D):
+    g = torch.Generator(device=DEV).manual_seed(5)
+    NB, H, T = 6, 3, 40
+    sentinel = torch.full((NB, H, 16, D), 7.0, dtype=dtype, device=DEV)
+    k = torch.randn((T, H, D), generator=g, device=DEV).to(dtype)
+    v = torch.randn((T, H, D), generator=g, device=DEV).to(dtype)
+    slots = torch.randperm(NB * 16, generator=torch.Generator().manual_seed(1))[:T].to(torch.int64)
+    slots[::7] = -1
+    slots[5] = NB * 16 + 3  # outside the pool: skipped and flagged
+    slots = slots.to(DEV)
+    kc, vc = sentinel.clone(), sentinel.clone()
+    pa.cache_write(k, v, slots, kc, vc)
+    torch.cuda.synchronize()
+    kc_o, vc_o, bad = oracle.cache_write(wl.as_numpy(k), wl.as_numpy(v), wl.as_numpy(slots),
+                                         wl.as_numpy(sentinel), wl.as_numpy(sentinel))
+    assert bad == 1
+    assert np.array_equal(_bits(wl.as_numpy(kc)), _bits(kc_o))
+    assert np.array_equal(_bits(wl.as_numpy(vc)), _bits(vc_o))
+    assert pa.device_error() == pa.PA_DEVERR_SLOT_OOB
+
+
+# ------------------------------------------------------------------ decode, full compare
+@pytest.mark.parametrize("pb", [0, -1, 1, 2])
+def test_tiny_fp32(pb):
+    """The tiny check (lens {35,1,16,17}, fp32, D=64, 2 q heads on 1 kv head)
+    after the cache write of each sequence's newest token."""
+    w = wl.make("tiny", device=DEV)
+    h = host(w)
+    pa.cache_write(w.new_k, w.new_v, w.slot_mapping, w.k_cache, w.v_cache)
+    h["kc"], h["vc"], _ = oracle.cache_write(h["nk"], h["nv"], h["sm"], h["kc"], h["vc"])
+    out = gpu_decode(w, partition_blocks=pb)
+    ref = oracle_decode(w, h)
+    assert_close(to_f64(out), ref, torch.float32, f"tiny pb={pb}")
+    assert pa.device_error() == 0
+
+
+EDGE_LENS = [1, 15, 16, 17, 0, 511, 512, 513, 33, 1000]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (32, 8), (16, 2), (32, 2)])
+@pytest.mark.parametrize("pb", [0, -1, 3, 32])
+def test_edge_lengths(dtype, D, Hq, Hkv, pb):
+    """Lengths at block and partition edges (and an empty sequence), group sizes
+    1..16, both head sizes, split and unsplit."""
+    w = wl.build(EDGE_LENS, Hq, Hkv, D, dtype, seed=D + Hq + Hkv, device=DEV, poison_unused=True)
+    out = gpu_decode(w, partition_blocks=pb)
+    ref = oracle_decode(w)
+    assert_close(to_f64(out), ref, dtype, f"edge {dtype} D={D} {Hq}/{Hkv} pb={pb}")
+    assert (to_f64(out)[EDGE_LENS.index(0)] == 0).all()
+    assert pa.device_error() == 0
+
+
+@pytest.mark.parametrize("name,Hq,Hkv", [("mha", 32, 32), ("gqa", 32, 8), ("long", 64, 8)])
+def test_config_shapes_reduced_lengths(name, Hq, Hkv):
+    """Each config's head layout on lengths the oracle covers in full (several
+    tiles per sequence and ragged tails), in the config's partition setting."""
+    rng = np.random.default_rng(3)
+    lens = [int(x) for x in rng.integers(1, 3000, size=12)] + [2048, 4097]
+    w = wl.build(lens, Hq, Hkv, 128, torch.bfloat16, seed=11, device=DEV,
+                 partition_blocks=32 if name == "long" else 0)
+    out = gpu_decode(w)
+    assert_close(to_f64(out), oracle_decode(w), torch.bfloat16, name)
+
+
+# ------------------------------------------------------------------ full-size configs, sampled rows
+def _sample_rows(w, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = {(int(rng.integers(w.num_seqs)), int(rng.integers(w.num_q_heads))) for _ in range(n)}
+    longest = int(np.argmax(w.lens_host))
+    rows |= {(longest, 0), (longest, w.num_q_heads - 1), (0, 0)}
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name,nrows", [("mha", 48), ("gqa", 48), ("prefix", 32), ("long", 12)])
+def test_full_size_config_sampled_rows(name, nrows):
+    """The config at full size, in the launch configuration the benchmark times
+    (cache write of the newest token, then decode with the config's partition
+    setting); sampled (sequence, head) rows against the oracle."""
+    w = wl.make(name, device=DEV)
+    h = host(w)  # pre-write pools
+    pa.cache_write(w.new_k, w.new_v, w.slot_mapping, w.k_cache, w.v_cache)
+    out = gpu_decode(w)
+    h["kc"], h["vc"], _ = oracle.cache_write(h["nk"], h["nv"], h["sm"], h["kc"], h["vc"])
+    rows = _sample_rows(w, nrows, seed=len(name))
+    ref = oracle_decode(w, h, rows=rows)
+    g = to_f64(out)
+    got = np.stack([g[s, qh] for s, qh in rows])
+    assert_close(got, ref, torch.bfloat16, name)
+    assert np.isfinite(g).all()
+    assert pa.device_error() == 0
+
+
+# ------------------------------------------------------------------ invariances (bitwise on the GPU)
+def test_physical_permutation_is_bitwise_invariant():
+    w = wl.build([35, 1, 16, 17, 700, 1500, 96], 32, 8, 128, torch.bfloat16, seed=21, device=DEV)
+    base = gpu_decode(w)
+    perm = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(2)).to(DEV)
+    kc = torch.empty_like(w.k_cache)
+    vc = torch.empty_like(w.v_cache)
+    kc[perm] = w.k_cache
+    vc[perm] = w.v_cache
+    bt = torch.where(w.block_tables >= 0, perm[w.block_tables.clamp(min=0).long()].int(), w.block_tables)
+    moved = gpu_decode(w, k_cache=kc, v_cache=vc, block_tables=bt)
+    assert torch.equal(base.view(torch.int16), moved.view(torch.int16))
+
+
+@pytest.mark.parametrize("prefix_len", [4096, 4090])
+def test_shared_prefix_matches_private_copies_bitwise(prefix_len):
+    """Sequences sharing prefix blocks give the same bits as the same sequences
+    holding private copies of every block (and, within tolerance, the oracle)."""
+    w = wl.make("prefix", device=DEV, prefix_len=prefix_len)
+    shared = gpu_decode(w)
+    refs = [b for t in w.tables_host for b in t]
+    src = torch.tensor(refs, dtype=torch.long, device=DEV)
+    kc = w.k_cache[src].contiguous()
+    vc = w.v_cache[src].contiguous()
+    bt = torch.full_like(w.block_tables, -1)
+    i = 0
+    for s, t in enumerate(w.tables_host):
+        bt[s, : len(t)] = torch.arange(i, i + len(t), dtype=torch.int32, device=DEV)
+        i += len(t)
+    private = gpu_decode(w, k_cache=kc, v_cache=vc, block_tables=bt)
+    assert torch.equal(shared.view(torch.int16), private.view(torch.int16))
+    rows = _sample_rows(w, 16, seed=prefix_len)
+    ref = oracle_decode(w, rows=rows)
+    g = to_f64(shared)
+    assert_close(np.stack([g[s, qh] for s, qh in rows]), ref, torch.bfloat16, "prefix")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_nan_in_unreachable_slots_changes_nothing(dtype):
+    lens = [35, 1, 16, 17, 513, 250]
+    clean = wl.build(lens, 8, 2, 128, dtype, seed=31, device=DEV)
+    dirty = wl.build(lens, 8, 2, 128, dtype, seed=31, device=DEV, poison_unused=True)
+    assert torch.isnan(dirty.k_cache.float()).any()
+    a, b = gpu_decode(clean, partition_blocks=4), gpu_decode(dirty, partition_blocks=4)
+    assert torch.isfinite(b.float()).all()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("pb", [1, 4, 32])
+def test_split_and_single_pass_agree(pb):
+    w = wl.build([3000, 600, 17, 4096], 64, 8, 128, torch.bfloat16, seed=41, device=DEV)
+    ref = oracle_decode(w)
+    single = gpu_decode(w, partition_blocks=-1)
+    split = gpu_decode(w, partition_blocks=pb)
+    assert_close(to_f64(single), ref, torch.bfloat16, "single")
+    assert_close(to_f64(split), ref, torch.bfloat16, f"split pb={pb}")
+
+
+# ------------------------------------------------------------------ the two steps separately
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_partition_partials_match_oracle(dtype):
+    """pa_decode_partitions alone: the workspace partials (m, l, acc) of every
+    partition against the oracle's split-K form."""
+    pb = 4
+    w = wl.build([300, 64, 65, 17], 8, 2, 128, dtype, seed=51, device=DEV)
+    msl = w.max_seq_len
+    ws = pa.alloc_workspace(w.num_seqs, 8, 2, 128, msl, pb, device=DEV)
+    ws.fill_(0)
+    out = torch.zeros_like(w.q)
+    pa.decode_partitions(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, out, msl, pb, ws)
+    torch.cuda.synchronize()
+    h = host(w)
+    m_o, l_o, acc_o, np_o = oracle.decode_partials(h["q"], h["kc"], h["vc"], h["bt"], h["sl"], w.scale, pb * 16)
+    P = -(-(-(-msl // 16)) // pb)  # ceil(ceil(msl / 16) / pb)
+    m_g, l_g, acc_g = (t.double().cpu().numpy() for t in pa.workspace_views(ws, w.num_seqs, 8, 128, P))
+    for s, L in enumerate(w.lens_host):
+        n = int(np_o[s])
+        if n <= 1:  # written straight to out
+            assert_close(to_f64(out)[s], (acc_o[s, :, 0] / l_o[s, :, 0, None]), dtype, "single-part row")
+            continue
+        tol = 2e-2 if dtype == torch.bfloat16 else 1e-5
+        np.testing.assert_allclose(m_g[s, :, :n], m_o[s, :, :n], rtol=0, atol=tol)
+        # normalised partition outputs and weights
+        assert_close(acc_g[s, :, :n] / l_g[s, :, :n, None], acc_o[s, :, :n] / l_o[s, :, :n, None], dtype, "acc/l")
+        lw_g = l_g[s, :, :n] * np.exp(m_g[s, :, :n] - m_o[s, :, :n])
+        np.testing.assert_allclose(lw_g, l_o[s, :, :n], rtol=1e-2 if dtype == torch.bfloat16 else 1e-5)
+
+
+def test_reduce_of_oracle_partials_matches_oracle_merge():
+    """pa_decode_reduce alone, fed with the oracle's own partials (fp32)."""
+    pb = 2
+    w = wl.build([100, 500, 33, 64, 7], 16, 4, 64, torch.float32, seed=61, device=DEV)
+    msl = w.max_seq_len
+    h = host(w)
+    m_o, l_o, acc_o, np_o = oracle.decode_partials(h["q"], h["kc"], h["vc"], h["bt"], h["sl"], w.scale, pb * 16)
+    P = -(-(-(-msl // 16)) // pb)  # ceil(ceil(msl / 16) / pb)
+    ws = pa.alloc_workspace(w.num_seqs, 16, 4, 64, msl, pb, device=DEV)
+    m_v, l_v, acc_v = pa.workspace_views(ws, w.num_seqs, 16, 64, P)
+    m_v.zero_(), l_v.zero_(), acc_v.zero_()
+    Po = m_o.shape[2]
+    m_v[:, :, :Po] = torch.from_numpy(m_o).float().to(DEV)
+    l_v[:, :, :Po] = torch.from_numpy(l_o).float().to(DEV)
+    acc_v[:, :, :Po] = torch.from_numpy(acc_o).float().to(DEV)
+    out = torch.full_like(w.q, 123.0)
+    pa.decode_reduce(w.seq_lens, out, 4, w.max_blocks_per_seq, msl, pb, ws)
+    torch.cuda.synchronize()
+    ref = oracle.lse_merge(m_o, l_o, acc_o, np_o)
+    g = to_f64(out)
+    for s in range(w.num_seqs):
+        if np_o[s] <= 1:
+            assert (g[s] == 123.0).all()  # left to the partition step
+        else:
+            np.testing.assert_allclose(g[s], ref[s], rtol=0, atol=2e-6)
+
+
+# ------------------------------------------------------------------ limits and device-side errors
+def test_many_sequences_span_several_launches():
+    """More sequences than one launch's item table holds (2048)."""
+    rng = np.random.default_rng(71)
+    lens = [int(x) for x in rng.integers(0, 80, size=2500)]
+    w = wl.build(lens, 4, 1, 64, torch.bfloat16, seed=71, device=DEV)
+    out = gpu_decode(w, partition_blocks=2)
+    assert_close(to_f64(out), oracle_decode(w), torch.bfloat16, "2500 seqs")
+
+
+def test_out_of_pool_block_id_is_masked_and_flagged():
+    w = wl.build([40, 40], 4, 1, 128, torch.bfloat16, seed=81, device=DEV)
+    bt = w.block_tables.clone()
+    bt[1, 1] = w.num_blocks + 5  # second block of sequence 1 points outside the pool
+    out = gpu_decode(w, block_tables=bt)
+    assert pa.device_error() & pa.PA_DEVERR_BLOCK_OOB
+    assert torch.isfinite(out.float()).all()
+    # sequence 0 is untouched by the bad entry
+    ref = oracle_decode(w, rows=[(0, i) for i in range(4)])
+    assert_close(to_f64(out)[0], ref, torch.bfloat16, "seq 0")
+    # sequence 1 equals attention over its remaining tokens (blocks 0 and 2),
+    # packed into a fresh two-block pool for the oracle
+    h = host(w)
+    keep = [t for t in range(40) if t // 16 != 1]
+    packed_k = np.zeros((2, 1, 16, 128), np.uint16)
+    packed_v = np.zeros_like(packed_k)
+    for i, t in enumerate(keep):
+        b = w.tables_host[1][t // 16]
+        packed_k[i // 16, 0, i % 16] = h["kc"][b, 0, t % 16]
+        packed_v[i // 16, 0, i % 16] = h["vc"][b, 0, t % 16]
+    ref1 = oracle.paged_decode(h["q"][1:2], packed_k, packed_v, np.array([[0, 1]], np.int32),
+                               np.array([len(keep)], np.int32), w.scale)
+    assert_close(to_f64(out)[1:2], ref1, torch.bfloat16, "seq 1 without the bad block")
+
+
+def test_sequence_longer_than_bound_is_clamped_and_flagged():
+    w = wl.build([100, 600], 4, 2, 128, torch.bfloat16, seed=91, device=DEV)
+    out = gpu_decode(w, max_seq_len=300, partition_blocks=4)
+    assert pa.device_error() & pa.PA_DEVERR_SEQ_LEN
+    h = host(w)
+    h["sl"] = np.array([100, 300], np.int32)
+    ref = oracle.paged_decode(h["q"], h["kc"], h["vc"], h["bt"], h["sl"], w.scale)
+    assert_close(to_f64(out), ref, torch.bfloat16, "clamped")
