@@ -196,24 +196,33 @@ def dist_setup():
     return ws, rank, local
 
 
-def max_over_ranks(x: float, ws: int) -> float:
+def _reduce(x: float, ws: int, op: str, device) -> float:
     if ws == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
 
 
-def sum_over_ranks(x: float, ws: int) -> float:
-    if ws == 1:
-        return x
-    import torch.distributed as dist
+def aggregate(step_ms: float, step_bytes: float, seqs: int, ws: int, device="cuda") -> dict:
+    """Whole-job numbers of a weak-scaling run: every rank processed its own
+    replica; the job took as long as the slowest rank."""
+    t = _reduce(step_ms, ws, "max", device)
+    b = _reduce(float(step_bytes), ws, "sum", device)
+    n = _reduce(float(seqs), ws, "sum", device)
+    return {"step_ms": t, "bytes": b, "seqs": n, "gbs": b / (t * 1e-3) / 1e9,
+            "tokens_per_s": n / (t * 1e-3)}
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+
+def max_over_ranks(x: float, ws: int, device="cuda") -> float:
+    return _reduce(x, ws, "max", device)
+
+
+def replica_seed(base: int, rank: int) -> int:
+    """Each rank draws its own replica of the workload."""
+    return base + rank
 
 
 def barrier(ws: int):
@@ -314,7 +323,7 @@ def run_ours(args) -> None:
         pa_build.build()
     barrier(ws)
     dev = torch.device("cuda", local)
-    w = wl.make(args.config, seed=args.seed + rank, device=dev)
+    w = wl.make(args.config, seed=replica_seed(args.seed, rank), device=dev)
     pb = w.partition_blocks if args.partition_blocks is None else args.partition_blocks
     msl = w.max_seq_len
     resolved_pb = pa.partition_blocks(w.num_seqs, w.num_kv_heads, msl, pb)
@@ -370,13 +379,11 @@ def run_ours(args) -> None:
         tot, dec, red, wr, clocks = timed()
         clocks["remeasured"] = True
     K = args.steps
-    step_ms = max_over_ranks(tot / K, ws)
+    agg = aggregate(tot / K, by["step"], w.num_seqs, ws)
+    step_ms, total_bytes, total_seqs, value = agg["step_ms"], agg["bytes"], agg["seqs"], agg["gbs"]
     dec_ms = max_over_ranks(dec / K, ws)
     red_ms = max_over_ranks(red / K, ws)
     wr_ms = max_over_ranks(wr / K, ws)
-    total_bytes = sum_over_ranks(by["step"], ws)
-    total_seqs = sum_over_ranks(w.num_seqs, ws)
-    value = total_bytes / (step_ms * 1e-3) / 1e9
 
     # ---- end to end through the public API: inputs from pinned host memory,
     # result read back, every step
