@@ -6,8 +6,9 @@
 One step = one pass of the hot path over one batch: the cache write of each
 sequence's newest token (pa_cache_write), then the decode (the block-table
 walk with split-K partials, pa_decode_partitions, and the log-sum-exp merge,
-pa_decode_reduce).  Inputs are resident in HBM; L2 is flushed (512 MiB write)
-before every step, outside the timed events.  Times are CUDA events on the
+pa_decode_reduce).  Inputs are resident in HBM; L2 is flushed before every
+step (a 512 MiB write, then a 256 MiB read so no dirty lines are left to
+write back inside the next step), outside the timed events.  Times are CUDA events on the
 launching stream; with N > 1 (torchrun) every rank runs its own replica of the
 workload (seed + rank, no data exchange) and the step time is the max over
 ranks.  Prints one JSON line.
@@ -78,10 +79,12 @@ def workload_config(w: wl.Workload, pb: int) -> dict:
         "block_size": w.block_size,
         "pool_blocks": w.num_blocks,
         "partition_blocks": pb,
+        "split": "balanced (equal blocks per warp)" if pb == 0 else (
+            "never" if pb >= (1 << 24) else f"fixed {pb}-block partitions"),
         "new_tokens": int(w.slot_mapping.numel()),
         "slot_utilisation": round(sum(w.lens_host) / (16 * sum(len(t) for t in w.tables_host)), 5),
-        "l2": "flushed before every step (512 MiB write, outside the timed events); KV footprint "
-              "exceeds L2",
+        "l2": "flushed before every step (512 MiB write + 256 MiB read, outside the timed "
+              "events); KV footprint exceeds L2",
     }
 
 
@@ -327,10 +330,18 @@ def run_ours(args) -> None:
     pb = w.partition_blocks if args.partition_blocks is None else args.partition_blocks
     msl = w.max_seq_len
     resolved_pb = pa.partition_blocks(w.num_seqs, w.num_kv_heads, msl, pb)
-    split = math.ceil(math.ceil(msl / 16) / resolved_pb) > 1
     wsp = pa.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, msl, pb, device=dev)
+    split = wsp is not None
     out = torch.empty_like(w.q)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(FLUSH_BYTES // 2, dtype=torch.uint8, device=dev)
+
+    def flush_l2():
+        # evict everything: write a buffer 4x the L2, then read another 2x the
+        # L2 so the lines left behind are clean (no write-back lands in the
+        # next timed step)
+        flush_w.zero_()
+        flush_r.view(torch.int32).sum()
     stream = torch.cuda.current_stream(dev)
     by = algorithmic_bytes(w)
     chunks = math.ceil(w.num_seqs / 2048)
@@ -352,7 +363,7 @@ def run_ours(args) -> None:
             ev[3].record(stream)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         step()
     torch.cuda.synchronize(dev)
     if pa.device_error() != 0:
@@ -364,7 +375,7 @@ def run_ours(args) -> None:
         torch.cuda.synchronize(dev)
         with ClockSampler(local) as cs:
             for k in range(args.steps):
-                flush.zero_()
+                flush_l2()
                 step(evs[k])
             torch.cuda.synchronize(dev)
         barrier(ws)
@@ -405,14 +416,14 @@ def run_ours(args) -> None:
             host_out.copy_(out, non_blocking=True)
 
         for _ in range(args.warmup):
-            flush.zero_()
+            flush_l2()
             e2e_step()
         n_e2e = max(3, min(K, 50))
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_e2e)]
         barrier(ws)
         torch.cuda.synchronize(dev)
         for k in range(n_e2e):
-            flush.zero_()
+            flush_l2()
             evs[k][0].record(stream)
             e2e_step()
             evs[k][1].record(stream)

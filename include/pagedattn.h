@@ -87,27 +87,38 @@ PA_API int pa_cache_write(const void* k, const void* v, const int64_t* slot_mapp
                    int32_t block_size, int32_t dtype, void* stream);
 
 /*
- * Blocks per partition the decode uses: partition_blocks > 0 is taken as is,
- * -1 means never split (one pass over the whole sequence), 0 lets the library
- * choose from the sizes.  Returns the resolved value (a value >= the blocks of
- * max_seq_len means no split), or a negative status on bad arguments.
+ * How the decode splits sequences, from partition_blocks:
+ *   0   (auto) balanced split.  All (sequence, kv head) units form one stream
+ *       of blocks and every warp of the persistent grid takes an equal share
+ *       (at least 32 blocks), so long and short sequences mix without load
+ *       imbalance.  A unit that spans several shares becomes several pieces.
+ *   > 0 fixed partitions of that many blocks.
+ *   -1  never split: one pass over each whole sequence.
+ * Returns 0 for the balanced split, the partition size otherwise (a value >=
+ * the blocks of max_seq_len means no split), or a negative status on bad
+ * arguments.
  */
 PA_API int32_t pa_decode_partition_blocks(int32_t num_seqs, int32_t num_kv_heads,
-                                   int32_t max_seq_len, int32_t block_size,
-                                   int32_t partition_blocks);
+                                          int32_t max_seq_len, int32_t block_size,
+                                          int32_t partition_blocks);
 
 /*
- * Bytes of workspace pa_decode needs for these sizes (0 when no sequence of
- * up to max_seq_len tokens is split).  Workspace layout, P = partitions per
- * sequence at max_seq_len, rows r = seq * num_q_heads + q_head:
- *   float m  [num_seqs*num_q_heads][P]     max score of the partition (natural log units)
- *   float l  [num_seqs*num_q_heads][P]     sum of exp(score - m)
- *   float acc[num_seqs*num_q_heads][P][D]  sum of exp(score - m) * v
- * each array starting on a 256-byte boundary.
+ * Bytes of workspace pa_decode needs for these sizes (0 when no sequence of up
+ * to max_seq_len tokens can be split).  Workspace layout: P is the number of
+ * pieces a unit can have at max_seq_len (fixed: ceil(nb / partition_blocks);
+ * balanced: ceil(nb / 32) + 1, with nb = ceil(max_seq_len / 16)), and rows
+ * r = seq * num_q_heads + q_head:
+ *   float   m    [num_seqs*num_q_heads][P]    max score of the piece (natural log units)
+ *   float   l    [num_seqs*num_q_heads][P]    sum of exp(score - m)
+ *   float   acc  [num_seqs*num_q_heads][P][D] sum of exp(score - m) * v
+ *   int32_t parts[num_seqs*num_kv_heads]      pieces of each (sequence, kv head)
+ * each array starting on a 256-byte boundary.  Its contents need no
+ * initialisation: every value read is written first in the same call.
  */
-PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
-                                int32_t head_dim, int32_t max_seq_len, int32_t block_size,
-                                int32_t partition_blocks);
+PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                       int32_t num_kv_heads, int32_t head_dim,
+                                       int32_t max_seq_len, int32_t block_size,
+                                       int32_t partition_blocks);
 
 /*
  * Paged decode attention: for each sequence s and query head i,
@@ -115,9 +126,10 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, in
  * where K_s[t] = k_cache[block_tables[s][t / bs]][i / group][t % bs] (same for V).
  * Accumulation is fp32 (bf16 inputs: scores and P.V on tensor cores with fp32
  * accumulators); out is rounded to the input dtype (round to nearest even).  A
- * zero-length sequence gives a zero row.  Sequences longer than
- * partition_blocks * block_size tokens are split into partitions whose partial
- * results are merged by a log-sum-exp reduction (pa_decode runs both steps).
+ * zero-length sequence gives a zero row.  Sequences are cut into pieces as
+ * partition_blocks says (pa_decode_partition_blocks) and the partial results of
+ * a split sequence are merged by a log-sum-exp reduction (pa_decode runs both
+ * steps).
  * max_seq_len is a host-side bound on seq_lens (<= 0: max_blocks_per_seq *
  * block_size); it sizes the workspace, and longer sequences are clamped to it
  * with PA_DEVERR_SEQ_LEN set.  Table entries past a sequence's last block are
@@ -137,9 +149,8 @@ PA_API int pa_decode(const void* q, const void* k_cache, const void* v_cache,
 
 /*
  * First step of pa_decode alone: walks the block tables and writes out[] for
- * every sequence with at most one partition, and the workspace partials
- * (layout above) for every partition of the longer ones.  Same arguments as
- * pa_decode.
+ * every (sequence, kv head) that is one piece, and the workspace partials
+ * (layout above) for every piece of the others.  Same arguments as pa_decode.
  */
 PA_API int pa_decode_partitions(const void* q, const void* k_cache, const void* v_cache,
                          const int32_t* block_tables, int32_t max_blocks_per_seq,
@@ -150,11 +161,12 @@ PA_API int pa_decode_partitions(const void* q, const void* k_cache, const void* 
                          void* out, int32_t dtype, void* stream);
 
 /*
- * Second step of pa_decode alone: for every sequence with more than one
- * partition, merges the workspace partials,
+ * Second step of pa_decode alone: for every (sequence, kv head) with more than
+ * one piece (the count recorded in the workspace), merges the partials of its
+ * query heads,
  *   M = max_p m_p,  out = sum_p e^(m_p - M) acc_p / sum_p e^(m_p - M) l_p,
- * and writes out[] in `dtype`.  Sequences with at most one partition are left
- * untouched.  The sizes must be those given to pa_decode_partitions.
+ * and writes out[] in `dtype`.  Rows of single-piece units are left untouched.
+ * The sizes must be those given to pa_decode_partitions.
  */
 PA_API int pa_decode_reduce(const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,

@@ -153,42 +153,57 @@ int encode_pool_map(CUtensorMap* map, const void* base, int64_t rows, int head_d
 }
 
 // ------------------------------------------------------------ planning
-int32_t resolve_part_blocks(int32_t max_seq_len, int32_t partition_blocks) {
+constexpr int32_t kMinChunk = 32;  // balanced split: fewest blocks in one warp's range
+
+// Fixed partition size for partition_blocks > 0 or -1 (never split); 0 for the
+// balanced split (partition_blocks = 0).
+int32_t resolve_part_blocks(int32_t partition_blocks) {
     if (partition_blocks > 0) return partition_blocks;
     if (partition_blocks == -1) return kNoSplit;
-    const int32_t nb = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
-    return nb <= kAutoPartBlocks ? kNoSplit : kAutoPartBlocks;
+    return 0;
 }
 
 struct Plan {
-    int32_t part_blocks;
-    int32_t max_parts;
-    int32_t max_len;  // effective max_seq_len (the workspace is sized for it)
+    bool balanced;
+    int32_t part_blocks;  // fixed mode
+    int32_t max_parts;    // pieces per unit the workspace holds
+    int32_t max_len;      // effective max_seq_len (the workspace is sized for it)
     bool split;
 };
 
 Plan make_plan(int32_t max_seq_len, int32_t partition_blocks) {
     Plan p;
     p.max_len = max_seq_len;
-    p.part_blocks = resolve_part_blocks(max_seq_len, partition_blocks);
     const int32_t nb = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
-    p.max_parts = nb == 0 ? 1 : 1 + (nb - 1) / p.part_blocks;
+    const int32_t pb = resolve_part_blocks(partition_blocks);
+    p.balanced = pb == 0;
+    if (p.balanced) {
+        // a unit of nb blocks meets at most ceil(nb / C) + 1 warp ranges of C >= kMinChunk
+        p.part_blocks = kNoSplit;
+        p.max_parts = nb == 0 ? 1 : (nb + kMinChunk - 1) / kMinChunk + 1;
+    } else {
+        p.part_blocks = pb;
+        p.max_parts = nb == 0 ? 1 : 1 + (nb - 1) / pb;
+    }
     p.split = p.max_parts > 1;
     return p;
 }
 
 struct WsLayout {
-    size_t off_m, off_l, off_acc, bytes;
+    size_t off_m, off_l, off_acc, off_parts, bytes;
 };
 
-WsLayout ws_layout(int64_t rows, int32_t max_parts, int32_t head_dim, bool split) {
-    WsLayout w{0, 0, 0, 0};
+WsLayout ws_layout(int64_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_parts,
+                   int32_t head_dim, bool split) {
+    WsLayout w{0, 0, 0, 0, 0};
     if (!split) return w;
+    const int64_t rows = num_seqs * num_q_heads;
     const size_t ml = align256(static_cast<size_t>(rows) * max_parts * sizeof(float));
     w.off_m = 0;
     w.off_l = ml;
     w.off_acc = 2 * ml;
-    w.bytes = 2 * ml + align256(static_cast<size_t>(rows) * max_parts * head_dim * sizeof(float));
+    w.off_parts = w.off_acc + align256(static_cast<size_t>(rows) * max_parts * head_dim * sizeof(float));
+    w.bytes = w.off_parts + align256(static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int32_t));
     return w;
 }
 
@@ -245,8 +260,8 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
                                 ? a.max_seq_len
                                 : static_cast<int32_t>(table_tokens > INT32_MAX ? INT32_MAX : table_tokens);
     *plan = make_plan(max_len, a.partition_blocks);
-    const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
-    const WsLayout ws = ws_layout(rows, plan->max_parts, a.head_dim, plan->split);
+    const WsLayout ws = ws_layout(a.num_seqs, a.num_q_heads, a.num_kv_heads, plan->max_parts,
+                                  a.head_dim, plan->split);
     std::memset(P, 0, sizeof *P);
     if (plan->split) {
         if (!a.workspace || !aligned(a.workspace, 256)) return PA_ERR_WORKSPACE;
@@ -255,6 +270,7 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
         P->ws_m = reinterpret_cast<float*>(w + ws.off_m);
         P->ws_l = reinterpret_cast<float*>(w + ws.off_l);
         P->ws_acc = reinterpret_cast<float*>(w + ws.off_acc);
+        P->ws_parts = reinterpret_cast<int32_t*>(w + ws.off_parts);
     }
     P->q = a.q;
     P->k_cache = a.k_cache;
@@ -270,11 +286,22 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
     P->max_blocks_per_seq = a.max_blocks_per_seq;
     P->num_blocks = a.num_blocks;
     P->part_blocks = plan->part_blocks;
+    P->balanced = plan->balanced ? 1 : 0;
+    P->min_chunk = kMinChunk;
     P->max_parts = plan->max_parts;
     P->len_cap = static_cast<int32_t>(max_len < table_tokens ? max_len : table_tokens);
     P->scale = a.scale;
     P->scale_log2 = a.scale * 1.4426950408889634f;
     return PA_OK;
+}
+
+// Sequences per launch: the per-CTA prefix holds at most kMaxSeqsPerLaunch
+// entries, and its running sums (blocks x kv heads) must fit in 32 bits.
+int32_t seqs_per_launch(const DecodeParams& P) {
+    const int64_t nb_cap = (static_cast<int64_t>(P.len_cap) + kBlockTokens - 1) / kBlockTokens;
+    const int64_t per_seq = (nb_cap > 0 ? nb_cap : 1) * P.num_kv_heads;
+    const int64_t lim = static_cast<int64_t>(INT32_MAX) / per_seq;
+    return static_cast<int32_t>(lim < kMaxSeqsPerLaunch ? (lim < 1 ? 1 : lim) : kMaxSeqsPerLaunch);
 }
 
 template <int D, int ROWS>
@@ -287,14 +314,15 @@ int launch_mma(const DecodeParams& base, cudaStream_t st) {
     alignas(64) CUtensorMap mk, mv;
     if ((rc = encode_pool_map(&mk, base.k_cache, rows, D)) != PA_OK) return rc;
     if ((rc = encode_pool_map(&mv, base.v_cache, rows, D)) != PA_OK) return rc;
-    for (int32_t b = 0; b < base.num_seqs; b += kMaxSeqsPerLaunch) {
+    const int32_t chunk = seqs_per_launch(base);
+    for (int32_t b = 0; b < base.num_seqs; b += chunk) {
         DecodeParams P = base;
         P.seq_begin = b;
-        P.seq_count = base.num_seqs - b < kMaxSeqsPerLaunch ? base.num_seqs - b : kMaxSeqsPerLaunch;
+        P.seq_count = base.num_seqs - b < chunk ? base.num_seqs - b : chunk;
         const size_t smem = Cfg::smem_bytes(P.seq_count);
-        const int64_t max_items = static_cast<int64_t>(P.seq_count) * P.num_kv_heads * P.max_parts;
+        const int64_t max_pieces = static_cast<int64_t>(P.seq_count) * P.num_kv_heads * P.max_parts;
         int grid = 0;
-        rc = persistent_grid(kernel, Cfg::kThreads, smem, (max_items + kMmaWarps - 1) / kMmaWarps,
+        rc = persistent_grid(kernel, Cfg::kThreads, smem, (max_pieces + kMmaWarps - 1) / kMmaWarps,
                              &grid);
         if (rc != PA_OK) return rc;
         kernel<<<grid, Cfg::kThreads, smem, st>>>(mk, mv, P);
@@ -307,15 +335,16 @@ int launch_mma(const DecodeParams& base, cudaStream_t st) {
 template <int D, int MAXG>
 int launch_simt(const DecodeParams& base, cudaStream_t st) {
     auto kernel = decode_f32_simt_kernel<D, MAXG>;
-    for (int32_t b = 0; b < base.num_seqs; b += kMaxSeqsPerLaunch) {
+    const int32_t chunk = seqs_per_launch(base);
+    for (int32_t b = 0; b < base.num_seqs; b += chunk) {
         DecodeParams P = base;
         P.seq_begin = b;
-        P.seq_count = base.num_seqs - b < kMaxSeqsPerLaunch ? base.num_seqs - b : kMaxSeqsPerLaunch;
+        P.seq_count = base.num_seqs - b < chunk ? base.num_seqs - b : chunk;
         const size_t smem = 8 * static_cast<size_t>(P.seq_count + 1);
-        const int64_t max_items = static_cast<int64_t>(P.seq_count) * P.num_kv_heads * P.max_parts;
+        const int64_t max_pieces = static_cast<int64_t>(P.seq_count) * P.num_kv_heads * P.max_parts;
         int grid = 0;
         int rc = persistent_grid(kernel, kSimtWarps * 32, smem,
-                                 (max_items + kSimtWarps - 1) / kSimtWarps, &grid);
+                                 (max_pieces + kSimtWarps - 1) / kSimtWarps, &grid);
         if (rc != PA_OK) return rc;
         kernel<<<grid, kSimtWarps * 32, smem, st>>>(P);
         cudaError_t e = cudaGetLastError();
@@ -336,10 +365,11 @@ int run_partitions(const DecodeParams& P, int32_t dtype, cudaStream_t st) {
 
 template <typename OutT, int D>
 int launch_reduce(const DecodeParams& base, cudaStream_t st) {
-    for (int32_t b = 0; b < base.num_seqs; b += kMaxSeqsPerLaunch) {
+    const int32_t chunk = seqs_per_launch(base);
+    for (int32_t b = 0; b < base.num_seqs; b += chunk) {
         DecodeParams P = base;
         P.seq_begin = b;
-        P.seq_count = base.num_seqs - b < kMaxSeqsPerLaunch ? base.num_seqs - b : kMaxSeqsPerLaunch;
+        P.seq_count = base.num_seqs - b < chunk ? base.num_seqs - b : chunk;
         const unsigned grid = static_cast<unsigned>(P.seq_count) * P.num_q_heads;
         lse_reduce_kernel<OutT, D><<<grid, kReduceWarps * 32, 0, st>>>(P);
         cudaError_t e = cudaGetLastError();
@@ -421,7 +451,7 @@ int32_t pa_decode_partition_blocks(int32_t num_seqs, int32_t num_kv_heads, int32
     if (num_seqs < 0 || num_kv_heads <= 0 || max_seq_len < 0 || partition_blocks < -1)
         return PA_ERR_INVALID_ARG;
     if (block_size != kBlockTokens) return PA_ERR_UNSUPPORTED;
-    return resolve_part_blocks(max_seq_len, partition_blocks);
+    return resolve_part_blocks(partition_blocks);
 }
 
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
@@ -431,9 +461,7 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t n
         max_seq_len < 0 || block_size != kBlockTokens || partition_blocks < -1)
         return 0;
     const Plan plan = make_plan(max_seq_len, partition_blocks);
-    return ws_layout(static_cast<int64_t>(num_seqs) * num_q_heads, plan.max_parts, head_dim,
-                     plan.split)
-        .bytes;
+    return ws_layout(num_seqs, num_q_heads, num_kv_heads, plan.max_parts, head_dim, plan.split).bytes;
 }
 
 int pa_decode_partitions(const void* q, const void* k_cache, const void* v_cache,

@@ -37,6 +37,7 @@ struct DecodeParams {
     float* ws_m;    // [num_seqs*num_q_heads][max_parts]        (null: no split)
     float* ws_l;    // [num_seqs*num_q_heads][max_parts]
     float* ws_acc;  // [num_seqs*num_q_heads][max_parts][head_dim]
+    int32_t* ws_parts;  // [num_seqs*num_kv_heads] pieces of each unit (split only)
     int32_t num_seqs;
     int32_t num_q_heads;
     int32_t num_kv_heads;
@@ -44,8 +45,10 @@ struct DecodeParams {
     int32_t group;               // num_q_heads / num_kv_heads
     int32_t max_blocks_per_seq;  // table row width
     int32_t num_blocks;          // pool size in blocks
-    int32_t part_blocks;         // blocks per partition (huge = never split)
-    int32_t max_parts;           // partitions per row in the workspace
+    int32_t part_blocks;         // fixed mode: blocks per partition (huge = never split)
+    int32_t balanced;            // 1: balanced stream split, 0: fixed partitions
+    int32_t min_chunk;           // balanced mode: fewest blocks a warp range holds
+    int32_t max_parts;           // pieces per row the workspace holds
     int32_t len_cap;             // longest sequence handled; longer ones are clamped
     int32_t seq_begin;           // first sequence of this launch
     int32_t seq_count;           // sequences in this launch

@@ -105,13 +105,14 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int st = 0; st < STAGES; ++st) mbar_init(smem_u32(&bars[st]), 1);
         fence_barrier_init();
     }
-    const int32_t total = build_item_prefix(P, prefix, lens);  // ends with __syncthreads
+    const Schedule sched = make_schedule(P, prefix, lens, WARPS);  // ends with __syncthreads
     zero_empty_sequences<__nv_bfloat16>(P, lens);
 
-    const int32_t nw = gridDim.x * WARPS;
-    int32_t prod_item = blockIdx.x * WARPS + warp;
-    if (prod_item >= total) return;
-    int32_t cons_item = prod_item;
+    const int32_t my_warp = blockIdx.x * WARPS + warp;
+    Cursor pc;  // producer: the piece whose next block is loaded next
+    sched.start(pc, my_warp);
+    if (!pc.valid) return;
+    Cursor cc = pc;  // consumer: the piece being computed
 
     const uint64_t policy = l2_policy_evict_first();
     const uint32_t ring_u32 = smem_u32(ring);
@@ -122,20 +123,20 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const CUtensorMap* map_v = &tmap_v;
 
     // ---------------- producer state (warp-uniform except `tbl`)
-    Item pi = decode_item(P, prefix, lens, prod_item);
-    int32_t pj = pi.jbeg;
+    int32_t pj = pc.jbeg;
     bool prod_live = true;
-    int32_t tbl = 0, tbase = 0, titem = -1;
-    uint32_t oob_mask = 0;  // stages whose block id was outside the pool
+    int32_t tbl = 0, tbase = 0;
+    bool tbl_fresh = false;  // tbl holds entries of the producer's current piece
+    uint32_t oob_mask = 0;   // stages whose block id was outside the pool
     uint32_t issued = 0, consumed = 0;
 
     auto produce = [&](int stage) {
-        if (titem != prod_item || pj >= tbase + 32) {
+        if (!tbl_fresh || pj >= tbase + 32) {
             tbase = pj;
-            titem = prod_item;
+            tbl_fresh = true;
             const int32_t jj = tbase + lane;
-            tbl = jj < pi.jend
-                      ? __ldg(P.block_tables + static_cast<size_t>(pi.s) * P.max_blocks_per_seq + jj)
+            tbl = jj < pc.jend
+                      ? __ldg(P.block_tables + static_cast<size_t>(pc.s) * P.max_blocks_per_seq + jj)
                       : 0;
         }
         int32_t pb = __shfl_sync(kFullMask, tbl, pj - tbase);
@@ -151,7 +152,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             fence_proxy_async_smem();
             const uint32_t bar = bar_u32 + stage * 8;
             mbar_arrive_expect_tx(bar, Cfg::kStageBytes);
-            const int32_t row = (pb * Hkv + pi.h) * kBlockTokens;
+            const int32_t row = (pb * Hkv + pc.h) * kBlockTokens;
             const uint32_t kdst = ring_u32 + stage * Cfg::kStageBytes;
 #pragma unroll
             for (int r = 0; r < Cfg::kRegions; ++r) {
@@ -161,22 +162,18 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
         ++issued;
-        if (++pj == pi.jend) {
-            prod_item += nw;
-            if (prod_item < total) {
-                pi = decode_item(P, prefix, lens, prod_item);
-                pj = pi.jbeg;
-            } else {
-                prod_live = false;
-            }
+        if (++pj == pc.jend) {
+            sched.next(pc);
+            tbl_fresh = false;
+            if (pc.valid) pj = pc.jbeg;
+            else prod_live = false;
         }
     };
 
     for (int st = 0; st < STAGES && prod_live; ++st) produce(st);
 
     // ---------------- consumer
-    Item ci = decode_item(P, prefix, lens, cons_item);
-    int32_t cj = ci.jbeg;
+    int32_t cj = cc.jbeg;
     int stage = 0;
     uint32_t phase = 0;
 
@@ -190,9 +187,9 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     float acc[NTD][4];
 
     while (true) {
-        if (cj == ci.jbeg) {  // new item: load its query rows as A fragments
+        if (cj == cc.jbeg) {  // new item: load its query rows as A fragments
             const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(P.q) +
-                                      (static_cast<size_t>(ci.s) * P.num_q_heads + ci.h * g) * D;
+                                      (static_cast<size_t>(cc.s) * P.num_q_heads + cc.h * g) * D;
             const uint32_t* q_lo = reinterpret_cast<const uint32_t*>(qg + r_lo * D + tq);
             const uint32_t* q_hi = reinterpret_cast<const uint32_t*>(qg + (r_lo + 8) * D + tq);
             const bool lo_ok = r_lo < g, hi_ok = HI && (r_lo + 8 < g);
@@ -222,7 +219,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         ++consumed;
         const uint32_t kbase = ring_u32 + stage * Cfg::kStageBytes;
         const uint32_t vbase = kbase + Cfg::kTileBytes;
-        const int valid = ((oob_mask >> stage) & 1u) ? 0 : min(kBlockTokens, ci.len - cj * kBlockTokens);
+        const int valid = ((oob_mask >> stage) & 1u) ? 0 : min(kBlockTokens, cc.len - cj * kBlockTokens);
         if (valid < kBlockTokens) {
             // zero V rows [valid, 16) so that 0 * (stale or NaN) never enters P V
             uint8_t* vs = ring + stage * Cfg::kStageBytes + Cfg::kTileBytes;
@@ -301,7 +298,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             phase ^= 1;
         }
 
-        if (++cj < ci.jend) continue;
+        if (++cj < cc.jend) continue;
 
         // ---- item done: final row or partition partials
         float lt_lo = l_lo + __shfl_xor_sync(kFullMask, l_lo, 1);
@@ -311,12 +308,12 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             lt_hi = l_hi + __shfl_xor_sync(kFullMask, l_hi, 1);
             lt_hi += __shfl_xor_sync(kFullMask, lt_hi, 2);
         }
-        const int qh_lo = ci.h * g + r_lo;
-        if (ci.parts == 1) {
+        const int qh_lo = cc.h * g + r_lo;
+        if (cc.parts == 1) {
             __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(P.out);
             if (r_lo < g) {
                 const float inv = lt_lo > 0.f ? 1.0f / lt_lo : 0.f;
-                __nv_bfloat16* o = ob + (static_cast<size_t>(ci.s) * P.num_q_heads + qh_lo) * D + tq;
+                __nv_bfloat16* o = ob + (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo) * D + tq;
 #pragma unroll
                 for (int n = 0; n < NTD; ++n)
                     *reinterpret_cast<__nv_bfloat162*>(o + 8 * n) =
@@ -324,7 +321,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             if (HI && r_lo + 8 < g) {
                 const float inv = lt_hi > 0.f ? 1.0f / lt_hi : 0.f;
-                __nv_bfloat16* o = ob + (static_cast<size_t>(ci.s) * P.num_q_heads + qh_lo + 8) * D + tq;
+                __nv_bfloat16* o = ob + (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo + 8) * D + tq;
 #pragma unroll
                 for (int n = 0; n < NTD; ++n)
                     *reinterpret_cast<__nv_bfloat162*>(o + 8 * n) =
@@ -333,7 +330,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         } else {
             constexpr float kLn2 = 0.693147180559945309f;
             if (r_lo < g) {
-                const size_t idx = (static_cast<size_t>(ci.s) * P.num_q_heads + qh_lo) * P.max_parts + ci.p;
+                const size_t idx = (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo) * P.max_parts + cc.p;
                 if ((lane & 3) == 0) {
                     P.ws_m[idx] = m_lo * kLn2;
                     P.ws_l[idx] = lt_lo;
@@ -345,7 +342,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             if (HI && r_lo + 8 < g) {
                 const size_t idx =
-                    (static_cast<size_t>(ci.s) * P.num_q_heads + qh_lo + 8) * P.max_parts + ci.p;
+                    (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo + 8) * P.max_parts + cc.p;
                 if ((lane & 3) == 0) {
                     P.ws_m[idx] = m_hi * kLn2;
                     P.ws_l[idx] = lt_hi;
@@ -357,10 +354,10 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
 
-        cons_item += nw;
-        if (cons_item >= total) break;
-        ci = decode_item(P, prefix, lens, cons_item);
-        cj = ci.jbeg;
+        record_parts(P, cc, lane);
+        sched.next(cc);
+        if (!cc.valid) break;
+        cj = cc.jbeg;
     }
 }
 

@@ -27,7 +27,7 @@ decode_f32_simt_kernel(const DecodeParams P) {
     __shared__ float pbuf[kSimtWarps][MAXG][kBlockTokens];
     int32_t* prefix = smem_i;
     int32_t* lens = prefix + P.seq_count + 1;
-    const int32_t total = build_item_prefix(P, prefix, lens);
+    const Schedule sched = make_schedule(P, prefix, lens, kSimtWarps);
     zero_empty_sequences<float>(P, lens);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -36,9 +36,8 @@ decode_f32_simt_kernel(const DecodeParams P) {
     const float* kc = static_cast<const float*>(P.k_cache);
     const float* vc = static_cast<const float*>(P.v_cache);
 
-    for (int32_t item = blockIdx.x * kSimtWarps + warp; item < total;
-         item += gridDim.x * kSimtWarps) {
-        const Item it = decode_item(P, prefix, lens, item);
+    Cursor it;
+    for (sched.start(it, blockIdx.x * kSimtWarps + warp); it.valid; sched.next(it)) {
         const float* qg = static_cast<const float*>(P.q) +
                           (static_cast<size_t>(it.s) * P.num_q_heads + it.h * g) * D + lane * DPL;
         float q[MAXG][DPL], acc[MAXG][DPL], m[MAXG], l[MAXG];
@@ -149,6 +148,7 @@ decode_f32_simt_kernel(const DecodeParams P) {
                 for (int e = 0; e < DPL; ++e) P.ws_acc[idx * D + lane * DPL + e] = acc[i][e];
             }
         }
+        record_parts(P, it, lane);
     }
 }
 

@@ -1,12 +1,26 @@
-// items.cuh -- how a decode launch cuts its sequences into work items.
+// items.cuh -- how a decode launch cuts its sequences into pieces of work.
 //
-// A work item is (sequence s, partition p, kv head h): the blocks
-// [p*part_blocks, min((p+1)*part_blocks, nb_s)) of sequence s, seen through
-// kv head h, for all query heads of that head's group.  Items are numbered
-// sequence-major, then partition, then kv head, so consecutive warps stream
-// neighbouring head slices of the same physical blocks.  Every CTA of a launch
-// builds the exclusive prefix sum of items per sequence in shared memory once
-// and then maps an item number to (s, p, h) by binary search.
+// A unit is (sequence s, kv head h): the ceil(len_s / 16) blocks of s seen
+// through kv head h, for all query heads of that head's group.  A piece is a
+// run of consecutive blocks of one unit; one warp processes it and writes
+// either the final rows (the piece is the whole unit) or the piece's partial
+// (m, l, acc) for the log-sum-exp reduction.  Two ways to cut:
+//
+//  * balanced (partition_blocks = 0): the blocks of all units form one stream,
+//    units ordered sequence-major then kv head (so neighbouring warps read
+//    neighbouring head slices of the same physical blocks), and warp w takes
+//    stream positions [w*C, (w+1)*C) with C = max(min_chunk, ceil(total / warps)).
+//    Every warp gets the same number of blocks (+-1), whatever the length mix;
+//    a unit that crosses a warp boundary becomes several pieces.  Piece p of a
+//    unit is the part that falls in the unit's p-th warp range.
+//  * fixed (partition_blocks > 0, or "never split"): piece p of a unit is
+//    blocks [p*PB, (p+1)*PB); pieces are numbered sequence-major, then piece,
+//    then kv head, and handed out round-robin over the warps.
+//
+// Every CTA builds a prefix sum over the launch's sequences in shared memory
+// once (blocks per sequence, or pieces per sequence) and then locates any
+// stream position or piece number by binary search.  The prefix and the
+// clamped lengths take 8 bytes of shared memory per sequence.
 #pragma once
 
 #include "common.cuh"
@@ -16,7 +30,7 @@ namespace pa {
 struct SeqGeom {
     int32_t len;    // tokens attended (clamped)
     int32_t nb;     // blocks: ceil(len / 16)
-    int32_t parts;  // partitions: ceil(nb / part_blocks), 0 for an empty sequence
+    int32_t parts;  // fixed mode: ceil(nb / part_blocks); 0 for an empty sequence
 };
 
 __device__ __forceinline__ SeqGeom seq_geometry(const DecodeParams& P, int32_t len) {
@@ -29,46 +43,42 @@ __device__ __forceinline__ SeqGeom seq_geometry(const DecodeParams& P, int32_t l
     return g;
 }
 
-__device__ __forceinline__ int32_t load_len_checked(const DecodeParams& P, int32_t s, bool report) {
-    int32_t len = P.seq_lens[s];
-    if (report && (len < 0 || len > P.len_cap)) flag_error(PA_DEVERR_SEQ_LEN);
-    return len;
-}
-
-// Builds prefix[0..n] (items before each sequence of the launch, prefix[n] =
-// total) and lens[0..n) (clamped lengths) in shared memory.  All threads of
-// the CTA must call it.  Returns the total number of items.
-__device__ __forceinline__ int32_t build_item_prefix(const DecodeParams& P, int32_t* prefix,
-                                                     int32_t* lens) {
+// Builds prefix[0..n] (exclusive sums of the per-sequence quantity: blocks in
+// balanced mode, pieces x kv heads in fixed mode; prefix[n] = total) and
+// lens[0..n) (clamped lengths) in shared memory.  All threads of the CTA must
+// call it.  Returns the total.
+__device__ __forceinline__ int32_t build_prefix(const DecodeParams& P, int32_t* prefix,
+                                                int32_t* lens) {
     __shared__ int32_t warp_tot[32];
     const int n = P.seq_count;
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int per = (n + nthr - 1) / nthr;
     const int beg = min(n, tid * per), end = min(n, beg + per);
-    // only CTA 0 reports bad lengths, so each bad length is counted once
+    // only CTA 0 reports bad lengths, so each is counted once per launch
     const bool report = blockIdx.x == 0;
     int32_t local = 0;
     for (int i = beg; i < end; ++i) {
-        SeqGeom g = seq_geometry(P, load_len_checked(P, P.seq_begin + i, report));
+        const int32_t raw = P.seq_lens[P.seq_begin + i];
+        if (report && (raw < 0 || raw > P.len_cap)) flag_error(PA_DEVERR_SEQ_LEN);
+        const SeqGeom g = seq_geometry(P, raw);
         lens[i] = g.len;
-        local += g.parts * P.num_kv_heads;
+        local += P.balanced ? g.nb : g.parts * P.num_kv_heads;
     }
-    // exclusive scan of `local` over the CTA
     const int lane = tid & 31, warp = tid >> 5, nwarps = (nthr + 31) >> 5;
     int32_t incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        int32_t v = __shfl_up_sync(kFullMask, incl, o);
+        const int32_t v = __shfl_up_sync(kFullMask, incl, o);
         if (lane >= o) incl += v;
     }
     if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        int32_t t = lane < nwarps ? warp_tot[lane] : 0;
+        const int32_t t = lane < nwarps ? warp_tot[lane] : 0;
         int32_t ti = t;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            int32_t v = __shfl_up_sync(kFullMask, ti, o);
+            const int32_t v = __shfl_up_sync(kFullMask, ti, o);
             if (lane >= o) ti += v;
         }
         warp_tot[lane] = ti - t;  // exclusive
@@ -77,47 +87,132 @@ __device__ __forceinline__ int32_t build_item_prefix(const DecodeParams& P, int3
     int32_t run = warp_tot[warp] + incl - local;
     for (int i = beg; i < end; ++i) {
         prefix[i] = run;
-        SeqGeom g = seq_geometry(P, lens[i]);
-        run += g.parts * P.num_kv_heads;
+        const SeqGeom g = seq_geometry(P, lens[i]);
+        run += P.balanced ? g.nb : g.parts * P.num_kv_heads;
     }
-    if (tid == nthr - 1) prefix[n] = run;  // last thread holds the grand total
+    if (tid == nthr - 1) prefix[n] = run;  // the last thread ends on the grand total
     __syncthreads();
     return prefix[n];
 }
 
-struct Item {
-    int32_t s;       // sequence (global index)
-    int32_t h;       // kv head
-    int32_t p;       // partition
-    int32_t len;     // tokens of the sequence
-    int32_t parts;   // partitions of the sequence
-    int32_t jbeg;    // first block of the item
-    int32_t jend;    // one past its last block
-};
-
-// Item number -> (s, p, h).  Warp-uniform; reads the shared prefix.
-__device__ __forceinline__ Item decode_item(const DecodeParams& P, const int32_t* prefix,
-                                            const int32_t* lens, int32_t item) {
-    int lo = 0, hi = P.seq_count;  // prefix[lo] <= item < prefix[hi]
+// Largest s in [0, n) with key(s) <= x, where key is non-decreasing and
+// key(0) <= x < key(n).
+template <typename Key>
+__device__ __forceinline__ int upper_index(int n, int64_t x, Key key) {
+    int lo = 0, hi = n;
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (prefix[mid] <= item) lo = mid;
+        if (key(mid) <= x) lo = mid;
         else hi = mid;
     }
-    Item it;
-    const int32_t r = item - prefix[lo];
-    it.p = r / P.num_kv_heads;
-    it.h = r - it.p * P.num_kv_heads;
-    it.s = P.seq_begin + lo;
-    SeqGeom g = seq_geometry(P, lens[lo]);
-    it.len = g.len;
-    it.parts = g.parts;
-    it.jbeg = it.p * P.part_blocks;
-    it.jend = min(g.nb, it.jbeg + P.part_blocks);
-    return it;
+    return lo;
 }
 
-// Zero-length sequences have no items; their rows of `out` are zero.  CTA b
+// Iterates the pieces one warp owns.  Warp-uniform.
+struct Cursor {
+    // the current piece
+    bool valid;
+    int32_t s;      // sequence (global index)
+    int32_t h;      // kv head
+    int32_t p;      // piece index within its unit
+    int32_t parts;  // pieces of the unit
+    int32_t len;    // tokens of the sequence
+    int32_t jbeg;   // first block of the piece
+    int32_t jend;   // one past its last block
+    // iteration state
+    int32_t item;    // fixed mode: piece number
+    int64_t pos;     // balanced mode: stream position of the current piece
+    int64_t end;     // balanced mode: end of this warp's range
+    int64_t chunk;   // balanced mode: C
+};
+
+struct Schedule {
+    const DecodeParams* P;
+    const int32_t* prefix;
+    const int32_t* lens;
+    int32_t total;  // blocks (balanced) or pieces (fixed)
+    int64_t chunk;  // balanced: blocks per warp range
+    int32_t nw;     // warps in the grid
+
+    __device__ __forceinline__ void locate_fixed(Cursor& c) const {
+        const int n = P->seq_count;
+        const int i = upper_index(n, c.item, [&](int k) { return (int64_t)prefix[k]; });
+        const int32_t r = c.item - prefix[i];
+        c.p = r / P->num_kv_heads;
+        c.h = r - c.p * P->num_kv_heads;
+        c.s = P->seq_begin + i;
+        const SeqGeom g = seq_geometry(*P, lens[i]);
+        c.len = g.len;
+        c.parts = g.parts;
+        c.jbeg = c.p * P->part_blocks;
+        c.jend = min(g.nb, c.jbeg + P->part_blocks);
+    }
+
+    __device__ __forceinline__ void locate_balanced(Cursor& c) const {
+        const int n = P->seq_count;
+        const int64_t hk = P->num_kv_heads;
+        const int i = upper_index(n, c.pos, [&](int k) { return hk * prefix[k]; });
+        const SeqGeom g = seq_geometry(*P, lens[i]);
+        const int64_t off = c.pos - hk * prefix[i];
+        c.h = static_cast<int32_t>(off / g.nb);
+        c.jbeg = static_cast<int32_t>(off - static_cast<int64_t>(c.h) * g.nb);
+        const int64_t ustart = c.pos - c.jbeg;
+        const int64_t uend = ustart + g.nb;
+        c.jend = static_cast<int32_t>(min(uend, c.end) - ustart);
+        c.s = P->seq_begin + i;
+        c.len = g.len;
+        c.p = static_cast<int32_t>(c.pos / c.chunk - ustart / c.chunk);
+        c.parts = static_cast<int32_t>((uend - 1) / c.chunk - ustart / c.chunk + 1);
+    }
+
+    __device__ __forceinline__ void start(Cursor& c, int32_t warp_global) const {
+        if (P->balanced) {
+            c.chunk = chunk;
+            c.pos = static_cast<int64_t>(warp_global) * chunk;
+            c.end = min(c.pos + chunk, static_cast<int64_t>(total) * P->num_kv_heads);
+            c.valid = c.pos < c.end;
+            if (c.valid) locate_balanced(c);
+        } else {
+            c.item = warp_global;
+            c.valid = c.item < total;
+            if (c.valid) locate_fixed(c);
+        }
+    }
+
+    // Move to the warp's next piece.
+    __device__ __forceinline__ void next(Cursor& c) const {
+        if (P->balanced) {
+            c.pos += c.jend - c.jbeg;
+            c.valid = c.pos < c.end;
+            if (c.valid) locate_balanced(c);
+        } else {
+            c.item += nw;
+            c.valid = c.item < total;
+            if (c.valid) locate_fixed(c);
+        }
+    }
+};
+
+// Sets up the schedule of a launch (all threads of the CTA call it).
+__device__ __forceinline__ Schedule make_schedule(const DecodeParams& P, int32_t* prefix,
+                                                  int32_t* lens, int warps_per_cta) {
+    Schedule sc;
+    sc.P = &P;
+    sc.prefix = prefix;
+    sc.lens = lens;
+    sc.total = build_prefix(P, prefix, lens);
+    sc.nw = gridDim.x * warps_per_cta;
+    if (P.balanced) {
+        const int64_t blocks = static_cast<int64_t>(sc.total) * P.num_kv_heads;
+        const int64_t even = (blocks + sc.nw - 1) / sc.nw;
+        sc.chunk = even > P.min_chunk ? even : P.min_chunk;
+    } else {
+        sc.chunk = 0;
+    }
+    return sc;
+}
+
+// Zero-length sequences have no pieces; their rows of `out` are zero.  CTA b
 // clears those of the sequences s = b, b + gridDim.x, ... of the launch.
 template <typename OutT>
 __device__ __forceinline__ void zero_empty_sequences(const DecodeParams& P, const int32_t* lens) {
@@ -127,6 +222,13 @@ __device__ __forceinline__ void zero_empty_sequences(const DecodeParams& P, cons
         OutT* o = static_cast<OutT*>(P.out) + static_cast<size_t>(P.seq_begin + i) * row;
         for (int e = threadIdx.x; e < row; e += blockDim.x) o[e] = OutT(0.0f);
     }
+}
+
+// Records how many pieces unit (s, h) has (written by the warp holding piece 0;
+// read by the reduction).
+__device__ __forceinline__ void record_parts(const DecodeParams& P, const Cursor& c, int lane) {
+    if (P.ws_parts != nullptr && c.p == 0 && lane == 0)
+        P.ws_parts[static_cast<size_t>(c.s) * P.num_kv_heads + c.h] = c.parts;
 }
 
 }  // namespace pa

@@ -11,10 +11,11 @@
 // §"L'avenir de PagedAttention et vLLM").
 //
 // One CTA (4 warps) per (sequence, query head) row: all threads find M and the
-// denominator, each warp accumulates a strided subset of the partitions'
-// acc rows with 16-byte loads, and the four warp sums are added in a fixed
-// order.  Rows of sequences with at most one partition are skipped (the decode
-// kernel wrote them).
+// denominator, each warp accumulates a strided subset of the pieces' acc rows
+// with 16-byte loads, and the four warp sums are added in a fixed order.  The
+// number of pieces of each (sequence, kv head) unit is read from the
+// workspace, where the decode kernel recorded it; rows of units with a single
+// piece are skipped (the decode kernel wrote them).
 #pragma once
 
 #include "items.cuh"
@@ -43,8 +44,9 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const Dec
     const int32_t s = P.seq_begin + static_cast<int32_t>(row / P.num_q_heads);
     const int32_t qh = static_cast<int32_t>(row % P.num_q_heads);
     const SeqGeom geo = seq_geometry(P, P.seq_lens[s]);
-    if (geo.parts <= 1) return;
-    const int parts = geo.parts;
+    if (geo.nb == 0) return;  // an empty sequence: the decode kernel zeroed its rows
+    const int parts = P.ws_parts[static_cast<size_t>(s) * P.num_kv_heads + qh / P.group];
+    if (parts <= 1) return;   // a single piece: the decode kernel wrote the row
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t base = (static_cast<size_t>(s) * P.num_q_heads + qh) * P.max_parts;

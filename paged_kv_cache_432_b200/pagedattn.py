@@ -176,15 +176,21 @@ def device_error(clear: bool = True, stream=None) -> int:
     return int(bits.value)
 
 
-def workspace_views(workspace: torch.Tensor, num_seqs, num_q_heads, head_dim, max_parts):
-    """(m, l, acc) float views of a workspace, following the layout the header
-    documents: arrays of [rows][P] and [rows][P][D] each on a 256-byte boundary."""
+def workspace_views(workspace: torch.Tensor, num_seqs, num_q_heads, head_dim, max_parts, num_kv_heads=None):
+    """(m, l, acc, parts) views of a workspace, following the layout the header
+    documents: float [rows][P], [rows][P], [rows][P][D] and int32 [N*Hkv], each
+    on a 256-byte boundary (parts is None when num_kv_heads is not given)."""
     rows = num_seqs * num_q_heads
     a256 = lambda x: (x + 255) // 256 * 256
     ml = a256(rows * max_parts * 4)
+    off_parts = 2 * ml + a256(rows * max_parts * head_dim * 4)
     f = workspace.view(torch.uint8)
     m = f[:rows * max_parts * 4].view(torch.float32).view(num_seqs, num_q_heads, max_parts)
     l = f[ml:ml + rows * max_parts * 4].view(torch.float32).view(num_seqs, num_q_heads, max_parts)
     acc = f[2 * ml:2 * ml + rows * max_parts * head_dim * 4].view(torch.float32).view(
         num_seqs, num_q_heads, max_parts, head_dim)
-    return m, l, acc
+    parts = None
+    if num_kv_heads is not None:
+        parts = f[off_parts:off_parts + num_seqs * num_kv_heads * 4].view(torch.int32).view(
+            num_seqs, num_kv_heads)
+    return m, l, acc, parts

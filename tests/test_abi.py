@@ -55,22 +55,29 @@ def test_status_strings(lib):
 def test_partition_policy(lib):
     assert pa.partition_blocks(8, 8, 131072, 32) == 32
     assert pa.partition_blocks(8, 8, 131072, -1) >= 131072 // 16
-    assert pa.partition_blocks(8, 8, 512, 0) >= 32          # short: never split
-    assert pa.partition_blocks(64, 32, 2048, 0) == 32       # long enough: 512-token partitions
+    assert pa.partition_blocks(8, 8, 512, 0) == 0           # auto: the balanced split
+    assert pa.partition_blocks(64, 32, 2048, 0) == 0
     assert lib.pa_decode_partition_blocks(8, 8, 100, 8, 0) == pa.PA_ERR_UNSUPPORTED
     assert lib.pa_decode_partition_blocks(8, 8, 100, 16, -2) == pa.PA_ERR_INVALID_ARG
 
 
 def test_workspace_size_matches_documented_layout(lib):
     a256 = lambda x: (x + 255) // 256 * 256
+
+    def layout(N, Hq, Hkv, D, P):
+        rows = N * Hq
+        return 2 * a256(rows * P * 4) + a256(rows * P * D * 4) + a256(N * Hkv * 4)
+
     N, Hq, Hkv, D, L = 8, 64, 8, 128, 131072
-    P = -(-(L // 16) // 32)
-    rows = N * Hq
-    expect = 2 * a256(rows * P * 4) + a256(rows * P * D * 4)
-    assert pa.workspace_size(N, Hq, Hkv, D, L, 32) == expect
+    nb = L // 16
+    assert pa.workspace_size(N, Hq, Hkv, D, L, 32) == layout(N, Hq, Hkv, D, -(-nb // 32))
     assert pa.workspace_size(N, Hq, Hkv, D, 512, 32) == 0        # one partition: no workspace
     assert pa.workspace_size(N, Hq, Hkv, D, L, -1) == 0
-    assert pa.workspace_size(N, Hq, Hkv, D, 513, 32) == 2 * a256(rows * 2 * 4) + a256(rows * 2 * D * 4)
+    assert pa.workspace_size(N, Hq, Hkv, D, 513, 32) == layout(N, Hq, Hkv, D, 2)
+    # balanced split: a unit of nb blocks meets at most ceil(nb / 32) + 1 warp ranges
+    assert pa.workspace_size(N, Hq, Hkv, D, L, 0) == layout(N, Hq, Hkv, D, -(-nb // 32) + 1)
+    assert pa.workspace_size(N, Hq, Hkv, D, 100, 0) == layout(N, Hq, Hkv, D, 2)
+    assert pa.workspace_size(N, Hq, Hkv, D, 0, 0) == 0
 
 
 def _decode_rc(lib, **over):

@@ -199,6 +199,17 @@ def test_split_and_single_pass_agree(pb):
     assert_close(to_f64(split), ref, torch.bfloat16, f"split pb={pb}")
 
 
+@pytest.mark.parametrize("lens,Hq,Hkv", [([30000, 5, 700, 0, 64], 8, 1), ([70000], 16, 2),
+                                          ([1] * 300 + [9000], 4, 4)])
+def test_balanced_split_long_unit_across_many_warps(lens, Hq, Hkv):
+    """Balanced split (partition_blocks = 0): a long unit is cut at warp-range
+    boundaries into many pieces, next to units that are one piece."""
+    w = wl.build(lens, Hq, Hkv, 128, torch.bfloat16, seed=sum(lens) % 1000, device=DEV)
+    out = gpu_decode(w, partition_blocks=0)
+    assert_close(to_f64(out), oracle_decode(w), torch.bfloat16, f"balanced {lens[:3]}")
+    assert pa.device_error() == 0
+
+
 # ------------------------------------------------------------------ the two steps separately
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_partition_partials_match_oracle(dtype):
@@ -215,7 +226,7 @@ def test_partition_partials_match_oracle(dtype):
     h = host(w)
     m_o, l_o, acc_o, np_o = oracle.decode_partials(h["q"], h["kc"], h["vc"], h["bt"], h["sl"], w.scale, pb * 16)
     P = -(-(-(-msl // 16)) // pb)  # ceil(ceil(msl / 16) / pb)
-    m_g, l_g, acc_g = (t.double().cpu().numpy() for t in pa.workspace_views(ws, w.num_seqs, 8, 128, P))
+    m_g, l_g, acc_g = (t.double().cpu().numpy() for t in pa.workspace_views(ws, w.num_seqs, 8, 128, P)[:3])
     for s, L in enumerate(w.lens_host):
         n = int(np_o[s])
         if n <= 1:  # written straight to out
@@ -238,8 +249,9 @@ def test_reduce_of_oracle_partials_matches_oracle_merge():
     m_o, l_o, acc_o, np_o = oracle.decode_partials(h["q"], h["kc"], h["vc"], h["bt"], h["sl"], w.scale, pb * 16)
     P = -(-(-(-msl // 16)) // pb)  # ceil(ceil(msl / 16) / pb)
     ws = pa.alloc_workspace(w.num_seqs, 16, 4, 64, msl, pb, device=DEV)
-    m_v, l_v, acc_v = pa.workspace_views(ws, w.num_seqs, 16, 64, P)
+    m_v, l_v, acc_v, parts_v = pa.workspace_views(ws, w.num_seqs, 16, 64, P, num_kv_heads=4)
     m_v.zero_(), l_v.zero_(), acc_v.zero_()
+    parts_v[:] = torch.from_numpy(np_o).int().to(DEV)[:, None]  # pieces of every kv head
     Po = m_o.shape[2]
     m_v[:, :, :Po] = torch.from_numpy(m_o).float().to(DEV)
     l_v[:, :, :Po] = torch.from_numpy(l_o).float().to(DEV)
