@@ -60,6 +60,7 @@ extern "C" {
 #define PA_ERR_UNSUPPORTED (-2) /* dtype, head_dim, block size or group size */
 #define PA_ERR_WORKSPACE (-3)   /* workspace missing or too small            */
 #define PA_ERR_CUDA (-4)        /* a CUDA call or launch failed              */
+#define PA_ERR_SCRATCH_LIMIT (-5) /* pa_decode_noalloc: sizes need more than its fixed buffer */
 
 /* Element types (q, caches, new k/v and out share one). */
 #define PA_DTYPE_F32 0
@@ -179,6 +180,40 @@ PA_API int pa_decode_reduce(const int32_t* seq_lens, int32_t max_seq_len, int32_
  * after synchronising `stream`; clears it when `clear` is non-zero.
  */
 PA_API int pa_get_device_error(uint32_t* bits, int32_t clear, void* stream);
+
+/*
+ * pa_decode without any device allocation, for callers that cannot allocate
+ * device memory themselves.  Examples: a plugin inside an inference engine
+ * that owns every byte of device memory through its own pool and forbids
+ * cudaMalloc, a runtime whose memory budget is fixed at start-up, or a
+ * foreign-language caller with no binding for CUDA allocation.  The pages
+ * have no counterpart: this is an interface convenience, not part of the
+ * method.
+ *
+ * Same arguments and result as pa_decode, minus the workspace.  The split-K
+ * partials live in a buffer of PA_NOALLOC_SCRATCH_BYTES (32 MiB) built into
+ * the library as a static device array.  Every GPU that loads the library
+ * holds that buffer until the process exits.  If the sizes need more than
+ * that (pa_decode_workspace_size > PA_NOALLOC_SCRATCH_BYTES) the call returns
+ * PA_ERR_SCRATCH_LIMIT and does nothing.  Use larger partitions or pa_decode
+ * with your own workspace instead.
+ *
+ * The first call on a device looks up the buffer's device address (a
+ * one-time set-up per device, done with that device current).  Make that
+ * first call before any stream capture.  All calls share the one buffer and
+ * it keeps the last call's contents.  Nothing in it needs to start at zero,
+ * since each partial is written before it is read.  Calls that overlap on the
+ * GPU race on that buffer (two streams, or two threads), so serialise them.
+ * Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+PA_API int pa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, int32_t max_blocks_per_seq,
+                             const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                             int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                             int32_t num_blocks, int32_t block_size, float scale,
+                             int32_t partition_blocks, void* out, int32_t dtype, void* stream);
+
+#define PA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 
 /* Human-readable text for a return code (for PA_ERR_CUDA: the last CUDA error
  * seen by the calling thread). */

@@ -517,6 +517,61 @@ int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int
     return run_reduce(P, plan, dtype, a.stream);
 }
 
+// ------------------------------------------------------------ no-allocation decode
+// The split-K scratch of pa_decode_noalloc: one file-scope device array of a
+// fixed size, present on every device that loads the library.  Host code must
+// not pass the name itself to a kernel (on the host it is only a stand-in);
+// its device address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device (looked up on
+// the first call per device, with that device current).
+int noalloc_scratch(void** ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return PA_OK;
+}
+}  // namespace
+
+int pa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, int32_t max_blocks_per_seq,
+                      const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                      int32_t num_blocks, int32_t block_size, float scale,
+                      int32_t partition_blocks, void* out, int32_t dtype, void* stream) {
+    int rc = check_shapes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, dtype);
+    if (rc != PA_OK) return rc;
+    if (max_blocks_per_seq <= 0 || partition_blocks < -1) return PA_ERR_INVALID_ARG;
+    // the same effective bound pa_decode sizes its workspace with
+    const int64_t table_tokens = static_cast<int64_t>(max_blocks_per_seq) * kBlockTokens;
+    const int32_t max_len = max_seq_len > 0
+                                ? max_seq_len
+                                : static_cast<int32_t>(table_tokens > INT32_MAX ? INT32_MAX : table_tokens);
+    const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                 max_len, block_size, partition_blocks);
+    if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_SCRATCH_LIMIT;
+    void* scratch = nullptr;
+    if (need > 0 && (rc = noalloc_scratch(&scratch)) != PA_OK) return rc;
+    return pa_decode(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, max_seq_len,
+                     num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale,
+                     partition_blocks, scratch, need > 0 ? PA_NOALLOC_SCRATCH_BYTES : 0, out,
+                     dtype, stream);
+}
+
 int pa_get_device_error(uint32_t* bits, int32_t clear, void* stream) {
     if (!bits) return PA_ERR_INVALID_ARG;
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
@@ -540,6 +595,9 @@ const char* pa_status_string(int status) {
         case PA_ERR_UNSUPPORTED: return "unsupported dtype, head_dim, block size or group size";
         case PA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case PA_ERR_CUDA: return g_last_cuda_error;
+        case PA_ERR_SCRATCH_LIMIT:
+            return "sizes need more split-K scratch than pa_decode_noalloc's built-in 32 MiB buffer "
+                   "(use larger partitions, or pa_decode with a caller-owned workspace)";
         default: return "unknown status";
     }
 }

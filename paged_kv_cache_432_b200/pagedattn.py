@@ -21,6 +21,8 @@ PA_ERR_INVALID_ARG = -1
 PA_ERR_UNSUPPORTED = -2
 PA_ERR_WORKSPACE = -3
 PA_ERR_CUDA = -4
+PA_ERR_SCRATCH_LIMIT = -5
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 PA_DTYPE_F32 = 0
 PA_DTYPE_BF16 = 1
@@ -40,6 +42,8 @@ SIGNATURES = {
     "pa_decode": (ctypes.c_int, _DECODE_ARGS),
     "pa_decode_partitions": (ctypes.c_int, _DECODE_ARGS),
     "pa_decode_reduce": (ctypes.c_int, [_P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ, _P, _I32, _P]),
+    "pa_decode_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _F,
+                                         _I32, _P, _I32, _P]),
     "pa_get_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _I32, _P]),
     "pa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -166,6 +170,20 @@ def decode_reduce(seq_lens, out, num_kv_heads, max_blocks_per_seq, max_seq_len, 
                                 max_blocks_per_seq, 16, partition_blocks, _ptr(workspace), ws_bytes,
                                 _ptr(out), dtype_code(out.dtype), _stream(stream))
     _check("pa_decode_reduce", rc)
+
+
+def decode_noalloc(q, k_cache, v_cache, block_tables, seq_lens, scale, out, max_seq_len=0,
+                   partition_blocks=0, stream=None) -> torch.Tensor:
+    """pa_decode_noalloc: the decode without any device allocation (its split-K
+    partials live in the library's fixed 32 MiB buffer); `out` is required."""
+    N, Hq, D = q.shape
+    NB, Hkv, B, _ = k_cache.shape
+    rc = lib().pa_decode_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1],
+        _ptr(seq_lens), max_seq_len, N, Hq, Hkv, D, NB, B, float(scale), partition_blocks,
+        _ptr(out), dtype_code(q.dtype), _stream(stream))
+    _check("pa_decode_noalloc", rc)
+    return out
 
 
 def device_error(clear: bool = True, stream=None) -> int:
