@@ -370,19 +370,31 @@ def run_ours(args) -> None:
         raise RuntimeError("device error flagged during warm-up")
 
     def timed():
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        """Two timed loops over the same steps: (a) events at step boundaries
+        only, so consecutive kernels overlap as they do in use (programmatic
+        dependent launch) -> the step time; (b) events between the kernels ->
+        each kernel's own duration (the roofline's)."""
+        K = args.steps
+        ev_step = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        ev_k = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
         barrier(ws)
         torch.cuda.synchronize(dev)
         with ClockSampler(local) as cs:
-            for k in range(args.steps):
+            for k in range(K):
                 flush_l2()
-                step(evs[k])
+                ev_step[k][0].record(stream)
+                step()
+                ev_step[k][1].record(stream)
+            torch.cuda.synchronize(dev)
+            for k in range(K):
+                flush_l2()
+                step(ev_k[k])
             torch.cuda.synchronize(dev)
         barrier(ws)
-        tot = sum(e[0].elapsed_time(e[3]) for e in evs)
-        dec = sum(e[1].elapsed_time(e[2]) for e in evs)
-        red = sum(e[2].elapsed_time(e[3]) for e in evs)
-        wr = sum(e[0].elapsed_time(e[1]) for e in evs)
+        tot = sum(a.elapsed_time(b) for a, b in ev_step)
+        dec = sum(e[1].elapsed_time(e[2]) for e in ev_k)
+        red = sum(e[2].elapsed_time(e[3]) for e in ev_k)
+        wr = sum(e[0].elapsed_time(e[1]) for e in ev_k)
         return tot, dec, red, wr, cs.summary()
 
     tot, dec, red, wr, clocks = timed()
@@ -400,16 +412,27 @@ def run_ours(args) -> None:
     # result read back, every step
     e2e = None
     if not args.no_e2e:
+        # the step's inputs travel in one pinned staging buffer (one H2D copy),
+        # each at a 256-byte aligned offset; the device tensors are views
         names = ["q", "new_k", "new_v", "slot_mapping", "block_tables", "seq_lens"]
-        host_in = {n: getattr(w, n).cpu().pin_memory() for n in names}
-        dev_in = {n: torch.empty_like(getattr(w, n)) for n in names}
+        src = {n: getattr(w, n).contiguous() for n in names}
+        offs, off = {}, 0
+        for n in names:
+            offs[n] = off
+            off += (src[n].numel() * src[n].element_size() + 255) // 256 * 256
+        host_buf = torch.empty(off, dtype=torch.uint8, pin_memory=True)
+        dev_buf = torch.empty(off, dtype=torch.uint8, device=dev)
+        dev_in = {}
+        for n in names:
+            nb = src[n].numel() * src[n].element_size()
+            host_buf[offs[n]:offs[n] + nb].copy_(src[n].view(-1).view(torch.uint8).cpu())
+            dev_in[n] = dev_buf[offs[n]:offs[n] + nb].view(src[n].dtype).view(src[n].shape)
         host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        h2d = sum(src[n].numel() * src[n].element_size() for n in names)
         d2h = host_out.numel() * host_out.element_size()
 
         def e2e_step():
-            for n in names:
-                dev_in[n].copy_(host_in[n], non_blocking=True)
+            dev_buf.copy_(host_buf, non_blocking=True)
             pa.cache_write(dev_in["new_k"], dev_in["new_v"], dev_in["slot_mapping"], w.k_cache, w.v_cache, stream)
             pa.decode(dev_in["q"], w.k_cache, w.v_cache, dev_in["block_tables"], dev_in["seq_lens"], w.scale,
                       out=out, max_seq_len=msl, partition_blocks=pb, workspace=wsp, stream=stream)
@@ -467,13 +490,15 @@ def run_ours(args) -> None:
         "config": workload_config(w, resolved_pb),
         "tokens_per_s": round(total_seqs / (step_ms * 1e-3), 1),
         "kernel_ms": {"cache_write": round(wr_ms, 5), "decode_partitions": round(dec_ms, 5),
-                      "lse_reduce": round(red_ms, 5)},
+                      "lse_reduce": round(red_ms, 5),
+                      "how": "CUDA events between the kernels, in a second timed loop of the same steps"},
         "bytes_per_step": by,
         "roofline": roof,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "clocks": clocks,
         "gpu_launches": launches_per_step * K,
+        "gpu_launches_note": "per timed loop: cache write, decode, reduce per step",
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

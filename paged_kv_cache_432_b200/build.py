@@ -44,13 +44,16 @@ def stale() -> bool:
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not verbose_ptxas and not stale():
+def build(force: bool = False, verbose_ptxas: bool = False, out: str = None, defines=()) -> str:
+    """Compile the library (to `out`, default in-tree) if a source is newer;
+    `defines` are extra -D macros (tuning variants)."""
+    target = out or LIB
+    if out is None and not force and not verbose_ptxas and not stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = target + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-cudart", "static", "-I", INCLUDE, "-I", CSRC,
-           "-o", tmp, os.path.join(CSRC, "api.cu")]
+           *[f"-D{d}" for d in defines], "-o", tmp, os.path.join(CSRC, "api.cu")]
     if verbose_ptxas:
         cmd[1:1] = ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -59,8 +62,8 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         raise RuntimeError("nvcc failed")
     if verbose_ptxas:
         sys.stderr.write(r.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 def main():

@@ -14,6 +14,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "pagedattn.h"
 
@@ -29,13 +30,23 @@ namespace {
 using namespace pa;
 
 constexpr int32_t kNoSplit = 1 << 24;       // partition size meaning "never split"
-constexpr int32_t kAutoPartBlocks = 32;     // 512 tokens per partition when splitting
 constexpr int32_t kMaxSeqsPerLaunch = 2048; // sequences whose item prefix one CTA holds
 constexpr int kMaxDevices = 64;
 
-// bf16 kernel configuration: warps per CTA and ring stages per warp.
-constexpr int kMmaWarps = 4;
-constexpr int kMmaStages = 3;
+// bf16 kernel configuration: warps per CTA and ring stages per warp (build-time
+// overridable, for tuning sweeps).
+#ifndef PA_MMA_WARPS
+#define PA_MMA_WARPS 4
+#endif
+#ifndef PA_MMA_STAGES
+#define PA_MMA_STAGES 2
+#endif
+#ifndef PA_MMA_MIN_CTAS
+#define PA_MMA_MIN_CTAS 2
+#endif
+constexpr int kMmaWarps = PA_MMA_WARPS;
+constexpr int kMmaStages = PA_MMA_STAGES;
+constexpr int kMmaMinCtas = PA_MMA_MIN_CTAS;  // CTAs per SM the register budget must allow
 
 thread_local char g_last_cuda_error[256] = "no CUDA error recorded";
 
@@ -304,53 +315,112 @@ int32_t seqs_per_launch(const DecodeParams& P) {
     return static_cast<int32_t>(lim < kMaxSeqsPerLaunch ? (lim < 1 ? 1 : lim) : kMaxSeqsPerLaunch);
 }
 
+// Launches `kernel` with programmatic stream serialization, so that it may
+// begin while the previous kernel in the stream finishes (the kernels call
+// griddepcontrol.wait before touching anything that kernel writes).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Shape of the decode launch for one chunk of sequences (shared by the decode
+// launch and by the balanced reduction, which recomputes the decode's warp
+// ranges).
+struct LaunchShape {
+    int grid;
+    int threads;
+    size_t smem;
+};
+
 template <int D, int ROWS>
-int launch_mma(const DecodeParams& base, cudaStream_t st) {
+auto mma_kernel() {
+    return decode_bf16_mma_kernel<D, ROWS, kMmaStages, kMmaWarps, kMmaMinCtas>;
+}
+
+template <typename K>
+int shape_of(K kernel, int warps, size_t smem, const DecodeParams& P, LaunchShape* L) {
+    const int64_t max_pieces = static_cast<int64_t>(P.seq_count) * P.num_kv_heads * P.max_parts;
+    L->threads = warps * 32;
+    L->smem = smem;
+    return persistent_grid(kernel, L->threads, smem, (max_pieces + warps - 1) / warps, &L->grid);
+}
+
+template <int D, int ROWS>
+int mma_shape(const DecodeParams& P, LaunchShape* L) {
     using Cfg = MmaCfg<D, kMmaStages, kMmaWarps>;
-    auto kernel = decode_bf16_mma_kernel<D, ROWS, kMmaStages, kMmaWarps>;
+    auto kernel = mma_kernel<D, ROWS>();
     int rc = ensure_smem_attr(kernel, Cfg::smem_bytes(kMaxSeqsPerLaunch));
     if (rc != PA_OK) return rc;
-    const int64_t rows = static_cast<int64_t>(base.num_blocks) * base.num_kv_heads * kBlockTokens;
-    alignas(64) CUtensorMap mk, mv;
-    if ((rc = encode_pool_map(&mk, base.k_cache, rows, D)) != PA_OK) return rc;
-    if ((rc = encode_pool_map(&mv, base.v_cache, rows, D)) != PA_OK) return rc;
+    return shape_of(kernel, kMmaWarps, Cfg::smem_bytes(P.seq_count), P, L);
+}
+
+template <int D, int MAXG>
+int simt_shape(const DecodeParams& P, LaunchShape* L) {
+    return shape_of(decode_f32_simt_kernel<D, MAXG>, kSimtWarps, 8 * static_cast<size_t>(P.seq_count + 1),
+                    P, L);
+}
+
+int decode_shape(const DecodeParams& P, int32_t dtype, LaunchShape* L) {
+    if (dtype == PA_DTYPE_BF16) {
+        if (P.head_dim == 128) return P.group <= 8 ? mma_shape<128, 8>(P, L) : mma_shape<128, 16>(P, L);
+        return P.group <= 8 ? mma_shape<64, 8>(P, L) : mma_shape<64, 16>(P, L);
+    }
+    if (P.head_dim == 128) return P.group <= 4 ? simt_shape<128, 4>(P, L) : simt_shape<128, 16>(P, L);
+    return P.group <= 4 ? simt_shape<64, 4>(P, L) : simt_shape<64, 16>(P, L);
+}
+
+// Calls fn(chunk_params) for each launch chunk of sequences.
+template <typename F>
+int for_each_chunk(const DecodeParams& base, F fn) {
     const int32_t chunk = seqs_per_launch(base);
     for (int32_t b = 0; b < base.num_seqs; b += chunk) {
         DecodeParams P = base;
         P.seq_begin = b;
         P.seq_count = base.num_seqs - b < chunk ? base.num_seqs - b : chunk;
-        const size_t smem = Cfg::smem_bytes(P.seq_count);
-        const int64_t max_pieces = static_cast<int64_t>(P.seq_count) * P.num_kv_heads * P.max_parts;
-        int grid = 0;
-        rc = persistent_grid(kernel, Cfg::kThreads, smem, (max_pieces + kMmaWarps - 1) / kMmaWarps,
-                             &grid);
+        const int rc = fn(P);
         if (rc != PA_OK) return rc;
-        kernel<<<grid, Cfg::kThreads, smem, st>>>(mk, mv, P);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "decode_bf16_mma_kernel launch");
     }
     return PA_OK;
 }
 
+template <int D, int ROWS>
+int launch_mma(const DecodeParams& base, cudaStream_t st) {
+    const int64_t rows = static_cast<int64_t>(base.num_blocks) * base.num_kv_heads * kBlockTokens;
+    alignas(64) CUtensorMap mk, mv;
+    int rc;
+    if ((rc = encode_pool_map(&mk, base.k_cache, rows, D)) != PA_OK) return rc;
+    if ((rc = encode_pool_map(&mv, base.v_cache, rows, D)) != PA_OK) return rc;
+    return for_each_chunk(base, [&](const DecodeParams& P) {
+        LaunchShape L;
+        int r = mma_shape<D, ROWS>(P, &L);
+        if (r != PA_OK) return r;
+        cudaError_t e = launch_pdl(mma_kernel<D, ROWS>(), dim3(L.grid), dim3(L.threads), L.smem, st,
+                                   mk, mv, P);
+        return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode_bf16_mma_kernel launch");
+    });
+}
+
 template <int D, int MAXG>
 int launch_simt(const DecodeParams& base, cudaStream_t st) {
-    auto kernel = decode_f32_simt_kernel<D, MAXG>;
-    const int32_t chunk = seqs_per_launch(base);
-    for (int32_t b = 0; b < base.num_seqs; b += chunk) {
-        DecodeParams P = base;
-        P.seq_begin = b;
-        P.seq_count = base.num_seqs - b < chunk ? base.num_seqs - b : chunk;
-        const size_t smem = 8 * static_cast<size_t>(P.seq_count + 1);
-        const int64_t max_pieces = static_cast<int64_t>(P.seq_count) * P.num_kv_heads * P.max_parts;
-        int grid = 0;
-        int rc = persistent_grid(kernel, kSimtWarps * 32, smem,
-                                 (max_pieces + kSimtWarps - 1) / kSimtWarps, &grid);
-        if (rc != PA_OK) return rc;
-        kernel<<<grid, kSimtWarps * 32, smem, st>>>(P);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "decode_f32_simt_kernel launch");
-    }
-    return PA_OK;
+    return for_each_chunk(base, [&](const DecodeParams& P) {
+        LaunchShape L;
+        int r = simt_shape<D, MAXG>(P, &L);
+        if (r != PA_OK) return r;
+        cudaError_t e = launch_pdl(decode_f32_simt_kernel<D, MAXG>, dim3(L.grid), dim3(L.threads),
+                                   L.smem, st, P);
+        return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode_f32_simt_kernel launch");
+    });
 }
 
 int run_partitions(const DecodeParams& P, int32_t dtype, cudaStream_t st) {
@@ -364,26 +434,33 @@ int run_partitions(const DecodeParams& P, int32_t dtype, cudaStream_t st) {
 }
 
 template <typename OutT, int D>
-int launch_reduce(const DecodeParams& base, cudaStream_t st) {
-    const int32_t chunk = seqs_per_launch(base);
-    for (int32_t b = 0; b < base.num_seqs; b += chunk) {
-        DecodeParams P = base;
-        P.seq_begin = b;
-        P.seq_count = base.num_seqs - b < chunk ? base.num_seqs - b : chunk;
-        const unsigned grid = static_cast<unsigned>(P.seq_count) * P.num_q_heads;
-        lse_reduce_kernel<OutT, D><<<grid, kReduceWarps * 32, 0, st>>>(P);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "lse_reduce_kernel launch");
-    }
-    return PA_OK;
+int launch_reduce(const DecodeParams& base, int32_t dtype, cudaStream_t st) {
+    return for_each_chunk(base, [&](const DecodeParams& P) {
+        cudaError_t e;
+        if (P.balanced) {
+            LaunchShape L;
+            int r = decode_shape(P, dtype, &L);
+            if (r != PA_OK) return r;
+            const int decode_warps = L.grid * (L.threads / 32);
+            if (decode_warps < 2) return PA_OK;  // one warp range: nothing was cut
+            e = launch_pdl(lse_reduce_balanced_kernel<OutT, D>, dim3(decode_warps - 1),
+                           dim3(kReduceWarps * 32), 8 * static_cast<size_t>(P.seq_count + 1), st, P,
+                           decode_warps);
+        } else {
+            const unsigned grid = static_cast<unsigned>(P.seq_count) * P.num_q_heads;
+            e = launch_pdl(lse_reduce_kernel<OutT, D>, dim3(grid), dim3(kReduceWarps * 32), 0, st, P);
+        }
+        return e == cudaSuccess ? PA_OK : cuda_fail(e, "lse_reduce_kernel launch");
+    });
 }
 
 int run_reduce(const DecodeParams& P, const Plan& plan, int32_t dtype, cudaStream_t st) {
     if (P.num_seqs == 0 || !plan.split) return PA_OK;
     if (dtype == PA_DTYPE_BF16)
-        return P.head_dim == 128 ? launch_reduce<__nv_bfloat16, 128>(P, st)
-                                 : launch_reduce<__nv_bfloat16, 64>(P, st);
-    return P.head_dim == 128 ? launch_reduce<float, 128>(P, st) : launch_reduce<float, 64>(P, st);
+        return P.head_dim == 128 ? launch_reduce<__nv_bfloat16, 128>(P, dtype, st)
+                                 : launch_reduce<__nv_bfloat16, 64>(P, dtype, st);
+    return P.head_dim == 128 ? launch_reduce<float, 128>(P, dtype, st)
+                             : launch_reduce<float, 64>(P, dtype, st);
 }
 
 DecodeArgs make_args(const void* q, const void* k_cache, const void* v_cache,

@@ -21,6 +21,7 @@ cache_write_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                    const int64_t* __restrict__ slot_mapping, int64_t total_chunks,
                    int32_t num_kv_heads, int32_t chunks_per_row, uint4* __restrict__ k_cache,
                    uint4* __restrict__ v_cache, int64_t num_slots) {
+    allow_dependents();  // a dependent decode may become resident now
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= total_chunks) return;
     const int64_t row = i / chunks_per_row;  // (token, head)

@@ -66,6 +66,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream is still
+// running; grid_dependency_wait() blocks until that kernel has completed and
+// its memory is visible (a no-op for a normal launch).  allow_dependents()
+// lets the next kernel in the stream begin launching.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void allow_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -155,6 +169,31 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
         "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The same with rows 8..15 of A and C known to be zero: only the two
+// accumulators of rows 0..7 are kept (the other two outputs are discarded), so
+// a query group of <= 8 heads holds half the accumulator registers.
+__device__ __forceinline__ void mma_bf16_rows8(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0,
+                                               uint32_t b1) {
+    float z2, z3;
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(z2), "=f"(z3)
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(0.f),
+          "f"(0.f));
+    (void)z2;
+    (void)z3;
+}
+
+// Fragment-array forms: 4 registers = all 16 rows, 2 registers = rows 0..7.
+__device__ __forceinline__ void mma_frag(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    mma_bf16(d, a[0], a[1], a[2], a[3], b0, b1);
+}
+__device__ __forceinline__ void mma_frag(float (&d)[2], const uint32_t (&a)[2], uint32_t b0,
+                                         uint32_t b1) {
+    mma_bf16_rows8(d, a[0], a[1], b0, b1);
 }
 
 __device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) {

@@ -82,14 +82,15 @@ __device__ __forceinline__ float softmax_update(float& m, float& l, const float 
     return alpha;
 }
 
-template <int D, int ROWS, int STAGES, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32)
+template <int D, int ROWS, int STAGES, int WARPS, int MIN_CTAS>
+__global__ void __launch_bounds__(WARPS * 32, MIN_CTAS)
 decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v, const DecodeParams P) {
     using Cfg = MmaCfg<D, STAGES, WARPS>;
     constexpr int KSTEPS = D / 16;  // k-steps of Q K^T
     constexpr int NTD = D / 8;      // n-tiles of P V
     constexpr bool HI = ROWS > 8;   // query rows 8..15 in use
+    constexpr int AR = HI ? 4 : 2;  // registers per A fragment / per C tile that are held
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -105,6 +106,12 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int st = 0; st < STAGES; ++st) mbar_init(smem_u32(&bars[st]), 1);
         fence_barrier_init();
     }
+    // Launched with programmatic stream serialization: the CTAs become
+    // resident while the previous kernel (typically the cache write) drains,
+    // and wait here until its results are visible.  Nothing above touched
+    // global memory.
+    grid_dependency_wait();
+    allow_dependents();  // the reduction may launch and wait for this grid
     const Schedule sched = make_schedule(P, prefix, lens, WARPS);  // ends with __syncthreads
     zero_empty_sequences<__nv_bfloat16>(P, lens);
 
@@ -182,9 +189,9 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const uint32_t sw = lane & 7;   // swizzle term: ldmatrix row index mod 8
     const float sl2 = P.scale_log2;
 
-    uint32_t qa[KSTEPS][4];
+    uint32_t qa[KSTEPS][AR];  // Q as A fragments: {lo, [hi,] lo+8 cols, [hi+8 cols]}
     float m_lo = -INFINITY, l_lo = 0.f, m_hi = -INFINITY, l_hi = 0.f;
-    float acc[NTD][4];
+    float acc[NTD][AR];
 
     while (true) {
         if (cj == cc.jbeg) {  // new item: load its query rows as A fragments
@@ -195,15 +202,22 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const bool lo_ok = r_lo < g, hi_ok = HI && (r_lo + 8 < g);
 #pragma unroll
             for (int ks = 0; ks < KSTEPS; ++ks) {
-                qa[ks][0] = lo_ok ? __ldg(q_lo + ks * 8) : 0u;
-                qa[ks][2] = lo_ok ? __ldg(q_lo + ks * 8 + 4) : 0u;
-                qa[ks][1] = hi_ok ? __ldg(q_hi + ks * 8) : 0u;
-                qa[ks][3] = hi_ok ? __ldg(q_hi + ks * 8 + 4) : 0u;
+                if constexpr (HI) {
+                    qa[ks][0] = lo_ok ? __ldg(q_lo + ks * 8) : 0u;
+                    qa[ks][2] = lo_ok ? __ldg(q_lo + ks * 8 + 4) : 0u;
+                    qa[ks][1] = hi_ok ? __ldg(q_hi + ks * 8) : 0u;
+                    qa[ks][3] = hi_ok ? __ldg(q_hi + ks * 8 + 4) : 0u;
+                } else {
+                    qa[ks][0] = lo_ok ? __ldg(q_lo + ks * 8) : 0u;
+                    qa[ks][1] = lo_ok ? __ldg(q_lo + ks * 8 + 4) : 0u;
+                }
             }
             m_lo = m_hi = -INFINITY;
             l_lo = l_hi = 0.f;
 #pragma unroll
-            for (int n = 0; n < NTD; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+            for (int n = 0; n < NTD; ++n)
+#pragma unroll
+                for (int r = 0; r < AR; ++r) acc[n][r] = 0.f;
         }
 
         const uint32_t bar = bar_u32 + stage * 8;
@@ -235,18 +249,20 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
 
         // ---- S = Q K^T : two n-tiles of 8 tokens
-        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+        float s0[AR], s1[AR];
+#pragma unroll
+        for (int r = 0; r < AR; ++r) s0[r] = s1[r] = 0.f;
 #pragma unroll
         for (int kp = 0; kp < KSTEPS / 2; ++kp) {
             const int cg = 4 * kp + (lane >> 3);  // 8-element column chunk 0 .. D/8-1
             const uint32_t col = (cg >> 3) * Cfg::kRegionBytes + ((((uint32_t)cg & 7u) ^ sw) << 4);
             uint32_t b0, b1, b2, b3;
             ldsm_x4(kbase + col + (lane & 7) * 128, b0, b1, b2, b3);
-            mma_bf16(s0, qa[2 * kp][0], qa[2 * kp][1], qa[2 * kp][2], qa[2 * kp][3], b0, b1);
-            mma_bf16(s0, qa[2 * kp + 1][0], qa[2 * kp + 1][1], qa[2 * kp + 1][2], qa[2 * kp + 1][3], b2, b3);
+            mma_frag(s0, qa[2 * kp], b0, b1);
+            mma_frag(s0, qa[2 * kp + 1], b2, b3);
             ldsm_x4(kbase + col + (8 + (lane & 7)) * 128, b0, b1, b2, b3);
-            mma_bf16(s1, qa[2 * kp][0], qa[2 * kp][1], qa[2 * kp][2], qa[2 * kp][3], b0, b1);
-            mma_bf16(s1, qa[2 * kp + 1][0], qa[2 * kp + 1][1], qa[2 * kp + 1][2], qa[2 * kp + 1][3], b2, b3);
+            mma_frag(s1, qa[2 * kp], b0, b1);
+            mma_frag(s1, qa[2 * kp + 1], b2, b3);
         }
 
         // ---- online softmax (rows r_lo and r_lo + 8)
@@ -264,7 +280,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 acc[n][1] *= alpha;
             }
         }
-        if (HI) {
+        if constexpr (HI) {
             float x[4] = {s0[2], s0[3], s1[2], s1[3]};
             x[0] = tq < valid ? x[0] * sl2 : -INFINITY;
             x[1] = tq + 1 < valid ? x[1] * sl2 : -INFINITY;
@@ -278,6 +294,13 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
 
+        uint32_t pa[AR];  // P as an A fragment
+        if constexpr (HI) {
+            pa[0] = pa0; pa[1] = pa1; pa[2] = pa2; pa[3] = pa3;
+        } else {
+            pa[0] = pa0; pa[1] = pa2;
+        }
+
         // ---- O += P V : n-tiles of 8 head dims, K = the 16 tokens
 #pragma unroll
         for (int dp = 0; dp < D / 16; ++dp) {
@@ -287,8 +310,8 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                   ((((uint32_t)cg & 7u) ^ sw) << 4);
             uint32_t b0, b1, b2, b3;
             ldsm_x4_trans(addr, b0, b1, b2, b3);
-            mma_bf16(acc[2 * dp], pa0, pa1, pa2, pa3, b0, b1);
-            mma_bf16(acc[2 * dp + 1], pa0, pa1, pa2, pa3, b2, b3);
+            mma_frag(acc[2 * dp], pa, b0, b1);
+            mma_frag(acc[2 * dp + 1], pa, b2, b3);
         }
         __syncwarp();
 
@@ -304,7 +327,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         float lt_lo = l_lo + __shfl_xor_sync(kFullMask, l_lo, 1);
         lt_lo += __shfl_xor_sync(kFullMask, lt_lo, 2);
         float lt_hi = 0.f;
-        if (HI) {
+        if constexpr (HI) {
             lt_hi = l_hi + __shfl_xor_sync(kFullMask, l_hi, 1);
             lt_hi += __shfl_xor_sync(kFullMask, lt_hi, 2);
         }
@@ -319,13 +342,16 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     *reinterpret_cast<__nv_bfloat162*>(o + 8 * n) =
                         __floats2bfloat162_rn(acc[n][0] * inv, acc[n][1] * inv);
             }
-            if (HI && r_lo + 8 < g) {
-                const float inv = lt_hi > 0.f ? 1.0f / lt_hi : 0.f;
-                __nv_bfloat16* o = ob + (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo + 8) * D + tq;
+            if constexpr (HI) {
+                if (r_lo + 8 < g) {
+                    const float inv = lt_hi > 0.f ? 1.0f / lt_hi : 0.f;
+                    __nv_bfloat16* o =
+                        ob + (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo + 8) * D + tq;
 #pragma unroll
-                for (int n = 0; n < NTD; ++n)
-                    *reinterpret_cast<__nv_bfloat162*>(o + 8 * n) =
-                        __floats2bfloat162_rn(acc[n][2] * inv, acc[n][3] * inv);
+                    for (int n = 0; n < NTD; ++n)
+                        *reinterpret_cast<__nv_bfloat162*>(o + 8 * n) =
+                            __floats2bfloat162_rn(acc[n][2] * inv, acc[n][3] * inv);
+                }
             }
         } else {
             constexpr float kLn2 = 0.693147180559945309f;
@@ -340,17 +366,19 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 for (int n = 0; n < NTD; ++n)
                     *reinterpret_cast<float2*>(a + 8 * n) = make_float2(acc[n][0], acc[n][1]);
             }
-            if (HI && r_lo + 8 < g) {
-                const size_t idx =
-                    (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo + 8) * P.max_parts + cc.p;
-                if ((lane & 3) == 0) {
-                    P.ws_m[idx] = m_hi * kLn2;
-                    P.ws_l[idx] = lt_hi;
-                }
-                float* a = P.ws_acc + idx * D + tq;
+            if constexpr (HI) {
+                if (r_lo + 8 < g) {
+                    const size_t idx =
+                        (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo + 8) * P.max_parts + cc.p;
+                    if ((lane & 3) == 0) {
+                        P.ws_m[idx] = m_hi * kLn2;
+                        P.ws_l[idx] = lt_hi;
+                    }
+                    float* a = P.ws_acc + idx * D + tq;
 #pragma unroll
-                for (int n = 0; n < NTD; ++n)
-                    *reinterpret_cast<float2*>(a + 8 * n) = make_float2(acc[n][2], acc[n][3]);
+                    for (int n = 0; n < NTD; ++n)
+                        *reinterpret_cast<float2*>(a + 8 * n) = make_float2(acc[n][2], acc[n][3]);
+                }
             }
         }
 

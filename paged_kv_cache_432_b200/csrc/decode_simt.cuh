@@ -27,6 +27,8 @@ decode_f32_simt_kernel(const DecodeParams P) {
     __shared__ float pbuf[kSimtWarps][MAXG][kBlockTokens];
     int32_t* prefix = smem_i;
     int32_t* lens = prefix + P.seq_count + 1;
+    grid_dependency_wait();  // global memory only once the previous kernel is done
+    allow_dependents();
     const Schedule sched = make_schedule(P, prefix, lens, kSimtWarps);
     zero_empty_sequences<float>(P, lens);
 

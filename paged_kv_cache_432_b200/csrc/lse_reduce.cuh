@@ -40,6 +40,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const Dec
     __shared__ float red[kReduceWarps][D];
     __shared__ float wmax[kReduceWarps], wden[kReduceWarps];
 
+    grid_dependency_wait();  // the partials of the decode launched just before
     const int64_t row = blockIdx.x;  // (sequence within launch) * Hq + query head
     const int32_t s = P.seq_begin + static_cast<int32_t>(row / P.num_q_heads);
     const int32_t qh = static_cast<int32_t>(row % P.num_q_heads);
@@ -90,6 +91,83 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const Dec
     const float inv = den > 0.f ? 1.0f / den : 0.f;
     for (int d = tid; d < D; d += blockDim.x)
         o[d] = from_float<OutT>(((red[0][d] + red[1][d]) + (red[2][d] + red[3][d])) * inv);
+}
+
+// One warp merges one row (sequence, query head) from its `parts` pieces
+// starting at partial index `base`; lanes hold D/32 consecutive head dims.
+template <typename OutT, int D>
+__device__ __forceinline__ void merge_row_warp(const DecodeParams& P, size_t base, int parts,
+                                               OutT* o, int lane) {
+    constexpr int DPL = D / 32;
+    using Vec = typename std::conditional<DPL == 4, float4, float2>::type;
+    const float* wm = P.ws_m + base;
+    const float* wl = P.ws_l + base;
+    const float* wa = P.ws_acc + base * D + lane * DPL;
+    float M = -INFINITY;
+    for (int p = lane; p < parts; p += 32) M = fmaxf(M, wm[p]);
+    M = warp_max(M);
+    if (M == -INFINITY) {  // every piece fully masked
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) o[lane * DPL + e] = from_float<OutT>(0.f);
+        return;
+    }
+    float den = 0.f;
+    for (int p = lane; p < parts; p += 32) den += expf(wm[p] - M) * wl[p];
+    den = warp_sum(den);
+    float a[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) a[e] = 0.f;
+#pragma unroll 4
+    for (int p = 0; p < parts; ++p) {
+        const float w = expf(wm[p] - M);
+        const Vec x = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(p) * D);
+        const float* f = reinterpret_cast<const float*>(&x);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) a[e] = fmaf(w, f[e], a[e]);
+    }
+    const float inv = den > 0.f ? 1.0f / den : 0.f;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) o[lane * DPL + e] = from_float<OutT>(a[e] * inv);
+}
+
+// Balanced split: only units that cross a boundary between two decode warps'
+// ranges were cut, so the merge walks those boundaries instead of every row.
+// CTA b looks at the boundary between decode warps b and b + 1 (stream
+// position (b + 1) * C, with C recomputed exactly as the decode did from the
+// same lengths and the decode's warp count).  If a unit crosses it and this is
+// the unit's first boundary, the CTA's warps merge the unit's query rows.
+template <typename OutT, int D>
+__global__ void __launch_bounds__(kReduceWarps * 32)
+lse_reduce_balanced_kernel(const DecodeParams P, int32_t decode_warps) {
+    grid_dependency_wait();  // the partials of the decode launched just before
+    extern __shared__ int32_t smem_i[];
+    int32_t* prefix = smem_i;
+    int32_t* lens = prefix + P.seq_count + 1;
+    const int32_t total = build_prefix(P, prefix, lens);  // blocks per sequence
+    const int64_t hk = P.num_kv_heads;
+    const int64_t T = static_cast<int64_t>(total) * hk;
+    const int64_t even = (T + decode_warps - 1) / decode_warps;
+    const int64_t C = even > P.min_chunk ? even : P.min_chunk;
+    const int64_t b = (static_cast<int64_t>(blockIdx.x) + 1) * C;
+    if (b >= T) return;
+    const int i = upper_index(P.seq_count, b, [&](int k) { return hk * prefix[k]; });
+    const SeqGeom geo = seq_geometry(P, lens[i]);
+    const int64_t off = b - hk * prefix[i];
+    const int32_t h = static_cast<int32_t>(off / geo.nb);
+    const int64_t j = off - static_cast<int64_t>(h) * geo.nb;
+    if (j == 0) return;  // a unit starts exactly here: nothing crosses
+    const int64_t ustart = b - j;
+    if (ustart / C != blockIdx.x) return;  // merged at the unit's first boundary
+    const int64_t uend = ustart + geo.nb;
+    const int parts = static_cast<int>((uend - 1) / C - ustart / C + 1);
+    const int32_t s = P.seq_begin + i;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int r = warp; r < P.group; r += kReduceWarps) {
+        const int32_t qh = h * P.group + r;
+        const size_t row = static_cast<size_t>(s) * P.num_q_heads + qh;
+        merge_row_warp<OutT, D>(P, row * P.max_parts, parts, static_cast<OutT*>(P.out) + row * D,
+                                lane);
+    }
 }
 
 }  // namespace pa
