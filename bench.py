@@ -82,6 +82,7 @@ def workload_config(w: wl.Workload, pb: int) -> dict:
         "split": "balanced (equal blocks per warp)" if pb == 0 else (
             "never" if pb >= (1 << 24) else f"fixed {pb}-block partitions"),
         "new_tokens": int(w.slot_mapping.numel()),
+        "shared_prefix_blocks": w.shared_prefix_blocks,
         "slot_utilisation": round(sum(w.lens_host) / (16 * sum(len(t) for t in w.tables_host)), 5),
         "l2": "flushed before every step (512 MiB write + 256 MiB read, outside the timed "
               "events); KV footprint exceeds L2",
@@ -330,7 +331,14 @@ def run_ours(args) -> None:
     pb = w.partition_blocks if args.partition_blocks is None else args.partition_blocks
     msl = w.max_seq_len
     resolved_pb = pa.partition_blocks(w.num_seqs, w.num_kv_heads, msl, pb)
-    wsp = pa.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, msl, pb, device=dev)
+    # a batch sharing a prompt prefix goes through the shared-prefix decode
+    use_sp = w.shared_prefix_blocks > 0 and not args.plain_decode
+    if use_sp:
+        n = pa.shared_prefix_workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, msl,
+                                            w.shared_prefix_blocks, pb)
+        wsp = torch.empty(n, dtype=torch.uint8, device=dev)
+    else:
+        wsp = pa.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, msl, pb, device=dev)
     split = wsp is not None
     out = torch.empty_like(w.q)
     flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -345,7 +353,7 @@ def run_ours(args) -> None:
     stream = torch.cuda.current_stream(dev)
     by = algorithmic_bytes(w)
     chunks = math.ceil(w.num_seqs / 2048)
-    launches_per_step = 1 + chunks + (chunks if split else 0)
+    launches_per_step = 1 + chunks + (chunks if split else 0) + (1 if use_sp else 0)
 
     def step(ev=None):
         if ev is not None:
@@ -353,6 +361,14 @@ def run_ours(args) -> None:
         pa.cache_write(w.new_k, w.new_v, w.slot_mapping, w.k_cache, w.v_cache, stream)
         if ev is not None:
             ev[1].record(stream)
+        if use_sp:  # prefix kernel + private-part decode + merge, one call
+            pa.decode_shared_prefix(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale,
+                                    w.shared_prefix_blocks, out=out, max_seq_len=msl, partition_blocks=pb,
+                                    workspace=wsp, stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
+                ev[3].record(stream)
+            return
         pa.decode_partitions(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, out, msl,
                              pb, wsp, stream)
         if ev is not None:
@@ -434,8 +450,13 @@ def run_ours(args) -> None:
         def e2e_step():
             dev_buf.copy_(host_buf, non_blocking=True)
             pa.cache_write(dev_in["new_k"], dev_in["new_v"], dev_in["slot_mapping"], w.k_cache, w.v_cache, stream)
-            pa.decode(dev_in["q"], w.k_cache, w.v_cache, dev_in["block_tables"], dev_in["seq_lens"], w.scale,
-                      out=out, max_seq_len=msl, partition_blocks=pb, workspace=wsp, stream=stream)
+            if use_sp:
+                pa.decode_shared_prefix(dev_in["q"], w.k_cache, w.v_cache, dev_in["block_tables"],
+                                        dev_in["seq_lens"], w.scale, w.shared_prefix_blocks, out=out,
+                                        max_seq_len=msl, partition_blocks=pb, workspace=wsp, stream=stream)
+            else:
+                pa.decode(dev_in["q"], w.k_cache, w.v_cache, dev_in["block_tables"], dev_in["seq_lens"], w.scale,
+                          out=out, max_seq_len=msl, partition_blocks=pb, workspace=wsp, stream=stream)
             host_out.copy_(out, non_blocking=True)
 
         for _ in range(args.warmup):
@@ -462,8 +483,10 @@ def run_ours(args) -> None:
 
     peak, peak_kind = load_peaks()
     achieved = by["decode"] / (dec_ms * 1e-3) / 1e9
-    roof = {"bound": "hbm", "kernel": "decode_bf16_mma_kernel" if w.dtype == torch.bfloat16 else
-            "decode_f32_simt_kernel", "achieved": round(achieved, 1), "peak": peak,
+    kname = "decode_bf16_mma_kernel" if w.dtype == torch.bfloat16 else "decode_f32_simt_kernel"
+    if use_sp:
+        kname = "pa_decode_shared_prefix (prefix kernel + decode_bf16_mma_kernel + reduce, timed together)"
+    roof = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1), "peak": peak,
             "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
             else "fallback 6650 GB/s", "unit": "GB/s", "frac": round(achieved / peak, 4),
             "frac_of_8TBs": round(achieved / 8000.0, 4),
@@ -518,6 +541,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition-blocks", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--plain-decode", action="store_true",
+                    help="decode a shared-prefix batch with pa_decode instead of pa_decode_shared_prefix")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
     ap.add_argument("--ref-seqs-per-step", type=int, default=2)

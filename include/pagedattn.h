@@ -71,6 +71,8 @@ extern "C" {
 #define PA_DEVERR_BLOCK_OOB 2u /* decode: table entry outside [0, num_blocks), block masked */
 #define PA_DEVERR_SEQ_LEN 4u   /* decode: seq_len < 0 or beyond capacity, clamped          */
 #define PA_DEVERR_TIMEOUT 8u   /* a bounded wait on an async copy gave up                  */
+#define PA_DEVERR_PREFIX 16u   /* shared-prefix decode: a table does not start with the
+                                  shared blocks, or a sequence is shorter than them      */
 
 /*
  * Cache write (the scatter of newly computed K/V into the paged pool).
@@ -174,6 +176,44 @@ PA_API int pa_decode_reduce(const int32_t* seq_lens, int32_t max_seq_len, int32_
                      int32_t max_blocks_per_seq, int32_t block_size,
                      int32_t partition_blocks, const void* workspace,
                      size_t workspace_bytes, void* out, int32_t dtype, void* stream);
+
+/*
+ * Decode for a batch whose sequences all start with the same prompt, stored
+ * once: the first `shared_blocks` entries of every block table are the same
+ * physical blocks (prefix caching: "Was ändert PagedAttention an der
+ * KV-Speicherzuweisung für LLMs?", slavadubrov.com, §"Gemeinsame Nutzung
+ * erfordert mehr als Speicherzuweisung"; "PagedAttention et vLLM",
+ * aiunderstanding.org, §"Questions fréquemment posées").  Same result as
+ * pa_decode, computed in three launches: the query rows of all sequences
+ * attend to the shared blocks together, so those blocks are read once per
+ * kv head rather than once per sequence (tensor-core tiles of 64 query rows);
+ * each sequence's own blocks go through the decode kernel; a log-sum-exp
+ * reduction merges the two.  Preconditions: every table starts with the
+ * prefix blocks of table 0, and every seq_len >= shared_blocks * block_size.
+ * A violation is flagged with PA_DEVERR_PREFIX (the result is then
+ * meaningless for the offending sequences).  Only PA_DTYPE_BF16.  The
+ * workspace is sized by pa_decode_shared_prefix_workspace_size; the other
+ * arguments are those of pa_decode.  shared_blocks = 0 is plain pa_decode.
+ */
+PA_API int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_cache,
+                                   const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   const int32_t* seq_lens, int32_t max_seq_len,
+                                   int32_t shared_blocks, int32_t num_seqs, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                                   int32_t block_size, float scale, int32_t partition_blocks,
+                                   void* workspace, size_t workspace_bytes, void* out,
+                                   int32_t dtype, void* stream);
+
+/*
+ * Workspace bytes pa_decode_shared_prefix needs.  Layout as for pa_decode, with
+ * P = prefix key splits + the pieces the private part of a sequence can have;
+ * pieces 0 .. splits-1 of every row hold the shared prefix's partials.
+ */
+PA_API size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                                     int32_t num_kv_heads, int32_t head_dim,
+                                                     int32_t max_seq_len, int32_t shared_blocks,
+                                                     int32_t block_size,
+                                                     int32_t partition_blocks);
 
 /*
  * Reads the sticky device error word of the current device (PA_DEVERR_* bits)

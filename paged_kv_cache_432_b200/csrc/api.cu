@@ -21,6 +21,7 @@
 #include "cache_write.cuh"
 #include "common.cuh"
 #include "decode_mma.cuh"
+#include "decode_prefix.cuh"
 #include "decode_simt.cuh"
 #include "items.cuh"
 #include "lse_reduce.cuh"
@@ -180,11 +181,17 @@ struct Plan {
     int32_t max_parts;    // pieces per unit the workspace holds
     int32_t max_len;      // effective max_seq_len (the workspace is sized for it)
     bool split;
+    // shared-prefix decode only
+    int32_t shared_blocks;
+    int32_t prefix_splits;        // key splits of the prefix = its pieces 0 .. splits-1
+    int32_t prefix_split_blocks;  // blocks per key split
+    int32_t prefix_row_tiles;     // ceil(num_seqs * group / 64)
 };
 
 Plan make_plan(int32_t max_seq_len, int32_t partition_blocks) {
     Plan p;
     p.max_len = max_seq_len;
+    p.shared_blocks = p.prefix_splits = p.prefix_split_blocks = p.prefix_row_tiles = 0;
     const int32_t nb = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
     const int32_t pb = resolve_part_blocks(partition_blocks);
     p.balanced = pb == 0;
@@ -197,6 +204,32 @@ Plan make_plan(int32_t max_seq_len, int32_t partition_blocks) {
         p.max_parts = nb == 0 ? 1 : 1 + (nb - 1) / pb;
     }
     p.split = p.max_parts > 1;
+    return p;
+}
+
+// Shared-prefix decode: the prefix kernel's key splits are pieces 0..splits-1
+// of every row; the private part of each sequence (blocks from shared_blocks
+// on) is cut as pa_decode would cut a sequence of the remaining length, and
+// its pieces follow.  Key splits are chosen for about kPrefixTargetCtas CTAs.
+constexpr int32_t kPrefixTargetCtas = 512;
+
+Plan make_prefix_plan(int32_t max_seq_len, int32_t partition_blocks, int32_t shared_blocks,
+                      int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads) {
+    const int32_t rest = max_seq_len - shared_blocks * kBlockTokens;
+    Plan p = make_plan(rest > 0 ? rest : 0, partition_blocks);
+    p.max_len = max_seq_len;
+    const int64_t rows = static_cast<int64_t>(num_seqs) * (num_q_heads / num_kv_heads);
+    p.prefix_row_tiles = static_cast<int32_t>((rows + kPrefixRows - 1) / kPrefixRows);
+    if (p.prefix_row_tiles < 1) p.prefix_row_tiles = 1;
+    const int64_t per_split = static_cast<int64_t>(num_kv_heads) * p.prefix_row_tiles;
+    int64_t splits = (kPrefixTargetCtas + per_split - 1) / per_split;
+    if (splits > shared_blocks) splits = shared_blocks;
+    if (splits < 1) splits = 1;
+    p.prefix_split_blocks = static_cast<int32_t>((shared_blocks + splits - 1) / splits);
+    p.prefix_splits = (shared_blocks + p.prefix_split_blocks - 1) / p.prefix_split_blocks;
+    p.shared_blocks = shared_blocks;
+    p.max_parts += p.prefix_splits;
+    p.split = true;
     return p;
 }
 
@@ -248,7 +281,9 @@ int check_shapes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, in
 }
 
 // Validates and fills the kernel parameter block (workspace pointers included).
-int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan* plan) {
+// shared_blocks > 0: the shared-prefix decode (plan from make_prefix_plan).
+int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan* plan,
+                   int32_t shared_blocks = 0) {
     int rc = check_shapes(a.num_seqs, a.num_q_heads, a.num_kv_heads, a.head_dim, a.block_size,
                           a.dtype);
     if (rc != PA_OK) return rc;
@@ -270,7 +305,16 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
     const int32_t max_len = a.max_seq_len > 0
                                 ? a.max_seq_len
                                 : static_cast<int32_t>(table_tokens > INT32_MAX ? INT32_MAX : table_tokens);
-    *plan = make_plan(max_len, a.partition_blocks);
+    if (shared_blocks > 0) {
+        if (a.dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
+        if (shared_blocks > a.max_blocks_per_seq ||
+            static_cast<int64_t>(shared_blocks) * kBlockTokens > max_len)
+            return PA_ERR_INVALID_ARG;
+        *plan = make_prefix_plan(max_len, a.partition_blocks, shared_blocks, a.num_seqs,
+                                 a.num_q_heads, a.num_kv_heads);
+    } else {
+        *plan = make_plan(max_len, a.partition_blocks);
+    }
     const WsLayout ws = ws_layout(a.num_seqs, a.num_q_heads, a.num_kv_heads, plan->max_parts,
                                   a.head_dim, plan->split);
     std::memset(P, 0, sizeof *P);
@@ -301,6 +345,8 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
     P->min_chunk = kMinChunk;
     P->max_parts = plan->max_parts;
     P->len_cap = static_cast<int32_t>(max_len < table_tokens ? max_len : table_tokens);
+    P->skip_blocks = plan->shared_blocks;
+    P->piece_base = plan->prefix_splits;
     P->scale = a.scale;
     P->scale_log2 = a.scale * 1.4426950408889634f;
     return PA_OK;
@@ -433,11 +479,45 @@ int run_partitions(const DecodeParams& P, int32_t dtype, cudaStream_t st) {
     return P.group <= 4 ? launch_simt<64, 4>(P, st) : launch_simt<64, 16>(P, st);
 }
 
+template <int D>
+int launch_prefix(const DecodeParams& P, const Plan& plan, cudaStream_t st) {
+    auto kernel = decode_prefix_mma_kernel<D>;
+    int rc = ensure_smem_attr(kernel, PrefixCfg<D>::kSmem);
+    if (rc != PA_OK) return rc;
+    const int64_t rows = static_cast<int64_t>(P.num_blocks) * P.num_kv_heads * kBlockTokens;
+    alignas(64) CUtensorMap mk, mv;
+    if ((rc = encode_pool_map(&mk, P.k_cache, rows, D)) != PA_OK) return rc;
+    if ((rc = encode_pool_map(&mv, P.v_cache, rows, D)) != PA_OK) return rc;
+    PrefixParams PP;
+    PP.q = P.q;
+    PP.block_tables = P.block_tables;
+    PP.seq_lens = P.seq_lens;
+    PP.ws_m = P.ws_m;
+    PP.ws_l = P.ws_l;
+    PP.ws_acc = P.ws_acc;
+    PP.num_seqs = P.num_seqs;
+    PP.num_q_heads = P.num_q_heads;
+    PP.num_kv_heads = P.num_kv_heads;
+    PP.group = P.group;
+    PP.max_blocks_per_seq = P.max_blocks_per_seq;
+    PP.num_blocks = P.num_blocks;
+    PP.shared_blocks = plan.shared_blocks;
+    PP.split_blocks = plan.prefix_split_blocks;
+    PP.row_tiles = plan.prefix_row_tiles;
+    PP.max_parts = P.max_parts;
+    PP.scale_log2 = P.scale_log2;
+    const dim3 grid(static_cast<unsigned>(plan.prefix_row_tiles) * plan.prefix_splits,
+                    static_cast<unsigned>(P.num_kv_heads));
+    cudaError_t e = launch_pdl(kernel, grid, dim3(PrefixCfg<D>::kThreads), PrefixCfg<D>::kSmem, st,
+                               mk, mv, PP);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode_prefix_mma_kernel launch");
+}
+
 template <typename OutT, int D>
 int launch_reduce(const DecodeParams& base, int32_t dtype, cudaStream_t st) {
     return for_each_chunk(base, [&](const DecodeParams& P) {
         cudaError_t e;
-        if (P.balanced) {
+        if (P.balanced && P.piece_base == 0) {
             LaunchShape L;
             int r = decode_shape(P, dtype, &L);
             if (r != PA_OK) return r;
@@ -647,6 +727,52 @@ int pa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                      num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale,
                      partition_blocks, scratch, need > 0 ? PA_NOALLOC_SCRATCH_BYTES : 0, out,
                      dtype, stream);
+}
+
+int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* seq_lens, int32_t max_seq_len, int32_t shared_blocks,
+                            int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                            int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
+                            int32_t partition_blocks, void* workspace, size_t workspace_bytes,
+                            void* out, int32_t dtype, void* stream) {
+    if (shared_blocks < 0) return PA_ERR_INVALID_ARG;
+    if (shared_blocks == 0)
+        return pa_decode(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                         max_seq_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                         block_size, scale, partition_blocks, workspace, workspace_bytes, out,
+                         dtype, stream);
+    const DecodeArgs a = make_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                                   max_seq_len, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                   num_blocks, block_size, scale, partition_blocks, workspace,
+                                   workspace_bytes, out, dtype, stream);
+    DecodeParams P;
+    Plan plan;
+    int rc = prepare_decode(a, true, &P, &plan, shared_blocks);
+    if (rc != PA_OK) return rc;
+    if (num_seqs == 0) return PA_OK;
+    rc = head_dim == 128 ? launch_prefix<128>(P, plan, a.stream) : launch_prefix<64>(P, plan, a.stream);
+    if (rc != PA_OK) return rc;
+    rc = run_partitions(P, dtype, a.stream);
+    if (rc != PA_OK) return rc;
+    return run_reduce(P, plan, dtype, a.stream);
+}
+
+size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                              int32_t num_kv_heads, int32_t head_dim,
+                                              int32_t max_seq_len, int32_t shared_blocks,
+                                              int32_t block_size, int32_t partition_blocks) {
+    if (shared_blocks == 0)
+        return pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len,
+                                        block_size, partition_blocks);
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        max_seq_len < 0 || block_size != kBlockTokens || partition_blocks < -1 ||
+        shared_blocks < 0 || num_q_heads % num_kv_heads != 0 ||
+        static_cast<int64_t>(shared_blocks) * kBlockTokens > max_seq_len)
+        return 0;
+    const Plan plan = make_prefix_plan(max_seq_len, partition_blocks, shared_blocks, num_seqs,
+                                       num_q_heads, num_kv_heads);
+    return ws_layout(num_seqs, num_q_heads, num_kv_heads, plan.max_parts, head_dim, plan.split).bytes;
 }
 
 int pa_get_device_error(uint32_t* bits, int32_t clear, void* stream) {

@@ -50,6 +50,9 @@ struct DecodeParams {
     int32_t min_chunk;           // balanced mode: fewest blocks a warp range holds
     int32_t max_parts;           // pieces per row the workspace holds
     int32_t len_cap;             // longest sequence handled; longer ones are clamped
+    int32_t skip_blocks;         // pieces cover blocks [skip_blocks, nb) of each sequence
+    int32_t piece_base;          // > 0: pieces are written as partials at index piece_base + p
+                                 //      (the first piece_base partials come from elsewhere)
     int32_t seq_begin;           // first sequence of this launch
     int32_t seq_count;           // sequences in this launch
     float scale;                 // softmax scale (natural units)
@@ -142,6 +145,13 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// L2 policy for data many CTAs read (a shared prefix): keep it.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
 

@@ -332,7 +332,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             lt_hi += __shfl_xor_sync(kFullMask, lt_hi, 2);
         }
         const int qh_lo = cc.h * g + r_lo;
-        if (cc.parts == 1) {
+        if (cc.parts == 1 && P.piece_base == 0) {
             __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(P.out);
             if (r_lo < g) {
                 const float inv = lt_lo > 0.f ? 1.0f / lt_lo : 0.f;
@@ -356,7 +356,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         } else {
             constexpr float kLn2 = 0.693147180559945309f;
             if (r_lo < g) {
-                const size_t idx = (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo) * P.max_parts + cc.p;
+                const size_t idx = (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo) * P.max_parts + P.piece_base + cc.p;
                 if ((lane & 3) == 0) {
                     P.ws_m[idx] = m_lo * kLn2;
                     P.ws_l[idx] = lt_lo;
@@ -369,7 +369,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if constexpr (HI) {
                 if (r_lo + 8 < g) {
                     const size_t idx =
-                        (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo + 8) * P.max_parts + cc.p;
+                        (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo + 8) * P.max_parts + P.piece_base + cc.p;
                     if ((lane & 3) == 0) {
                         P.ws_m[idx] = m_hi * kLn2;
                         P.ws_l[idx] = lt_hi;

@@ -126,7 +126,7 @@ decode_f32_simt_kernel(const DecodeParams P) {
             __syncwarp();
         }
 
-        if (it.parts == 1) {
+        if (it.parts == 1 && P.piece_base == 0) {
             float* o = static_cast<float*>(P.out) +
                        (static_cast<size_t>(it.s) * P.num_q_heads + it.h * g) * D + lane * DPL;
 #pragma unroll
@@ -141,7 +141,7 @@ decode_f32_simt_kernel(const DecodeParams P) {
             for (int i = 0; i < MAXG; ++i) {
                 if (i >= g) break;
                 const size_t idx =
-                    (static_cast<size_t>(it.s) * P.num_q_heads + it.h * g + i) * P.max_parts + it.p;
+                    (static_cast<size_t>(it.s) * P.num_q_heads + it.h * g + i) * P.max_parts + P.piece_base + it.p;
                 if (lane == 0) {
                     P.ws_m[idx] = m[i];
                     P.ws_l[idx] = l[i];

@@ -30,7 +30,9 @@ namespace pa {
 struct SeqGeom {
     int32_t len;    // tokens attended (clamped)
     int32_t nb;     // blocks: ceil(len / 16)
-    int32_t parts;  // fixed mode: ceil(nb / part_blocks); 0 for an empty sequence
+    int32_t first;  // first block the pieces cover (skip_blocks, at most nb)
+    int32_t work;   // blocks the pieces cover: nb - first
+    int32_t parts;  // fixed mode: ceil(work / part_blocks); 0 when there is no work
 };
 
 __device__ __forceinline__ SeqGeom seq_geometry(const DecodeParams& P, int32_t len) {
@@ -39,7 +41,9 @@ __device__ __forceinline__ SeqGeom seq_geometry(const DecodeParams& P, int32_t l
     if (len > P.len_cap) len = P.len_cap;
     g.len = len;
     g.nb = (len + kBlockTokens - 1) / kBlockTokens;
-    g.parts = g.nb == 0 ? 0 : 1 + (g.nb - 1) / P.part_blocks;
+    g.first = min(P.skip_blocks, g.nb);
+    g.work = g.nb - g.first;
+    g.parts = g.work == 0 ? 0 : 1 + (g.work - 1) / P.part_blocks;
     return g;
 }
 
@@ -62,7 +66,7 @@ __device__ __forceinline__ int32_t build_prefix(const DecodeParams& P, int32_t* 
         if (report && (raw < 0 || raw > P.len_cap)) flag_error(PA_DEVERR_SEQ_LEN);
         const SeqGeom g = seq_geometry(P, raw);
         lens[i] = g.len;
-        local += P.balanced ? g.nb : g.parts * P.num_kv_heads;
+        local += P.balanced ? g.work : g.parts * P.num_kv_heads;
     }
     const int lane = tid & 31, warp = tid >> 5, nwarps = (nthr + 31) >> 5;
     int32_t incl = local;
@@ -88,7 +92,7 @@ __device__ __forceinline__ int32_t build_prefix(const DecodeParams& P, int32_t* 
     for (int i = beg; i < end; ++i) {
         prefix[i] = run;
         const SeqGeom g = seq_geometry(P, lens[i]);
-        run += P.balanced ? g.nb : g.parts * P.num_kv_heads;
+        run += P.balanced ? g.work : g.parts * P.num_kv_heads;
     }
     if (tid == nthr - 1) prefix[n] = run;  // the last thread ends on the grand total
     __syncthreads();
@@ -144,7 +148,7 @@ struct Schedule {
         const SeqGeom g = seq_geometry(*P, lens[i]);
         c.len = g.len;
         c.parts = g.parts;
-        c.jbeg = c.p * P->part_blocks;
+        c.jbeg = g.first + c.p * P->part_blocks;
         c.jend = min(g.nb, c.jbeg + P->part_blocks);
     }
 
@@ -154,11 +158,12 @@ struct Schedule {
         const int i = upper_index(n, c.pos, [&](int k) { return hk * prefix[k]; });
         const SeqGeom g = seq_geometry(*P, lens[i]);
         const int64_t off = c.pos - hk * prefix[i];
-        c.h = static_cast<int32_t>(off / g.nb);
-        c.jbeg = static_cast<int32_t>(off - static_cast<int64_t>(c.h) * g.nb);
-        const int64_t ustart = c.pos - c.jbeg;
-        const int64_t uend = ustart + g.nb;
-        c.jend = static_cast<int32_t>(min(uend, c.end) - ustart);
+        c.h = static_cast<int32_t>(off / g.work);
+        const int64_t jrel = off - static_cast<int64_t>(c.h) * g.work;
+        const int64_t ustart = c.pos - jrel;
+        const int64_t uend = ustart + g.work;
+        c.jbeg = g.first + static_cast<int32_t>(jrel);
+        c.jend = g.first + static_cast<int32_t>(min(uend, c.end) - ustart);
         c.s = P->seq_begin + i;
         c.len = g.len;
         c.p = static_cast<int32_t>(c.pos / c.chunk - ustart / c.chunk);
@@ -182,7 +187,7 @@ struct Schedule {
     // Move to the warp's next piece.
     __device__ __forceinline__ void next(Cursor& c) const {
         if (P->balanced) {
-            c.pos += c.jend - c.jbeg;
+            c.pos += c.jend - c.jbeg;  // the piece's length
             c.valid = c.pos < c.end;
             if (c.valid) locate_balanced(c);
         } else {
@@ -213,9 +218,11 @@ __device__ __forceinline__ Schedule make_schedule(const DecodeParams& P, int32_t
 }
 
 // Zero-length sequences have no pieces; their rows of `out` are zero.  CTA b
-// clears those of the sequences s = b, b + gridDim.x, ... of the launch.
+// clears those of the sequences s = b, b + gridDim.x, ... of the launch.  (With
+// piece_base > 0 the rows are written by the merge instead.)
 template <typename OutT>
 __device__ __forceinline__ void zero_empty_sequences(const DecodeParams& P, const int32_t* lens) {
+    if (P.piece_base > 0) return;
     const int row = P.num_q_heads * P.head_dim;
     for (int i = blockIdx.x; i < P.seq_count; i += gridDim.x) {
         if (lens[i] != 0) continue;

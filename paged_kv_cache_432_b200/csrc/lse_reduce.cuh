@@ -45,9 +45,11 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const Dec
     const int32_t s = P.seq_begin + static_cast<int32_t>(row / P.num_q_heads);
     const int32_t qh = static_cast<int32_t>(row % P.num_q_heads);
     const SeqGeom geo = seq_geometry(P, P.seq_lens[s]);
-    if (geo.nb == 0) return;  // an empty sequence: the decode kernel zeroed its rows
-    const int parts = P.ws_parts[static_cast<size_t>(s) * P.num_kv_heads + qh / P.group];
-    if (parts <= 1) return;   // a single piece: the decode kernel wrote the row
+    // pieces: piece_base partials written elsewhere (a shared prefix), then
+    // the decode kernel's pieces of blocks [first, nb), counted in ws_parts
+    const int own = geo.work > 0 ? P.ws_parts[static_cast<size_t>(s) * P.num_kv_heads + qh / P.group] : 0;
+    const int parts = P.piece_base + own;
+    if (P.piece_base == 0 && parts <= 1) return;  // empty or a single piece: the decode wrote the row
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t base = (static_cast<size_t>(s) * P.num_q_heads + qh) * P.max_parts;
@@ -153,12 +155,12 @@ lse_reduce_balanced_kernel(const DecodeParams P, int32_t decode_warps) {
     const int i = upper_index(P.seq_count, b, [&](int k) { return hk * prefix[k]; });
     const SeqGeom geo = seq_geometry(P, lens[i]);
     const int64_t off = b - hk * prefix[i];
-    const int32_t h = static_cast<int32_t>(off / geo.nb);
-    const int64_t j = off - static_cast<int64_t>(h) * geo.nb;
+    const int32_t h = static_cast<int32_t>(off / geo.work);
+    const int64_t j = off - static_cast<int64_t>(h) * geo.work;
     if (j == 0) return;  // a unit starts exactly here: nothing crosses
     const int64_t ustart = b - j;
     if (ustart / C != blockIdx.x) return;  // merged at the unit's first boundary
-    const int64_t uend = ustart + geo.nb;
+    const int64_t uend = ustart + geo.work;
     const int parts = static_cast<int>((uend - 1) / C - ustart / C + 1);
     const int32_t s = P.seq_begin + i;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -31,6 +31,7 @@ PA_DEVERR_SLOT_OOB = 1
 PA_DEVERR_BLOCK_OOB = 2
 PA_DEVERR_SEQ_LEN = 4
 PA_DEVERR_TIMEOUT = 8
+PA_DEVERR_PREFIX = 16
 
 # every symbol the header declares, with (restype, argtypes)
 _P, _I32, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -44,6 +45,9 @@ SIGNATURES = {
     "pa_decode_reduce": (ctypes.c_int, [_P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ, _P, _I32, _P]),
     "pa_decode_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _F,
                                          _I32, _P, _I32, _P]),
+    "pa_decode_shared_prefix": (ctypes.c_int, [_P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32,
+                                               _I32, _F, _I32, _P, _SZ, _P, _I32, _P]),
+    "pa_decode_shared_prefix_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "pa_get_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _I32, _P]),
     "pa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -151,6 +155,34 @@ def decode(q, k_cache, v_cache, block_tables, seq_lens, scale, out=None, max_seq
                                     partition_blocks, device=q.device)
     _decode_call("pa_decode", q, k_cache, v_cache, block_tables, seq_lens, scale, out, max_seq_len,
                  partition_blocks, workspace, stream)
+    return out
+
+
+def shared_prefix_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len, shared_blocks,
+                                 partition_blocks=0, block_size=16) -> int:
+    return int(lib().pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                            max_seq_len, shared_blocks, block_size,
+                                                            partition_blocks))
+
+
+def decode_shared_prefix(q, k_cache, v_cache, block_tables, seq_lens, scale, shared_blocks, out=None,
+                         max_seq_len=0, partition_blocks=0, workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode_shared_prefix: the decode when the first `shared_blocks` blocks of
+    every table are one shared prefix (read once per kv head for all sequences)."""
+    N, Hq, D = q.shape
+    NB, Hkv, B, _ = k_cache.shape
+    msl = max_seq_len if max_seq_len > 0 else block_tables.shape[1] * 16
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        n = shared_prefix_workspace_size(N, Hq, Hkv, D, msl, shared_blocks, partition_blocks)
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().pa_decode_shared_prefix(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens),
+        max_seq_len, shared_blocks, N, Hq, Hkv, D, NB, B, float(scale), partition_blocks, _ptr(workspace),
+        ws_bytes, _ptr(out), dtype_code(q.dtype), _stream(stream))
+    _check("pa_decode_shared_prefix", rc)
     return out
 
 

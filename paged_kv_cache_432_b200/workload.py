@@ -85,6 +85,7 @@ class Workload:
     slot_mapping: torch.Tensor  # int64 [T]; -1 = padding (nothing written)
     partition_blocks: int = 0  # 0 = let the library choose
     shared_blocks: list = field(default_factory=list)  # physical ids referenced by >1 seq
+    shared_prefix_blocks: int = 0  # leading table entries every sequence shares (whole blocks)
     desc: str = ""
 
     @property
@@ -308,6 +309,7 @@ def build(
         slot_mapping=slot_mapping.to(device),
         partition_blocks=partition_blocks,
         shared_blocks=sorted(p.shared + [src for src, _ in p.cow_pairs[:1]]),
+        shared_prefix_blocks=len(p.shared),
         desc=desc,
     )
 

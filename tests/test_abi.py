@@ -80,6 +80,22 @@ def test_workspace_size_matches_documented_layout(lib):
     assert pa.workspace_size(N, Hq, Hkv, D, 0, 0) == 0
 
 
+def test_shared_prefix_workspace_size(lib):
+    a256 = lambda x: (x + 255) // 256 * 256
+    N, Hq, Hkv, D = 128, 32, 8, 128
+    # 512 query rows per kv head -> 8 row tiles x 8 heads = 64 CTAs per key split -> 8 splits
+    # private part: (4604 - 4096) tokens -> 32 blocks -> balanced bound ceil(32/32)+1 = 2 pieces
+    P = 8 + 2
+    rows = N * Hq
+    expect = 2 * a256(rows * P * 4) + a256(rows * P * D * 4) + a256(N * Hkv * 4)
+    assert lib.pa_decode_shared_prefix_workspace_size(N, Hq, Hkv, D, 4604, 256, 16, 0) == expect
+    # no shared blocks: the plain decode's size
+    assert lib.pa_decode_shared_prefix_workspace_size(N, Hq, Hkv, D, 4604, 0, 16, 0) == \
+        lib.pa_decode_workspace_size(N, Hq, Hkv, D, 4604, 16, 0)
+    # a prefix longer than the longest sequence is rejected
+    assert lib.pa_decode_shared_prefix_workspace_size(N, Hq, Hkv, D, 1000, 256, 16, 0) == 0
+
+
 def _decode_rc(lib, **over):
     args = dict(q=16, k=16, v=16, bt=16, mb=4, sl=16, msl=64, N=2, Hq=4, Hkv=2, D=128, NB=8, B=16,
                 scale=0.1, pb=0, ws=None, wsb=0, out=16, dt=pa.PA_DTYPE_BF16)

@@ -210,6 +210,61 @@ def test_balanced_split_long_unit_across_many_warps(lens, Hq, Hkv):
     assert pa.device_error() == 0
 
 
+# ------------------------------------------------------------------ shared-prefix decode
+def _shared_prefix_decode(w, pb=0, **kw):
+    out = pa.decode_shared_prefix(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale,
+                                  w.shared_prefix_blocks, max_seq_len=w.max_seq_len, partition_blocks=pb, **kw)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("prefix_len,suffixes,Hq,Hkv,D", [
+    (64, [5, 40, 17, 0, 200], 8, 2, 128),
+    (4096, [64, 1, 300, 512, 16], 32, 8, 128),
+    (4090, [5, 40, 700], 16, 2, 64),        # prefix ends mid-block: 255 shared blocks + private copies
+    (1600, [33] * 40, 4, 4, 128),           # many sequences: several row tiles per kv head
+    (512, [9, 100], 32, 2, 128),            # group of 16
+])
+@pytest.mark.parametrize("pb", [0, 4])
+def test_shared_prefix_decode_matches_oracle(prefix_len, suffixes, Hq, Hkv, D, pb):
+    lens = [prefix_len + x for x in suffixes]
+    w = wl.build(lens, Hq, Hkv, D, torch.bfloat16, seed=prefix_len + len(lens), device=DEV,
+                 prefix_len=prefix_len, poison_unused=True)
+    assert w.shared_prefix_blocks == prefix_len // 16
+    out = _shared_prefix_decode(w, pb)
+    assert_close(to_f64(out), oracle_decode(w), torch.bfloat16, f"shared prefix {prefix_len}")
+    assert pa.device_error() == 0
+
+
+def test_shared_prefix_full_size_workload_sampled_rows():
+    """The prefix-sharing workload at full size through the shared-prefix path,
+    after the cache write of each sequence's newest token."""
+    w = wl.make("prefix", device=DEV)
+    h = host(w)
+    pa.cache_write(w.new_k, w.new_v, w.slot_mapping, w.k_cache, w.v_cache)
+    out = _shared_prefix_decode(w)
+    h["kc"], h["vc"], _ = oracle.cache_write(h["nk"], h["nv"], h["sm"], h["kc"], h["vc"])
+    rows = _sample_rows(w, 40, seed=7)
+    ref = oracle_decode(w, h, rows=rows)
+    g = to_f64(out)
+    assert_close(np.stack([g[s, qh] for s, qh in rows]), ref, torch.bfloat16, "prefix full size")
+    plain = to_f64(gpu_decode(w))
+    assert_close(g, plain, torch.bfloat16, "shared-prefix vs plain decode")
+    assert pa.device_error() == 0
+
+
+def test_shared_prefix_preconditions_are_flagged():
+    w = wl.build([600, 700], 8, 2, 128, torch.bfloat16, seed=5, device=DEV, prefix_len=512)
+    bt = w.block_tables.clone()
+    bt[1, 3] = w.tables_host[1][-1]  # sequence 1 no longer starts with the shared blocks
+    pa.decode_shared_prefix(w.q, w.k_cache, w.v_cache, bt, w.seq_lens, w.scale, 32, max_seq_len=700)
+    assert pa.device_error() & pa.PA_DEVERR_PREFIX
+    short = w.seq_lens.clone()
+    short[0] = 100  # shorter than the prefix
+    pa.decode_shared_prefix(w.q, w.k_cache, w.v_cache, w.block_tables, short, w.scale, 32, max_seq_len=700)
+    assert pa.device_error() & pa.PA_DEVERR_PREFIX
+
+
 # ------------------------------------------------------------------ the two steps separately
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_partition_partials_match_oracle(dtype):
