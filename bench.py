@@ -7,8 +7,8 @@ One step = one pass of the hot path over one batch: the cache write of each
 sequence's newest token (pa_cache_write), then the decode (the block-table
 walk with split-K partials, pa_decode_partitions, and the log-sum-exp merge,
 pa_decode_reduce).  Inputs are resident in HBM; L2 is flushed before every
-step (a 512 MiB write, then a 256 MiB read so no dirty lines are left to
-write back inside the next step), outside the timed events.  Times are CUDA events on the
+step (a 512 MiB write, then a 512 MiB read so no dirty lines or pending
+write-backs are left for the next step), outside the timed events.  Times are CUDA events on the
 launching stream; with N > 1 (torchrun) every rank runs its own replica of the
 workload (seed + rank, no data exchange) and the step time is the max over
 ranks.  Prints one JSON line.
@@ -84,7 +84,7 @@ def workload_config(w: wl.Workload, pb: int) -> dict:
         "new_tokens": int(w.slot_mapping.numel()),
         "shared_prefix_blocks": w.shared_prefix_blocks,
         "slot_utilisation": round(sum(w.lens_host) / (16 * sum(len(t) for t in w.tables_host)), 5),
-        "l2": "flushed before every step (512 MiB write + 256 MiB read, outside the timed "
+        "l2": "flushed before every step (512 MiB write + 512 MiB read, outside the timed "
               "events); KV footprint exceeds L2",
     }
 
@@ -342,12 +342,12 @@ def run_ours(args) -> None:
     split = wsp is not None
     out = torch.empty_like(w.q)
     flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    flush_r = torch.zeros(FLUSH_BYTES // 2, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def flush_l2():
-        # evict everything: write a buffer 4x the L2, then read another 2x the
-        # L2 so the lines left behind are clean (no write-back lands in the
-        # next timed step)
+        # evict everything: write a buffer 4x the L2, then read another 4x the
+        # L2 so the lines left behind are clean and the write-backs of the
+        # written lines have drained (none lands in the next timed step)
         flush_w.zero_()
         flush_r.view(torch.float32).sum()  # a read-only reduction (no dtype-converting copy)
     stream = torch.cuda.current_stream(dev)

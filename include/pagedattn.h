@@ -93,7 +93,7 @@ PA_API int pa_cache_write(const void* k, const void* v, const int64_t* slot_mapp
  * How the decode splits sequences, from partition_blocks:
  *   0   (auto) balanced split.  All (sequence, kv head) units form one stream
  *       of blocks and every warp of the persistent grid takes an equal share
- *       (at least 32 blocks), so long and short sequences mix without load
+ *       (at least 16 blocks), so long and short sequences mix without load
  *       imbalance.  A unit that spans several shares becomes several pieces.
  *   > 0 fixed partitions of that many blocks.
  *   -1  never split: one pass over each whole sequence.
@@ -109,7 +109,7 @@ PA_API int32_t pa_decode_partition_blocks(int32_t num_seqs, int32_t num_kv_heads
  * Bytes of workspace pa_decode needs for these sizes (0 when no sequence of up
  * to max_seq_len tokens can be split).  Workspace layout: P is the number of
  * pieces a unit can have at max_seq_len (fixed: ceil(nb / partition_blocks);
- * balanced: ceil(nb / 32) + 1, with nb = ceil(max_seq_len / 16)), and rows
+ * balanced: ceil(nb / 16) + 1, with nb = ceil(max_seq_len / 16)), and rows
  * r = seq * num_q_heads + q_head:
  *   float   m    [num_seqs*num_q_heads][P]    max score of the piece (natural log units)
  *   float   l    [num_seqs*num_q_heads][P]    sum of exp(score - m)
@@ -206,8 +206,10 @@ PA_API int pa_decode_shared_prefix(const void* q, const void* k_cache, const voi
 
 /*
  * Workspace bytes pa_decode_shared_prefix needs.  Layout as for pa_decode, with
- * P = prefix key splits + the pieces the private part of a sequence can have;
- * pieces 0 .. splits-1 of every row hold the shared prefix's partials.
+ * P = min(16, shared_blocks) slots for the prefix's key splits + the pieces the
+ * private part of a sequence can have; pieces 0 .. splits-1 of every row hold
+ * the shared prefix's partials (the split count, at most 16, is chosen at
+ * launch to fill one wave of the device) and the private pieces follow.
  */
 PA_API size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                                      int32_t num_kv_heads, int32_t head_dim,

@@ -165,7 +165,7 @@ int encode_pool_map(CUtensorMap* map, const void* base, int64_t rows, int head_d
 }
 
 // ------------------------------------------------------------ planning
-constexpr int32_t kMinChunk = 32;  // balanced split: fewest blocks in one warp's range
+constexpr int32_t kMinChunk = 16;  // balanced split: fewest blocks in one warp's range
 
 // Fixed partition size for partition_blocks > 0 or -1 (never split); 0 for the
 // balanced split (partition_blocks = 0).
@@ -210,8 +210,11 @@ Plan make_plan(int32_t max_seq_len, int32_t partition_blocks) {
 // Shared-prefix decode: the prefix kernel's key splits are pieces 0..splits-1
 // of every row; the private part of each sequence (blocks from shared_blocks
 // on) is cut as pa_decode would cut a sequence of the remaining length, and
-// its pieces follow.  Key splits are chosen for about kPrefixTargetCtas CTAs.
-constexpr int32_t kPrefixTargetCtas = 512;
+// its pieces follow.  The workspace reserves kMaxPrefixSplits slots; the launch
+// picks the split count that fills one wave of the prefix kernel on the
+// device (choose_prefix_splits).
+constexpr int32_t kMaxPrefixSplits = 16;
+constexpr int32_t kWideReducePieces = 32;  // rows that can have more pieces merge with 4 warps each
 
 Plan make_prefix_plan(int32_t max_seq_len, int32_t partition_blocks, int32_t shared_blocks,
                       int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads) {
@@ -221,14 +224,11 @@ Plan make_prefix_plan(int32_t max_seq_len, int32_t partition_blocks, int32_t sha
     const int64_t rows = static_cast<int64_t>(num_seqs) * (num_q_heads / num_kv_heads);
     p.prefix_row_tiles = static_cast<int32_t>((rows + kPrefixRows - 1) / kPrefixRows);
     if (p.prefix_row_tiles < 1) p.prefix_row_tiles = 1;
-    const int64_t per_split = static_cast<int64_t>(num_kv_heads) * p.prefix_row_tiles;
-    int64_t splits = (kPrefixTargetCtas + per_split - 1) / per_split;
-    if (splits > shared_blocks) splits = shared_blocks;
-    if (splits < 1) splits = 1;
-    p.prefix_split_blocks = static_cast<int32_t>((shared_blocks + splits - 1) / splits);
-    p.prefix_splits = (shared_blocks + p.prefix_split_blocks - 1) / p.prefix_split_blocks;
     p.shared_blocks = shared_blocks;
-    p.max_parts += p.prefix_splits;
+    const int32_t slots = shared_blocks < kMaxPrefixSplits ? shared_blocks : kMaxPrefixSplits;
+    p.prefix_splits = slots;  // reserved; narrowed at launch
+    p.prefix_split_blocks = (shared_blocks + slots - 1) / slots;
+    p.max_parts += slots;
     p.split = true;
     return p;
 }
@@ -479,6 +479,31 @@ int run_partitions(const DecodeParams& P, int32_t dtype, cudaStream_t st) {
     return P.group <= 4 ? launch_simt<64, 4>(P, st) : launch_simt<64, 16>(P, st);
 }
 
+// Key splits of the shared prefix: as many as fill one wave of the prefix
+// kernel (resident CTAs on the device / CTAs per split), within the slots the
+// workspace reserves.  Sets plan->prefix_splits / prefix_split_blocks.
+template <int D>
+int choose_prefix_splits(const DecodeParams& P, Plan* plan) {
+    auto kernel = decode_prefix_mma_kernel<D>;
+    int rc = ensure_smem_attr(kernel, PrefixCfg<D>::kSmem);
+    if (rc != PA_OK) return rc;
+    DeviceInfo di;
+    if ((rc = device_info(&di)) != PA_OK) return rc;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, PrefixCfg<D>::kThreads,
+                                                                  PrefixCfg<D>::kSmem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    const int64_t wave = static_cast<int64_t>(di.sms) * (per_sm > 0 ? per_sm : 1);
+    const int64_t per_split = static_cast<int64_t>(P.num_kv_heads) * plan->prefix_row_tiles;
+    int64_t splits = wave / per_split;
+    const int32_t slots = plan->prefix_splits;
+    if (splits > slots) splits = slots;
+    if (splits < 1) splits = 1;
+    plan->prefix_split_blocks = static_cast<int32_t>((plan->shared_blocks + splits - 1) / splits);
+    plan->prefix_splits = (plan->shared_blocks + plan->prefix_split_blocks - 1) / plan->prefix_split_blocks;
+    return PA_OK;
+}
+
 template <int D>
 int launch_prefix(const DecodeParams& P, const Plan& plan, cudaStream_t st) {
     auto kernel = decode_prefix_mma_kernel<D>;
@@ -527,8 +552,14 @@ int launch_reduce(const DecodeParams& base, int32_t dtype, cudaStream_t st) {
                            dim3(kReduceWarps * 32), 8 * static_cast<size_t>(P.seq_count + 1), st, P,
                            decode_warps);
         } else {
-            const unsigned grid = static_cast<unsigned>(P.seq_count) * P.num_q_heads;
-            e = launch_pdl(lse_reduce_kernel<OutT, D>, dim3(grid), dim3(kReduceWarps * 32), 0, st, P);
+            const int64_t rows = static_cast<int64_t>(P.seq_count) * P.num_q_heads;
+            if (P.max_parts > kWideReducePieces) {  // many pieces per row: 4 warps per row
+                e = launch_pdl(lse_reduce_wide_kernel<OutT, D>, dim3(static_cast<unsigned>(rows)),
+                               dim3(kReduceWarps * 32), 0, st, P);
+            } else {
+                const unsigned grid = static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps);
+                e = launch_pdl(lse_reduce_kernel<OutT, D>, dim3(grid), dim3(kReduceWarps * 32), 0, st, P);
+            }
         }
         return e == cudaSuccess ? PA_OK : cuda_fail(e, "lse_reduce_kernel launch");
     });
@@ -751,6 +782,9 @@ int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_ca
     int rc = prepare_decode(a, true, &P, &plan, shared_blocks);
     if (rc != PA_OK) return rc;
     if (num_seqs == 0) return PA_OK;
+    rc = head_dim == 128 ? choose_prefix_splits<128>(P, &plan) : choose_prefix_splits<64>(P, &plan);
+    if (rc != PA_OK) return rc;
+    P.piece_base = plan.prefix_splits;  // the private pieces follow the splits actually used
     rc = head_dim == 128 ? launch_prefix<128>(P, plan, a.stream) : launch_prefix<64>(P, plan, a.stream);
     if (rc != PA_OK) return rc;
     rc = run_partitions(P, dtype, a.stream);

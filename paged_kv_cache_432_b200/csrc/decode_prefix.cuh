@@ -15,9 +15,12 @@
 // Grid: (row tiles x key splits, kv heads).  A CTA owns 64 query rows (4
 // consumer warps x 16 rows, any (sequence, query head) pairs of the group) and
 // one key split (a run of prefix blocks).  A producer warp streams the split's
-// blocks with TMA (64 x 16 boxes, 128-byte swizzle) into a 4-stage ring shared
-// by the 4 consumers: `full` barriers carry the TMA byte counts, `empty`
-// barriers collect one arrival per consumer warp before a stage is refilled.
+// blocks with TMA (64 x 16 boxes, 128-byte swizzle), two blocks (32 keys) per
+// stage, into a 4-stage ring shared by the 4 consumers: `full` barriers carry
+// the TMA byte counts, `empty` barriers collect one arrival per consumer warp
+// before a stage is refilled.  Each 32-key step costs one softmax update per
+// row, and the accumulators are rescaled only when some row's running max
+// moved.
 // Each consumer runs mma.sync m16n8k16 (bf16, fp32 accumulate) on its 16 rows,
 // the same fragment layout as the decode kernel, and writes the split's
 // partial (m, l, acc) per row to the workspace at piece index = split.  The
@@ -49,18 +52,51 @@ struct PrefixParams {
     float scale_log2;
 };
 
+#ifndef PA_PREFIX_MIN_CTAS
+#define PA_PREFIX_MIN_CTAS 2
+#endif
 constexpr int kPrefixConsumers = 4;
 constexpr int kPrefixStages = 4;
 constexpr int kPrefixRows = 16 * kPrefixConsumers;  // query rows per CTA
 
+constexpr int kPrefixBlocksPerStage = 2;  // 32 keys per softmax step
+
 template <int D>
 struct PrefixCfg {
     static constexpr int kRegions = D / 64;
-    static constexpr int kTileBytes = kRegions * 2048;
-    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kTileBytes = kRegions * 2048;  // K (or V) of one block, one head
+    // stage: K of block 0, K of block 1, V of block 0, V of block 1
+    static constexpr int kStageBytes = 2 * kPrefixBlocksPerStage * kTileBytes;
     static constexpr int kThreads = (kPrefixConsumers + 1) * 32;
     static constexpr size_t kSmem = 1024 + kPrefixStages * kStageBytes + 2 * kPrefixStages * 8 + 16 * 4;
 };
+
+// Online-softmax update of one row set over a 32-key step.  x[] are the row's
+// scores (log2 units, -inf where masked) for keys tq, tq+1, 8+tq, 9+tq, then
+// the same + 16.  Packs the probabilities as bf16 pairs p[0..3] (keys tq..,
+// 8+tq.., 16+tq.., 24+tq..) and returns the accumulator rescale factor.
+__device__ __forceinline__ float softmax_update32(float& m, float& l, const float (&x)[8],
+                                                  uint32_t (&p)[4]) {
+    float bm = x[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) bm = fmaxf(bm, x[k]);
+    bm = fmaxf(bm, __shfl_xor_sync(kFullMask, bm, 1));
+    bm = fmaxf(bm, __shfl_xor_sync(kFullMask, bm, 2));
+    const float mn = fmaxf(m, bm);
+    const float mu = mn == -INFINITY ? 0.0f : mn;
+    const float alpha = exp2f(m - mu);
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(exp2f(x[2 * k] - mu), exp2f(x[2 * k + 1] - mu));
+        const float2 f = __bfloat1622float2(v);
+        sum += f.x + f.y;
+        p[k] = bf162_bits(v);
+    }
+    l = l * alpha + sum;
+    m = mn;
+    return alpha;
+}
 
 // Single-thread bounded wait (the producer lane).
 __device__ __forceinline__ bool mbar_wait_bounded_thread(uint32_t bar, uint32_t parity) {
@@ -78,7 +114,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(PrefixCfg<D>::kThreads)
+__global__ void __launch_bounds__(PrefixCfg<D>::kThreads, PA_PREFIX_MIN_CTAS)
 decode_prefix_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                          const __grid_constant__ CUtensorMap tmap_v, const PrefixParams P) {
     using Cfg = PrefixCfg<D>;
@@ -135,29 +171,50 @@ decode_prefix_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         // ---------------- producer: one lane streams the split's blocks
         if (lane != 0) return;
         const uint64_t policy = l2_policy_evict_last();  // every row tile of this head reads them
-        for (int n = 0; n < nblk; ++n) {
+        const int nst = (nblk + kPrefixBlocksPerStage - 1) / kPrefixBlocksPerStage;
+        for (int n = 0; n < nst; ++n) {
             const int st = n % S;
             const uint32_t fill = n / S;
             if (fill > 0 && !mbar_wait_bounded_thread(empty_u32 + st * 8, (fill - 1) & 1u)) {
                 flag_error(PA_DEVERR_TIMEOUT);
                 return;
             }
-            int32_t pb = P.block_tables[jbeg + n];
-            const bool bad = static_cast<uint32_t>(pb) >= static_cast<uint32_t>(P.num_blocks);
-            if (bad) {
-                flag_error(PA_DEVERR_BLOCK_OOB);
-                pb = 0;
+            // bit b: block b of the stage is absent or outside the pool (masked)
+            int32_t pbs[kPrefixBlocksPerStage];
+            int32_t mask = 0, loaded = 0;
+#pragma unroll
+            for (int b = 0; b < kPrefixBlocksPerStage; ++b) {
+                const int j = jbeg + n * kPrefixBlocksPerStage + b;
+                pbs[b] = -1;
+                if (j >= jend) {
+                    mask |= 1 << b;
+                    continue;
+                }
+                int32_t pb = P.block_tables[j];
+                if (static_cast<uint32_t>(pb) >= static_cast<uint32_t>(P.num_blocks)) {
+                    flag_error(PA_DEVERR_BLOCK_OOB);
+                    mask |= 1 << b;
+                    continue;
+                }
+                pbs[b] = pb;
+                ++loaded;
             }
-            oob[st] = bad ? 1 : 0;  // published by the mbarrier arrive below
+            oob[st] = mask;  // published by the mbarrier arrive below
             fence_proxy_async_smem();
             const uint32_t bar = full_u32 + st * 8;
-            mbar_arrive_expect_tx(bar, Cfg::kStageBytes);
-            const int32_t row = (pb * P.num_kv_heads + h) * kBlockTokens;
-            const uint32_t kdst = ring_u32 + st * Cfg::kStageBytes;
+            mbar_arrive_expect_tx(bar, loaded * 2 * Cfg::kTileBytes);
+            const uint32_t sbase = ring_u32 + st * Cfg::kStageBytes;
 #pragma unroll
-            for (int r = 0; r < Cfg::kRegions; ++r) {
-                tma_load_2d(kdst + r * 2048, &tmap_k, r * 64, row, bar, policy);
-                tma_load_2d(kdst + Cfg::kTileBytes + r * 2048, &tmap_v, r * 64, row, bar, policy);
+            for (int b = 0; b < kPrefixBlocksPerStage; ++b) {
+                if (pbs[b] < 0) continue;
+                const int32_t row = (pbs[b] * P.num_kv_heads + h) * kBlockTokens;
+                const uint32_t kdst = sbase + b * Cfg::kTileBytes;
+                const uint32_t vdst = sbase + (kPrefixBlocksPerStage + b) * Cfg::kTileBytes;
+#pragma unroll
+                for (int r = 0; r < Cfg::kRegions; ++r) {
+                    tma_load_2d(kdst + r * 2048, &tmap_k, r * 64, row, bar, policy);
+                    tma_load_2d(vdst + r * 2048, &tmap_v, r * 64, row, bar, policy);
+                }
             }
         }
         return;
@@ -189,48 +246,65 @@ decode_prefix_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     for (int n = 0; n < NTD; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
     const float sl2 = P.scale_log2;
 
-    for (int n = 0; n < nblk; ++n) {
+    const int nst = (nblk + kPrefixBlocksPerStage - 1) / kPrefixBlocksPerStage;
+    for (int n = 0; n < nst; ++n) {
         const int st = n % S;
         if (!mbar_wait_bounded(full_u32 + st * 8, (n / S) & 1u)) {
             if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
             return;
         }
-        const bool bad = oob[st] != 0;
-        const uint32_t kbase = ring_u32 + st * Cfg::kStageBytes;
-        const uint32_t vbase = kbase + Cfg::kTileBytes;
-        if (!bad) {
-            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+        const int32_t mask = oob[st];
+        const uint32_t sbase = ring_u32 + st * Cfg::kStageBytes;
+        // ---- S = Q K^T over 32 keys: n-tiles 0,1 from block 0, 2,3 from block 1
+        float sc[4][4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) sc[t][0] = sc[t][1] = sc[t][2] = sc[t][3] = 0.f;
+#pragma unroll
+        for (int b = 0; b < kPrefixBlocksPerStage; ++b) {
+            if (mask & (1 << b)) continue;  // warp-uniform
+            const uint32_t kbase = sbase + b * Cfg::kTileBytes;
 #pragma unroll
             for (int kp = 0; kp < KSTEPS / 2; ++kp) {
                 const int cg = 4 * kp + (lane >> 3);
                 const uint32_t col = (cg >> 3) * 2048 + ((((uint32_t)cg & 7u) ^ sw) << 4);
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(kbase + col + (lane & 7) * 128, b0, b1, b2, b3);
-                mma_frag(s0, qa[2 * kp], b0, b1);
-                mma_frag(s0, qa[2 * kp + 1], b2, b3);
+                mma_frag(sc[2 * b], qa[2 * kp], b0, b1);
+                mma_frag(sc[2 * b], qa[2 * kp + 1], b2, b3);
                 ldsm_x4(kbase + col + (8 + (lane & 7)) * 128, b0, b1, b2, b3);
-                mma_frag(s1, qa[2 * kp], b0, b1);
-                mma_frag(s1, qa[2 * kp + 1], b2, b3);
+                mma_frag(sc[2 * b + 1], qa[2 * kp], b0, b1);
+                mma_frag(sc[2 * b + 1], qa[2 * kp + 1], b2, b3);
             }
-            uint32_t pa[4];
-            {
-                const float x[4] = {s0[0] * sl2, s0[1] * sl2, s1[0] * sl2, s1[1] * sl2};
-                const float alpha = softmax_update(m_lo, l_lo, x, pa[0], pa[2]);
+        }
+        // ---- online softmax of rows r_lo (accumulator regs 0,1) and r_hi (2,3)
+        const bool m0 = (mask & 1) != 0, m1 = (mask & 2) != 0;
+        float xl[8], xh[8];
 #pragma unroll
-                for (int k = 0; k < NTD; ++k) {
-                    acc[k][0] *= alpha;
-                    acc[k][1] *= alpha;
-                }
-            }
-            {
-                const float x[4] = {s0[2] * sl2, s0[3] * sl2, s1[2] * sl2, s1[3] * sl2};
-                const float alpha = softmax_update(m_hi, l_hi, x, pa[1], pa[3]);
+        for (int t = 0; t < 4; ++t) {
+            const bool dead = t < 2 ? m0 : m1;
+            xl[2 * t] = dead ? -INFINITY : sc[t][0] * sl2;
+            xl[2 * t + 1] = dead ? -INFINITY : sc[t][1] * sl2;
+            xh[2 * t] = dead ? -INFINITY : sc[t][2] * sl2;
+            xh[2 * t + 1] = dead ? -INFINITY : sc[t][3] * sl2;
+        }
+        uint32_t pl[4], ph[4];
+        const float alpha_lo = softmax_update32(m_lo, l_lo, xl, pl);
+        const float alpha_hi = softmax_update32(m_hi, l_hi, xh, ph);
+        if (__any_sync(kFullMask, alpha_lo != 1.f || alpha_hi != 1.f)) {  // a row max moved
 #pragma unroll
-                for (int k = 0; k < NTD; ++k) {
-                    acc[k][2] *= alpha;
-                    acc[k][3] *= alpha;
-                }
+            for (int k = 0; k < NTD; ++k) {
+                acc[k][0] *= alpha_lo;
+                acc[k][1] *= alpha_lo;
+                acc[k][2] *= alpha_hi;
+                acc[k][3] *= alpha_hi;
             }
+        }
+        // ---- O += P V, one k-step of 16 keys per present block
+#pragma unroll
+        for (int b = 0; b < kPrefixBlocksPerStage; ++b) {
+            if (mask & (1 << b)) continue;
+            const uint32_t pa[4] = {pl[2 * b], ph[2 * b], pl[2 * b + 1], ph[2 * b + 1]};
+            const uint32_t vbase = sbase + (kPrefixBlocksPerStage + b) * Cfg::kTileBytes;
 #pragma unroll
             for (int dp = 0; dp < D / 16; ++dp) {
                 const int cg = 2 * dp + (lane >> 4);

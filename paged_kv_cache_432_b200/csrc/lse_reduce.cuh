@@ -10,12 +10,11 @@
 // matters most: "PagedAttention et vLLM", aiunderstanding.org,
 // §"L'avenir de PagedAttention et vLLM").
 //
-// One CTA (4 warps) per (sequence, query head) row: all threads find M and the
-// denominator, each warp accumulates a strided subset of the pieces' acc rows
-// with 16-byte loads, and the four warp sums are added in a fixed order.  The
-// number of pieces of each (sequence, kv head) unit is read from the
-// workspace, where the decode kernel recorded it; rows of units with a single
-// piece are skipped (the decode kernel wrote them).
+// A warp merges one (sequence, query head) row: lanes read the pieces' m and
+// l in parallel, then accumulate the pieces' acc rows (lanes across head dims,
+// 16-byte loads, eight pieces in flight).  Two kernels choose the rows: the
+// row-wise one (fixed partitions, shared prefix) and the boundary-walking one
+// (balanced split).
 #pragma once
 
 #include "items.cuh"
@@ -31,68 +30,6 @@ __device__ __forceinline__ float from_float<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) {
     return __float2bfloat16_rn(x);
-}
-
-template <typename OutT, int D>
-__global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const DecodeParams P) {
-    constexpr int DPL = D / 32;
-    using Vec = typename std::conditional<DPL == 4, float4, float2>::type;
-    __shared__ float red[kReduceWarps][D];
-    __shared__ float wmax[kReduceWarps], wden[kReduceWarps];
-
-    grid_dependency_wait();  // the partials of the decode launched just before
-    const int64_t row = blockIdx.x;  // (sequence within launch) * Hq + query head
-    const int32_t s = P.seq_begin + static_cast<int32_t>(row / P.num_q_heads);
-    const int32_t qh = static_cast<int32_t>(row % P.num_q_heads);
-    const SeqGeom geo = seq_geometry(P, P.seq_lens[s]);
-    // pieces: piece_base partials written elsewhere (a shared prefix), then
-    // the decode kernel's pieces of blocks [first, nb), counted in ws_parts
-    const int own = geo.work > 0 ? P.ws_parts[static_cast<size_t>(s) * P.num_kv_heads + qh / P.group] : 0;
-    const int parts = P.piece_base + own;
-    if (P.piece_base == 0 && parts <= 1) return;  // empty or a single piece: the decode wrote the row
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const size_t base = (static_cast<size_t>(s) * P.num_q_heads + qh) * P.max_parts;
-    const float* wm = P.ws_m + base;
-    const float* wl = P.ws_l + base;
-    const float* wa = P.ws_acc + base * D;
-
-    float M = -INFINITY;
-    for (int p = tid; p < parts; p += blockDim.x) M = fmaxf(M, wm[p]);
-    M = warp_max(M);
-    if (lane == 0) wmax[warp] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
-
-    OutT* o = static_cast<OutT*>(P.out) + (static_cast<size_t>(s) * P.num_q_heads + qh) * D;
-    if (M == -INFINITY) {  // every partition fully masked
-        for (int d = tid; d < D; d += blockDim.x) o[d] = from_float<OutT>(0.f);
-        return;
-    }
-
-    float den = 0.f;
-    for (int p = tid; p < parts; p += blockDim.x) den += expf(wm[p] - M) * wl[p];
-    den = warp_sum(den);
-    if (lane == 0) wden[warp] = den;
-
-    float a[DPL];
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) a[e] = 0.f;
-#pragma unroll 4
-    for (int p = warp; p < parts; p += kReduceWarps) {
-        const float w = expf(wm[p] - M);
-        const Vec x = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(p) * D + lane * DPL);
-        const float* f = reinterpret_cast<const float*>(&x);
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) a[e] = fmaf(w, f[e], a[e]);
-    }
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) red[warp][lane * DPL + e] = a[e];
-    __syncthreads();
-    den = (wden[0] + wden[1]) + (wden[2] + wden[3]);
-    const float inv = den > 0.f ? 1.0f / den : 0.f;
-    for (int d = tid; d < D; d += blockDim.x)
-        o[d] = from_float<OutT>(((red[0][d] + red[1][d]) + (red[2][d] + red[3][d])) * inv);
 }
 
 // One warp merges one row (sequence, query head) from its `parts` pieces
@@ -119,7 +56,7 @@ __device__ __forceinline__ void merge_row_warp(const DecodeParams& P, size_t bas
     float a[DPL];
 #pragma unroll
     for (int e = 0; e < DPL; ++e) a[e] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
     for (int p = 0; p < parts; ++p) {
         const float w = expf(wm[p] - M);
         const Vec x = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(p) * D);
@@ -130,6 +67,85 @@ __device__ __forceinline__ void merge_row_warp(const DecodeParams& P, size_t bas
     const float inv = den > 0.f ? 1.0f / den : 0.f;
 #pragma unroll
     for (int e = 0; e < DPL; ++e) o[lane * DPL + e] = from_float<OutT>(a[e] * inv);
+}
+
+// Row-wise merge (fixed partitions, or a shared prefix): one warp per
+// (sequence, query head) row, four rows per CTA.  The pieces of a row are
+// piece_base partials written by another kernel (a shared prefix's key
+// splits) followed by the decode kernel's pieces of blocks [first, nb), whose
+// number the decode recorded in ws_parts.  Rows with a single piece of their
+// own and nothing before it were written by the decode and are skipped.
+template <typename OutT, int D>
+__global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const DecodeParams P) {
+    grid_dependency_wait();  // the partials of the decode launched just before
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kReduceWarps + warp;
+    if (row >= static_cast<int64_t>(P.seq_count) * P.num_q_heads) return;
+    const int32_t s = P.seq_begin + static_cast<int32_t>(row / P.num_q_heads);
+    const int32_t qh = static_cast<int32_t>(row % P.num_q_heads);
+    const SeqGeom geo = seq_geometry(P, P.seq_lens[s]);
+    const int own = geo.work > 0 ? P.ws_parts[static_cast<size_t>(s) * P.num_kv_heads + qh / P.group] : 0;
+    const int parts = P.piece_base + own;
+    if (P.piece_base == 0 && parts <= 1) return;
+    const size_t r = static_cast<size_t>(s) * P.num_q_heads + qh;
+    merge_row_warp<OutT, D>(P, r * P.max_parts, parts, static_cast<OutT*>(P.out) + r * D, lane);
+}
+
+// Row-wise merge for rows with many pieces (long sequences in fixed
+// partitions): one CTA per row, the 4 warps split the pieces and their sums
+// are added in a fixed order.
+template <typename OutT, int D>
+__global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_wide_kernel(const DecodeParams P) {
+    constexpr int DPL = D / 32;
+    using Vec = typename std::conditional<DPL == 4, float4, float2>::type;
+    __shared__ float red[kReduceWarps][D];
+    __shared__ float wmax[kReduceWarps], wden[kReduceWarps];
+    grid_dependency_wait();
+    const int64_t row = blockIdx.x;  // (sequence within launch) * Hq + query head
+    const int32_t s = P.seq_begin + static_cast<int32_t>(row / P.num_q_heads);
+    const int32_t qh = static_cast<int32_t>(row % P.num_q_heads);
+    const SeqGeom geo = seq_geometry(P, P.seq_lens[s]);
+    const int own = geo.work > 0 ? P.ws_parts[static_cast<size_t>(s) * P.num_kv_heads + qh / P.group] : 0;
+    const int parts = P.piece_base + own;
+    if (P.piece_base == 0 && parts <= 1) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t base = (static_cast<size_t>(s) * P.num_q_heads + qh) * P.max_parts;
+    const float* wm = P.ws_m + base;
+    const float* wl = P.ws_l + base;
+    const float* wa = P.ws_acc + base * D;
+    float M = -INFINITY;
+    for (int p = tid; p < parts; p += blockDim.x) M = fmaxf(M, wm[p]);
+    M = warp_max(M);
+    if (lane == 0) wmax[warp] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+    OutT* o = static_cast<OutT*>(P.out) + (static_cast<size_t>(s) * P.num_q_heads + qh) * D;
+    if (M == -INFINITY) {
+        for (int d = tid; d < D; d += blockDim.x) o[d] = from_float<OutT>(0.f);
+        return;
+    }
+    float den = 0.f;
+    for (int p = tid; p < parts; p += blockDim.x) den += expf(wm[p] - M) * wl[p];
+    den = warp_sum(den);
+    if (lane == 0) wden[warp] = den;
+    float a[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) a[e] = 0.f;
+#pragma unroll 4
+    for (int p = warp; p < parts; p += kReduceWarps) {
+        const float w = expf(wm[p] - M);
+        const Vec x = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(p) * D + lane * DPL);
+        const float* f = reinterpret_cast<const float*>(&x);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) a[e] = fmaf(w, f[e], a[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) red[warp][lane * DPL + e] = a[e];
+    __syncthreads();
+    den = (wden[0] + wden[1]) + (wden[2] + wden[3]);
+    const float inv = den > 0.f ? 1.0f / den : 0.f;
+    for (int d = tid; d < D; d += blockDim.x)
+        o[d] = from_float<OutT>(((red[0][d] + red[1][d]) + (red[2][d] + red[3][d])) * inv);
 }
 
 // Balanced split: only units that cross a boundary between two decode warps'

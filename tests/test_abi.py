@@ -74,8 +74,8 @@ def test_workspace_size_matches_documented_layout(lib):
     assert pa.workspace_size(N, Hq, Hkv, D, 512, 32) == 0        # one partition: no workspace
     assert pa.workspace_size(N, Hq, Hkv, D, L, -1) == 0
     assert pa.workspace_size(N, Hq, Hkv, D, 513, 32) == layout(N, Hq, Hkv, D, 2)
-    # balanced split: a unit of nb blocks meets at most ceil(nb / 32) + 1 warp ranges
-    assert pa.workspace_size(N, Hq, Hkv, D, L, 0) == layout(N, Hq, Hkv, D, -(-nb // 32) + 1)
+    # balanced split: a unit of nb blocks meets at most ceil(nb / 16) + 1 warp ranges
+    assert pa.workspace_size(N, Hq, Hkv, D, L, 0) == layout(N, Hq, Hkv, D, -(-nb // 16) + 1)
     assert pa.workspace_size(N, Hq, Hkv, D, 100, 0) == layout(N, Hq, Hkv, D, 2)
     assert pa.workspace_size(N, Hq, Hkv, D, 0, 0) == 0
 
@@ -83,9 +83,9 @@ def test_workspace_size_matches_documented_layout(lib):
 def test_shared_prefix_workspace_size(lib):
     a256 = lambda x: (x + 255) // 256 * 256
     N, Hq, Hkv, D = 128, 32, 8, 128
-    # 512 query rows per kv head -> 8 row tiles x 8 heads = 64 CTAs per key split -> 8 splits
-    # private part: (4604 - 4096) tokens -> 32 blocks -> balanced bound ceil(32/32)+1 = 2 pieces
-    P = 8 + 2
+    # 16 reserved key-split slots for the prefix, then the private part:
+    # (4604 - 4096) tokens -> 32 blocks -> balanced bound ceil(32/16)+1 = 3 pieces
+    P = 16 + 3
     rows = N * Hq
     expect = 2 * a256(rows * P * 4) + a256(rows * P * D * 4) + a256(N * Hkv * 4)
     assert lib.pa_decode_shared_prefix_workspace_size(N, Hq, Hkv, D, 4604, 256, 16, 0) == expect
