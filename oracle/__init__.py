@@ -54,6 +54,8 @@ def _load():
         lib.oracle_decode_partials.restype = ctypes.c_int
         lib.oracle_decode_partials.argtypes = [P, P, P, P, I32, P, I32, I32, I32, I32, I32, I64,
                                                I32, D, I32, I32, P, P, P, P]
+        lib.oracle_copy_blocks.restype = I64
+        lib.oracle_copy_blocks.argtypes = [P, P, P, P, I64, I64, I64]
         lib.oracle_lse_merge.restype = None
         lib.oracle_lse_merge.argtypes = [P, P, P, P, I32, I32, I32, I32, P]
         _lib = lib
@@ -115,6 +117,20 @@ def cache_write(k, v, slot_mapping, k_cache, v_cache, inplace=False):
     NB, H2, B, D2 = kc.shape
     assert (H, D) == (H2, D2)
     bad = _load().oracle_cache_write(_ptr(k), _ptr(v), _ptr(sm), T, H, D, dt, _ptr(kc), _ptr(vc), NB, B)
+    return kc, vc, int(bad)
+
+
+def copy_blocks(k_cache, v_cache, src, dst):
+    """Copies of the pools where block dst[i] = block src[i] (both pools, all
+    heads); returns (k_cache, v_cache, n_bad)."""
+    kc = np.array(k_cache, copy=True, order="C")
+    vc = np.array(v_cache, copy=True, order="C")
+    src = np.ascontiguousarray(src, dtype=np.int32)
+    dst = np.ascontiguousarray(dst, dtype=np.int32)
+    assert src.shape == dst.shape
+    NB = kc.shape[0]
+    bb = kc[0].nbytes
+    bad = _load().oracle_copy_blocks(_ptr(kc), _ptr(vc), _ptr(src), _ptr(dst), len(src), NB, bb)
     return kc, vc, int(bad)
 
 

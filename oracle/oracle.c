@@ -87,6 +87,24 @@ int64_t oracle_cache_write(const void* k, const void* v, const int64_t* slot_map
 }
 
 /*
+ * Block copy (copy-on-write of a shared block): for every pair i, block
+ * dst[i] of both pools becomes a byte copy of block src[i] (all kv heads).
+ * Pairs with an id outside the pool are skipped and counted.
+ */
+int64_t oracle_copy_blocks(void* k_cache, void* v_cache, const int32_t* src, const int32_t* dst,
+                           int64_t num_pairs, int64_t num_blocks, int64_t block_bytes) {
+    int64_t bad = 0;
+    for (int64_t i = 0; i < num_pairs; ++i) {
+        if (src[i] < 0 || src[i] >= num_blocks || dst[i] < 0 || dst[i] >= num_blocks) { ++bad; continue; }
+        memmove((char*)k_cache + (size_t)dst[i] * block_bytes, (const char*)k_cache + (size_t)src[i] * block_bytes,
+                (size_t)block_bytes);
+        memmove((char*)v_cache + (size_t)dst[i] * block_bytes, (const char*)v_cache + (size_t)src[i] * block_bytes,
+                (size_t)block_bytes);
+    }
+    return bad;
+}
+
+/*
  * Gather the first `len` tokens of kv head h of sequence s through its block
  * table into contiguous [len][D] fp64 arrays.  Logical position p sits in
  * physical block table[p / block_size] at offset p % block_size.

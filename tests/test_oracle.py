@@ -306,3 +306,20 @@ def test_single_partition_is_the_unnormalised_softmax():
     scores = [w.scale * float(h["q"][0, 0].astype(np.float64) @ h["kc"][b[t // 16], 0, t % 16].astype(np.float64))
               for t in range(30)]
     assert m[0, 0, 0] == pytest.approx(max(scores), abs=1e-14)
+
+
+# ------------------------------------------------------------------ block copy
+def test_copy_blocks_matches_numpy_indexing():
+    """dst blocks become byte copies of src blocks in both pools; others untouched;
+    pairs outside the pool are skipped."""
+    rng = np.random.default_rng(21)
+    kc = rng.integers(0, 1 << 16, size=(9, 3, 16, 8), dtype=np.uint16)
+    vc = rng.integers(0, 1 << 16, size=(9, 3, 16, 8), dtype=np.uint16)
+    src = np.array([1, 4, 7, 2], np.int32)
+    dst = np.array([0, 5, 3, 9], np.int32)  # the last pair points outside the pool
+    k2, v2, bad = oracle.copy_blocks(kc, vc, src, dst)
+    assert bad == 1
+    ek, ev = kc.copy(), vc.copy()
+    ek[dst[:3]] = kc[src[:3]]
+    ev[dst[:3]] = vc[src[:3]]
+    assert np.array_equal(k2, ek) and np.array_equal(v2, ev)
