@@ -531,6 +531,63 @@ def run_ours(args) -> None:
         dist.destroy_process_group()
 
 
+def run_copy_blocks(args) -> None:
+    """Copy-on-write block copies (pa_copy_blocks) on the workload's pool: 2048
+    pairs of distinct random blocks per step, L2 flushed between steps."""
+    from paged_kv_cache_432_b200 import build as pa_build
+    from paged_kv_cache_432_b200 import pagedattn as pa
+
+    ws, rank, local = dist_setup()
+    if rank == 0:
+        pa_build.build()
+    barrier(ws)
+    dev = torch.device("cuda", local)
+    w = wl.make(args.config, seed=replica_seed(args.seed, rank), device=dev)
+    n = min(2048, w.num_blocks // 2)
+    perm = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(args.seed + rank))
+    src = perm[:n].to(torch.int32).to(dev)
+    dst = perm[n:2 * n].to(torch.int32).to(dev)
+    block_bytes = w.k_cache[0].numel() * w.elem_bytes
+    moved = 2 * 2 * n * block_bytes  # both pools, read + write
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        pa.copy_blocks(w.k_cache, w.v_cache, src, dst, stream)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as cs:
+        for e in evs:
+            flush_w.zero_()
+            flush_r.view(torch.float32).sum()
+            e[0].record(stream)
+            pa.copy_blocks(w.k_cache, w.v_cache, src, dst, stream)
+            e[1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(ws)
+    agg = aggregate(sum(a.elapsed_time(b) for a, b in evs) / args.steps, moved, n, ws)
+    peak, peak_kind = load_peaks()
+    if pa.device_error() != 0:
+        raise RuntimeError("device error flagged")
+    line = {"metric": "copy-on-write block copy GB/s (read + write)", "value": round(agg["gbs"], 1),
+            "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(agg["step_ms"], 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "op": "pa_copy_blocks", "pairs": n, "block_bytes_per_pool": block_bytes,
+                       "l2": "flushed before every step (512 MiB write + 512 MiB read)"},
+            "roofline": {"bound": "hbm", "kernel": "copy_blocks_kernel", "achieved": round(agg["gbs"] / ws, 1),
+                         "peak": peak, "unit": "GB/s", "frac": round(agg["gbs"] / ws / peak, 4),
+                         "peak_source": peak_kind, "traffic": None},
+            "clocks": cs.summary(), "gpu_launches": args.steps}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -539,6 +596,8 @@ def main():
     ap.add_argument("--config", default="mha", choices=list(wl.CONFIGS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--op", default="step", choices=["step", "copy_blocks"],
+                    help="step: cache write + decode (the headline); copy_blocks: copy-on-write copies")
     ap.add_argument("--partition-blocks", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--plain-decode", action="store_true",
@@ -550,6 +609,8 @@ def main():
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.op == "copy_blocks":
+        run_copy_blocks(args)
     else:
         run_ours(args)
 

@@ -61,6 +61,7 @@ extern "C" {
 #define PA_ERR_WORKSPACE (-3)   /* workspace missing or too small            */
 #define PA_ERR_CUDA (-4)        /* a CUDA call or launch failed              */
 #define PA_ERR_SCRATCH_LIMIT (-5) /* pa_decode_noalloc: sizes need more than its fixed buffer */
+#define PA_ERR_OUT_OF_BLOCKS (-6) /* block manager: the pool has too few free blocks     */
 
 /* Element types (q, caches, new k/v and out share one). */
 #define PA_DTYPE_F32 0
@@ -88,6 +89,22 @@ PA_API int pa_cache_write(const void* k, const void* v, const int64_t* slot_mapp
                    int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
                    void* k_cache, void* v_cache, int32_t num_blocks,
                    int32_t block_size, int32_t dtype, void* stream);
+
+/*
+ * Block copy, the device half of copy-on-write: for every i, physical block
+ * dst[i] of both pools becomes a byte copy of block src[i] (all kv heads).
+ * A shared, partly filled block is copied before one of its sequences writes
+ * into it ("Was ändert PagedAttention an der KV-Speicherzuweisung für LLMs?",
+ * slavadubrov.com, §"Gemeinsame Nutzung erfordert mehr als
+ * Speicherzuweisung"; "PagedAttention et vLLM", aiunderstanding.org,
+ * §"Questions fréquemment posées").  src/dst are device int32 arrays; no dst
+ * may appear as another pair's src or dst in the same call (the block manager
+ * below only produces fresh destinations).  Ids outside the pool skip the pair
+ * and set PA_DEVERR_BLOCK_OOB.
+ */
+PA_API int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src, const int32_t* dst,
+                          int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t num_blocks, int32_t block_size, int32_t dtype, void* stream);
 
 /*
  * How the decode splits sequences, from partition_blocks:
@@ -216,6 +233,50 @@ PA_API size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t n
                                                      int32_t max_seq_len, int32_t shared_blocks,
                                                      int32_t block_size,
                                                      int32_t partition_blocks);
+
+/*
+ * Host-side block manager: the bookkeeping that hands out physical blocks.
+ * A sequence holds ceil(len / block_size) blocks, taken first-in first-out
+ * from a free list (initially in ascending id order) as it grows and returned
+ * when it is freed ("Was ändert PagedAttention an der KV-Speicherzuweisung
+ * für LLMs?", slavadubrov.com, §"Ungenutzten Platz in Blöcken berechnen").
+ * Forking shares every block of the parent (reference counts); appending to a
+ * sequence whose last block is shared and partly filled first replaces that
+ * block with a fresh copy, and reports the (src, dst) pair for pa_copy_blocks
+ * (copy-on-write).  Full shared blocks are never written and stay shared.
+ * Pure host code: no CUDA call, no device memory; thread-safe.
+ */
+typedef struct pa_block_manager pa_block_manager;
+
+/* NULL on bad sizes or allocation failure. */
+PA_API pa_block_manager* pa_bm_create(int32_t num_blocks, int32_t block_size,
+                                      int32_t max_blocks_per_seq);
+PA_API void pa_bm_destroy(pa_block_manager* m);
+/* A new empty sequence; PA_ERR_INVALID_ARG if the id is in use. */
+PA_API int pa_bm_add_sequence(pa_block_manager* m, int32_t seq);
+/* `child` starts as a copy of `parent`, sharing all of its blocks. */
+PA_API int pa_bm_fork(pa_block_manager* m, int32_t parent, int32_t child);
+/*
+ * Reserves num_tokens slots at the end of `seq` and writes them (block *
+ * block_size + offset, the input of pa_cache_write) to slots_out.  If the last
+ * block had to be copied first, its (src, dst) pair goes to copy_src[0] /
+ * copy_dst[0] and *num_copies = 1 (else 0); run pa_copy_blocks on it before
+ * writing the new tokens.  PA_ERR_OUT_OF_BLOCKS (nothing changed) when the
+ * free list is too short; PA_ERR_INVALID_ARG when the sequence would exceed
+ * max_blocks_per_seq.
+ */
+PA_API int pa_bm_append(pa_block_manager* m, int32_t seq, int32_t num_tokens, int64_t* slots_out,
+                        int32_t* copy_src, int32_t* copy_dst, int32_t* num_copies);
+/* Releases the sequence's blocks (those no other sequence holds go back to the free list). */
+PA_API int pa_bm_free_sequence(pa_block_manager* m, int32_t seq);
+PA_API int32_t pa_bm_num_free(pa_block_manager* m);
+PA_API int32_t pa_bm_refcount(pa_block_manager* m, int32_t block);
+/*
+ * Block tables ([num_seqs][width], unused entries -1) and lengths of the given
+ * sequences, ready to upload for pa_decode.
+ */
+PA_API int pa_bm_export_tables(pa_block_manager* m, const int32_t* seq_ids, int32_t num_seqs,
+                               int32_t* tables_out, int32_t width, int32_t* lens_out);
 
 /*
  * Reads the sticky device error word of the current device (PA_DEVERR_* bits)

@@ -3,9 +3,10 @@
     python -m paged_kv_cache_432_b200.build [--verbose-ptxas] [--force]
 
 The library is one CUDA translation unit (csrc/api.cu including the kernel
-headers), linked with the static CUDA runtime so that it loads next to any
-PyTorch build; it needs no libcuda at link time (the tensor-map encoder is
-fetched from the driver at run time).
+headers) plus the host-only block manager (csrc/block_manager.cpp), linked
+with the static CUDA runtime so that it loads next to any PyTorch build; it
+needs no libcuda at link time (the tensor-map encoder is fetched from the
+driver at run time).
 """
 from __future__ import annotations
 
@@ -34,7 +35,7 @@ def nvcc() -> str:
 
 def sources() -> list:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-                  + [os.path.join(INCLUDE, "pagedattn.h")])
+                  + glob.glob(os.path.join(CSRC, "*.cpp")) + [os.path.join(INCLUDE, "pagedattn.h")])
 
 
 def stale() -> bool:
@@ -53,7 +54,8 @@ def build(force: bool = False, verbose_ptxas: bool = False, out: str = None, def
     tmp = target + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-cudart", "static", "-I", INCLUDE, "-I", CSRC,
-           *[f"-D{d}" for d in defines], "-o", tmp, os.path.join(CSRC, "api.cu")]
+           *[f"-D{d}" for d in defines], "-o", tmp, os.path.join(CSRC, "api.cu"),
+           os.path.join(CSRC, "block_manager.cpp")]
     if verbose_ptxas:
         cmd[1:1] = ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)

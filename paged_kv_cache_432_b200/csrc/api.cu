@@ -634,6 +634,30 @@ int pa_cache_write(const void* k, const void* v, const int64_t* slot_mapping, in
     return PA_OK;
 }
 
+int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src, const int32_t* dst,
+                   int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                   int32_t block_size, int32_t dtype, void* stream) {
+    int rc = check_shapes(0, num_kv_heads, num_kv_heads, head_dim, block_size, dtype);
+    if (rc != PA_OK) return rc;
+    if (num_pairs < 0 || num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !src || !dst || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(src, 4) || !aligned(dst, 4))
+        return PA_ERR_INVALID_ARG;
+    const int32_t elem = dtype == PA_DTYPE_F32 ? 4 : 2;
+    const int64_t chunks = static_cast<int64_t>(num_kv_heads) * kBlockTokens * head_dim * elem / 16;
+    DeviceInfo di;
+    if ((rc = device_info(&di)) != PA_OK) return rc;
+    const int64_t want = (static_cast<int64_t>(num_pairs) * chunks + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(di.sms) * 8;
+    const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
+    copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), src, dst, num_pairs, chunks,
+        num_blocks);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks_kernel launch");
+}
+
 int32_t pa_decode_partition_blocks(int32_t num_seqs, int32_t num_kv_heads, int32_t max_seq_len,
                                    int32_t block_size, int32_t partition_blocks) {
     if (num_seqs < 0 || num_kv_heads <= 0 || max_seq_len < 0 || partition_blocks < -1)
@@ -832,6 +856,7 @@ const char* pa_status_string(int status) {
         case PA_ERR_UNSUPPORTED: return "unsupported dtype, head_dim, block size or group size";
         case PA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case PA_ERR_CUDA: return g_last_cuda_error;
+        case PA_ERR_OUT_OF_BLOCKS: return "the block pool has too few free blocks";
         case PA_ERR_SCRATCH_LIMIT:
             return "sizes need more split-K scratch than pa_decode_noalloc's built-in 32 MiB buffer "
                    "(use larger partitions, or pa_decode with a caller-owned workspace)";

@@ -43,4 +43,30 @@ cache_write_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
     v_cache[dst] = vv;
 }
 
+// Block copy for copy-on-write: grid-stride over (pair, 16-byte chunk) of a
+// whole physical block (all kv heads, both pools); consecutive threads move
+// consecutive chunks of one block, so both the reads and the writes are fully
+// coalesced.
+__global__ void __launch_bounds__(256)
+copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                   const int32_t* __restrict__ src, const int32_t* __restrict__ dst,
+                   int32_t num_pairs, int64_t chunks_per_block, int32_t num_blocks) {
+    const int64_t total = static_cast<int64_t>(num_pairs) * chunks_per_block;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t pair = i / chunks_per_block;
+        const int64_t c = i - pair * chunks_per_block;
+        const int32_t s = src[pair], d = dst[pair];
+        if (static_cast<uint32_t>(s) >= static_cast<uint32_t>(num_blocks) ||
+            static_cast<uint32_t>(d) >= static_cast<uint32_t>(num_blocks)) {
+            if (c == 0) flag_error(PA_DEVERR_BLOCK_OOB);
+            continue;
+        }
+        const uint4 kv = k_cache[static_cast<int64_t>(s) * chunks_per_block + c];
+        const uint4 vv = v_cache[static_cast<int64_t>(s) * chunks_per_block + c];
+        k_cache[static_cast<int64_t>(d) * chunks_per_block + c] = kv;
+        v_cache[static_cast<int64_t>(d) * chunks_per_block + c] = vv;
+    }
+}
+
 }  // namespace pa

@@ -22,6 +22,7 @@ PA_ERR_UNSUPPORTED = -2
 PA_ERR_WORKSPACE = -3
 PA_ERR_CUDA = -4
 PA_ERR_SCRATCH_LIMIT = -5
+PA_ERR_OUT_OF_BLOCKS = -6
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 PA_DTYPE_F32 = 0
@@ -48,6 +49,16 @@ SIGNATURES = {
     "pa_decode_shared_prefix": (ctypes.c_int, [_P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32,
                                                _I32, _F, _I32, _P, _SZ, _P, _I32, _P]),
     "pa_decode_shared_prefix_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32]),
+    "pa_copy_blocks": (ctypes.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P]),
+    "pa_bm_create": (_P, [_I32, _I32, _I32]),
+    "pa_bm_destroy": (None, [_P]),
+    "pa_bm_add_sequence": (ctypes.c_int, [_P, _I32]),
+    "pa_bm_fork": (ctypes.c_int, [_P, _I32, _I32]),
+    "pa_bm_append": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _P]),
+    "pa_bm_free_sequence": (ctypes.c_int, [_P, _I32]),
+    "pa_bm_num_free": (_I32, [_P]),
+    "pa_bm_refcount": (_I32, [_P, _I32]),
+    "pa_bm_export_tables": (ctypes.c_int, [_P, _P, _I32, _P, _I32, _P]),
     "pa_get_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _I32, _P]),
     "pa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -216,6 +227,61 @@ def decode_noalloc(q, k_cache, v_cache, block_tables, seq_lens, scale, out, max_
         _ptr(out), dtype_code(q.dtype), _stream(stream))
     _check("pa_decode_noalloc", rc)
     return out
+
+
+def copy_blocks(k_cache, v_cache, src, dst, stream=None) -> None:
+    """pa_copy_blocks: block dst[i] of both pools <- block src[i] (int32 device tensors)."""
+    NB, Hkv, B, D = k_cache.shape
+    rc = lib().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(src), _ptr(dst), int(src.numel()), Hkv, D,
+                              NB, B, dtype_code(k_cache.dtype), _stream(stream))
+    _check("pa_copy_blocks", rc)
+
+
+class BlockManager:
+    """The library's host-side block manager (pa_bm_*): free list, reference
+    counts, per-sequence tables; copy-on-write of shared partial blocks."""
+
+    def __init__(self, num_blocks: int, block_size: int = 16, max_blocks_per_seq: int = 1 << 20):
+        self.h = lib().pa_bm_create(num_blocks, block_size, max_blocks_per_seq)
+        if not self.h:
+            raise PagedAttnError("pa_bm_create", PA_ERR_INVALID_ARG)
+
+    def __del__(self):
+        if getattr(self, "h", None):
+            lib().pa_bm_destroy(self.h)
+            self.h = None
+
+    def add(self, seq: int):
+        _check("pa_bm_add_sequence", lib().pa_bm_add_sequence(self.h, seq))
+
+    def fork(self, parent: int, child: int):
+        _check("pa_bm_fork", lib().pa_bm_fork(self.h, parent, child))
+
+    def append(self, seq: int, n: int):
+        """-> (slots: list[int], copies: list[(src, dst)])"""
+        slots = (ctypes.c_int64 * max(n, 1))()
+        src, dst, nc = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        rc = lib().pa_bm_append(self.h, seq, n, slots, ctypes.byref(src), ctypes.byref(dst), ctypes.byref(nc))
+        _check("pa_bm_append", rc)
+        return list(slots[:n]), ([(src.value, dst.value)] if nc.value else [])
+
+    def release(self, seq: int):
+        _check("pa_bm_free_sequence", lib().pa_bm_free_sequence(self.h, seq))
+
+    def num_free(self) -> int:
+        return int(lib().pa_bm_num_free(self.h))
+
+    def refcount(self, block: int) -> int:
+        return int(lib().pa_bm_refcount(self.h, block))
+
+    def tables(self, seq_ids, width: int):
+        """-> (int32 tables [n][width] padded with -1, int32 lens [n]) as CPU tensors."""
+        ids = (ctypes.c_int32 * max(len(seq_ids), 1))(*seq_ids)
+        tab = torch.empty((len(seq_ids), width), dtype=torch.int32)
+        lens = torch.empty(len(seq_ids), dtype=torch.int32)
+        rc = lib().pa_bm_export_tables(self.h, ids, len(seq_ids), tab.data_ptr(), width, lens.data_ptr())
+        _check("pa_bm_export_tables", rc)
+        return tab, lens
 
 
 def device_error(clear: bool = True, stream=None) -> int:
