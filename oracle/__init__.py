@@ -54,6 +54,9 @@ def _load():
         lib.oracle_decode_partials.restype = ctypes.c_int
         lib.oracle_decode_partials.argtypes = [P, P, P, P, I32, P, I32, I32, I32, I32, I32, I64,
                                                I32, D, I32, I32, P, P, P, P]
+        lib.oracle_paged_decode_multi.restype = ctypes.c_int
+        lib.oracle_paged_decode_multi.argtypes = [P, P, P, P, I32, P, P, I32, I32, I32, I32, I32, I64,
+                                                  I32, D, P]
         lib.oracle_copy_blocks.restype = I64
         lib.oracle_copy_blocks.argtypes = [P, P, P, P, I64, I64, I64]
         lib.oracle_lse_merge.restype = None
@@ -173,6 +176,26 @@ def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, rows=None):
         _ptr(sel_h) if sel_h is not None else None, nsel, _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle_paged_decode failed ({rc})")
+    return out
+
+
+def paged_decode_multi(q, k_cache, v_cache, block_tables, seq_lens, q_start, scale):
+    """fp64 attention of several new query tokens per sequence (causal among
+    them).  q [rows, Hq, D] packs each sequence's query tokens (rows
+    q_start[s] .. q_start[s+1]-1), which are the sequence's last positions.
+    Returns [rows, Hq, D]."""
+    q, kc, vc, bt, sl = _decode_args(q, k_cache, v_cache, block_tables, seq_lens)
+    qs = np.ascontiguousarray(q_start, dtype=np.int32)
+    T, Hq, D = q.shape
+    NB, Hkv, B, _ = kc.shape
+    N = len(sl)
+    assert len(qs) == N + 1 and qs[-1] == T
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    rc = _load().oracle_paged_decode_multi(_ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), bt.shape[1], _ptr(sl),
+                                           _ptr(qs), N, Hq, Hkv, D, B, NB, _dtype_code(q), float(scale),
+                                           _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_paged_decode_multi failed ({rc})")
     return out
 
 

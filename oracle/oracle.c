@@ -215,6 +215,65 @@ int oracle_paged_decode(const void* q, const void* k_cache, const void* v_cache,
 }
 
 /*
+ * Several new query tokens per sequence (a speculative-decoding check, a small
+ * prefill chunk), rows packed without padding: the query tokens of sequence s
+ * are rows q_start[s] .. q_start[s+1]-1 of q / out ([rows][num_q_heads][D]).
+ * They are the sequence's last n = q_start[s+1] - q_start[s] positions, so
+ * token r (0-based) sits at position p = seq_lens[s] - n + r and attends to
+ * keys 0 .. p (causal).  Returns 0, -1 (table entry outside the pool), -2 (bad
+ * sizes, or n > seq_len).
+ */
+int oracle_paged_decode_multi(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, int32_t max_blocks,
+                              const int32_t* seq_lens, const int32_t* q_start, int32_t num_seqs,
+                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                              int32_t block_size, int64_t num_blocks, int32_t dtype, double scale,
+                              double* out) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0)
+        return -2;
+    const int32_t group = num_q_heads / num_kv_heads;
+    const int32_t D = head_dim;
+    int32_t max_len = 0;
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        const int32_t n = q_start[s + 1] - q_start[s];
+        if (seq_lens[s] < 0 || seq_lens[s] > max_blocks * block_size || n < 0 || n > seq_lens[s])
+            return -2;
+        if (seq_lens[s] > max_len) max_len = seq_lens[s];
+    }
+    double* K = (double*)malloc(sizeof(double) * ((size_t)max_len * D + 1));
+    double* V = (double*)malloc(sizeof(double) * ((size_t)max_len * D + 1));
+    double* z = (double*)malloc(sizeof(double) * ((size_t)max_len + 1));
+    double* qv = (double*)malloc(sizeof(double) * (size_t)D);
+    double* acc = (double*)malloc(sizeof(double) * (size_t)D);
+    int rc = 0;
+    for (int32_t s = 0; s < num_seqs && rc == 0; ++s) {
+        const int32_t L = seq_lens[s], n = q_start[s + 1] - q_start[s];
+        for (int32_t h = 0; h < num_kv_heads && rc == 0; ++h) {
+            if (gather_sequence(k_cache, v_cache, block_tables + (size_t)s * max_blocks, L, h,
+                                num_kv_heads, D, block_size, num_blocks, dtype, K, V)) {
+                rc = -1;
+                break;
+            }
+            for (int32_t r = 0; r < n; ++r) {
+                const int32_t pos = L - n + r;
+                const size_t qrow = (size_t)q_start[s] + r;
+                for (int32_t i = 0; i < group; ++i) {
+                    const int32_t qh = h * group + i;
+                    for (int32_t d = 0; d < D; ++d)
+                        qv[d] = load_elem(q, (qrow * num_q_heads + qh) * D + d, dtype);
+                    double M, l;
+                    attend_range(qv, K, V, 0, pos + 1, D, scale, z, &M, &l, acc);
+                    double* o = out + (qrow * num_q_heads + qh) * D;
+                    for (int32_t d = 0; d < D; ++d) o[d] = acc[d] / l;
+                }
+            }
+        }
+    }
+    free(K); free(V); free(z); free(qv); free(acc);
+    return rc;
+}
+
+/*
  * Split-K form of the same computation, used to pin the log-sum-exp merge:
  * the tokens of each sequence are cut into partitions of partition_tokens
  * consecutive logical positions; for partition p of (s, qh) it returns

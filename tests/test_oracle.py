@@ -323,3 +323,53 @@ def test_copy_blocks_matches_numpy_indexing():
     ek[dst[:3]] = kc[src[:3]]
     ev[dst[:3]] = vc[src[:3]]
     assert np.array_equal(k2, ek) and np.array_equal(v2, ev)
+
+
+# ------------------------------------------------------------------ several query tokens
+def test_multi_query_with_one_token_each_is_decode():
+    w = wl.build([35, 1, 16, 17, 90], 4, 2, 32, torch.bfloat16, seed=31)
+    h = _np_host(w)
+    qs = np.arange(w.num_seqs + 1, dtype=np.int32)
+    multi = oracle.paged_decode_multi(h["q"], h["kc"], h["vc"], h["bt"], h["sl"], qs, w.scale)
+    assert np.array_equal(multi, _decode(w))
+
+
+def test_multi_query_token_equals_decode_of_the_truncated_sequence():
+    """Query token r of n sees exactly the first L - n + r + 1 tokens."""
+    lens = [40, 17, 70]
+    nq = [3, 1, 5]
+    w = wl.build(lens, 2, 1, 32, torch.float32, seed=32)
+    h = _np_host(w)
+    rng = np.random.default_rng(0)
+    q = rng.standard_normal((sum(nq), 2, 32)).astype(np.float32)
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    multi = oracle.paged_decode_multi(q, h["kc"], h["vc"], h["bt"], h["sl"], qs, w.scale)
+    for s, (L, n) in enumerate(zip(lens, nq)):
+        for r in range(n):
+            row = qs[s] + r
+            sl = np.array([L - n + r + 1], np.int32)
+            one = oracle.paged_decode(q[row:row + 1], h["kc"], h["vc"], h["bt"][s:s + 1], sl, w.scale)
+            assert np.array_equal(multi[row], one[0])
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(2, 1), (4, 2)])
+def test_multi_query_equals_library_sdpa_with_causal_mask(Hq, Hkv):
+    """Against torch SDPA in fp64 with an explicit mask on the contiguous K/V the
+    pool was built from: new token r of n may see keys 0 .. L - n + r."""
+    lens = [35, 18, 64]
+    nq = [4, 2, 7]
+    D = 32
+    w, Ks, Vs, _, kc, vc = _truth_pool(lens, Hq, Hkv, D, seed=33)
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((sum(nq), Hq, D)).astype(np.float32)
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    out = oracle.paged_decode_multi(q, kc, vc, wl.as_numpy(w.block_tables), np.array(lens, np.int32), qs, 0.29)
+    g = Hq // Hkv
+    for s, (L, n) in enumerate(zip(lens, nq)):
+        K = torch.from_numpy(Ks[s].astype(np.float64)).permute(1, 0, 2).repeat_interleave(g, dim=0)
+        V = torch.from_numpy(Vs[s].astype(np.float64)).permute(1, 0, 2).repeat_interleave(g, dim=0)
+        Q = torch.from_numpy(q[qs[s]:qs[s + 1]].astype(np.float64)).permute(1, 0, 2)  # [Hq, n, D]
+        mask = torch.arange(L)[None, :] <= (L - n + torch.arange(n))[:, None]     # [n, L]
+        ref = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None], attn_mask=mask,
+                                                               scale=0.29)[0]
+        np.testing.assert_allclose(out[qs[s]:qs[s + 1]], ref.permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
