@@ -588,6 +588,75 @@ def run_copy_blocks(args) -> None:
         dist.destroy_process_group()
 
 
+def run_multi(args) -> None:
+    """Several query tokens per sequence (pa_decode_multi): the check step of
+    speculative decoding with q_len - 1 drafted tokens.  The KV of every
+    sequence is read once for all its query tokens."""
+    from paged_kv_cache_432_b200 import build as pa_build
+    from paged_kv_cache_432_b200 import pagedattn as pa
+
+    ws, rank, local = dist_setup()
+    if rank == 0:
+        pa_build.build()
+    barrier(ws)
+    dev = torch.device("cuda", local)
+    w = wl.make(args.config, seed=replica_seed(args.seed, rank), device=dev)
+    nq = args.q_len
+    gen = torch.Generator(device=dev).manual_seed(args.seed + 7)
+    q = torch.randn((w.num_seqs * nq, w.num_q_heads, w.head_dim), generator=gen, device=dev).to(w.dtype)
+    qs = torch.arange(0, w.num_seqs * nq + 1, nq, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    pb = w.partition_blocks if args.partition_blocks is None else args.partition_blocks
+    msl = w.max_seq_len
+    n = pa.multi_workspace_size(w.num_seqs, q.shape[0], w.num_q_heads, w.num_kv_heads, w.head_dim, msl, pb)
+    wsp = torch.empty(n, dtype=torch.uint8, device=dev) if n else None
+    by = algorithmic_bytes(w)
+    step_bytes = by["kv_unique"] + by["meta"] + 2 * q.numel() * w.elem_bytes
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        pa.decode_multi(q, qs, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, nq, out=out,
+                        max_seq_len=msl, partition_blocks=pb, workspace=wsp, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as cs:
+        for e in evs:
+            flush_w.zero_()
+            flush_r.view(torch.float32).sum()
+            e[0].record(stream)
+            step()
+            e[1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(ws)
+    agg = aggregate(sum(a.elapsed_time(b) for a, b in evs) / args.steps, step_bytes, w.num_seqs * nq, ws)
+    peak, peak_kind = load_peaks()
+    if pa.device_error() != 0:
+        raise RuntimeError("device error flagged")
+    line = {"metric": f"multi-token paged decode KV GB/s ({nq} query tokens per sequence)",
+            "value": round(agg["gbs"], 1), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(agg["step_ms"], 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(w, pa.partition_blocks(w.num_seqs, w.num_kv_heads, msl, pb)),
+                           op="pa_decode_multi", q_len=nq),
+            "query_tokens_per_s": round(agg["tokens_per_s"], 1),
+            "roofline": {"bound": "hbm", "kernel": "decode_bf16_mma_kernel + reduce", "achieved": round(agg["gbs"] / ws, 1),
+                         "peak": peak, "unit": "GB/s", "frac": round(agg["gbs"] / ws / peak, 4),
+                         "peak_source": peak_kind, "traffic": None},
+            "clocks": cs.summary(), "gpu_launches": 2 * args.steps}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -596,8 +665,10 @@ def main():
     ap.add_argument("--config", default="mha", choices=list(wl.CONFIGS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="step", choices=["step", "copy_blocks"],
-                    help="step: cache write + decode (the headline); copy_blocks: copy-on-write copies")
+    ap.add_argument("--op", default="step", choices=["step", "copy_blocks", "multi"],
+                    help="step: cache write + decode (the headline); copy_blocks: copy-on-write copies; "
+                         "multi: several query tokens per sequence")
+    ap.add_argument("--q-len", type=int, default=4, help="query tokens per sequence for --op multi")
     ap.add_argument("--partition-blocks", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--plain-decode", action="store_true",
@@ -611,6 +682,8 @@ def main():
         run_reference(args)
     elif args.op == "copy_blocks":
         run_copy_blocks(args)
+    elif args.op == "multi":
+        run_multi(args)
     else:
         run_ours(args)
 

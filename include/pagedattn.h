@@ -91,6 +91,40 @@ PA_API int pa_cache_write(const void* k, const void* v, const int64_t* slot_mapp
                    int32_t block_size, int32_t dtype, void* stream);
 
 /*
+ * Several new query tokens per sequence: the check step of speculative
+ * decoding, or a short prefill chunk ("vLLM PagedAttention: eine Revolution
+ * für den Durchsatz bei der LLM-Inferenz", de.news.hada.io, list of advanced
+ * features; "Внутреннее устройство vLLM", artificials.ru, paragraphs on
+ * chunked prefill and on speculative decoding).  The rows are packed without
+ * padding, as in the engine's super-batch (same page, super-batch paragraph):
+ * the query tokens of sequence s are rows q_start[s] .. q_start[s+1]-1
+ * (int32 [num_seqs+1], q_start[num_seqs] = num_q_rows) of q and out, both
+ * [num_q_rows][num_q_heads][head_dim].  They are the sequence's last n
+ * positions (their K/V already in the cache), so token k attends to keys
+ * 0 .. seq_lens[s] - n + k (causal among the new tokens).  Needs PA_DTYPE_BF16
+ * and group * max_q_len <= 16; a sequence with more than max_q_len or more
+ * than seq_lens[s] query tokens has the excess ignored (its rows are not
+ * written) and PA_DEVERR_SEQ_LEN set.  Workspace from
+ * pa_decode_multi_workspace_size (rows are query-token rows); other arguments
+ * as for pa_decode.  With one query token per sequence this is pa_decode.
+ */
+PA_API int pa_decode_multi(const void* q, const int32_t* q_start, int32_t num_q_rows,
+                           int32_t max_q_len, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                           int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                           int32_t num_blocks, int32_t block_size, float scale,
+                           int32_t partition_blocks, void* workspace, size_t workspace_bytes,
+                           void* out, int32_t dtype, void* stream);
+
+/* Workspace bytes pa_decode_multi needs: the pa_decode layout with
+ * num_q_rows * num_q_heads rows. */
+PA_API size_t pa_decode_multi_workspace_size(int32_t num_seqs, int32_t num_q_rows,
+                                             int32_t num_q_heads, int32_t num_kv_heads,
+                                             int32_t head_dim, int32_t max_seq_len,
+                                             int32_t block_size, int32_t partition_blocks);
+
+/*
  * Block copy, the device half of copy-on-write: for every i, physical block
  * dst[i] of both pools becomes a byte copy of block src[i] (all kv heads).
  * A shared, partly filled block is copied before one of its sequences writes

@@ -237,11 +237,12 @@ struct WsLayout {
     size_t off_m, off_l, off_acc, off_parts, bytes;
 };
 
+// q_rows: query-token rows (num_seqs with one query token per sequence).
 WsLayout ws_layout(int64_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_parts,
-                   int32_t head_dim, bool split) {
+                   int32_t head_dim, bool split, int64_t q_rows = -1) {
     WsLayout w{0, 0, 0, 0, 0};
     if (!split) return w;
-    const int64_t rows = num_seqs * num_q_heads;
+    const int64_t rows = (q_rows >= 0 ? q_rows : num_seqs) * num_q_heads;
     const size_t ml = align256(static_cast<size_t>(rows) * max_parts * sizeof(float));
     w.off_m = 0;
     w.off_l = ml;
@@ -252,6 +253,9 @@ WsLayout ws_layout(int64_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, 
 }
 
 struct DecodeArgs {
+    const int32_t* q_start = nullptr;  // several query tokens per sequence (null: one)
+    int32_t max_q_len = 1;
+    int32_t num_q_rows = -1;           // query-token rows (-1: num_seqs)
     const void* q;
     const void* k_cache;
     const void* v_cache;
@@ -315,8 +319,9 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
     } else {
         *plan = make_plan(max_len, a.partition_blocks);
     }
+    const int64_t q_rows = a.q_start ? a.num_q_rows : a.num_seqs;
     const WsLayout ws = ws_layout(a.num_seqs, a.num_q_heads, a.num_kv_heads, plan->max_parts,
-                                  a.head_dim, plan->split);
+                                  a.head_dim, plan->split, q_rows);
     std::memset(P, 0, sizeof *P);
     if (plan->split) {
         if (!a.workspace || !aligned(a.workspace, 256)) return PA_ERR_WORKSPACE;
@@ -328,6 +333,9 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
         P->ws_parts = reinterpret_cast<int32_t*>(w + ws.off_parts);
     }
     P->q = a.q;
+    P->q_start = a.q_start;
+    P->max_q_len = a.q_start ? a.max_q_len : 1;
+    P->num_q_rows = static_cast<int32_t>(q_rows);
     P->k_cache = a.k_cache;
     P->v_cache = a.v_cache;
     P->block_tables = a.block_tables;
@@ -419,8 +427,9 @@ int simt_shape(const DecodeParams& P, LaunchShape* L) {
 
 int decode_shape(const DecodeParams& P, int32_t dtype, LaunchShape* L) {
     if (dtype == PA_DTYPE_BF16) {
-        if (P.head_dim == 128) return P.group <= 8 ? mma_shape<128, 8>(P, L) : mma_shape<128, 16>(P, L);
-        return P.group <= 8 ? mma_shape<64, 8>(P, L) : mma_shape<64, 16>(P, L);
+        const int rows = P.group * P.max_q_len;
+        if (P.head_dim == 128) return rows <= 8 ? mma_shape<128, 8>(P, L) : mma_shape<128, 16>(P, L);
+        return rows <= 8 ? mma_shape<64, 8>(P, L) : mma_shape<64, 16>(P, L);
     }
     if (P.head_dim == 128) return P.group <= 4 ? simt_shape<128, 4>(P, L) : simt_shape<128, 16>(P, L);
     return P.group <= 4 ? simt_shape<64, 4>(P, L) : simt_shape<64, 16>(P, L);
@@ -472,8 +481,9 @@ int launch_simt(const DecodeParams& base, cudaStream_t st) {
 int run_partitions(const DecodeParams& P, int32_t dtype, cudaStream_t st) {
     if (P.num_seqs == 0) return PA_OK;
     if (dtype == PA_DTYPE_BF16) {
-        if (P.head_dim == 128) return P.group <= 8 ? launch_mma<128, 8>(P, st) : launch_mma<128, 16>(P, st);
-        return P.group <= 8 ? launch_mma<64, 8>(P, st) : launch_mma<64, 16>(P, st);
+        const int rows = P.group * P.max_q_len;  // query rows of one (sequence, kv head) unit
+        if (P.head_dim == 128) return rows <= 8 ? launch_mma<128, 8>(P, st) : launch_mma<128, 16>(P, st);
+        return rows <= 8 ? launch_mma<64, 8>(P, st) : launch_mma<64, 16>(P, st);
     }
     if (P.head_dim == 128) return P.group <= 4 ? launch_simt<128, 4>(P, st) : launch_simt<128, 16>(P, st);
     return P.group <= 4 ? launch_simt<64, 4>(P, st) : launch_simt<64, 16>(P, st);
@@ -540,6 +550,24 @@ int launch_prefix(const DecodeParams& P, const Plan& plan, cudaStream_t st) {
 
 template <typename OutT, int D>
 int launch_reduce(const DecodeParams& base, int32_t dtype, cudaStream_t st) {
+    if (base.q_start && !(base.balanced && base.piece_base == 0)) {
+        // row-wise merge over every query-token row at once (rows locate their
+        // sequence through q_start)
+        DecodeParams P = base;
+        P.seq_begin = 0;
+        P.seq_count = base.num_seqs;
+        const int64_t rows = static_cast<int64_t>(P.num_q_rows) * P.num_q_heads;
+        if (rows == 0) return PA_OK;
+        cudaError_t e;
+        if (P.max_parts > kWideReducePieces)
+            e = launch_pdl(lse_reduce_wide_kernel<OutT, D>, dim3(static_cast<unsigned>(rows)),
+                           dim3(kReduceWarps * 32), 0, st, P);
+        else
+            e = launch_pdl(lse_reduce_kernel<OutT, D>,
+                           dim3(static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps)),
+                           dim3(kReduceWarps * 32), 0, st, P);
+        return e == cudaSuccess ? PA_OK : cuda_fail(e, "lse_reduce_kernel launch");
+    }
     return for_each_chunk(base, [&](const DecodeParams& P) {
         cudaError_t e;
         if (P.balanced && P.piece_base == 0) {
@@ -814,6 +842,45 @@ int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_ca
     rc = run_partitions(P, dtype, a.stream);
     if (rc != PA_OK) return rc;
     return run_reduce(P, plan, dtype, a.stream);
+}
+
+int pa_decode_multi(const void* q, const int32_t* q_start, int32_t num_q_rows, int32_t max_q_len,
+                    const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                    int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t max_seq_len,
+                    int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                    int32_t num_blocks, int32_t block_size, float scale, int32_t partition_blocks,
+                    void* workspace, size_t workspace_bytes, void* out, int32_t dtype,
+                    void* stream) {
+    if (!q_start || !aligned(q_start, 4) || num_q_rows < 0 || max_q_len < 1) return PA_ERR_INVALID_ARG;
+    if (dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(num_q_heads / num_kv_heads) * max_q_len > 16) return PA_ERR_UNSUPPORTED;
+    DecodeArgs a = make_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                             max_seq_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                             block_size, scale, partition_blocks, workspace, workspace_bytes, out,
+                             dtype, stream);
+    a.q_start = q_start;
+    a.max_q_len = max_q_len;
+    a.num_q_rows = num_q_rows;
+    DecodeParams P;
+    Plan plan;
+    int rc = prepare_decode(a, true, &P, &plan);
+    if (rc != PA_OK) return rc;
+    rc = run_partitions(P, dtype, a.stream);
+    if (rc != PA_OK) return rc;
+    return run_reduce(P, plan, dtype, a.stream);
+}
+
+size_t pa_decode_multi_workspace_size(int32_t num_seqs, int32_t num_q_rows, int32_t num_q_heads,
+                                      int32_t num_kv_heads, int32_t head_dim, int32_t max_seq_len,
+                                      int32_t block_size, int32_t partition_blocks) {
+    if (num_seqs < 0 || num_q_rows < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        max_seq_len < 0 || block_size != kBlockTokens || partition_blocks < -1)
+        return 0;
+    const Plan plan = make_plan(max_seq_len, partition_blocks);
+    return ws_layout(num_seqs, num_q_heads, num_kv_heads, plan.max_parts, head_dim, plan.split,
+                     num_q_rows)
+        .bytes;
 }
 
 size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads,

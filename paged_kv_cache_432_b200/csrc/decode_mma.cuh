@@ -191,25 +191,41 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     uint32_t qa[KSTEPS][AR];  // Q as A fragments: {lo, [hi,] lo+8 cols, [hi+8 cols]}
     float m_lo = -INFINITY, l_lo = 0.f, m_hi = -INFINITY, l_hi = 0.f;
+    // this lane's two query rows in the current piece: in use?, row of q / out,
+    // last key position they may see
+    bool ok_lo = false, ok_hi = false;
+    size_t orow_lo = 0, orow_hi = 0;
+    int32_t lim_lo = 0, lim_hi = 0;
     float acc[NTD][AR];
 
     while (true) {
-        if (cj == cc.jbeg) {  // new item: load its query rows as A fragments
-            const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(P.q) +
-                                      (static_cast<size_t>(cc.s) * P.num_q_heads + cc.h * g) * D;
-            const uint32_t* q_lo = reinterpret_cast<const uint32_t*>(qg + r_lo * D + tq);
-            const uint32_t* q_hi = reinterpret_cast<const uint32_t*>(qg + (r_lo + 8) * D + tq);
-            const bool lo_ok = r_lo < g, hi_ok = HI && (r_lo + 8 < g);
+        if (cj == cc.jbeg) {  // new piece: load its query rows as A fragments
+            // Row R of the unit is (query token R / g, query head h*g + R % g);
+            // token k of n new tokens sits at position len - n + k and may
+            // see keys 0 .. len - n + k.  One token per sequence: R = head.
+            const QRows qr = query_rows(P, cc.s, cc.len);
+            if (qr.clamped && cc.p == 0 && lane == 0) flag_error(PA_DEVERR_SEQ_LEN);
+            const int rows_used = g * qr.n;
+            const int tok_lo = r_lo / g, tok_hi = (r_lo + 8) / g;
+            ok_lo = r_lo < rows_used;
+            ok_hi = HI && (r_lo + 8 < rows_used);
+            orow_lo = (static_cast<size_t>(qr.base) + tok_lo) * P.num_q_heads + cc.h * g + r_lo % g;
+            orow_hi = (static_cast<size_t>(qr.base) + tok_hi) * P.num_q_heads + cc.h * g + (r_lo + 8) % g;
+            lim_lo = cc.len - qr.n + tok_lo;
+            lim_hi = cc.len - qr.n + tok_hi;
+            const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(P.q);
+            const uint32_t* q_lo = reinterpret_cast<const uint32_t*>(qb + (ok_lo ? orow_lo : 0) * D + tq);
+            const uint32_t* q_hi = reinterpret_cast<const uint32_t*>(qb + (ok_hi ? orow_hi : 0) * D + tq);
 #pragma unroll
             for (int ks = 0; ks < KSTEPS; ++ks) {
                 if constexpr (HI) {
-                    qa[ks][0] = lo_ok ? __ldg(q_lo + ks * 8) : 0u;
-                    qa[ks][2] = lo_ok ? __ldg(q_lo + ks * 8 + 4) : 0u;
-                    qa[ks][1] = hi_ok ? __ldg(q_hi + ks * 8) : 0u;
-                    qa[ks][3] = hi_ok ? __ldg(q_hi + ks * 8 + 4) : 0u;
+                    qa[ks][0] = ok_lo ? __ldg(q_lo + ks * 8) : 0u;
+                    qa[ks][2] = ok_lo ? __ldg(q_lo + ks * 8 + 4) : 0u;
+                    qa[ks][1] = ok_hi ? __ldg(q_hi + ks * 8) : 0u;
+                    qa[ks][3] = ok_hi ? __ldg(q_hi + ks * 8 + 4) : 0u;
                 } else {
-                    qa[ks][0] = lo_ok ? __ldg(q_lo + ks * 8) : 0u;
-                    qa[ks][1] = lo_ok ? __ldg(q_lo + ks * 8 + 4) : 0u;
+                    qa[ks][0] = ok_lo ? __ldg(q_lo + ks * 8) : 0u;
+                    qa[ks][1] = ok_lo ? __ldg(q_lo + ks * 8 + 4) : 0u;
                 }
             }
             m_lo = m_hi = -INFINITY;
@@ -265,14 +281,16 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             mma_frag(s1, qa[2 * kp + 1], b2, b3);
         }
 
-        // ---- online softmax (rows r_lo and r_lo + 8)
+        // ---- online softmax (rows r_lo and r_lo + 8); key t of the block is
+        // visible to a row iff t < valid and cj*16 + t <= the row's limit
         uint32_t pa0, pa1 = 0u, pa2, pa3 = 0u;
         {
+            const int vis = min(valid - 1, lim_lo - cj * kBlockTokens);  // last visible key
             float x[4] = {s0[0], s0[1], s1[0], s1[1]};
-            x[0] = tq < valid ? x[0] * sl2 : -INFINITY;
-            x[1] = tq + 1 < valid ? x[1] * sl2 : -INFINITY;
-            x[2] = tq + 8 < valid ? x[2] * sl2 : -INFINITY;
-            x[3] = tq + 9 < valid ? x[3] * sl2 : -INFINITY;
+            x[0] = tq <= vis ? x[0] * sl2 : -INFINITY;
+            x[1] = tq + 1 <= vis ? x[1] * sl2 : -INFINITY;
+            x[2] = tq + 8 <= vis ? x[2] * sl2 : -INFINITY;
+            x[3] = tq + 9 <= vis ? x[3] * sl2 : -INFINITY;
             const float alpha = softmax_update(m_lo, l_lo, x, pa0, pa2);
 #pragma unroll
             for (int n = 0; n < NTD; ++n) {
@@ -281,11 +299,12 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
         if constexpr (HI) {
+            const int vis = min(valid - 1, lim_hi - cj * kBlockTokens);
             float x[4] = {s0[2], s0[3], s1[2], s1[3]};
-            x[0] = tq < valid ? x[0] * sl2 : -INFINITY;
-            x[1] = tq + 1 < valid ? x[1] * sl2 : -INFINITY;
-            x[2] = tq + 8 < valid ? x[2] * sl2 : -INFINITY;
-            x[3] = tq + 9 < valid ? x[3] * sl2 : -INFINITY;
+            x[0] = tq <= vis ? x[0] * sl2 : -INFINITY;
+            x[1] = tq + 1 <= vis ? x[1] * sl2 : -INFINITY;
+            x[2] = tq + 8 <= vis ? x[2] * sl2 : -INFINITY;
+            x[3] = tq + 9 <= vis ? x[3] * sl2 : -INFINITY;
             const float alpha = softmax_update(m_hi, l_hi, x, pa1, pa3);
 #pragma unroll
             for (int n = 0; n < NTD; ++n) {
@@ -331,22 +350,20 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             lt_hi = l_hi + __shfl_xor_sync(kFullMask, l_hi, 1);
             lt_hi += __shfl_xor_sync(kFullMask, lt_hi, 2);
         }
-        const int qh_lo = cc.h * g + r_lo;
         if (cc.parts == 1 && P.piece_base == 0) {
             __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(P.out);
-            if (r_lo < g) {
+            if (ok_lo) {
                 const float inv = lt_lo > 0.f ? 1.0f / lt_lo : 0.f;
-                __nv_bfloat16* o = ob + (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo) * D + tq;
+                __nv_bfloat16* o = ob + orow_lo * D + tq;
 #pragma unroll
                 for (int n = 0; n < NTD; ++n)
                     *reinterpret_cast<__nv_bfloat162*>(o + 8 * n) =
                         __floats2bfloat162_rn(acc[n][0] * inv, acc[n][1] * inv);
             }
             if constexpr (HI) {
-                if (r_lo + 8 < g) {
+                if (ok_hi) {
                     const float inv = lt_hi > 0.f ? 1.0f / lt_hi : 0.f;
-                    __nv_bfloat16* o =
-                        ob + (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo + 8) * D + tq;
+                    __nv_bfloat16* o = ob + orow_hi * D + tq;
 #pragma unroll
                     for (int n = 0; n < NTD; ++n)
                         *reinterpret_cast<__nv_bfloat162*>(o + 8 * n) =
@@ -355,8 +372,8 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         } else {
             constexpr float kLn2 = 0.693147180559945309f;
-            if (r_lo < g) {
-                const size_t idx = (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo) * P.max_parts + P.piece_base + cc.p;
+            if (ok_lo) {
+                const size_t idx = orow_lo * P.max_parts + P.piece_base + cc.p;
                 if ((lane & 3) == 0) {
                     P.ws_m[idx] = m_lo * kLn2;
                     P.ws_l[idx] = lt_lo;
@@ -367,9 +384,8 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     *reinterpret_cast<float2*>(a + 8 * n) = make_float2(acc[n][0], acc[n][1]);
             }
             if constexpr (HI) {
-                if (r_lo + 8 < g) {
-                    const size_t idx =
-                        (static_cast<size_t>(cc.s) * P.num_q_heads + qh_lo + 8) * P.max_parts + P.piece_base + cc.p;
+                if (ok_hi) {
+                    const size_t idx = orow_hi * P.max_parts + P.piece_base + cc.p;
                     if ((lane & 3) == 0) {
                         P.ws_m[idx] = m_hi * kLn2;
                         P.ws_l[idx] = lt_hi;

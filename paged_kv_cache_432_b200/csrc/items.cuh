@@ -226,9 +226,40 @@ __device__ __forceinline__ void zero_empty_sequences(const DecodeParams& P, cons
     const int row = P.num_q_heads * P.head_dim;
     for (int i = blockIdx.x; i < P.seq_count; i += gridDim.x) {
         if (lens[i] != 0) continue;
-        OutT* o = static_cast<OutT*>(P.out) + static_cast<size_t>(P.seq_begin + i) * row;
-        for (int e = threadIdx.x; e < row; e += blockDim.x) o[e] = OutT(0.0f);
+        const int32_t s = P.seq_begin + i;
+        const int32_t r0 = P.q_start ? P.q_start[s] : s;
+        const int32_t r1 = P.q_start ? P.q_start[s + 1] : s + 1;
+        OutT* o = static_cast<OutT*>(P.out) + static_cast<size_t>(r0) * row;
+        for (int64_t e = threadIdx.x; e < static_cast<int64_t>(r1 - r0) * row; e += blockDim.x)
+            o[e] = OutT(0.0f);
     }
+}
+
+// Query-token rows of sequence s: first row and count (clamped to
+// max_q_len and to the sequence length).  One row per sequence without
+// q_start.
+struct QRows {
+    int32_t base;
+    int32_t n;
+    bool clamped;  // the raw count exceeded max_q_len or the sequence length
+};
+
+__device__ __forceinline__ QRows query_rows(const DecodeParams& P, int32_t s, int32_t len) {
+    QRows q;
+    q.clamped = false;
+    if (!P.q_start) {
+        q.base = s;
+        q.n = 1;
+        return q;
+    }
+    q.base = __ldg(P.q_start + s);
+    q.n = __ldg(P.q_start + s + 1) - q.base;
+    const int32_t cap = min(P.max_q_len, len);
+    if (q.n > cap || q.n < 0) {
+        q.clamped = true;
+        q.n = q.n < 0 ? 0 : cap;
+    }
+    return q;
 }
 
 // Records how many pieces unit (s, h) has (written by the warp holding piece 0;

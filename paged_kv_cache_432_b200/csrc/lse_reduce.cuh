@@ -69,6 +69,31 @@ __device__ __forceinline__ void merge_row_warp(const DecodeParams& P, size_t bas
     for (int e = 0; e < DPL; ++e) o[lane * DPL + e] = from_float<OutT>(a[e] * inv);
 }
 
+// The (sequence, query head, query-token row) of output row `row` of a
+// launch: rows are sequence-major without q_start, token-row-major with it
+// (the sequence then found by binary search over q_start).  Returns false
+// when the row was not computed (a token beyond the clamped count).
+struct RowRef {
+    int32_t s, qh;
+    size_t r;  // output row (query token row * Hq + qh)
+};
+
+__device__ __forceinline__ bool locate_row(const DecodeParams& P, int64_t row, RowRef* R) {
+    if (!P.q_start) {
+        R->s = P.seq_begin + static_cast<int32_t>(row / P.num_q_heads);
+        R->qh = static_cast<int32_t>(row % P.num_q_heads);
+        R->r = static_cast<size_t>(R->s) * P.num_q_heads + R->qh;
+        return true;
+    }
+    const int32_t t = static_cast<int32_t>(row / P.num_q_heads);
+    R->qh = static_cast<int32_t>(row % P.num_q_heads);
+    R->s = upper_index(P.num_seqs, t, [&](int k) { return static_cast<int64_t>(__ldg(P.q_start + k)); });
+    R->r = static_cast<size_t>(row);
+    const int32_t len = seq_geometry(P, P.seq_lens[R->s]).len;
+    const QRows qr = query_rows(P, R->s, len);
+    return t - qr.base < qr.n;
+}
+
 // Row-wise merge (fixed partitions, or a shared prefix): one warp per
 // (sequence, query head) row, four rows per CTA.  The pieces of a row are
 // piece_base partials written by another kernel (a shared prefix's key
@@ -80,15 +105,15 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const Dec
     grid_dependency_wait();  // the partials of the decode launched just before
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kReduceWarps + warp;
-    if (row >= static_cast<int64_t>(P.seq_count) * P.num_q_heads) return;
-    const int32_t s = P.seq_begin + static_cast<int32_t>(row / P.num_q_heads);
-    const int32_t qh = static_cast<int32_t>(row % P.num_q_heads);
-    const SeqGeom geo = seq_geometry(P, P.seq_lens[s]);
-    const int own = geo.work > 0 ? P.ws_parts[static_cast<size_t>(s) * P.num_kv_heads + qh / P.group] : 0;
+    const int64_t rows = static_cast<int64_t>(P.q_start ? P.num_q_rows : P.seq_count) * P.num_q_heads;
+    if (row >= rows) return;
+    RowRef R;
+    if (!locate_row(P, row, &R)) return;
+    const SeqGeom geo = seq_geometry(P, P.seq_lens[R.s]);
+    const int own = geo.work > 0 ? P.ws_parts[static_cast<size_t>(R.s) * P.num_kv_heads + R.qh / P.group] : 0;
     const int parts = P.piece_base + own;
     if (P.piece_base == 0 && parts <= 1) return;
-    const size_t r = static_cast<size_t>(s) * P.num_q_heads + qh;
-    merge_row_warp<OutT, D>(P, r * P.max_parts, parts, static_cast<OutT*>(P.out) + r * D, lane);
+    merge_row_warp<OutT, D>(P, R.r * P.max_parts, parts, static_cast<OutT*>(P.out) + R.r * D, lane);
 }
 
 // Row-wise merge for rows with many pieces (long sequences in fixed
@@ -101,15 +126,14 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_wide_kernel(cons
     __shared__ float red[kReduceWarps][D];
     __shared__ float wmax[kReduceWarps], wden[kReduceWarps];
     grid_dependency_wait();
-    const int64_t row = blockIdx.x;  // (sequence within launch) * Hq + query head
-    const int32_t s = P.seq_begin + static_cast<int32_t>(row / P.num_q_heads);
-    const int32_t qh = static_cast<int32_t>(row % P.num_q_heads);
-    const SeqGeom geo = seq_geometry(P, P.seq_lens[s]);
-    const int own = geo.work > 0 ? P.ws_parts[static_cast<size_t>(s) * P.num_kv_heads + qh / P.group] : 0;
+    RowRef R;
+    if (!locate_row(P, blockIdx.x, &R)) return;
+    const SeqGeom geo = seq_geometry(P, P.seq_lens[R.s]);
+    const int own = geo.work > 0 ? P.ws_parts[static_cast<size_t>(R.s) * P.num_kv_heads + R.qh / P.group] : 0;
     const int parts = P.piece_base + own;
     if (P.piece_base == 0 && parts <= 1) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const size_t base = (static_cast<size_t>(s) * P.num_q_heads + qh) * P.max_parts;
+    const size_t base = R.r * P.max_parts;
     const float* wm = P.ws_m + base;
     const float* wl = P.ws_l + base;
     const float* wa = P.ws_acc + base * D;
@@ -119,7 +143,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_wide_kernel(cons
     if (lane == 0) wmax[warp] = M;
     __syncthreads();
     M = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
-    OutT* o = static_cast<OutT*>(P.out) + (static_cast<size_t>(s) * P.num_q_heads + qh) * D;
+    OutT* o = static_cast<OutT*>(P.out) + R.r * D;
     if (M == -INFINITY) {
         for (int d = tid; d < D; d += blockDim.x) o[d] = from_float<OutT>(0.f);
         return;
@@ -179,10 +203,11 @@ lse_reduce_balanced_kernel(const DecodeParams P, int32_t decode_warps) {
     const int64_t uend = ustart + geo.work;
     const int parts = static_cast<int>((uend - 1) / C - ustart / C + 1);
     const int32_t s = P.seq_begin + i;
+    const QRows qr = query_rows(P, s, geo.len);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int r = warp; r < P.group; r += kReduceWarps) {
-        const int32_t qh = h * P.group + r;
-        const size_t row = static_cast<size_t>(s) * P.num_q_heads + qh;
+    for (int r = warp; r < P.group * qr.n; r += kReduceWarps) {  // (query token, head) rows
+        const size_t row = (static_cast<size_t>(qr.base) + r / P.group) * P.num_q_heads +
+                           h * P.group + r % P.group;
         merge_row_warp<OutT, D>(P, row * P.max_parts, parts, static_cast<OutT*>(P.out) + row * D,
                                 lane);
     }

@@ -49,6 +49,9 @@ SIGNATURES = {
     "pa_decode_shared_prefix": (ctypes.c_int, [_P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32,
                                                _I32, _F, _I32, _P, _SZ, _P, _I32, _P]),
     "pa_decode_shared_prefix_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32]),
+    "pa_decode_multi": (ctypes.c_int, [_P, _P, _I32, _I32, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
+                                       _I32, _I32, _F, _I32, _P, _SZ, _P, _I32, _P]),
+    "pa_decode_multi_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "pa_copy_blocks": (ctypes.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P]),
     "pa_bm_create": (_P, [_I32, _I32, _I32]),
     "pa_bm_destroy": (None, [_P]),
@@ -226,6 +229,34 @@ def decode_noalloc(q, k_cache, v_cache, block_tables, seq_lens, scale, out, max_
         _ptr(seq_lens), max_seq_len, N, Hq, Hkv, D, NB, B, float(scale), partition_blocks,
         _ptr(out), dtype_code(q.dtype), _stream(stream))
     _check("pa_decode_noalloc", rc)
+    return out
+
+
+def multi_workspace_size(num_seqs, num_q_rows, num_q_heads, num_kv_heads, head_dim, max_seq_len,
+                         partition_blocks=0, block_size=16) -> int:
+    return int(lib().pa_decode_multi_workspace_size(num_seqs, num_q_rows, num_q_heads, num_kv_heads, head_dim,
+                                                    max_seq_len, block_size, partition_blocks))
+
+
+def decode_multi(q, q_start, k_cache, v_cache, block_tables, seq_lens, scale, max_q_len, out=None, max_seq_len=0,
+                 partition_blocks=0, workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode_multi: q [rows, Hq, D] packs each sequence's new query tokens
+    (rows q_start[s] .. q_start[s+1]-1); causal among them.  Returns out [rows, Hq, D]."""
+    T, Hq, D = q.shape
+    NB, Hkv, B, _ = k_cache.shape
+    N = seq_lens.numel()
+    msl = max_seq_len if max_seq_len > 0 else block_tables.shape[1] * 16
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        n = multi_workspace_size(N, T, Hq, Hkv, D, msl, partition_blocks)
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().pa_decode_multi(_ptr(q), _ptr(q_start), T, max_q_len, _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                               block_tables.shape[1], _ptr(seq_lens), max_seq_len, N, Hq, Hkv, D, NB, B,
+                               float(scale), partition_blocks, _ptr(workspace), ws_bytes, _ptr(out),
+                               dtype_code(q.dtype), _stream(stream))
+    _check("pa_decode_multi", rc)
     return out
 
 

@@ -96,6 +96,22 @@ def test_shared_prefix_workspace_size(lib):
     assert lib.pa_decode_shared_prefix_workspace_size(N, Hq, Hkv, D, 1000, 256, 16, 0) == 0
 
 
+def test_multi_query_workspace_and_limits(lib):
+    a256 = lambda x: (x + 255) // 256 * 256
+    N, T, Hq, Hkv, D, L = 4, 13, 8, 2, 128, 3000
+    P = -(-(-(-L // 16)) // 16) + 1  # balanced bound
+    rows = T * Hq
+    assert lib.pa_decode_multi_workspace_size(N, T, Hq, Hkv, D, L, 16, 0) == \
+        2 * a256(rows * P * 4) + a256(rows * P * D * 4) + a256(N * Hkv * 4)
+    # group 4 x 5 query tokens = 20 rows > 16: unsupported; fp32: unsupported
+    assert lib.pa_decode_multi(16, 16, T, 5, 16, 16, 16, 64, 16, L, N, 8, 2, D, 64, 16, 0.1, 0, None, 0, 16,
+                               pa.PA_DTYPE_BF16, None) == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_decode_multi(16, 16, T, 2, 16, 16, 16, 64, 16, L, N, 8, 2, D, 64, 16, 0.1, 0, None, 0, 16,
+                               pa.PA_DTYPE_F32, None) == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_decode_multi(16, None, T, 2, 16, 16, 16, 64, 16, L, N, 8, 2, D, 64, 16, 0.1, 0, None, 0, 16,
+                               pa.PA_DTYPE_BF16, None) == pa.PA_ERR_INVALID_ARG
+
+
 def _decode_rc(lib, **over):
     args = dict(q=16, k=16, v=16, bt=16, mb=4, sl=16, msl=64, N=2, Hq=4, Hkv=2, D=128, NB=8, B=16,
                 scale=0.1, pb=0, ws=None, wsb=0, out=16, dt=pa.PA_DTYPE_BF16)
