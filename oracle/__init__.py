@@ -57,6 +57,14 @@ def _load():
         lib.oracle_paged_decode_multi.restype = ctypes.c_int
         lib.oracle_paged_decode_multi.argtypes = [P, P, P, P, I32, P, P, I32, I32, I32, I32, I32, I64,
                                                   I32, D, P]
+        lib.oracle_e4m3_decode.restype = D
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_cache_write_fp8.restype = I64
+        lib.oracle_cache_write_fp8.argtypes = [P, P, P, I64, I32, I32, P, P, I64, I32, P, P]
+        lib.oracle_paged_decode_fp8.restype = ctypes.c_int
+        lib.oracle_paged_decode_fp8.argtypes = [P, P, P, P, I32, P, I32, I32, I32, I32, I32, I64, P, P, D, P]
         lib.oracle_copy_blocks.restype = I64
         lib.oracle_copy_blocks.argtypes = [P, P, P, P, I64, I64, I64]
         lib.oracle_lse_merge.restype = None
@@ -121,6 +129,53 @@ def cache_write(k, v, slot_mapping, k_cache, v_cache, inplace=False):
     assert (H, D) == (H2, D2)
     bad = _load().oracle_cache_write(_ptr(k), _ptr(v), _ptr(sm), T, H, D, dt, _ptr(kc), _ptr(vc), NB, B)
     return kc, vc, int(bad)
+
+
+def e4m3_decode(code: int) -> float:
+    """Value of an FP8 E4M3 code (NaN for S.1111.111)."""
+    return _load().oracle_e4m3_decode(int(code) & 0xFF)
+
+
+def e4m3_encode(y: float) -> int:
+    """Nearest E4M3 code of a float32 value (ties to even, saturating at 448)."""
+    return int(_load().oracle_e4m3_encode(float(np.float32(y))))
+
+
+def cache_write_fp8(k, v, slot_mapping, k_cache, v_cache, k_inv_scale, v_inv_scale):
+    """Quantising scatter into E4M3 caches (uint8 [NB, Hkv, B, D]); k, v bf16 bits.
+    Returns (k_cache, v_cache, n_bad) as copies."""
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    kc = np.array(k_cache, dtype=np.uint8, copy=True, order="C")
+    vc = np.array(v_cache, dtype=np.uint8, copy=True, order="C")
+    ks = np.ascontiguousarray(k_inv_scale, dtype=np.float32)
+    vs = np.ascontiguousarray(v_inv_scale, dtype=np.float32)
+    T, H, D = k.shape
+    NB, _, B, _ = kc.shape
+    bad = _load().oracle_cache_write_fp8(_ptr(k), _ptr(v), _ptr(sm), T, H, D, _ptr(kc), _ptr(vc), NB, B,
+                                         _ptr(ks), _ptr(vs))
+    return kc, vc, int(bad)
+
+
+def paged_decode_fp8(q, k_cache, v_cache, block_tables, seq_lens, k_scale, v_scale, scale):
+    """fp64 decode over E4M3 caches (value = decode(code) * scale of the kv head);
+    q as bf16 bits.  Returns [N, Hq, D]."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    kc = np.ascontiguousarray(k_cache, dtype=np.uint8)
+    vc = np.ascontiguousarray(v_cache, dtype=np.uint8)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    ks = np.ascontiguousarray(k_scale, dtype=np.float32)
+    vs = np.ascontiguousarray(v_scale, dtype=np.float32)
+    N, Hq, D = q.shape
+    NB, Hkv, B, _ = kc.shape
+    out = np.zeros((N, Hq, D), dtype=np.float64)
+    rc = _load().oracle_paged_decode_fp8(_ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), bt.shape[1], _ptr(sl), N, Hq, Hkv,
+                                         D, B, NB, _ptr(ks), _ptr(vs), float(scale), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_paged_decode_fp8 failed ({rc})")
+    return out
 
 
 def copy_blocks(k_cache, v_cache, src, dst):

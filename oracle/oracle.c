@@ -39,7 +39,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { ORACLE_F32 = 0, ORACLE_BF16 = 1 };
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2 };
 
 /* bf16 is the top half of an IEEE float32: widen the bits, exact. */
 static double bf16_bits_to_double(uint16_t bits) {
@@ -49,12 +49,85 @@ static double bf16_bits_to_double(uint16_t bits) {
     return (double)f;
 }
 
+double oracle_e4m3_decode(uint8_t c);
+
 static double load_elem(const void* base, size_t idx, int dtype) {
     if (dtype == ORACLE_F32) return (double)((const float*)base)[idx];
+    if (dtype == ORACLE_E4M3) return oracle_e4m3_decode(((const uint8_t*)base)[idx]);
     return bf16_bits_to_double(((const uint16_t*)base)[idx]);
 }
 
 static size_t elem_size(int dtype) { return dtype == ORACLE_F32 ? 4u : 2u; }
+
+/*
+ * FP8 E4M3 (the 8-bit format with 4 exponent bits of bias 7 and 3 mantissa
+ * bits; no infinities; S.1111.111 is NaN; largest finite 1.75 * 2^8 = 448;
+ * smallest normal 2^-6; subnormals m * 2^-9).  Written from that definition.
+ */
+double oracle_e4m3_decode(uint8_t c) {
+    const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Round to the nearest E4M3 value, ties to even; magnitudes above 448
+ * saturate to 448; NaN gives 0x7F. */
+uint8_t oracle_e4m3_encode(float y) {
+    if (isnan(y)) return 0x7F;
+    const uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    const double a = fabs((double)y);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);   /* a = f * 2^e with f in [0.5, 1): floor(log2 a) = e - 1 */
+    int ex = e - 1;
+    if (ex < -6) ex = -6; /* subnormal range shares the quantum of the lowest binade */
+    const double quantum = ldexp(1.0, ex - 3);
+    const double n = rint(a / quantum); /* exact division; rint rounds half to even */
+    const double m = n * quantum;
+    if (m == 0.0) return sign;
+    if (m < ldexp(1.0, -6)) return sign | (uint8_t)(m / ldexp(1.0, -9));
+    int e2;
+    frexp(m, &e2);
+    const int ex2 = e2 - 1;
+    const int mant = (int)((m / ldexp(1.0, ex2) - 1.0) * 8.0);
+    return sign | (uint8_t)(((ex2 + 7) << 3) | mant);
+}
+
+/*
+ * Cache write into an FP8 E4M3 cache: every element of the new k / v (bf16)
+ * is multiplied in fp32 by its kv head's inverse scale and rounded to E4M3
+ * (oracle_e4m3_encode).  Slots as for oracle_cache_write.
+ */
+int64_t oracle_cache_write_fp8(const uint16_t* k, const uint16_t* v, const int64_t* slot_mapping,
+                               int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                               uint8_t* k_cache, uint8_t* v_cache, int64_t num_blocks,
+                               int32_t block_size, const float* k_inv_scale,
+                               const float* v_inv_scale) {
+    int64_t bad = 0;
+    for (int64_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= num_blocks * (int64_t)block_size) { ++bad; continue; }
+        int64_t blk = slot / block_size, off = slot % block_size;
+        for (int32_t h = 0; h < num_kv_heads; ++h) {
+            size_t src = ((size_t)t * num_kv_heads + h) * head_dim;
+            size_t dst = (((size_t)blk * num_kv_heads + h) * block_size + off) * head_dim;
+            for (int32_t d = 0; d < head_dim; ++d) {
+                const float xk = (float)bf16_bits_to_double(k[src + d]);
+                const float xv = (float)bf16_bits_to_double(v[src + d]);
+                const float yk = xk * k_inv_scale[h];
+                const float yv = xv * v_inv_scale[h];
+                k_cache[dst + d] = oracle_e4m3_encode(yk);
+                v_cache[dst + d] = oracle_e4m3_encode(yv);
+            }
+        }
+    }
+    return bad;
+}
 
 /*
  * Cache write: each new token t with slot s = slot_mapping[t] >= 0 lands in
@@ -266,6 +339,63 @@ int oracle_paged_decode_multi(const void* q, const void* k_cache, const void* v_
                     double* o = out + (qrow * num_q_heads + qh) * D;
                     for (int32_t d = 0; d < D; ++d) o[d] = acc[d] / l;
                 }
+            }
+        }
+    }
+    free(K); free(V); free(z); free(qv); free(acc);
+    return rc;
+}
+
+/*
+ * Decode over an FP8 E4M3 cache: K_s[t] = decode(code) * k_scale[h] (same for
+ * V), in fp64; q is bf16.  Otherwise as oracle_paged_decode (all rows).
+ */
+int oracle_paged_decode_fp8(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                            const int32_t* block_tables, int32_t max_blocks,
+                            const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                            int64_t num_blocks, const float* k_scale, const float* v_scale,
+                            double scale, double* out) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0)
+        return -2;
+    const int32_t group = num_q_heads / num_kv_heads;
+    const int32_t D = head_dim;
+    int32_t max_len = 0;
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        if (seq_lens[s] < 0 || seq_lens[s] > max_blocks * block_size) return -2;
+        if (seq_lens[s] > max_len) max_len = seq_lens[s];
+    }
+    double* K = (double*)malloc(sizeof(double) * ((size_t)max_len * D + 1));
+    double* V = (double*)malloc(sizeof(double) * ((size_t)max_len * D + 1));
+    double* z = (double*)malloc(sizeof(double) * ((size_t)max_len + 1));
+    double* qv = (double*)malloc(sizeof(double) * (size_t)D);
+    double* acc = (double*)malloc(sizeof(double) * (size_t)D);
+    int rc = 0;
+    for (int32_t s = 0; s < num_seqs && rc == 0; ++s) {
+        const int32_t L = seq_lens[s];
+        for (int32_t h = 0; h < num_kv_heads && rc == 0; ++h) {
+            for (int32_t i = 0; i < group; ++i) {
+                double* o = out + ((size_t)s * num_q_heads + h * group + i) * D;
+                for (int32_t d = 0; d < D; ++d) o[d] = 0.0;
+            }
+            if (L == 0) continue;
+            if (gather_sequence(k_cache, v_cache, block_tables + (size_t)s * max_blocks, L, h,
+                                num_kv_heads, D, block_size, num_blocks, ORACLE_E4M3, K, V)) {
+                rc = -1;
+                break;
+            }
+            for (size_t e = 0; e < (size_t)L * D; ++e) {
+                K[e] *= (double)k_scale[h];
+                V[e] *= (double)v_scale[h];
+            }
+            for (int32_t i = 0; i < group; ++i) {
+                const int32_t qh = h * group + i;
+                for (int32_t d = 0; d < D; ++d)
+                    qv[d] = bf16_bits_to_double(q[((size_t)s * num_q_heads + qh) * D + d]);
+                double M, l;
+                attend_range(qv, K, V, 0, L, D, scale, z, &M, &l, acc);
+                double* o = out + ((size_t)s * num_q_heads + qh) * D;
+                for (int32_t d = 0; d < D; ++d) o[d] = acc[d] / l;
             }
         }
     }

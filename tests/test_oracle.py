@@ -373,3 +373,80 @@ def test_multi_query_equals_library_sdpa_with_causal_mask(Hq, Hkv):
         ref = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None], attn_mask=mask,
                                                                scale=0.29)[0]
         np.testing.assert_allclose(out[qs[s]:qs[s + 1]], ref.permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------ FP8 E4M3
+@pytest.mark.parametrize("value,code", [
+    (0.0, 0x00), (-0.0, 0x80), (1.0, 0x38), (-1.0, 0xB8), (448.0, 0x7E), (-448.0, 0xFE),
+    (2.0 ** -9, 0x01), (2.0 ** -6, 0x08), (7 * 2.0 ** -9, 0x07), (1.125, 0x39), (240.0, 0x77),
+    (2.0 ** -10, 0x00),            # half the smallest subnormal: tie, to even (zero)
+    (3 * 2.0 ** -10, 0x02),        # 1.5 quanta: tie, to even (2)
+    (1.0625, 0x38),                # halfway 1.0 / 1.125: to even (1.0)
+    (1.1875, 0x3A),                # halfway 1.125 / 1.25: to even (1.25)
+    (1.0626, 0x39),                # just above the tie
+    (500.0, 0x7E), (1e30, 0x7E), (float("inf"), 0x7E), (-1e30, 0xFE),  # saturate at 448
+])
+def test_e4m3_known_codes(value, code):
+    assert oracle.e4m3_encode(value) == code
+
+
+def test_e4m3_nan_and_round_trip_of_every_code():
+    assert oracle.e4m3_encode(float("nan")) == 0x7F
+    assert math.isnan(oracle.e4m3_decode(0x7F)) and math.isnan(oracle.e4m3_decode(0xFF))
+    values = []
+    for c in range(256):
+        if c & 0x7F == 0x7F:
+            continue
+        v = oracle.e4m3_decode(c)
+        assert oracle.e4m3_encode(v) == c          # every finite code is its own nearest value
+        values.append(v)
+    pos = sorted(set(v for v in values if v > 0))
+    assert len(pos) == 126 and pos[0] == 2.0 ** -9 and pos[-1] == 448.0
+    # between neighbours, values round to the nearer one
+    for a, b in zip(pos, pos[1:]):
+        assert oracle.e4m3_decode(oracle.e4m3_encode(a + (b - a) * 0.49)) == a
+        assert oracle.e4m3_decode(oracle.e4m3_encode(a + (b - a) * 0.51)) == b
+
+
+def test_fp8_cache_write_quantises_and_places_codes():
+    rng = np.random.default_rng(40)
+    NB, H, B, D, T = 5, 2, 16, 16, 6
+    k = torch.from_numpy(rng.standard_normal((T, H, D)).astype(np.float32)).to(torch.bfloat16)
+    v = torch.from_numpy(rng.standard_normal((T, H, D)).astype(np.float32)).to(torch.bfloat16)
+    inv = np.array([40.0, 0.5], np.float32)
+    slots = np.array([3, 17, -1, 40, 79, 0], np.int64)
+    kc0 = np.full((NB, H, B, D), 0xAA, np.uint8)
+    kc, vc, bad = oracle.cache_write_fp8(wl.as_numpy(k), wl.as_numpy(v), slots, kc0, kc0, inv, inv)
+    assert bad == 0
+    kf = k.float().numpy()
+    for t, s in enumerate(slots):
+        if s < 0:
+            continue
+        for hh in range(H):
+            want = [oracle.e4m3_encode(np.float32(x) * inv[hh]) for x in kf[t, hh]]
+            assert list(kc[s // 16, hh, s % 16]) == want
+    assert (kc[0, :, 1] == 0xAA).all()  # an untouched slot
+
+
+def test_fp8_decode_reduces_to_the_bf16_oracle_on_representable_values():
+    """Codes whose values (times a power-of-two scale) are exact in bf16 give the
+    bf16 oracle's result."""
+    w = wl.build([35, 1, 16, 70], 4, 2, 32, torch.bfloat16, seed=41)
+    rng = np.random.default_rng(41)
+    NB = w.num_blocks
+    codes_k = rng.integers(0, 256, size=(NB, 2, 16, 32)).astype(np.uint8)
+    codes_v = rng.integers(0, 256, size=(NB, 2, 16, 32)).astype(np.uint8)
+    codes_k[(codes_k & 0x7F) == 0x7F] = 0x38   # no NaN codes
+    codes_v[(codes_v & 0x7F) == 0x7F] = 0x38
+    codes_k &= 0xBF  # keep magnitudes moderate (exponent field < 8)
+    scales = np.array([0.25, 2.0], np.float32)
+    dec = np.vectorize(oracle.e4m3_decode)
+    kv = (dec(codes_k) * scales[None, :, None, None]).astype(np.float32)
+    vv = (dec(codes_v) * scales[None, :, None, None]).astype(np.float32)
+    kb = torch.from_numpy(kv).to(torch.bfloat16)
+    vb = torch.from_numpy(vv).to(torch.bfloat16)
+    assert torch.equal(kb.float(), torch.from_numpy(kv)) and torch.equal(vb.float(), torch.from_numpy(vv))
+    h = _np_host(w)
+    fp8 = oracle.paged_decode_fp8(h["q"], codes_k, codes_v, h["bt"], h["sl"], scales, scales, w.scale)
+    bf = oracle.paged_decode(h["q"], wl.as_numpy(kb), wl.as_numpy(vb), h["bt"], h["sl"], w.scale)
+    assert np.array_equal(fp8, bf)
