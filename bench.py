@@ -44,23 +44,26 @@ METRIC = "paged decode attention KV GB/s and decode tokens/s on 1 B200 vs 8 TB/s
 
 
 # ---------------------------------------------------------------- bytes accounting
-def algorithmic_bytes(w: wl.Workload) -> dict:
+def algorithmic_bytes(w: wl.Workload, kv_bytes=None) -> dict:
     """Bytes a step must move at minimum.  KV: every (distinct physical block,
-    kv head) slice attended, counted once, with the valid slots only."""
+    kv head) slice attended, counted once, with the valid slots only.
+    kv_bytes: bytes per cached element (1 for E4M3 pools; default the
+    workload's element size)."""
     e = w.elem_bytes
+    ek = e if kv_bytes is None else kv_bytes
     D, Hkv, Hq = w.head_dim, w.num_kv_heads, w.num_q_heads
     valid = {}
     for L, t in zip(w.lens_host, w.tables_host):
         for j, b in enumerate(t):
             valid[b] = max(valid.get(b, 0), min(16, L - 16 * j))
-    kv_unique = 2 * sum(valid.values()) * Hkv * D * e
-    kv_logical = 2 * sum(w.lens_host) * Hkv * D * e
+    kv_unique = 2 * sum(valid.values()) * Hkv * D * ek
+    kv_logical = 2 * sum(w.lens_host) * Hkv * D * ek
     n_blocks_read = sum(len(t) for t in w.tables_host)
     q_out = 2 * w.num_seqs * Hq * D * e
     meta = 4 * n_blocks_read + 4 * w.num_seqs
     decode = kv_unique + q_out + meta
     T = int(w.slot_mapping.numel())
-    write = 2 * (2 * T * Hkv * D * e) + 8 * T
+    write = 2 * T * Hkv * D * (e + ek) + 8 * T  # new k, v read; their slots written
     return dict(decode=decode, write=write, step=decode + write, kv_unique=kv_unique,
                 kv_logical=kv_logical, q_out=q_out, meta=meta)
 
@@ -105,10 +108,10 @@ def load_peaks() -> tuple:
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def load_traffic(workload: str):
-    """dram bytes per launch of the decode kernel from a committed ncu summary,
-    if it was taken on the current kernel sources."""
-    p = os.path.join(ROOT, "profiles", f"decode_bf16_mma_{workload}.json")
+def load_traffic(tag: str):
+    """dram bytes per launch of the decode kernel from a committed ncu summary
+    (profiles/<tag>.json), if it was taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", f"{tag}.json")
     try:
         d = json.load(open(p))
     except Exception:
@@ -331,8 +334,15 @@ def run_ours(args) -> None:
     pb = w.partition_blocks if args.partition_blocks is None else args.partition_blocks
     msl = w.max_seq_len
     resolved_pb = pa.partition_blocks(w.num_seqs, w.num_kv_heads, msl, pb)
+    fp8 = args.kv == "fp8"
+    if fp8:  # E4M3 pools with the workload's structure, per-head scales
+        if w.dtype != torch.bfloat16:
+            raise SystemExit("--kv fp8 needs a bf16 workload")
+        w.k_cache, w.v_cache, k_scale, v_scale = wl.fp8_pools(w)
+        k_inv, v_inv = (1.0 / k_scale).float(), (1.0 / v_scale).float()
+        torch.cuda.empty_cache()
     # a batch sharing a prompt prefix goes through the shared-prefix decode
-    use_sp = w.shared_prefix_blocks > 0 and not args.plain_decode
+    use_sp = w.shared_prefix_blocks > 0 and not args.plain_decode and not fp8
     if use_sp:
         n = pa.shared_prefix_workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, msl,
                                             w.shared_prefix_blocks, pb)
@@ -351,13 +361,23 @@ def run_ours(args) -> None:
         flush_w.zero_()
         flush_r.view(torch.float32).sum()  # a read-only reduction (no dtype-converting copy)
     stream = torch.cuda.current_stream(dev)
-    by = algorithmic_bytes(w)
+    by = algorithmic_bytes(w, kv_bytes=1 if fp8 else None)
     chunks = math.ceil(w.num_seqs / 2048)
     launches_per_step = 1 + chunks + (chunks if split else 0) + (1 if use_sp else 0)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
+        if fp8:  # quantising write, then decode + merge in one call
+            pa.cache_write_fp8(w.new_k, w.new_v, w.slot_mapping, w.k_cache, w.v_cache, k_inv, v_inv, stream)
+            if ev is not None:
+                ev[1].record(stream)
+            pa.decode_fp8(w.q, w.k_cache, w.v_cache, k_scale, v_scale, w.block_tables, w.seq_lens, w.scale,
+                          out=out, max_seq_len=msl, partition_blocks=pb, workspace=wsp, stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
+                ev[3].record(stream)
+            return
         pa.cache_write(w.new_k, w.new_v, w.slot_mapping, w.k_cache, w.v_cache, stream)
         if ev is not None:
             ev[1].record(stream)
@@ -449,6 +469,14 @@ def run_ours(args) -> None:
 
         def e2e_step():
             dev_buf.copy_(host_buf, non_blocking=True)
+            if fp8:
+                pa.cache_write_fp8(dev_in["new_k"], dev_in["new_v"], dev_in["slot_mapping"], w.k_cache, w.v_cache,
+                                   k_inv, v_inv, stream)
+                pa.decode_fp8(dev_in["q"], w.k_cache, w.v_cache, k_scale, v_scale, dev_in["block_tables"],
+                              dev_in["seq_lens"], w.scale, out=out, max_seq_len=msl, partition_blocks=pb,
+                              workspace=wsp, stream=stream)
+                host_out.copy_(out, non_blocking=True)
+                return
             pa.cache_write(dev_in["new_k"], dev_in["new_v"], dev_in["slot_mapping"], w.k_cache, w.v_cache, stream)
             if use_sp:
                 pa.decode_shared_prefix(dev_in["q"], w.k_cache, w.v_cache, dev_in["block_tables"],
@@ -486,15 +514,17 @@ def run_ours(args) -> None:
     kname = "decode_bf16_mma_kernel" if w.dtype == torch.bfloat16 else "decode_f32_simt_kernel"
     if use_sp:
         kname = "pa_decode_shared_prefix (prefix kernel + decode_bf16_mma_kernel + reduce, timed together)"
+    if fp8:
+        kname = "pa_decode_fp8 (decode_bf16_mma_kernel<E4M3> + reduce, timed together)"
     roof = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1), "peak": peak,
             "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
             else "fallback 6650 GB/s", "unit": "GB/s", "frac": round(achieved / peak, 4),
             "frac_of_8TBs": round(achieved / 8000.0, 4),
             "algorithmic_bytes_per_launch": by["decode"],
-            "traffic": load_traffic(w.name)}
+            "traffic": load_traffic(f"decode_{'fp8' if fp8 else 'bf16'}_mma_{w.name}")}
 
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and not fp8:
         cpu = cpu_baseline(w, budget_s=args.cpu_budget_s)
 
     line = {
@@ -508,9 +538,10 @@ def run_ours(args) -> None:
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+        "dtype": ("e4m3 KV, f16 MMA" if fp8 else "bf16") if w.dtype == torch.bfloat16 else "f32",
         "data": "synthetic",
-        "config": workload_config(w, resolved_pb),
+        "config": dict(workload_config(w, resolved_pb), kv="e4m3 codes, per-head fp32 scales" if fp8 else
+                       ("bf16" if w.dtype == torch.bfloat16 else "f32")),
         "tokens_per_s": round(total_seqs / (step_ms * 1e-3), 1),
         "kernel_ms": {"cache_write": round(wr_ms, 5), "decode_partitions": round(dec_ms, 5),
                       "lse_reduce": round(red_ms, 5),
@@ -669,6 +700,8 @@ def main():
                     help="step: cache write + decode (the headline); copy_blocks: copy-on-write copies; "
                          "multi: several query tokens per sequence")
     ap.add_argument("--q-len", type=int, default=4, help="query tokens per sequence for --op multi")
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
+                    help="KV pool element type for --op step (fp8: E4M3 codes with per-head scales)")
     ap.add_argument("--partition-blocks", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--plain-decode", action="store_true",

@@ -91,6 +91,54 @@ PA_API int pa_cache_write(const void* k, const void* v, const int64_t* slot_mapp
                    int32_t block_size, int32_t dtype, void* stream);
 
 /*
+ * FP8 KV cache, quantising cache write.  The caches hold one byte per element,
+ * an FP8 E4M3 code (sign, 4 exponent bits of bias 7, 3 mantissa bits; largest
+ * finite 448; S.1111.111 is NaN), with one scale per kv head and pool, so a
+ * token costs half the bytes of a bf16 cache (cache quantisation as a remedy
+ * when the KV data do not fit: "Was ändert PagedAttention an der
+ * KV-Speicherzuweisung für LLMs?", slavadubrov.com, §"Gemeinsame Nutzung
+ * erfordert mehr als Speicherzuweisung", last paragraph).  Layout as for
+ * pa_cache_write with uint8 elements: k_cache[num_blocks][num_kv_heads][16][head_dim].
+ * For every token t with slot s = slot_mapping[t] >= 0, kv head h and d:
+ *   k_cache[s / 16][h][s % 16][d] = E4M3(float(k[t][h][d]) * k_inv_scale[h])
+ * (same for v), where the product is one fp32 multiply rounded to nearest and
+ * E4M3() rounds to the nearest code, ties to even, saturates magnitudes above
+ * 448 to +-448 (infinities too) and gives 0x7F for NaN.  k and v are bf16
+ * [num_tokens][num_kv_heads][head_dim]; k_inv_scale and v_inv_scale are fp32
+ * device arrays [num_kv_heads] (the inverses of the scales pa_decode_fp8 takes).
+ * Slots: as pa_cache_write (< 0 skipped, beyond the pool skipped with
+ * PA_DEVERR_SLOT_OOB).  block_size 16; head_dim 64 or 128.  Pointers 16-byte
+ * aligned (scales 4-byte).  Errors: PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED as
+ * pa_cache_write; nothing is launched then.
+ */
+PA_API int pa_cache_write_fp8(const void* k, const void* v, const int64_t* slot_mapping,
+                              int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                              void* k_cache, void* v_cache, int32_t num_blocks,
+                              int32_t block_size, const float* k_inv_scale,
+                              const float* v_inv_scale, void* stream);
+
+/*
+ * Paged decode attention over FP8 E4M3 caches (written by pa_cache_write_fp8):
+ * as pa_decode with dtype BF16 (q and out bf16), where
+ *   K_s[t] = decode(k_cache[block_tables[s][t / 16]][h][t % 16]) * k_scale[h]
+ * (same for V with v_scale), decode() being the exact value of the code.
+ * The kernel widens the codes to f16 (exact), computes q . code and P . code
+ * on tensor cores (f16 in, fp32 accumulate; q rounded to f16, exact for bf16
+ * values of magnitude 2^-14 .. 65504), and applies the scales in fp32.
+ * k_scale and v_scale are fp32 device arrays [num_kv_heads].  Workspace: the
+ * size pa_decode_workspace_size gives for the same arguments.  Same errors
+ * and device error bits as pa_decode; null scales give PA_ERR_INVALID_ARG.
+ */
+PA_API int pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
+                         const float* k_scale, const float* v_scale,
+                         const int32_t* block_tables, int32_t max_blocks_per_seq,
+                         const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                         int32_t num_blocks, int32_t block_size, float scale,
+                         int32_t partition_blocks, void* workspace, size_t workspace_bytes,
+                         void* out, void* stream);
+
+/*
  * Several new query tokens per sequence: the check step of speculative
  * decoding, or a short prefill chunk ("vLLM PagedAttention: eine Revolution
  * für den Durchsatz bei der LLM-Inferenz", de.news.hada.io, list of advanced

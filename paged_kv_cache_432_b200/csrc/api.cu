@@ -45,9 +45,20 @@ constexpr int kMaxDevices = 64;
 #ifndef PA_MMA_MIN_CTAS
 #define PA_MMA_MIN_CTAS 2
 #endif
+// E4M3 stages are half the bytes: twice as many keep the same bytes in flight
+#ifndef PA_MMA_STAGES_FP8
+#define PA_MMA_STAGES_FP8 4
+#endif
+#ifndef PA_MMA_MIN_CTAS_FP8
+#define PA_MMA_MIN_CTAS_FP8 2
+#endif
 constexpr int kMmaWarps = PA_MMA_WARPS;
 constexpr int kMmaStages = PA_MMA_STAGES;
 constexpr int kMmaMinCtas = PA_MMA_MIN_CTAS;  // CTAs per SM the register budget must allow
+template <bool FP8>
+constexpr int mma_stages() { return FP8 ? PA_MMA_STAGES_FP8 : kMmaStages; }
+template <bool FP8>
+constexpr int mma_min_ctas() { return FP8 ? PA_MMA_MIN_CTAS_FP8 : kMmaMinCtas; }
 
 thread_local char g_last_cuda_error[256] = "no CUDA error recorded";
 
@@ -143,18 +154,23 @@ int get_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
     return PA_OK;
 }
 
-// The pool seen as a 2-D bf16 tensor [num_blocks*Hkv*16 rows][head_dim],
-// loaded in 64-column x 16-row boxes with the 128-byte swizzle.
-int encode_pool_map(CUtensorMap* map, const void* base, int64_t rows, int head_dim) {
+// The pool seen as a 2-D tensor [num_blocks*Hkv*16 rows][head_dim].  bf16:
+// loaded in 64-column x 16-row boxes with the 128-byte swizzle.  E4M3 (fp8):
+// one box of 16 rows x head_dim bytes, with the 128-byte swizzle (64-byte at
+// head_dim 64, where a row is 64 bytes).
+int encode_pool_map(CUtensorMap* map, const void* base, int64_t rows, int head_dim,
+                    bool fp8 = false) {
     PFN_cuTensorMapEncodeTiled_v12000 enc;
     int rc = get_encoder(&enc);
     if (rc != PA_OK) return rc;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
-    cuuint32_t box[2] = {64, 16};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * (fp8 ? 1 : 2)};
+    cuuint32_t box[2] = {fp8 ? static_cast<cuuint32_t>(head_dim) : 64u, 16};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     (fp8 && head_dim == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
@@ -253,6 +269,8 @@ WsLayout ws_layout(int64_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, 
 }
 
 struct DecodeArgs {
+    const float* k_scale = nullptr;    // E4M3 caches: per-kv-head scales (null: bf16/f32 caches)
+    const float* v_scale = nullptr;
     const int32_t* q_start = nullptr;  // several query tokens per sequence (null: one)
     int32_t max_q_len = 1;
     int32_t num_q_rows = -1;           // query-token rows (-1: num_seqs)
@@ -305,6 +323,11 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
             return PA_ERR_UNSUPPORTED;
         if (!std::isfinite(a.scale)) return PA_ERR_INVALID_ARG;
     }
+    if (a.k_scale || a.v_scale) {  // E4M3 caches: bf16 queries and output
+        if (a.dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
+        if (!a.k_scale || !a.v_scale || !aligned(a.k_scale, 4) || !aligned(a.v_scale, 4))
+            return PA_ERR_INVALID_ARG;
+    }
     const int64_t table_tokens = static_cast<int64_t>(a.max_blocks_per_seq) * kBlockTokens;
     const int32_t max_len = a.max_seq_len > 0
                                 ? a.max_seq_len
@@ -338,6 +361,8 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
     P->num_q_rows = static_cast<int32_t>(q_rows);
     P->k_cache = a.k_cache;
     P->v_cache = a.v_cache;
+    P->k_scale = a.k_scale;
+    P->v_scale = a.v_scale;
     P->block_tables = a.block_tables;
     P->seq_lens = a.seq_lens;
     P->out = a.out;
@@ -397,9 +422,9 @@ struct LaunchShape {
     size_t smem;
 };
 
-template <int D, int ROWS>
+template <int D, int ROWS, bool FP8>
 auto mma_kernel() {
-    return decode_bf16_mma_kernel<D, ROWS, kMmaStages, kMmaWarps, kMmaMinCtas>;
+    return decode_bf16_mma_kernel<D, ROWS, mma_stages<FP8>(), kMmaWarps, mma_min_ctas<FP8>(), FP8>;
 }
 
 template <typename K>
@@ -410,10 +435,10 @@ int shape_of(K kernel, int warps, size_t smem, const DecodeParams& P, LaunchShap
     return persistent_grid(kernel, L->threads, smem, (max_pieces + warps - 1) / warps, &L->grid);
 }
 
-template <int D, int ROWS>
+template <int D, int ROWS, bool FP8>
 int mma_shape(const DecodeParams& P, LaunchShape* L) {
-    using Cfg = MmaCfg<D, kMmaStages, kMmaWarps>;
-    auto kernel = mma_kernel<D, ROWS>();
+    using Cfg = MmaCfg<D, mma_stages<FP8>(), kMmaWarps, FP8>;
+    auto kernel = mma_kernel<D, ROWS, FP8>();
     int rc = ensure_smem_attr(kernel, Cfg::smem_bytes(kMaxSeqsPerLaunch));
     if (rc != PA_OK) return rc;
     return shape_of(kernel, kMmaWarps, Cfg::smem_bytes(P.seq_count), P, L);
@@ -425,12 +450,17 @@ int simt_shape(const DecodeParams& P, LaunchShape* L) {
                     P, L);
 }
 
+template <bool FP8>
+int mma_shape_for(const DecodeParams& P, LaunchShape* L) {
+    const int rows = P.group * P.max_q_len;
+    if (P.head_dim == 128)
+        return rows <= 8 ? mma_shape<128, 8, FP8>(P, L) : mma_shape<128, 16, FP8>(P, L);
+    return rows <= 8 ? mma_shape<64, 8, FP8>(P, L) : mma_shape<64, 16, FP8>(P, L);
+}
+
 int decode_shape(const DecodeParams& P, int32_t dtype, LaunchShape* L) {
-    if (dtype == PA_DTYPE_BF16) {
-        const int rows = P.group * P.max_q_len;
-        if (P.head_dim == 128) return rows <= 8 ? mma_shape<128, 8>(P, L) : mma_shape<128, 16>(P, L);
-        return rows <= 8 ? mma_shape<64, 8>(P, L) : mma_shape<64, 16>(P, L);
-    }
+    if (dtype == PA_DTYPE_BF16)
+        return P.k_scale ? mma_shape_for<true>(P, L) : mma_shape_for<false>(P, L);
     if (P.head_dim == 128) return P.group <= 4 ? simt_shape<128, 4>(P, L) : simt_shape<128, 16>(P, L);
     return P.group <= 4 ? simt_shape<64, 4>(P, L) : simt_shape<64, 16>(P, L);
 }
@@ -449,19 +479,19 @@ int for_each_chunk(const DecodeParams& base, F fn) {
     return PA_OK;
 }
 
-template <int D, int ROWS>
+template <int D, int ROWS, bool FP8>
 int launch_mma(const DecodeParams& base, cudaStream_t st) {
     const int64_t rows = static_cast<int64_t>(base.num_blocks) * base.num_kv_heads * kBlockTokens;
     alignas(64) CUtensorMap mk, mv;
     int rc;
-    if ((rc = encode_pool_map(&mk, base.k_cache, rows, D)) != PA_OK) return rc;
-    if ((rc = encode_pool_map(&mv, base.v_cache, rows, D)) != PA_OK) return rc;
+    if ((rc = encode_pool_map(&mk, base.k_cache, rows, D, FP8)) != PA_OK) return rc;
+    if ((rc = encode_pool_map(&mv, base.v_cache, rows, D, FP8)) != PA_OK) return rc;
     return for_each_chunk(base, [&](const DecodeParams& P) {
         LaunchShape L;
-        int r = mma_shape<D, ROWS>(P, &L);
+        int r = mma_shape<D, ROWS, FP8>(P, &L);
         if (r != PA_OK) return r;
-        cudaError_t e = launch_pdl(mma_kernel<D, ROWS>(), dim3(L.grid), dim3(L.threads), L.smem, st,
-                                   mk, mv, P);
+        cudaError_t e = launch_pdl(mma_kernel<D, ROWS, FP8>(), dim3(L.grid), dim3(L.threads), L.smem,
+                                   st, mk, mv, P);
         return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode_bf16_mma_kernel launch");
     });
 }
@@ -478,13 +508,18 @@ int launch_simt(const DecodeParams& base, cudaStream_t st) {
     });
 }
 
+template <bool FP8>
+int launch_mma_for(const DecodeParams& P, cudaStream_t st) {
+    const int rows = P.group * P.max_q_len;  // query rows of one (sequence, kv head) unit
+    if (P.head_dim == 128)
+        return rows <= 8 ? launch_mma<128, 8, FP8>(P, st) : launch_mma<128, 16, FP8>(P, st);
+    return rows <= 8 ? launch_mma<64, 8, FP8>(P, st) : launch_mma<64, 16, FP8>(P, st);
+}
+
 int run_partitions(const DecodeParams& P, int32_t dtype, cudaStream_t st) {
     if (P.num_seqs == 0) return PA_OK;
-    if (dtype == PA_DTYPE_BF16) {
-        const int rows = P.group * P.max_q_len;  // query rows of one (sequence, kv head) unit
-        if (P.head_dim == 128) return rows <= 8 ? launch_mma<128, 8>(P, st) : launch_mma<128, 16>(P, st);
-        return rows <= 8 ? launch_mma<64, 8>(P, st) : launch_mma<64, 16>(P, st);
-    }
+    if (dtype == PA_DTYPE_BF16)
+        return P.k_scale ? launch_mma_for<true>(P, st) : launch_mma_for<false>(P, st);
     if (P.head_dim == 128) return P.group <= 4 ? launch_simt<128, 4>(P, st) : launch_simt<128, 16>(P, st);
     return P.group <= 4 ? launch_simt<64, 4>(P, st) : launch_simt<64, 16>(P, st);
 }
@@ -662,6 +697,31 @@ int pa_cache_write(const void* k, const void* v, const int64_t* slot_mapping, in
     return PA_OK;
 }
 
+int pa_cache_write_fp8(const void* k, const void* v, const int64_t* slot_mapping,
+                       int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim, void* k_cache,
+                       void* v_cache, int32_t num_blocks, int32_t block_size,
+                       const float* k_inv_scale, const float* v_inv_scale, void* stream) {
+    int rc = check_shapes(0, num_kv_heads, num_kv_heads, head_dim, block_size, PA_DTYPE_BF16);
+    if (rc != PA_OK) return rc;
+    if (num_tokens < 0 || num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache || !k_inv_scale || !v_inv_scale)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(slot_mapping, 8) || !aligned(k_inv_scale, 4) || !aligned(v_inv_scale, 4))
+        return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    const int32_t chunks_per_row = head_dim / 16;  // 16 values per thread
+    const int64_t total = static_cast<int64_t>(num_tokens) * num_kv_heads * chunks_per_row;
+    const int64_t grid = (total + 255) / 256;
+    if (grid > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    cache_write_fp8_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, total,
+        num_kv_heads, chunks_per_row, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+        static_cast<int64_t>(num_blocks) * kBlockTokens, k_inv_scale, v_inv_scale);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "cache_write_fp8_kernel launch");
+}
+
 int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src, const int32_t* dst,
                    int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
                    int32_t block_size, int32_t dtype, void* stream) {
@@ -755,6 +815,28 @@ int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int
     rc = run_partitions(P, dtype, a.stream);
     if (rc != PA_OK) return rc;
     return run_reduce(P, plan, dtype, a.stream);
+}
+
+int pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                  const float* v_scale, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                  const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                  int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                  int32_t block_size, float scale, int32_t partition_blocks, void* workspace,
+                  size_t workspace_bytes, void* out, void* stream) {
+    if (!k_scale || !v_scale) return PA_ERR_INVALID_ARG;
+    DecodeArgs a = make_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                             max_seq_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                             block_size, scale, partition_blocks, workspace, workspace_bytes, out,
+                             PA_DTYPE_BF16, stream);
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    DecodeParams P;
+    Plan plan;
+    int rc = prepare_decode(a, true, &P, &plan);
+    if (rc != PA_OK) return rc;
+    rc = run_partitions(P, PA_DTYPE_BF16, a.stream);
+    if (rc != PA_OK) return rc;
+    return run_reduce(P, plan, PA_DTYPE_BF16, a.stream);
 }
 
 // ------------------------------------------------------------ no-allocation decode

@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -33,6 +34,8 @@ struct DecodeParams {
     const void* v_cache;
     const int32_t* block_tables;
     const int32_t* seq_lens;
+    const float* k_scale;  // E4M3 caches: dequantisation scale per kv head (else null)
+    const float* v_scale;
     void* out;
     float* ws_m;    // [num_seqs*num_q_heads][max_parts]        (null: no split)
     float* ws_l;    // [num_seqs*num_q_heads][max_parts]
@@ -208,6 +211,111 @@ __device__ __forceinline__ void mma_frag(float (&d)[4], const uint32_t (&a)[4], 
 __device__ __forceinline__ void mma_frag(float (&d)[2], const uint32_t (&a)[2], uint32_t b0,
                                          uint32_t b1) {
     mma_bf16_rows8(d, a[0], a[1], b0, b1);
+}
+
+// f16 inputs (the FP8 path widens E4M3 to f16, which is exact).
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16_rows8(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0,
+                                              uint32_t b1) {
+    float z2, z3;
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(z2), "=f"(z3)
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(0.f),
+          "f"(0.f));
+    (void)z2;
+    (void)z3;
+}
+
+template <bool F16>
+__device__ __forceinline__ void mma_frag_t(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                           uint32_t b1) {
+    if constexpr (F16) mma_f16(d, a[0], a[1], a[2], a[3], b0, b1);
+    else mma_bf16(d, a[0], a[1], a[2], a[3], b0, b1);
+}
+template <bool F16>
+__device__ __forceinline__ void mma_frag_t(float (&d)[2], const uint32_t (&a)[2], uint32_t b0,
+                                           uint32_t b1) {
+    if constexpr (F16) mma_f16_rows8(d, a[0], a[1], b0, b1);
+    else mma_bf16_rows8(d, a[0], a[1], b0, b1);
+}
+
+// Two fp32 values to a packed pair (lo in the low half) of bf16 or f16.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    if constexpr (F16) {
+        __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&h);
+    } else {
+        __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&b);
+    }
+}
+template <bool F16>
+__device__ __forceinline__ float2 unpack2(uint32_t u) {
+    if constexpr (F16) return __half22float2(*reinterpret_cast<__half2*>(&u));
+    else return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+}
+
+// E4M3 pair (low byte = first value) -> f16 pair; exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+    return r;
+}
+
+// Four E4M3 codes (bytes 0..3 of x) -> two f16 pairs: lo = (byte 0, byte 1),
+// hi = (byte 2, byte 3), first value in the low half; exact.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(x));
+}
+
+// 2^x with the hardware approximation (relative error about 2^-22; -inf
+// gives 0, results below 2^-126 flush to 0).  The softmax weights it feeds
+// are rounded to 16-bit floats right after.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Byte i of the result is byte (sel >> 4i) & 7 of {x (bytes 0..3), x (4..7)}.
+__device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %1, %2;" : "=r"(r) : "r"(x), "r"(sel));
+    return r;
+}
+
+// A bf16 pair -> an f16 pair (round to nearest; exact for magnitudes in
+// 2^-14 .. 65504).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
+    const float2 f = unpack2<false>(u);
+    return pack2<true>(f.x, f.y);
+}
+
+// Two fp32 values to an E4M3 pair (first value in the low byte), rounding to
+// nearest even and saturating at +-448.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float first, float second) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(second), "f"(first));
+    return r;
+}
+
+// Four packed E4M3 codes with every NaN (S.1111.111) made the one NaN code
+// 0x7F, whatever its sign.
+__device__ __forceinline__ uint32_t e4m3x4_canonical_nan(uint32_t w) {
+    const uint32_t nan = __vcmpeq4(w & 0x7f7f7f7fu, 0x7f7f7f7fu);  // 0xff in each NaN byte
+    return (w & ~nan) | (0x7f7f7f7fu & nan);
 }
 
 __device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) {

@@ -1,4 +1,4 @@
-// decode_mma.cuh -- paged decode attention, bf16, one warp per work item.
+// decode_mma.cuh -- paged decode attention, bf16 or E4M3 caches, one warp per work item.
 //
 // Decoding reads the whole KV cache once per step and does little arithmetic
 // per byte: it is bound by memory bandwidth ("vLLM PagedAttention: eine
@@ -37,6 +37,19 @@
 //    (acc / l, rounded to bf16) when the sequence has one partition, or the
 //    partition's (m, l, acc) to the workspace for the log-sum-exp reduction.
 //
+// E4M3 (fp8) caches (FP8 = true): a stage holds the 8-bit codes of the K and
+// V tile, one TMA box each (16 rows x D bytes, 128-byte swizzle).  The codes
+// go from shared memory straight into MMA fragments: ldmatrix on the codes
+// seen as 16-bit pairs, then cvt.f16x2.e4m3x2 (exact), and the MMAs run in
+// f16.  For K, a lane receives 4 consecutive dims of one token; the k index of
+// Q K^T is permuted to match (the Q fragments take the same dims), which
+// changes nothing in the sum.  For V, ldmatrix.trans gives each lane two
+// tokens of a dim pair; one byte permute splits that into the even and the
+// odd dim's token pair, so the P V n-tiles hold the even and the odd dims of
+// each 16-dim chunk.  The kv head's K scale is folded into the score scale
+// and its V scale multiplies the accumulators once at the end of the piece,
+// so the result is that of attention over decode(code) * scale.
+//
 // Every wait on an mbarrier is bounded: on timeout the warp flags
 // PA_DEVERR_TIMEOUT, waits (bounded) for its copies in flight and returns.
 #pragma once
@@ -45,10 +58,14 @@
 
 namespace pa {
 
-template <int D, int STAGES, int WARPS>
+template <int D, int STAGES, int WARPS, bool FP8 = false>
 struct MmaCfg {
-    static constexpr int kRegions = D / 64;            // 64-element (128 B) column slabs
-    static constexpr int kRegionBytes = 16 * 128;      // 16 token rows x 128 B
+    // bf16 tiles: D/64 column slabs of 16 rows x 128 B (64 values), one TMA
+    // box each.  E4M3 tiles: one box of 16 rows x D bytes.  Both with the
+    // 128-byte swizzle (64-byte for E4M3 at D = 64).
+    static constexpr int kRegions = FP8 ? 1 : D / 64;
+    static constexpr int kRowBytes = FP8 ? D : 128;
+    static constexpr int kRegionBytes = 16 * kRowBytes;
     static constexpr int kTileBytes = kRegions * kRegionBytes;  // K (or V) of one block, one head
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kRingBytes = WARPS * STAGES * kStageBytes;
@@ -57,40 +74,58 @@ struct MmaCfg {
     static size_t smem_bytes(int seq_count) {
         return 1024 + kRingBytes + kBarBytes + 8 * static_cast<size_t>(seq_count + 1);
     }
+    // 16-byte chunk c of row t sits at chunk c ^ swz(t) (the TMA swizzle pattern)
+    static __device__ __forceinline__ uint32_t swz(int t) {
+        return (FP8 && D == 64) ? static_cast<uint32_t>((t >> 1) & 3) : static_cast<uint32_t>(t & 7);
+    }
 };
 
-// Online-softmax update of one row set: x[] are four raw scores (tokens
-// tq, tq+1, 8+tq, 9+tq), already masked to -inf where invalid and scaled to
-// log2 units.  Returns the rescale factor for the accumulators and packs the
-// probabilities as bf16 pairs (lo: tokens tq..tq+1, hi: tokens 8+tq..9+tq).
-__device__ __forceinline__ float softmax_update(float& m, float& l, const float (&x)[4],
-                                                uint32_t& p_lo, uint32_t& p_hi) {
-    float bm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+// Online-softmax update of one row set over NB blocks: x[4b..4b+3] are four
+// raw scores of block b (tokens tq, tq+1, 8+tq, 9+tq), already masked to -inf
+// where invalid and scaled to log2 units.  Returns the rescale factor for the
+// accumulators and packs the probabilities as bf16 (or f16) pairs: p[b][0]
+// tokens tq..tq+1, p[b][1] tokens 8+tq..9+tq of block b.
+template <bool F16, int NB>
+__device__ __forceinline__ float softmax_update(float& m, float& l, const float (&x)[4 * NB],
+                                                uint32_t (&p)[NB][2]) {
+    float bm = x[0];
+#pragma unroll
+    for (int i = 1; i < 4 * NB; ++i) bm = fmaxf(bm, x[i]);
     bm = fmaxf(bm, __shfl_xor_sync(kFullMask, bm, 1));
     bm = fmaxf(bm, __shfl_xor_sync(kFullMask, bm, 2));
     const float mn = fmaxf(m, bm);
     const float mu = mn == -INFINITY ? 0.0f : mn;  // a row with nothing valid yet
-    const float alpha = exp2f(m - mu);
-    const __nv_bfloat162 a = __floats2bfloat162_rn(exp2f(x[0] - mu), exp2f(x[1] - mu));
-    const __nv_bfloat162 b = __floats2bfloat162_rn(exp2f(x[2] - mu), exp2f(x[3] - mu));
-    // the denominator sums the same (rounded) weights the numerator uses
-    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
-    l = l * alpha + ((fa.x + fa.y) + (fb.x + fb.y));
+    const float alpha = fast_exp2(m - mu);
+    float sum = 0.f;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        p[b][0] = pack2<F16>(fast_exp2(x[4 * b] - mu), fast_exp2(x[4 * b + 1] - mu));
+        p[b][1] = pack2<F16>(fast_exp2(x[4 * b + 2] - mu), fast_exp2(x[4 * b + 3] - mu));
+        // the denominator sums the same (rounded) weights the numerator uses
+        const float2 fa = unpack2<F16>(p[b][0]), fb = unpack2<F16>(p[b][1]);
+        sum += (fa.x + fa.y) + (fb.x + fb.y);
+    }
+    l = l * alpha + sum;
     m = mn;
-    p_lo = bf162_bits(a);
-    p_hi = bf162_bits(b);
     return alpha;
 }
 
-template <int D, int ROWS, int STAGES, int WARPS, int MIN_CTAS>
+template <int D, int ROWS, int STAGES, int WARPS, int MIN_CTAS, bool FP8 = false>
 __global__ void __launch_bounds__(WARPS * 32, MIN_CTAS)
 decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v, const DecodeParams P) {
-    using Cfg = MmaCfg<D, STAGES, WARPS>;
+    using Cfg = MmaCfg<D, STAGES, WARPS, FP8>;
     constexpr int KSTEPS = D / 16;  // k-steps of Q K^T
     constexpr int NTD = D / 8;      // n-tiles of P V
     constexpr bool HI = ROWS > 8;   // query rows 8..15 in use
     constexpr int AR = HI ? 4 : 2;  // registers per A fragment / per C tile that are held
+    // blocks per consumer step (one max / sum reduction and one rescale per
+    // step); one measured fastest for both element types
+#ifndef PA_FP8_BLOCKS_PER_STEP
+#define PA_FP8_BLOCKS_PER_STEP 1
+#endif
+    constexpr int BPS = FP8 ? PA_FP8_BLOCKS_PER_STEP : 1;
+    static_assert(STAGES >= 2 * BPS, "a step's stages plus as many in flight");
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -187,7 +222,8 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int tq = 2 * (lane & 3);  // first token (S) / first dim (O) of this lane's pair
     const int r_lo = lane >> 2;     // query row within the group
     const uint32_t sw = lane & 7;   // swizzle term: ldmatrix row index mod 8
-    const float sl2 = P.scale_log2;
+    float sl2 = P.scale_log2;  // times the kv head's K scale for E4M3 caches
+    float vscale = 1.f;         // the kv head's V scale for E4M3 caches
 
     uint32_t qa[KSTEPS][AR];  // Q as A fragments: {lo, [hi,] lo+8 cols, [hi+8 cols]}
     float m_lo = -INFINITY, l_lo = 0.f, m_hi = -INFINITY, l_hi = 0.f;
@@ -214,6 +250,30 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             lim_lo = cc.len - qr.n + tok_lo;
             lim_hi = cc.len - qr.n + tok_hi;
             const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(P.q);
+            if constexpr (FP8) {
+                // k-step ks covers dims 16ks..16ks+15; the K fragments hold
+                // dims 16ks+2tq..+3 (b0: first pair, b1: second), so the A
+                // fragment takes the same dims: a0/a1 the first pair, a2/a3
+                // the second.  Widened to f16 (exact for |q| in 2^-14..65504).
+                const uint2* q_lo = reinterpret_cast<const uint2*>(qb + (ok_lo ? orow_lo : 0) * D + 2 * tq);
+                const uint2* q_hi = reinterpret_cast<const uint2*>(qb + (ok_hi ? orow_hi : 0) * D + 2 * tq);
+#pragma unroll
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    const uint2 lo = ok_lo ? __ldg(q_lo + 4 * ks) : make_uint2(0u, 0u);
+                    if constexpr (HI) {
+                        const uint2 hi = ok_hi ? __ldg(q_hi + 4 * ks) : make_uint2(0u, 0u);
+                        qa[ks][0] = bf16x2_to_f16x2(lo.x);
+                        qa[ks][1] = bf16x2_to_f16x2(hi.x);
+                        qa[ks][2] = bf16x2_to_f16x2(lo.y);
+                        qa[ks][3] = bf16x2_to_f16x2(hi.y);
+                    } else {
+                        qa[ks][0] = bf16x2_to_f16x2(lo.x);
+                        qa[ks][1] = bf16x2_to_f16x2(lo.y);
+                    }
+                }
+                sl2 = P.scale_log2 * __ldg(P.k_scale + cc.h);
+                vscale = __ldg(P.v_scale + cc.h);
+            } else {
             const uint32_t* q_lo = reinterpret_cast<const uint32_t*>(qb + (ok_lo ? orow_lo : 0) * D + tq);
             const uint32_t* q_hi = reinterpret_cast<const uint32_t*>(qb + (ok_hi ? orow_hi : 0) * D + tq);
 #pragma unroll
@@ -228,6 +288,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     qa[ks][1] = ok_lo ? __ldg(q_lo + ks * 8 + 4) : 0u;
                 }
             }
+            }
             m_lo = m_hi = -INFINITY;
             l_lo = l_hi = 0.f;
 #pragma unroll
@@ -236,113 +297,219 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 for (int r = 0; r < AR; ++r) acc[n][r] = 0.f;
         }
 
-        const uint32_t bar = bar_u32 + stage * 8;
-        if (!mbar_wait_bounded(bar, phase)) {
-            if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
-            // drain: wait (bounded) for the copies still in flight, then leave
-            for (uint32_t k = 1; k < issued - consumed; ++k) {
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                mbar_wait_bounded(bar_u32 + stage * 8, phase);
+        // ---- this step: BPS blocks (fewer at the end of the piece); wait for
+        // their stages and mask what they hold
+        const int nb = BPS == 1 ? 1 : min(BPS, cc.jend - cj);
+        uint32_t kb[BPS], vb[BPS];
+        int valid[BPS];
+#pragma unroll
+        for (int b = 0; b < BPS; ++b) {
+            valid[b] = 0;
+            kb[b] = vb[b] = 0;
+            if (b >= nb) continue;
+            int sb = stage + b;
+            uint32_t pb = phase;
+            if (sb >= STAGES) {
+                sb -= STAGES;
+                pb ^= 1u;
             }
-            return;
-        }
-        ++consumed;
-        const uint32_t kbase = ring_u32 + stage * Cfg::kStageBytes;
-        const uint32_t vbase = kbase + Cfg::kTileBytes;
-        const int valid = ((oob_mask >> stage) & 1u) ? 0 : min(kBlockTokens, cc.len - cj * kBlockTokens);
-        if (valid < kBlockTokens) {
-            // zero V rows [valid, 16) so that 0 * (stale or NaN) never enters P V
-            uint8_t* vs = ring + stage * Cfg::kStageBytes + Cfg::kTileBytes;
-            const int chunks = (kBlockTokens - valid) * Cfg::kRegions * 8;
-            for (int c = lane; c < chunks; c += 32) {
-                const int row = valid + c / (Cfg::kRegions * 8);
-                const int rem = c % (Cfg::kRegions * 8);
-                *reinterpret_cast<uint4*>(vs + (rem >> 3) * Cfg::kRegionBytes + row * 128 +
-                                          (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
+            if (!mbar_wait_bounded(bar_u32 + sb * 8, pb)) {
+                if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
+                // drain: wait (bounded) for the copies still in flight, then leave
+                for (uint32_t k = 1; k < issued - consumed; ++k) {
+                    if (++sb == STAGES) { sb = 0; pb ^= 1u; }
+                    mbar_wait_bounded(bar_u32 + sb * 8, pb);
+                }
+                return;
             }
-            fence_proxy_async_smem();
-            __syncwarp();
+            ++consumed;
+            valid[b] = ((oob_mask >> sb) & 1u) ? 0 : min(kBlockTokens, cc.len - (cj + b) * kBlockTokens);
+            kb[b] = ring_u32 + sb * Cfg::kStageBytes;
+            vb[b] = kb[b] + Cfg::kTileBytes;
+            if (valid[b] < kBlockTokens) {
+                // zero V rows [valid, 16) so that 0 * (stale or NaN) never enters P V
+                uint8_t* vs = ring + sb * Cfg::kStageBytes + Cfg::kTileBytes;
+                constexpr int kRowChunks = Cfg::kRegions * Cfg::kRowBytes / 16;  // 16-byte chunks per row
+                constexpr int kSlabChunks = Cfg::kRowBytes / 16;
+                const int chunks = (kBlockTokens - valid[b]) * kRowChunks;
+                for (int c = lane; c < chunks; c += 32) {
+                    const int row = valid[b] + c / kRowChunks;
+                    const int rem = c % kRowChunks;
+                    *reinterpret_cast<uint4*>(vs + (rem / kSlabChunks) * Cfg::kRegionBytes +
+                                              row * Cfg::kRowBytes + (rem % kSlabChunks) * 16) =
+                        make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
         }
 
-        // ---- S = Q K^T : two n-tiles of 8 tokens
-        float s0[AR], s1[AR];
+        // ---- S = Q K^T per block: two n-tiles of 8 tokens, each with two
+        // accumulators (even / odd k-steps) so that the dependent MMA chains
+        // are KSTEPS/2 long
+        float sc[BPS][2][AR];
 #pragma unroll
-        for (int r = 0; r < AR; ++r) s0[r] = s1[r] = 0.f;
+        for (int b = 0; b < BPS; ++b) {
 #pragma unroll
-        for (int kp = 0; kp < KSTEPS / 2; ++kp) {
-            const int cg = 4 * kp + (lane >> 3);  // 8-element column chunk 0 .. D/8-1
-            const uint32_t col = (cg >> 3) * Cfg::kRegionBytes + ((((uint32_t)cg & 7u) ^ sw) << 4);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(kbase + col + (lane & 7) * 128, b0, b1, b2, b3);
-            mma_frag(s0, qa[2 * kp], b0, b1);
-            mma_frag(s0, qa[2 * kp + 1], b2, b3);
-            ldsm_x4(kbase + col + (8 + (lane & 7)) * 128, b0, b1, b2, b3);
-            mma_frag(s1, qa[2 * kp], b0, b1);
-            mma_frag(s1, qa[2 * kp + 1], b2, b3);
+            for (int r = 0; r < AR; ++r) sc[b][0][r] = sc[b][1][r] = 0.f;
+            if (b >= nb) continue;
+            float s0[AR], s1[AR], t0[AR], t1[AR];
+#pragma unroll
+            for (int r = 0; r < AR; ++r) s0[r] = s1[r] = t0[r] = t1[r] = 0.f;
+            const uint32_t kbase = kb[b];
+            if constexpr (FP8) {
+                // E4M3 K: ldmatrix on the codes seen as b16 gives each lane dims
+                // 4(lane%4)..+3 of one token per 16-dim chunk; matrices: (tokens
+                // 0-7, chunk j), (8-15, j), (0-7, j+1), (8-15, j+1)
+                const int tok = (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+                for (int j = 0; j < KSTEPS; j += 2) {
+                    const uint32_t ch = static_cast<uint32_t>(j + (lane >> 4));
+                    uint32_t r0, r1, r2, r3, b0, b1;
+                    ldsm_x4(kbase + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
+                    e4m3x4_to_f16x2x2(r0, b0, b1);
+                    mma_frag_t<true>(s0, qa[j], b0, b1);
+                    e4m3x4_to_f16x2x2(r1, b0, b1);
+                    mma_frag_t<true>(s1, qa[j], b0, b1);
+                    e4m3x4_to_f16x2x2(r2, b0, b1);
+                    mma_frag_t<true>(t0, qa[j + 1], b0, b1);
+                    e4m3x4_to_f16x2x2(r3, b0, b1);
+                    mma_frag_t<true>(t1, qa[j + 1], b0, b1);
+                }
+            } else {
+#pragma unroll
+                for (int kp = 0; kp < KSTEPS / 2; ++kp) {
+                    const int cg = 4 * kp + (lane >> 3);  // 8-element column chunk 0 .. D/8-1
+                    const uint32_t col = (cg >> 3) * Cfg::kRegionBytes + ((((uint32_t)cg & 7u) ^ sw) << 4);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(kbase + col + (lane & 7) * 128, b0, b1, b2, b3);
+                    mma_frag(s0, qa[2 * kp], b0, b1);
+                    mma_frag(t0, qa[2 * kp + 1], b2, b3);
+                    ldsm_x4(kbase + col + (8 + (lane & 7)) * 128, b0, b1, b2, b3);
+                    mma_frag(s1, qa[2 * kp], b0, b1);
+                    mma_frag(t1, qa[2 * kp + 1], b2, b3);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < AR; ++r) {
+                sc[b][0][r] += s0[r] + t0[r];
+                sc[b][1][r] += s1[r] + t1[r];
+            }
         }
 
-        // ---- online softmax (rows r_lo and r_lo + 8); key t of the block is
-        // visible to a row iff t < valid and cj*16 + t <= the row's limit
-        uint32_t pa0, pa1 = 0u, pa2, pa3 = 0u;
+        // ---- online softmax over the step's keys (rows r_lo and r_lo + 8);
+        // key t of block b is visible to a row iff t < valid[b] and
+        // (cj + b)*16 + t <= the row's limit
+        uint32_t plo[BPS][2], phi[BPS][2];  // P as bf16 / f16 pairs: [block][tokens tq.. / 8+tq..]
+        float alpha_lo, alpha_hi = 1.f;
         {
-            const int vis = min(valid - 1, lim_lo - cj * kBlockTokens);  // last visible key
-            float x[4] = {s0[0], s0[1], s1[0], s1[1]};
-            x[0] = tq <= vis ? x[0] * sl2 : -INFINITY;
-            x[1] = tq + 1 <= vis ? x[1] * sl2 : -INFINITY;
-            x[2] = tq + 8 <= vis ? x[2] * sl2 : -INFINITY;
-            x[3] = tq + 9 <= vis ? x[3] * sl2 : -INFINITY;
-            const float alpha = softmax_update(m_lo, l_lo, x, pa0, pa2);
+            float x[4 * BPS];
 #pragma unroll
-            for (int n = 0; n < NTD; ++n) {
-                acc[n][0] *= alpha;
-                acc[n][1] *= alpha;
+            for (int b = 0; b < BPS; ++b) {
+                const int vis = min(valid[b] - 1, lim_lo - (cj + b) * kBlockTokens);  // last visible key
+                x[4 * b + 0] = tq <= vis ? sc[b][0][0] * sl2 : -INFINITY;
+                x[4 * b + 1] = tq + 1 <= vis ? sc[b][0][1] * sl2 : -INFINITY;
+                x[4 * b + 2] = tq + 8 <= vis ? sc[b][1][0] * sl2 : -INFINITY;
+                x[4 * b + 3] = tq + 9 <= vis ? sc[b][1][1] * sl2 : -INFINITY;
             }
+            alpha_lo = softmax_update<FP8, BPS>(m_lo, l_lo, x, plo);
         }
         if constexpr (HI) {
-            const int vis = min(valid - 1, lim_hi - cj * kBlockTokens);
-            float x[4] = {s0[2], s0[3], s1[2], s1[3]};
-            x[0] = tq <= vis ? x[0] * sl2 : -INFINITY;
-            x[1] = tq + 1 <= vis ? x[1] * sl2 : -INFINITY;
-            x[2] = tq + 8 <= vis ? x[2] * sl2 : -INFINITY;
-            x[3] = tq + 9 <= vis ? x[3] * sl2 : -INFINITY;
-            const float alpha = softmax_update(m_hi, l_hi, x, pa1, pa3);
+            float x[4 * BPS];
+#pragma unroll
+            for (int b = 0; b < BPS; ++b) {
+                const int vis = min(valid[b] - 1, lim_hi - (cj + b) * kBlockTokens);
+                x[4 * b + 0] = tq <= vis ? sc[b][0][2] * sl2 : -INFINITY;
+                x[4 * b + 1] = tq + 1 <= vis ? sc[b][0][3] * sl2 : -INFINITY;
+                x[4 * b + 2] = tq + 8 <= vis ? sc[b][1][2] * sl2 : -INFINITY;
+                x[4 * b + 3] = tq + 9 <= vis ? sc[b][1][3] * sl2 : -INFINITY;
+            }
+            alpha_hi = softmax_update<FP8, BPS>(m_hi, l_hi, x, phi);
+        }
+        // rescale the accumulators only when some row's max moved (alpha is
+        // exactly 1 otherwise): after the first blocks of a sequence it rarely does
+        if (__any_sync(kFullMask, alpha_lo != 1.f || alpha_hi != 1.f)) {
 #pragma unroll
             for (int n = 0; n < NTD; ++n) {
-                acc[n][2] *= alpha;
-                acc[n][3] *= alpha;
+                acc[n][0] *= alpha_lo;
+                acc[n][1] *= alpha_lo;
+                if constexpr (HI) {
+                    acc[n][2] *= alpha_hi;
+                    acc[n][3] *= alpha_hi;
+                }
             }
         }
 
-        uint32_t pa[AR];  // P as an A fragment
-        if constexpr (HI) {
-            pa[0] = pa0; pa[1] = pa1; pa[2] = pa2; pa[3] = pa3;
-        } else {
-            pa[0] = pa0; pa[1] = pa2;
-        }
-
-        // ---- O += P V : n-tiles of 8 head dims, K = the 16 tokens
+        // ---- O += P V : n-tiles of 8 head dims, K = the 16 tokens of a block
 #pragma unroll
-        for (int dp = 0; dp < D / 16; ++dp) {
-            const int cg = 2 * dp + (lane >> 4);
-            const int t = 8 * ((lane >> 3) & 1) + (lane & 7);
-            const uint32_t addr = vbase + (cg >> 3) * Cfg::kRegionBytes + t * 128 +
-                                  ((((uint32_t)cg & 7u) ^ sw) << 4);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_trans(addr, b0, b1, b2, b3);
-            mma_frag(acc[2 * dp], pa, b0, b1);
-            mma_frag(acc[2 * dp + 1], pa, b2, b3);
+        for (int b = 0; b < BPS; ++b) {
+            if (b >= nb) continue;
+            uint32_t pa[AR];  // P as an A fragment
+            if constexpr (HI) {
+                pa[0] = plo[b][0]; pa[1] = phi[b][0]; pa[2] = plo[b][1]; pa[3] = phi[b][1];
+            } else {
+                pa[0] = plo[b][0]; pa[1] = plo[b][1];
+            }
+            const uint32_t vbase = vb[b];
+            if constexpr (FP8) {
+                // E4M3 V: ldmatrix.trans on the codes seen as b16 gives each lane
+                // tokens 2(lane%4), +1 of the dim pair 2(lane/4), +1 of a 16-dim
+                // chunk; one byte permute splits it into the even and the odd
+                // dim's token pair.  n-tile 2c of the accumulators holds the even
+                // dims 16c + 2n of chunk c, n-tile 2c+1 the odd dims.
+                const int tok = (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+                for (int c = 0; c < D / 16; c += 2) {
+                    const uint32_t ch = static_cast<uint32_t>(c + (lane >> 4));
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4_trans(vbase + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
+                    uint32_t e0, o0, e1, o1;
+                    e4m3x4_to_f16x2x2(byte_perm(r0, 0x3120), e0, o0);  // tokens 2(lane%4), +1
+                    e4m3x4_to_f16x2x2(byte_perm(r1, 0x3120), e1, o1);  // tokens 8 + 2(lane%4), +1
+                    mma_frag_t<true>(acc[2 * c], pa, e0, e1);
+                    mma_frag_t<true>(acc[2 * c + 1], pa, o0, o1);
+                    e4m3x4_to_f16x2x2(byte_perm(r2, 0x3120), e0, o0);
+                    e4m3x4_to_f16x2x2(byte_perm(r3, 0x3120), e1, o1);
+                    mma_frag_t<true>(acc[2 * c + 2], pa, e0, e1);
+                    mma_frag_t<true>(acc[2 * c + 3], pa, o0, o1);
+                }
+            } else {
+#pragma unroll
+                for (int dp = 0; dp < D / 16; ++dp) {
+                    const int cg = 2 * dp + (lane >> 4);
+                    const int t = 8 * ((lane >> 3) & 1) + (lane & 7);
+                    const uint32_t addr = vbase + (cg >> 3) * Cfg::kRegionBytes + t * 128 +
+                                          ((((uint32_t)cg & 7u) ^ sw) << 4);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_trans(addr, b0, b1, b2, b3);
+                    mma_frag(acc[2 * dp], pa, b0, b1);
+                    mma_frag(acc[2 * dp + 1], pa, b2, b3);
+                }
+            }
         }
         __syncwarp();
 
-        if (prod_live) produce(stage);
-        if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
+        // ---- hand the stages back to the producer
+#pragma unroll
+        for (int b = 0; b < BPS; ++b) {
+            if (b >= nb) continue;
+            if (prod_live) produce(stage);
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
         }
 
-        if (++cj < cc.jend) continue;
+        cj += nb;
+        if (cj < cc.jend) continue;
 
         // ---- item done: final row or partition partials
+        if constexpr (FP8) {  // the sums of P V used the V codes: apply the V scale once
+#pragma unroll
+            for (int n = 0; n < NTD; ++n)
+#pragma unroll
+                for (int r = 0; r < AR; ++r) acc[n][r] *= vscale;
+        }
         float lt_lo = l_lo + __shfl_xor_sync(kFullMask, l_lo, 1);
         lt_lo += __shfl_xor_sync(kFullMask, lt_lo, 2);
         float lt_hi = 0.f;
@@ -350,25 +517,43 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             lt_hi = l_hi + __shfl_xor_sync(kFullMask, l_hi, 1);
             lt_hi += __shfl_xor_sync(kFullMask, lt_hi, 2);
         }
-        if (cc.parts == 1 && P.piece_base == 0) {
-            __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(P.out);
-            if (ok_lo) {
-                const float inv = lt_lo > 0.f ? 1.0f / lt_lo : 0.f;
-                __nv_bfloat16* o = ob + orow_lo * D + tq;
+        // This lane's accumulators of a row (r = 0: row r_lo, r = 2: row
+        // r_lo + 8) go to dims 8n + tq, +1 of n-tile n (bf16); for E4M3 to
+        // dims 16c + 2tq .. +3 of chunk c as (even, odd, even, odd) n-tiles.
+        auto put_out = [&](size_t orow, int r, float inv) {
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(P.out) + orow * D;
+            if constexpr (FP8) {
+#pragma unroll
+                for (int c = 0; c < D / 16; ++c) {
+                    uint2 u;
+                    u.x = pack2<false>(acc[2 * c][r] * inv, acc[2 * c + 1][r] * inv);
+                    u.y = pack2<false>(acc[2 * c][r + 1] * inv, acc[2 * c + 1][r + 1] * inv);
+                    *reinterpret_cast<uint2*>(o + 16 * c + 2 * tq) = u;
+                }
+            } else {
 #pragma unroll
                 for (int n = 0; n < NTD; ++n)
-                    *reinterpret_cast<__nv_bfloat162*>(o + 8 * n) =
-                        __floats2bfloat162_rn(acc[n][0] * inv, acc[n][1] * inv);
+                    *reinterpret_cast<__nv_bfloat162*>(o + 8 * n + tq) =
+                        __floats2bfloat162_rn(acc[n][r] * inv, acc[n][r + 1] * inv);
             }
-            if constexpr (HI) {
-                if (ok_hi) {
-                    const float inv = lt_hi > 0.f ? 1.0f / lt_hi : 0.f;
-                    __nv_bfloat16* o = ob + orow_hi * D + tq;
+        };
+        auto put_partial = [&](size_t idx, int r) {
+            float* a = P.ws_acc + idx * D;
+            if constexpr (FP8) {
 #pragma unroll
-                    for (int n = 0; n < NTD; ++n)
-                        *reinterpret_cast<__nv_bfloat162*>(o + 8 * n) =
-                            __floats2bfloat162_rn(acc[n][2] * inv, acc[n][3] * inv);
-                }
+                for (int c = 0; c < D / 16; ++c)
+                    *reinterpret_cast<float4*>(a + 16 * c + 2 * tq) =
+                        make_float4(acc[2 * c][r], acc[2 * c + 1][r], acc[2 * c][r + 1], acc[2 * c + 1][r + 1]);
+            } else {
+#pragma unroll
+                for (int n = 0; n < NTD; ++n)
+                    *reinterpret_cast<float2*>(a + 8 * n + tq) = make_float2(acc[n][r], acc[n][r + 1]);
+            }
+        };
+        if (cc.parts == 1 && P.piece_base == 0) {
+            if (ok_lo) put_out(orow_lo, 0, lt_lo > 0.f ? 1.0f / lt_lo : 0.f);
+            if constexpr (HI) {
+                if (ok_hi) put_out(orow_hi, 2, lt_hi > 0.f ? 1.0f / lt_hi : 0.f);
             }
         } else {
             constexpr float kLn2 = 0.693147180559945309f;
@@ -378,10 +563,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     P.ws_m[idx] = m_lo * kLn2;
                     P.ws_l[idx] = lt_lo;
                 }
-                float* a = P.ws_acc + idx * D + tq;
-#pragma unroll
-                for (int n = 0; n < NTD; ++n)
-                    *reinterpret_cast<float2*>(a + 8 * n) = make_float2(acc[n][0], acc[n][1]);
+                put_partial(idx, 0);
             }
             if constexpr (HI) {
                 if (ok_hi) {
@@ -390,10 +572,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         P.ws_m[idx] = m_hi * kLn2;
                         P.ws_l[idx] = lt_hi;
                     }
-                    float* a = P.ws_acc + idx * D + tq;
-#pragma unroll
-                    for (int n = 0; n < NTD; ++n)
-                        *reinterpret_cast<float2*>(a + 8 * n) = make_float2(acc[n][2], acc[n][3]);
+                    put_partial(idx, 2);
                 }
             }
         }

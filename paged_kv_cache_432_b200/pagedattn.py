@@ -39,6 +39,9 @@ _P, _I32, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctype
 _DECODE_ARGS = [_P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _F, _I32, _P, _SZ, _P, _I32, _P]
 SIGNATURES = {
     "pa_cache_write": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _P, _P, _I32, _I32, _I32, _P]),
+    "pa_cache_write_fp8": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _P, _P, _I32, _I32, _P, _P, _P]),
+    "pa_decode_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32,
+                                     _F, _I32, _P, _SZ, _P, _P]),
     "pa_decode_partition_blocks": (_I32, [_I32, _I32, _I32, _I32, _I32]),
     "pa_decode_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "pa_decode": (ctypes.c_int, _DECODE_ARGS),
@@ -122,6 +125,36 @@ def cache_write(k, v, slot_mapping, k_cache, v_cache, stream=None) -> None:
     rc = lib().pa_cache_write(_ptr(k), _ptr(v), _ptr(slot_mapping), T, H, D, _ptr(k_cache),
                               _ptr(v_cache), NB, B, dtype_code(k.dtype), _stream(stream))
     _check("pa_cache_write", rc)
+
+
+def cache_write_fp8(k, v, slot_mapping, k_cache, v_cache, k_inv_scale, v_inv_scale, stream=None) -> None:
+    """pa_cache_write_fp8: k, v bf16 [T, Hkv, D]; caches uint8 (E4M3 codes)
+    [NB, Hkv, 16, D]; inverse scales fp32 [Hkv]; slots int64 [T]."""
+    T, H, D = k.shape
+    NB, H2, B, D2 = k_cache.shape
+    rc = lib().pa_cache_write_fp8(_ptr(k), _ptr(v), _ptr(slot_mapping), T, H, D, _ptr(k_cache), _ptr(v_cache),
+                                  NB, B, _ptr(k_inv_scale), _ptr(v_inv_scale), _stream(stream))
+    _check("pa_cache_write_fp8", rc)
+
+
+def decode_fp8(q, k_cache, v_cache, k_scale, v_scale, block_tables, seq_lens, scale, out=None, max_seq_len=0,
+               partition_blocks=0, workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode_fp8: q bf16 [N, Hq, D]; caches uint8 E4M3 [NB, Hkv, 16, D];
+    scales fp32 [Hkv].  Returns out (bf16 [N, Hq, D])."""
+    N, Hq, D = q.shape
+    NB, Hkv, B, _ = k_cache.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(N, Hq, Hkv, D, max_seq_len if max_seq_len > 0 else block_tables.shape[1] * 16,
+                                    partition_blocks, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().pa_decode_fp8(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+                             _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), max_seq_len, N, Hq, Hkv, D,
+                             NB, B, float(scale), partition_blocks, _ptr(workspace), ws_bytes, _ptr(out),
+                             _stream(stream))
+    _check("pa_decode_fp8", rc)
+    return out
 
 
 def partition_blocks(num_seqs, num_kv_heads, max_seq_len, partition_blocks=0, block_size=16) -> int:

@@ -278,11 +278,7 @@ def build(
     slot_mapping = torch.tensor(new_token_slots(p), dtype=torch.int64)
 
     if poison_unused:
-        used = torch.zeros((num_blocks, B), dtype=torch.bool)
-        for L, t in zip(lens, tables):
-            for j, b in enumerate(t):
-                used[b, : min(B, L - j * B)] = True
-        used = used.to(device)[:, None, :, None]
+        used = _used_slots(lens, tables, num_blocks).to(device)[:, None, :, None]
         nan = torch.tensor(float("nan"), dtype=dtype, device=device)
         k_cache = torch.where(used, k_cache, nan)
         v_cache = torch.where(used, v_cache, nan)
@@ -312,6 +308,53 @@ def build(
         shared_prefix_blocks=len(p.shared),
         desc=desc,
     )
+
+
+def _used_slots(lens, tables, num_blocks: int) -> torch.Tensor:
+    """[num_blocks, 16] bool: the slots some sequence's table reaches."""
+    B = BLOCK_SIZE
+    used = torch.zeros((num_blocks, B), dtype=torch.bool)
+    for L, t in zip(lens, tables):
+        for j, b in enumerate(t):
+            used[b, : min(B, L - j * B)] = True
+    return used
+
+
+E4M3_NAN = 0x7F  # S.1111.111, the code pa_cache_write_fp8 writes for NaN
+
+
+def fp8_pools(w: Workload, seed: Optional[int] = None, poison_unused: bool = False) -> tuple:
+    """E4M3 KV pools with the structure (pool size, tables) of ``w``.
+
+    Returns (k_codes, v_codes, k_scale, v_scale): uint8 [NB, Hkv, 16, D] codes
+    drawn uniformly from the 254 codes that are not NaN (bit patterns only: no
+    rounding or conversion here), and one fp32 scale per kv head and pool drawn
+    uniformly from [1/160, 1/112], so that decoded values stay within about
+    +-4, the range of the N(0, 1) values of the bf16 pools; all on ``w.device``.  Values come from a device
+    generator seeded with ``seed + 2`` (``seed`` defaults to ``w.seed``).
+    ``poison_unused`` sets every slot no table reaches to the NaN code.
+    """
+    seed = w.seed if seed is None else seed
+    dev = w.device
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed + 2)
+    shape = (w.num_blocks, w.num_kv_heads, BLOCK_SIZE, w.head_dim)
+    pools = []
+    for _ in range(2):
+        out = torch.empty(shape, dtype=torch.uint8, device=dev)
+        flat = out.view(-1)
+        chunk = 1 << 28
+        for off in range(0, flat.numel(), chunk):
+            m = min(chunk, flat.numel() - off)
+            c = torch.randint(0, 254, (m,), generator=gen, device=dev, dtype=torch.uint8)
+            flat[off : off + m] = c + (c >= E4M3_NAN).to(torch.uint8)  # 0..126, 128..254: no NaN code
+        pools.append(out)
+    scales = [1.0 / (112.0 + 48.0 * torch.rand(w.num_kv_heads, generator=gen, device=dev)) for _ in range(2)]
+    if poison_unused:
+        used = _used_slots(w.lens_host, w.tables_host, w.num_blocks).to(dev)[:, None, :, None]
+        nan = torch.tensor(E4M3_NAN, dtype=torch.uint8, device=dev)
+        pools = [torch.where(used, p, nan) for p in pools]
+    return pools[0], pools[1], scales[0].float(), scales[1].float()
 
 
 def new_token_slots(p: Plan) -> list:

@@ -24,7 +24,7 @@ def lib():
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(pa_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_declares_the_boundary():
@@ -38,7 +38,7 @@ def test_header_declares_the_boundary():
 
 def test_every_declared_symbol_is_exported(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True, text=True).stdout
-    exported = set(re.findall(r"\bT (pa_[a-z_]+)\b", out))
+    exported = set(re.findall(r"\bT (pa_[a-z0-9_]+)\b", out))
     for n in declared_functions():
         assert n in exported, n
         assert hasattr(lib, n)
@@ -156,6 +156,40 @@ def test_cache_write_rejects_bad_arguments_on_the_host(lib):
     assert rc(D=80) == pa.PA_ERR_UNSUPPORTED
     assert rc(B=8) == pa.PA_ERR_UNSUPPORTED
     assert rc(T=0) == pa.PA_OK                      # nothing to do, nothing launched
+
+
+def test_fp8_entry_points_reject_bad_arguments_on_the_host(lib):
+    f = lib.pa_cache_write_fp8
+    ok = dict(k=16, v=16, s=16, T=4, H=2, D=128, kc=16, vc=16, NB=8, B=16, ks=32, vs=32)
+
+    def rc(**o):
+        a = dict(ok, **o)
+        return f(a["k"], a["v"], a["s"], a["T"], a["H"], a["D"], a["kc"], a["vc"], a["NB"], a["B"], a["ks"],
+                 a["vs"], None)
+
+    assert rc(ks=None) == pa.PA_ERR_INVALID_ARG      # inverse scales are required
+    assert rc(vs=34) == pa.PA_ERR_INVALID_ARG        # not 4-byte aligned
+    assert rc(kc=8) == pa.PA_ERR_INVALID_ARG
+    assert rc(D=96) == pa.PA_ERR_UNSUPPORTED
+    assert rc(B=32) == pa.PA_ERR_UNSUPPORTED
+    assert rc(T=0) == pa.PA_OK
+
+    d = lib.pa_decode_fp8
+    base = [16, 16, 16, 32, 32, 16, 4, 16, 64, 2, 8, 2, 128, 8, 16, 0.1, -1, None, 0, 16, None]
+
+    def drc(i=None, val=None):
+        a = list(base)
+        if i is not None:
+            a[i] = val
+        return d(*a)
+
+    assert drc(3, None) == pa.PA_ERR_INVALID_ARG     # k_scale
+    assert drc(4, None) == pa.PA_ERR_INVALID_ARG     # v_scale
+    assert drc(4, 33) == pa.PA_ERR_INVALID_ARG       # misaligned v_scale
+    assert drc(0, 8) == pa.PA_ERR_INVALID_ARG        # misaligned q
+    assert drc(12, 96) == pa.PA_ERR_UNSUPPORTED      # head_dim
+    assert drc(10, 34) == pa.PA_ERR_UNSUPPORTED      # 34 / 2 = group of 17
+    assert drc(15, float("inf")) == pa.PA_ERR_INVALID_ARG
 
 
 def test_get_device_error_rejects_null(lib):

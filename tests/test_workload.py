@@ -78,3 +78,22 @@ def test_poison_marks_only_unreachable_slots():
         for t in range(L):
             assert not nan[w.tables_host[s][t // 16], t % 16]
     assert int(nan.sum()) == w.num_blocks * 16 - sum(w.lens_host)
+
+
+def test_fp8_pools_draw_no_nan_code_and_poison_only_unreachable_slots():
+    w = wl.build([35, 1, 300], 4, 2, 64, torch.bfloat16, seed=6)
+    kc, vc, ks, vs = wl.fp8_pools(w)
+    for c in (kc, vc):
+        assert c.dtype == torch.uint8 and c.shape == (w.num_blocks, 2, 16, 64)
+        assert not bool(((c & 0x7F) == 0x7F).any())  # neither NaN code is drawn
+        assert int(c.unique().numel()) > 200          # the other codes all appear
+    assert ks.shape == (2,) and bool(((ks >= 1 / 160) & (ks <= 1 / 112)).all())
+    kc2, _, ks2, _ = wl.fp8_pools(w)
+    assert torch.equal(kc, kc2) and torch.equal(ks, ks2)  # seeded
+    assert not torch.equal(kc, wl.fp8_pools(w, seed=9)[0])
+    kp, _, _, _ = wl.fp8_pools(w, poison_unused=True)
+    nan = kp[:, 0, :, 0] == wl.E4M3_NAN
+    for s, L in enumerate(w.lens_host):
+        for t in range(L):
+            assert not nan[w.tables_host[s][t // 16], t % 16]
+    assert int(nan.sum()) == w.num_blocks * 16 - sum(w.lens_host)
