@@ -22,6 +22,7 @@
 #include "common.cuh"
 #include "decode_mma.cuh"
 #include "decode_prefix.cuh"
+#include "decode_prefix_tc.cuh"
 #include "decode_simt.cuh"
 #include "items.cuh"
 #include "lse_reduce.cuh"
@@ -201,7 +202,7 @@ struct Plan {
     int32_t shared_blocks;
     int32_t prefix_splits;        // key splits of the prefix = its pieces 0 .. splits-1
     int32_t prefix_split_blocks;  // blocks per key split
-    int32_t prefix_row_tiles;     // ceil(num_seqs * group / 64)
+    int32_t prefix_row_tiles;     // ceil(num_seqs * group / rows per prefix CTA)
 };
 
 Plan make_plan(int32_t max_seq_len, int32_t partition_blocks) {
@@ -230,6 +231,26 @@ Plan make_plan(int32_t max_seq_len, int32_t partition_blocks) {
 // picks the split count that fills one wave of the prefix kernel on the
 // device (choose_prefix_splits).
 constexpr int32_t kMaxPrefixSplits = 16;
+
+// The shared-prefix kernel: tcgen05 with TMEM accumulators (128 query rows per
+// CTA), or the mma.sync kernel (64 rows per CTA) when built with PA_PREFIX_TC=0.
+#ifndef PA_PREFIX_TC
+#define PA_PREFIX_TC 1
+#endif
+constexpr bool kPrefixTc = PA_PREFIX_TC != 0;
+constexpr int kPrefixTileRows = kPrefixTc ? PrefixTcCfg<128>::kRows : kPrefixRows;
+
+template <int D>
+struct PrefixKernel {
+    using Fn = void (*)(CUtensorMap, CUtensorMap, PrefixParams);
+    static Fn fn() {
+        if constexpr (kPrefixTc) return decode_prefix_tc_kernel<D>;
+        else return decode_prefix_mma_kernel<D>;
+    }
+    static constexpr size_t kSmem = kPrefixTc ? PrefixTcCfg<D>::kSmem : PrefixCfg<D>::kSmem;
+    static constexpr int kThreads = kPrefixTc ? PrefixTcCfg<D>::kThreads : PrefixCfg<D>::kThreads;
+    static constexpr const char* kName = kPrefixTc ? "decode_prefix_tc_kernel" : "decode_prefix_mma_kernel";
+};
 constexpr int32_t kWideReducePieces = 32;  // rows that can have more pieces merge with 4 warps each
 
 Plan make_prefix_plan(int32_t max_seq_len, int32_t partition_blocks, int32_t shared_blocks,
@@ -238,7 +259,7 @@ Plan make_prefix_plan(int32_t max_seq_len, int32_t partition_blocks, int32_t sha
     Plan p = make_plan(rest > 0 ? rest : 0, partition_blocks);
     p.max_len = max_seq_len;
     const int64_t rows = static_cast<int64_t>(num_seqs) * (num_q_heads / num_kv_heads);
-    p.prefix_row_tiles = static_cast<int32_t>((rows + kPrefixRows - 1) / kPrefixRows);
+    p.prefix_row_tiles = static_cast<int32_t>((rows + kPrefixTileRows - 1) / kPrefixTileRows);
     if (p.prefix_row_tiles < 1) p.prefix_row_tiles = 1;
     p.shared_blocks = shared_blocks;
     const int32_t slots = shared_blocks < kMaxPrefixSplits ? shared_blocks : kMaxPrefixSplits;
@@ -529,14 +550,14 @@ int run_partitions(const DecodeParams& P, int32_t dtype, cudaStream_t st) {
 // workspace reserves.  Sets plan->prefix_splits / prefix_split_blocks.
 template <int D>
 int choose_prefix_splits(const DecodeParams& P, Plan* plan) {
-    auto kernel = decode_prefix_mma_kernel<D>;
-    int rc = ensure_smem_attr(kernel, PrefixCfg<D>::kSmem);
+    using K = PrefixKernel<D>;
+    auto kernel = K::fn();
+    int rc = ensure_smem_attr(kernel, K::kSmem);
     if (rc != PA_OK) return rc;
     DeviceInfo di;
     if ((rc = device_info(&di)) != PA_OK) return rc;
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, PrefixCfg<D>::kThreads,
-                                                                  PrefixCfg<D>::kSmem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, K::kThreads, K::kSmem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     const int64_t wave = static_cast<int64_t>(di.sms) * (per_sm > 0 ? per_sm : 1);
     const int64_t per_split = static_cast<int64_t>(P.num_kv_heads) * plan->prefix_row_tiles;
@@ -551,8 +572,9 @@ int choose_prefix_splits(const DecodeParams& P, Plan* plan) {
 
 template <int D>
 int launch_prefix(const DecodeParams& P, const Plan& plan, cudaStream_t st) {
-    auto kernel = decode_prefix_mma_kernel<D>;
-    int rc = ensure_smem_attr(kernel, PrefixCfg<D>::kSmem);
+    using K = PrefixKernel<D>;
+    auto kernel = K::fn();
+    int rc = ensure_smem_attr(kernel, K::kSmem);
     if (rc != PA_OK) return rc;
     const int64_t rows = static_cast<int64_t>(P.num_blocks) * P.num_kv_heads * kBlockTokens;
     alignas(64) CUtensorMap mk, mv;
@@ -578,9 +600,8 @@ int launch_prefix(const DecodeParams& P, const Plan& plan, cudaStream_t st) {
     PP.scale_log2 = P.scale_log2;
     const dim3 grid(static_cast<unsigned>(plan.prefix_row_tiles) * plan.prefix_splits,
                     static_cast<unsigned>(P.num_kv_heads));
-    cudaError_t e = launch_pdl(kernel, grid, dim3(PrefixCfg<D>::kThreads), PrefixCfg<D>::kSmem, st,
-                               mk, mv, PP);
-    return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode_prefix_mma_kernel launch");
+    cudaError_t e = launch_pdl(kernel, grid, dim3(K::kThreads), K::kSmem, st, mk, mv, PP);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, K::kName);
 }
 
 template <typename OutT, int D>
