@@ -232,13 +232,14 @@ Plan make_plan(int32_t max_seq_len, int32_t partition_blocks) {
 // device (choose_prefix_splits).
 constexpr int32_t kMaxPrefixSplits = 16;
 
-// The shared-prefix kernel: tcgen05 with TMEM accumulators (128 query rows per
-// CTA), or the mma.sync kernel (64 rows per CTA) when built with PA_PREFIX_TC=0.
+// The shared-prefix kernel: tcgen05 with TMEM accumulators (two tiles of 128
+// query rows per CTA), or the mma.sync kernel (64 rows per CTA) when built
+// with PA_PREFIX_TC=0.
 #ifndef PA_PREFIX_TC
 #define PA_PREFIX_TC 1
 #endif
 constexpr bool kPrefixTc = PA_PREFIX_TC != 0;
-constexpr int kPrefixTileRows = kPrefixTc ? PrefixTcCfg<128>::kRows : kPrefixRows;
+constexpr int kPrefixTileRows = kPrefixTc ? PrefixTcCfg<128>::kRows : kPrefixRows;  // query rows per CTA
 
 template <int D>
 struct PrefixKernel {

@@ -6,31 +6,34 @@
 // KV-Speicherzuweisung für LLMs?", slavadubrov.com, §"Gemeinsame Nutzung
 // erfordert mehr als Speicherzuweisung"; "PagedAttention et vLLM",
 // aiunderstanding.org, §"Questions fréquemment posées") attend to the prefix
-// keys, which are read once per CTA for 128 rows.  S = Q K^T and O += P V are
-// real matrix products here (M = 128 query rows, N = 128 keys or D dims), so
+// keys, which are read once per CTA for 256 rows.  S = Q K^T and O += P V are
+// real matrix products here (M = 128 query rows, N = 64 keys or D dims), so
 // they run as tcgen05.mma with the accumulators in TMEM:
 //
-//  * one CTA per SM: 128 query rows (TMEM lanes) x one key split; 10 warps.
-//    Warps 0-7: two threads per query row.  Warp w reaches TMEM lanes
-//    32 (w mod 4) .. +31 (its rows) and takes half w / 4 of each step's keys
-//    and of O's columns.  They load Q into shared memory, run the online
-//    softmax of their row half straight from TMEM (tcgen05.ld gives a thread
-//    its own row: the max and sum of a half need no shuffles; the two halves
-//    swap their maxima through shared memory once per step), write P as bf16
-//    into shared memory, rescale their half of O in TMEM when the row max
-//    moved, and finally write the split's partial (m, l, acc).
-//    Warp 8: TMA producer; 4 blocks (64 keys) of K and V per stage, a ring of
-//    PA_PREFIX_TC_STAGES stages (4 by default, 128 KB): each CTA keeps enough
-//    bytes in flight to cover the load latency.  It starts as soon as the
-//    barriers exist, while the softmax warps load Q.
-//    Warp 9: allocates TMEM and issues the MMAs from one thread.
-//  * TMEM: S in two buffers of 64 columns (the MMA of step j+1 runs while the
-//    softmax of step j reads the other), O in D columns; 256 columns.
+//  * one CTA per SM: two tiles of 128 query rows (each tile's rows are the
+//    TMEM lanes of its own columns) x one key split; 18 warps.  Both tiles use
+//    every K/V stage, so the TMA boxes per query row are halved.
+//    Warps 0-15: two threads per query row.  Warp w serves tile w / 8, reaches
+//    TMEM lanes 32 (w mod 4) .. +31 (its rows) and takes half (w / 4) mod 2 of
+//    each step's keys and of O's columns.  They load Q into shared memory,
+//    run the online softmax of their row half straight from TMEM (tcgen05.ld
+//    gives a thread its own row: the max and sum of a half need no shuffles;
+//    the two halves swap their maxima through shared memory once per step,
+//    one named barrier per tile), write P as bf16 into shared memory, rescale
+//    their half of O in TMEM when the row max moved, and finally write the
+//    split's partial (m, l, acc).
+//    Warp 16: TMA producer; 4 blocks (64 keys) of K and V per stage, a ring of
+//    PA_PREFIX_TC_STAGES stages (3 by default, 96 KB).  It starts as soon as
+//    the barriers exist, while the softmax warps load Q.
+//    Warp 17: allocates TMEM and issues the MMAs from one thread.
+//  * TMEM, per tile: S in two buffers of 64 columns (the MMA of step j+1 runs
+//    while the softmax of step j reads the other), O in D columns; 512
+//    columns in all.
 //  * shared memory operands all use the 128-byte swizzle (rows of 128 bytes,
 //    16-byte chunk c of row r at c ^ (r mod 8), 1 KB atoms of 8 rows): Q and K
 //    K-major for S, P K-major and V MN-major for O.
-//  * mbarriers: full/empty per stage (TMA <-> MMA), s_full per S buffer
-//    (tcgen05.commit -> softmax), p_full (128 softmax arrivals -> MMA),
+//  * mbarriers: full/empty per stage (TMA <-> MMA); per tile s_full per S
+//    buffer (tcgen05.commit -> softmax), p_full (256 softmax arrivals -> MMA),
 //    o_done (tcgen05.commit after each P V -> softmax).  Every wait is
 //    bounded; on timeout the CTA flags PA_DEVERR_TIMEOUT, drains what it
 //    issued and still frees its TMEM.
@@ -46,34 +49,47 @@ namespace pa {
 
 template <int D>
 struct PrefixTcCfg {
-    static constexpr int kRows = 128;                  // query rows per CTA = TMEM lanes
-    static constexpr int kKeys = 64;                   // keys per step
-    static constexpr int kStepBlocks = kKeys / kBlockTokens;
-    static constexpr int kSlabs = D / 64;              // 64-dim slabs (128-byte rows)
-    static constexpr int kQBytes = kSlabs * kRows * 128;
-    static constexpr int kKVSlab = kKeys * 128;        // one slab of K (or V) for a step
-    static constexpr int kStageBytes = 2 * kSlabs * kKVSlab;  // K slabs, then V slabs
+// One tile per CTA measured fastest (two tiles halve the K/V boxes per row
+// but double the softmax work per SM, which is what bounds the kernel).
+#ifndef PA_PREFIX_TC_TILES
+#define PA_PREFIX_TC_TILES 1
+#endif
 #ifndef PA_PREFIX_TC_STAGES
 #define PA_PREFIX_TC_STAGES 4
 #endif
+    static constexpr int kTiles = PA_PREFIX_TC_TILES;  // 128-row query tiles sharing each K/V stage
+    static constexpr int kTileRows = 128;              // rows of a tile = TMEM lanes
+    static constexpr int kRows = kTiles * kTileRows;   // query rows per CTA
+    static constexpr int kKeys = 64;                   // keys per step
+    static constexpr int kStepBlocks = kKeys / kBlockTokens;
+    static constexpr int kSlabs = D / 64;              // 64-dim slabs (128-byte rows)
+    static constexpr int kQBytes = kSlabs * kTileRows * 128;  // Q of one tile
+    static constexpr int kKVSlab = kKeys * 128;        // one slab of K (or V) for a step
+    static constexpr int kStageBytes = 2 * kSlabs * kKVSlab;  // K slabs, then V slabs
     static constexpr int kStages = PA_PREFIX_TC_STAGES;
-    static constexpr int kPBytes = (kKeys / 64) * kRows * 128;
-    static constexpr int kSoftmaxWarps = 8;            // two per TMEM lane quarter
-    static constexpr int kProducerWarp = 8, kMmaWarp = 9;
-    static constexpr int kThreads = 10 * 32;
-    static constexpr uint32_t kTmemCols = 256;         // S0 | S1 | O
+    static constexpr int kPBytes = kTileRows * 128;   // P of one tile (64 keys of bf16 per row)
+    static constexpr int kSoftmaxWarps = 8 * kTiles;  // two per TMEM lane quarter and tile
+    static constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
+    static constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+    // per tile: S0 | S1 | O; 256 columns each
+    static constexpr uint32_t kTileCols = 256;
+    static constexpr uint32_t kTmemCols = kTiles * kTileCols;
     static constexpr uint32_t kColS = 0, kColO = 2 * kKeys;
-    static constexpr int kBars = 2 * kStages + 2 + 4;  // full, empty, s_full x2, p_full, o_done, drain, q_ready
-    // exchange between the two halves of a row: [3][2 halves][128 rows]
+    // full, empty per stage; s_full x2, p_full, o_done per tile; drain, q_ready
+    static constexpr int kBars = 2 * kStages + 4 * kTiles + 2;
+    // exchange between the two halves of a row, per tile: [3][2 halves][128 rows]
     // (maxima of even / odd steps, then the row sums)
-    static constexpr int kXBytes = 3 * 2 * kRows * 4;
+    static constexpr int kXBytes = 3 * 2 * kTileRows * 4;
     // at least 120 KB so that one CTA fills an SM (its TMEM request never waits)
-    static constexpr size_t kSmemUsed =
-        1024 + kQBytes + kStages * kStageBytes + kPBytes + kXBytes + 8 * kBars + 16 + 8 * kStages;
+    static constexpr size_t kSmemUsed = 1024 + kTiles * kQBytes + kStages * kStageBytes + kTiles * kPBytes +
+                                        kTiles * kXBytes + 8 * kBars + 16 + 8 * kStages;
     static constexpr size_t kSmem = kSmemUsed > (120u << 10) ? kSmemUsed : (120u << 10);
-    static_assert(kColO + D <= kTmemCols, "TMEM columns");
-    static_assert(kKeys == 64, "one 128-byte P slab per row");
+    static_assert(kColO + D <= kTileCols, "TMEM columns");
+    static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation");
+    static_assert(kKeys == 64, "one 128-byte P row per query row");
     static_assert(kSmem <= 227u * 1024u, "shared memory per CTA");
+    static_assert(kTiles * kQBytes + kStages * kStageBytes >= kSoftmaxWarps * 32 * (D / 2) * 4,
+                  "epilogue staging fits in Q and the ring");
 };
 
 // ------------------------------------------------------------------ tcgen05 helpers
@@ -169,9 +185,9 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Named barrier over the softmax warps only.
-__device__ __forceinline__ void softmax_bar_sync(int nthreads) {
-    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+// Named barrier `id` (1.. : barrier 0 is __syncthreads) over `nthreads` softmax threads.
+__device__ __forceinline__ void softmax_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ... and the store, which has read its registers when the statement ends.
@@ -215,9 +231,12 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, const PrefixParams P) {
     using Cfg = PrefixTcCfg<D>;
     constexpr int S = Cfg::kStages;
-    constexpr int kHalfKeys = Cfg::kKeys / 2;  // keys of a step per softmax thread
-    constexpr int kHalfD = D / 2;              // O columns per softmax thread
+    constexpr int T = Cfg::kTiles;
+    constexpr int kHalfKeys = Cfg::kKeys / 2;      // keys of a step per softmax thread
+    constexpr int kHalfD = D / 2;                  // O columns per softmax thread
+    constexpr int kTileThreads = 8 * 32;           // softmax threads of one tile
     constexpr int kSoftmaxThreads = Cfg::kSoftmaxWarps * 32;
+    static_assert(T == 1 || T == 2, "one or two query tiles");
 
     grid_dependency_wait();
     allow_dependents();
@@ -225,25 +244,28 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+    // layout: Q[T] | ring[S] | P[T] | exchange[T] | barriers | TMEM address, stage masks
     const uint32_t q_u32 = smem_u32(smem);
-    const uint32_t ring_u32 = q_u32 + Cfg::kQBytes;
+    const uint32_t ring_u32 = q_u32 + T * Cfg::kQBytes;
     const uint32_t p_u32 = ring_u32 + S * Cfg::kStageBytes;
-    uint8_t* p_smem = smem + Cfg::kQBytes + S * Cfg::kStageBytes;
-    float* xchg = reinterpret_cast<float*>(p_smem + Cfg::kPBytes);  // [3][2][kRows]
-    const uint32_t bars_u32 = p_u32 + Cfg::kPBytes + Cfg::kXBytes;
-    const uint32_t full_u32 = bars_u32;               // [S]
-    const uint32_t empty_u32 = bars_u32 + 8 * S;      // [S]
-    const uint32_t sfull_u32 = bars_u32 + 16 * S;     // [2]
-    const uint32_t pfull_u32 = sfull_u32 + 16;
-    const uint32_t odone_u32 = pfull_u32 + 8;
-    const uint32_t drain_u32 = odone_u32 + 8;
+    uint8_t* ring_smem = smem + T * Cfg::kQBytes;
+    uint8_t* p_smem = ring_smem + S * Cfg::kStageBytes;
+    float* xchg_all = reinterpret_cast<float*>(p_smem + T * Cfg::kPBytes);
+    const uint32_t bars_u32 = p_u32 + T * Cfg::kPBytes + T * Cfg::kXBytes;
+    const uint32_t full_u32 = bars_u32;                // [S]
+    const uint32_t empty_u32 = bars_u32 + 8 * S;       // [S]
+    const uint32_t tile_bars_u32 = bars_u32 + 16 * S;  // per tile: s_full[2], p_full, o_done
+    const uint32_t drain_u32 = tile_bars_u32 + 32 * T;
     const uint32_t qready_u32 = drain_u32 + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (qready_u32 + 8 - q_u32));
     uint32_t* stage_present = tmem_slot + 2;  // [S]: blocks of the stage that were loaded
+    auto sfull_of = [&](int t, int b) { return tile_bars_u32 + 32 * t + 8 * b; };
+    auto pfull_of = [&](int t) { return tile_bars_u32 + 32 * t + 16; };
+    auto odone_of = [&](int t) { return tile_bars_u32 + 32 * t + 24; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y;
-    const int tile = blockIdx.x % P.row_tiles;
+    const int tile = blockIdx.x % P.row_tiles;  // a group of T tiles of 128 rows
     const int split = blockIdx.x / P.row_tiles;
     const int jbeg = split * P.split_blocks;
     const int jend = min(P.shared_blocks, jbeg + P.split_blocks);
@@ -251,11 +273,12 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int nsteps = (nblk + Cfg::kStepBlocks - 1) / Cfg::kStepBlocks;
     const int g = P.group;
     const int rows_total = P.num_seqs * g;
+    const int64_t check_me = static_cast<int64_t>(blockIdx.y * gridDim.x + blockIdx.x) * 64 + threadIdx.x -
+                             Cfg::kProducerWarp * 32;
+    const int64_t check_n = static_cast<int64_t>(gridDim.x) * gridDim.y * 64;
 
     if (nsteps == 0) {  // (uniform over the CTA: nothing allocated yet)
-        if (threadIdx.x >= 256)
-            check_prefix_tables(P, (blockIdx.y * gridDim.x + blockIdx.x) * 64 + threadIdx.x - 256,
-                                static_cast<int64_t>(gridDim.x) * gridDim.y * 64);
+        if (warp >= Cfg::kProducerWarp) check_prefix_tables(P, check_me, check_n);
         return;
     }
 
@@ -264,10 +287,12 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
             mbar_init(full_u32 + 8 * st, 1);
             mbar_init(empty_u32 + 8 * st, 1);
         }
-        mbar_init(sfull_u32, 1);
-        mbar_init(sfull_u32 + 8, 1);
-        mbar_init(pfull_u32, kSoftmaxThreads);
-        mbar_init(odone_u32, 1);
+        for (int t = 0; t < T; ++t) {
+            mbar_init(sfull_of(t, 0), 1);
+            mbar_init(sfull_of(t, 1), 1);
+            mbar_init(pfull_of(t), kTileThreads);
+            mbar_init(odone_of(t), 1);
+        }
         mbar_init(drain_u32, 1);
         mbar_init(qready_u32, kSoftmaxThreads);
         fence_barrier_init();
@@ -279,31 +304,33 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // softmax threads: row of the tile (= TMEM lane) and half of the keys / of O
+    // softmax threads: tile, row of the tile (= TMEM lane), half of the keys / of O
     const bool is_softmax = warp < Cfg::kSoftmaxWarps;
+    const int tl = warp >> 3;
     const int row = 32 * (warp & 3) + lane;
     const int hf = (warp >> 2) & 1;
-    const int r = tile * Cfg::kRows + row;
+    const int r = (tile * T + tl) * Cfg::kTileRows + row;
     const bool row_ok = is_softmax && r < rows_total;
     const size_t qrow = row_ok ? static_cast<size_t>(r / g) * P.num_q_heads + h * g + r % g : 0;
     if (is_softmax) {
         // this thread's half of the Q row into shared memory (K-major, 128-byte
         // swizzle), while the producer already streams K and V
+        uint8_t* qt = smem + tl * Cfg::kQBytes;
         const uint4* q = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(P.q) + qrow * D);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
             const int cc = hf * (D / 16) + k;  // 16-byte chunk of the row
-            const int s = cc >> 3, c = cc & 7;
+            const int sl = cc >> 3, c = cc & 7;
             const uint4 v = row_ok ? __ldg(q + cc) : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(smem + s * Cfg::kRows * 128 + row * 128 + ((c ^ (row & 7)) << 4)) = v;
+            *reinterpret_cast<uint4*>(qt + sl * Cfg::kTileRows * 128 + row * 128 + ((c ^ (row & 7)) << 4)) = v;
         }
         fence_proxy_async_smem();  // generic writes, read by the tensor cores
         mbar_arrive(qready_u32);
     }
 
     if (warp == Cfg::kProducerWarp) {
-        // ---------------- producer: 8 blocks of K and V per stage
-        const uint64_t policy = l2_policy_evict_last();  // every row tile of this head reads them
+        // ---------------- producer: 4 blocks of K and V per stage
+        const uint64_t policy = l2_policy_evict_last();  // every tile group of this head reads them
         int issued = 0;
         // table entries of the split, 32 at a time: lane l holds block
         // win + l (-1 where absent or outside the pool); the next window is
@@ -342,18 +369,17 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const int b = c / (Cfg::kSlabs * kBlockTokens * 8);
                     if ((present >> b) & 1u) continue;
                     const int rem = c % (Cfg::kSlabs * kBlockTokens * 8);
-                    const int s = rem / (kBlockTokens * 8), rr = rem % (kBlockTokens * 8);
+                    const int sl = rem / (kBlockTokens * 8), rr = rem % (kBlockTokens * 8);
                     const int t = b * kBlockTokens + rr / 8;
-                    *reinterpret_cast<uint4*>(smem + (sbase - q_u32) + (Cfg::kSlabs + s) * Cfg::kKVSlab + t * 128 +
-                                              (rr % 8) * 16) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(ring_smem + st * Cfg::kStageBytes + (Cfg::kSlabs + sl) * Cfg::kKVSlab +
+                                              t * 128 + (rr % 8) * 16) = make_uint4(0, 0, 0, 0);
                 }
                 fence_proxy_async_smem();
             }
             __syncwarp();
             if (lane == 0) {
                 stage_present[st] = present;  // read by the softmax after this barrier's phase
-                const uint32_t bar = full_u32 + 8 * st;
-                mbar_arrive_expect_tx(bar, __popc(present) * 2 * Cfg::kSlabs * 2048);
+                mbar_arrive_expect_tx(full_u32 + 8 * st, __popc(present) * 2 * Cfg::kSlabs * 2048);
             }
 #pragma unroll
             for (int b = 0; b < Cfg::kStepBlocks; ++b) {
@@ -362,11 +388,11 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const int32_t trow = (pbb * P.num_kv_heads + h) * kBlockTokens;
                     const uint32_t bar = full_u32 + 8 * st;
 #pragma unroll
-                    for (int s = 0; s < Cfg::kSlabs; ++s) {
-                        tma_load_2d(sbase + s * Cfg::kKVSlab + b * kBlockTokens * 128, &tmap_k, s * 64, trow, bar,
+                    for (int sl = 0; sl < Cfg::kSlabs; ++sl) {
+                        tma_load_2d(sbase + sl * Cfg::kKVSlab + b * kBlockTokens * 128, &tmap_k, sl * 64, trow, bar,
                                     policy);
-                        tma_load_2d(sbase + (Cfg::kSlabs + s) * Cfg::kKVSlab + b * kBlockTokens * 128, &tmap_v,
-                                    s * 64, trow, bar, policy);
+                        tma_load_2d(sbase + (Cfg::kSlabs + sl) * Cfg::kKVSlab + b * kBlockTokens * 128, &tmap_v,
+                                    sl * 64, trow, bar, policy);
                     }
                 }
             }
@@ -381,21 +407,26 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     } else if (warp == Cfg::kMmaWarp) {
         // ---------------- MMA issue (one thread)
         if (lane == 0) {
-            constexpr uint32_t kIdescS = umma_idesc_bf16(Cfg::kRows, Cfg::kKeys, 0);
-            constexpr uint32_t kIdescO = umma_idesc_bf16(Cfg::kRows, D, 1);
+            constexpr uint32_t kIdescS = umma_idesc_bf16(Cfg::kTileRows, Cfg::kKeys, 0);
+            constexpr uint32_t kIdescO = umma_idesc_bf16(Cfg::kTileRows, D, 1);
             auto issue_s = [&](int j) -> bool {
                 const int st = j % S;
                 if (!mbar_wait_bounded_thread(full_u32 + 8 * st, (j / S) & 1u)) return false;
                 tc_fence_after();
                 const uint32_t kb = ring_u32 + st * Cfg::kStageBytes;
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks % 4) * 32u;  // k-step within the 128-byte row
-                    const uint64_t a = umma_desc_sw128(q_u32 + (ks / 4) * Cfg::kRows * 128 + off, 16, 1024);
-                    const uint64_t b = umma_desc_sw128(kb + (ks / 4) * Cfg::kKVSlab + off, 16, 1024);
-                    umma_bf16(tmem + Cfg::kColS + (j & 1) * Cfg::kKeys, a, b, kIdescS, ks > 0);
+                for (int t = 0; t < T; ++t) {
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t off = (ks % 4) * 32u;  // k-step within the 128-byte row
+                        const uint64_t a = umma_desc_sw128(
+                            q_u32 + t * Cfg::kQBytes + (ks / 4) * Cfg::kTileRows * 128 + off, 16, 1024);
+                        const uint64_t b = umma_desc_sw128(kb + (ks / 4) * Cfg::kKVSlab + off, 16, 1024);
+                        umma_bf16(tmem + t * Cfg::kTileCols + Cfg::kColS + (j & 1) * Cfg::kKeys, a, b, kIdescS,
+                                  ks > 0);
+                    }
+                    umma_commit(sfull_of(t, j & 1));
                 }
-                umma_commit(sfull_u32 + 8 * (j & 1));
                 return true;
             };
             bool ok = mbar_wait_bounded_thread(qready_u32, 0);
@@ -405,16 +436,20 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             for (int j = 0; j < nsteps && ok; ++j) {
                 if (j + 1 < nsteps && !(ok = issue_s(j + 1))) break;
-                if (!(ok = mbar_wait_bounded_thread(pfull_u32, j & 1u))) break;
-                tc_fence_after();
                 const uint32_t vb = ring_u32 + (j % S) * Cfg::kStageBytes + Cfg::kSlabs * Cfg::kKVSlab;
 #pragma unroll
-                for (int ks = 0; ks < Cfg::kKeys / 16; ++ks) {
-                    const uint64_t a = umma_desc_sw128(p_u32 + ks * 32u, 16, 1024);
-                    const uint64_t b = umma_desc_sw128(vb + ks * 16 * 128, Cfg::kKVSlab, 1024);
-                    umma_bf16(tmem + Cfg::kColO, a, b, kIdescO, j > 0 || ks > 0);
+                for (int t = 0; t < T; ++t) {
+                    if (!(ok = mbar_wait_bounded_thread(pfull_of(t), j & 1u))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < Cfg::kKeys / 16; ++ks) {
+                        const uint64_t a = umma_desc_sw128(p_u32 + t * Cfg::kPBytes + ks * 32u, 16, 1024);
+                        const uint64_t b = umma_desc_sw128(vb + ks * 16 * 128, Cfg::kKVSlab, 1024);
+                        umma_bf16(tmem + t * Cfg::kTileCols + Cfg::kColO, a, b, kIdescO, j > 0 || ks > 0);
+                    }
+                    umma_commit(odone_of(t));
                 }
-                umma_commit(odone_u32);
+                if (!ok) break;
                 umma_commit(empty_u32 + 8 * (j % S));
             }
             if (!ok) flag_error(PA_DEVERR_TIMEOUT);
@@ -426,10 +461,14 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     } else {
         // ---------------- softmax: two threads per query row (keys and O split in halves)
         // Every softmax thread runs all nsteps steps and takes every named
-        // barrier, so that the halves of a row stay paired whatever happens; a
-        // wait that gives up marks the warp dead (warp-uniform), and a dead
-        // warp skips its tensor-memory work and its arrivals.
-        const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp & 3) * 32u) << 16);
+        // barrier of its tile, so that the halves of a row stay paired
+        // whatever happens; a wait that gives up marks the warp dead
+        // (warp-uniform), and a dead warp skips its tensor-memory work and its
+        // arrivals.
+        const uint32_t lane_base = tmem + tl * Cfg::kTileCols + ((static_cast<uint32_t>(warp & 3) * 32u) << 16);
+        uint8_t* p_tile = p_smem + tl * Cfg::kPBytes;
+        float* xchg = xchg_all + tl * (Cfg::kXBytes / 4);
+        const int bar_id = 1 + tl;
         const float sl2 = P.scale_log2;
         float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
         bool ok = true;
@@ -437,7 +476,7 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int st = j % S;
             // S of this step is in TMEM; the stage's block mask was published
             // with the stage's load barrier (already complete)
-            ok = ok && mbar_wait_bounded(sfull_u32 + 8 * (j & 1), (j >> 1) & 1u);
+            ok = ok && mbar_wait_bounded(sfull_of(tl, j & 1), (j >> 1) & 1u);
             ok = ok && mbar_wait_bounded(full_u32 + 8 * st, (j / S) & 1u);
             tc_fence_after();
             float x[kHalfKeys];
@@ -445,36 +484,38 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (ok) {
                 const uint32_t present = stage_present[st] >> (hf * kHalfKeys / kBlockTokens);
                 tmem_ld32(lane_base + Cfg::kColS + (j & 1) * Cfg::kKeys + hf * kHalfKeys, x);
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent chains
 #pragma unroll
                 for (int i = 0; i < kHalfKeys; ++i) {
                     x[i] = ((present >> (i / kBlockTokens)) & 1u) ? x[i] * sl2 : -INFINITY;
-                    mx = fmaxf(mx, x[i]);
+                    m4[i & 3] = fmaxf(m4[i & 3], x[i]);
                 }
+                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             } else {
 #pragma unroll
                 for (int i = 0; i < kHalfKeys; ++i) x[i] = -INFINITY;
             }
             // the row max over both halves
-            float* xs = xchg + (j & 1) * 2 * Cfg::kRows;
-            xs[hf * Cfg::kRows + row] = mx;
-            softmax_bar_sync(kSoftmaxThreads);
-            mx = fmaxf(mx, xs[(1 - hf) * Cfg::kRows + row]);
+            float* xs = xchg + (j & 1) * 2 * Cfg::kTileRows;
+            xs[hf * Cfg::kTileRows + row] = mx;
+            softmax_bar_sync(bar_id, kTileThreads);
+            mx = fmaxf(mx, xs[(1 - hf) * Cfg::kTileRows + row]);
             const float mn = fmaxf(m, mx);
             const float mu = mn == -INFINITY ? 0.0f : mn;
             const float alpha = fast_exp2(m - mu);
             m = mn;
             // P as bf16 pairs; the denominator sums the rounded weights
             uint32_t pw[kHalfKeys / 2];
-            float sum = 0.f;
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
             for (int i = 0; i < kHalfKeys / 2; ++i) {
                 pw[i] = pack2<false>(fast_exp2(x[2 * i] - mu), fast_exp2(x[2 * i + 1] - mu));
-                sum += __uint_as_float(pw[i] << 16) + __uint_as_float(pw[i] & 0xffff0000u);
+                s4[i & 3] += __uint_as_float(pw[i] << 16) + __uint_as_float(pw[i] & 0xffff0000u);
             }
-            l = l * alpha + sum;
+            l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
             if (j > 0) {
                 // P V of the previous step is done: the P buffer is free, O holds the sum up to it
-                ok = ok && mbar_wait_bounded(odone_u32, (j - 1) & 1u);
+                ok = ok && mbar_wait_bounded(odone_of(tl), (j - 1) & 1u);
                 tc_fence_after();
                 if (ok && __any_sync(kFullMask, alpha != 1.f)) {
 #pragma unroll
@@ -493,20 +534,23 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
                 for (int c = 0; c < kHalfKeys / 8; ++c) {
                     const int cc = hf * (kHalfKeys / 8) + c;
-                    *reinterpret_cast<uint4*>(p_smem + row * 128 + ((cc ^ (row & 7)) << 4)) =
+                    *reinterpret_cast<uint4*>(p_tile + row * 128 + ((cc ^ (row & 7)) << 4)) =
                         make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                mbar_arrive(pfull_u32);
+                mbar_arrive(pfull_of(tl));
             }
         }
         // the row sum over both halves (its own buffer: the partner may still
         // read the last step's maximum)
-        xchg[4 * Cfg::kRows + hf * Cfg::kRows + row] = l;
-        softmax_bar_sync(kSoftmaxThreads);
-        l += xchg[4 * Cfg::kRows + (1 - hf) * Cfg::kRows + row];
-        ok = ok && mbar_wait_bounded(odone_u32, (nsteps - 1) & 1u);
+        xchg[4 * Cfg::kTileRows + hf * Cfg::kTileRows + row] = l;
+        softmax_bar_sync(bar_id, kTileThreads);
+        l += xchg[4 * Cfg::kTileRows + (1 - hf) * Cfg::kTileRows + row];
+        ok = ok && mbar_wait_bounded(odone_of(tl), (nsteps - 1) & 1u);
+        // the last tile's last commit covers every MMA the CTA issued: after
+        // it, Q and the ring are idle and serve as staging below
+        ok = ok && mbar_wait_bounded(odone_of(T - 1), (nsteps - 1) & 1u);
         if (ok) {
             tc_fence_after();
             // the split's partial of this row: m, l by half 0; each half its O columns
@@ -516,12 +560,12 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 P.ws_m[idx] = m * kLn2;
                 P.ws_l[idx] = l;
             }
-            // the warp's 32 half-rows go through shared memory (the ring is
-            // idle now: every MMA has completed) so that each store instruction
+            // the warp's 32 half-rows go through shared memory (Q and the ring
+            // are idle now) so that each store instruction
             // writes one contiguous half-row; 16-byte chunk c of lane l's
             // half-row sits at c ^ (l mod 16)
             constexpr int kChunks = kHalfD / 4;  // 16-byte chunks of a half-row
-            float* stage = reinterpret_cast<float*>(smem + Cfg::kQBytes) + warp * 32 * kHalfD;
+            float* stage = reinterpret_cast<float*>(smem) + warp * 32 * kHalfD;
 #pragma unroll
             for (int c = 0; c < kHalfD / 32; ++c) {
                 float v[32];
@@ -550,8 +594,7 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
     }
 
-    if (!is_softmax) check_prefix_tables(P, (blockIdx.y * gridDim.x + blockIdx.x) * 64 + threadIdx.x - 256,
-                                         static_cast<int64_t>(gridDim.x) * gridDim.y * 64);
+    if (!is_softmax) check_prefix_tables(P, check_me, check_n);
     tc_fence_before();
     __syncthreads();
     if (warp == Cfg::kMmaWarp) {
