@@ -265,6 +265,33 @@ def test_shared_prefix_preconditions_are_flagged():
     assert pa.device_error() & pa.PA_DEVERR_PREFIX
 
 
+def test_shared_prefix_block_outside_the_pool_is_masked_and_flagged():
+    """A shared block id outside the pool (in every table, so the prefix stays
+    shared): flagged, its tokens take no part, the rest is exact attention."""
+    lens = [160 + x for x in (40, 3, 97)]
+    w = wl.build(lens, 8, 2, 128, torch.bfloat16, seed=91, device=DEV, prefix_len=160, poison_unused=True)
+    bt = w.block_tables.clone()
+    bt[:, 3] = w.num_blocks + 7
+    out = pa.decode_shared_prefix(w.q, w.k_cache, w.v_cache, bt, w.seq_lens, w.scale, w.shared_prefix_blocks,
+                                  max_seq_len=w.max_seq_len)
+    torch.cuda.synchronize()
+    assert pa.device_error() & pa.PA_DEVERR_BLOCK_OOB
+    assert torch.isfinite(out.float()).all()
+    h = host(w)
+    for s, L in enumerate(lens):
+        keep = [t for t in range(L) if t // 16 != 3]
+        nb = -(-len(keep) // 16)
+        packed_k = np.zeros((nb, 2, 16, 128), np.uint16)
+        packed_v = np.zeros_like(packed_k)
+        for i, t in enumerate(keep):
+            b = w.tables_host[s][t // 16]
+            packed_k[i // 16, :, i % 16] = h["kc"][b, :, t % 16]
+            packed_v[i // 16, :, i % 16] = h["vc"][b, :, t % 16]
+        ref = oracle.paged_decode(h["q"][s:s + 1], packed_k, packed_v, np.arange(nb, dtype=np.int32)[None, :],
+                                  np.array([len(keep)], np.int32), w.scale)
+        assert_close(to_f64(out)[s:s + 1], ref, torch.bfloat16, f"seq {s} without the bad shared block")
+
+
 # ------------------------------------------------------------------ the two steps separately
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_partition_partials_match_oracle(dtype):
