@@ -53,13 +53,26 @@ constexpr int kMaxDevices = 64;
 #ifndef PA_MMA_MIN_CTAS_FP8
 #define PA_MMA_MIN_CTAS_FP8 2
 #endif
+// E4M3 with <= 8 query rows runs the transposed products, which hold far
+// fewer registers: four CTAs per SM, each warp with a 2-stage ring (measured
+// faster than 3 or 4 stages at 3-4 CTAs)
+#ifndef PA_MMA_STAGES_FP8_T
+#define PA_MMA_STAGES_FP8_T 2
+#endif
+#ifndef PA_MMA_MIN_CTAS_FP8_T
+#define PA_MMA_MIN_CTAS_FP8_T 4
+#endif
 constexpr int kMmaWarps = PA_MMA_WARPS;
 constexpr int kMmaStages = PA_MMA_STAGES;
 constexpr int kMmaMinCtas = PA_MMA_MIN_CTAS;  // CTAs per SM the register budget must allow
-template <bool FP8>
-constexpr int mma_stages() { return FP8 ? PA_MMA_STAGES_FP8 : kMmaStages; }
-template <bool FP8>
-constexpr int mma_min_ctas() { return FP8 ? PA_MMA_MIN_CTAS_FP8 : kMmaMinCtas; }
+template <bool FP8, int ROWS>
+constexpr int mma_stages() {
+    return !FP8 ? kMmaStages : ROWS <= 8 ? PA_MMA_STAGES_FP8_T : PA_MMA_STAGES_FP8;
+}
+template <bool FP8, int ROWS>
+constexpr int mma_min_ctas() {
+    return !FP8 ? kMmaMinCtas : ROWS <= 8 ? PA_MMA_MIN_CTAS_FP8_T : PA_MMA_MIN_CTAS_FP8;
+}
 
 thread_local char g_last_cuda_error[256] = "no CUDA error recorded";
 
@@ -446,7 +459,7 @@ struct LaunchShape {
 
 template <int D, int ROWS, bool FP8>
 auto mma_kernel() {
-    return decode_bf16_mma_kernel<D, ROWS, mma_stages<FP8>(), kMmaWarps, mma_min_ctas<FP8>(), FP8>;
+    return decode_bf16_mma_kernel<D, ROWS, mma_stages<FP8, ROWS>(), kMmaWarps, mma_min_ctas<FP8, ROWS>(), FP8>;
 }
 
 template <typename K>
@@ -459,7 +472,7 @@ int shape_of(K kernel, int warps, size_t smem, const DecodeParams& P, LaunchShap
 
 template <int D, int ROWS, bool FP8>
 int mma_shape(const DecodeParams& P, LaunchShape* L) {
-    using Cfg = MmaCfg<D, mma_stages<FP8>(), kMmaWarps, FP8>;
+    using Cfg = MmaCfg<D, mma_stages<FP8, ROWS>(), kMmaWarps, FP8>;
     auto kernel = mma_kernel<D, ROWS, FP8>();
     int rc = ensure_smem_attr(kernel, Cfg::smem_bytes(kMaxSeqsPerLaunch));
     if (rc != PA_OK) return rc;

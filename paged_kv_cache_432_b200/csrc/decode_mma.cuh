@@ -50,6 +50,16 @@
 // and its V scale multiplies the accumulators once at the end of the piece,
 // so the result is that of attention over decode(code) * scale.
 //
+// E4M3 with at most 8 query rows (MHA, GQA up to 8 heads per kv head) runs
+// the transposed products S^T = K Q^T and O^T = V^T P^T: the block's 16
+// tokens (for S^T) and 16 head dims (for O^T) fill the MMA's M dimension and
+// the query rows its N = 8, so no register holds padding and each product
+// takes D/16 MMAs instead of D/8.  The widened codes are the A fragments
+// directly (K: token rows, V: even dims in rows 0-7, odd dims in rows 8-15);
+// a row's scores sit in the 8 lanes of equal lane % 4, and four shuffles plus
+// two byte permutes turn P into the B fragment of P^T.  The kernel then fits
+// 128 registers, four CTAs per SM.
+//
 // Every wait on an mbarrier is bounded: on timeout the warp flags
 // PA_DEVERR_TIMEOUT, waits (bounded) for its copies in flight and returns.
 #pragma once
@@ -110,6 +120,25 @@ __device__ __forceinline__ float softmax_update(float& m, float& l, const float 
     return alpha;
 }
 
+// The same for one row of the transposed layout, where the lane holds two of
+// the row's 16 scores (x0: token lane/4, x1: token 8 + lane/4) and the 8
+// lanes of equal lane % 4 hold the rest.  p gets the f16 pair (x0's, x1's
+// weight); l is this lane's share of the row sum.
+__device__ __forceinline__ float softmax_update_col(float& m, float& l, float x0, float x1, uint32_t& p) {
+    float bm = fmaxf(x0, x1);
+    bm = fmaxf(bm, __shfl_xor_sync(kFullMask, bm, 4));
+    bm = fmaxf(bm, __shfl_xor_sync(kFullMask, bm, 8));
+    bm = fmaxf(bm, __shfl_xor_sync(kFullMask, bm, 16));
+    const float mn = fmaxf(m, bm);
+    const float mu = mn == -INFINITY ? 0.0f : mn;  // a row with nothing valid yet
+    const float alpha = fast_exp2(m - mu);
+    p = pack2<true>(fast_exp2(x0 - mu), fast_exp2(x1 - mu));
+    const float2 f = unpack2<true>(p);  // the denominator sums the rounded weights
+    l = l * alpha + (f.x + f.y);
+    m = mn;
+    return alpha;
+}
+
 template <int D, int ROWS, int STAGES, int WARPS, int MIN_CTAS, bool FP8 = false>
 __global__ void __launch_bounds__(WARPS * 32, MIN_CTAS)
 decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
@@ -119,12 +148,17 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     constexpr int NTD = D / 8;      // n-tiles of P V
     constexpr bool HI = ROWS > 8;   // query rows 8..15 in use
     constexpr int AR = HI ? 4 : 2;  // registers per A fragment / per C tile that are held
+    // E4M3 with <= 8 query rows: the transposed products S^T = K Q^T and
+    // O^T = V^T P^T, tokens / head dims in M and the query rows in N
+    constexpr bool TR = FP8 && !HI;
+    constexpr int ACC_N = TR ? D / 16 : NTD;  // accumulator tiles
+    constexpr int ACC_R = TR ? 4 : AR;        // registers held per tile
     // blocks per consumer step (one max / sum reduction and one rescale per
     // step); one measured fastest for both element types
 #ifndef PA_FP8_BLOCKS_PER_STEP
 #define PA_FP8_BLOCKS_PER_STEP 1
 #endif
-    constexpr int BPS = FP8 ? PA_FP8_BLOCKS_PER_STEP : 1;
+    constexpr int BPS = (FP8 && !TR) ? PA_FP8_BLOCKS_PER_STEP : 1;
     static_assert(STAGES >= 2 * BPS, "a step's stages plus as many in flight");
 
     extern __shared__ uint8_t smem_raw[];
@@ -221,6 +255,9 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     const int tq = 2 * (lane & 3);  // first token (S) / first dim (O) of this lane's pair
     const int r_lo = lane >> 2;     // query row within the group
+    // The lane's two rows of S and O: r_lo and r_lo + 8, or, transposed, the
+    // C columns tq and tq + 1 (its Q row stays r_lo, the B-operand column).
+    const int row_a = TR ? tq : r_lo, row_b = TR ? tq + 1 : r_lo + 8;
     const uint32_t sw = lane & 7;   // swizzle term: ldmatrix row index mod 8
     float sl2 = P.scale_log2;  // times the kv head's K scale for E4M3 caches
     float vscale = 1.f;         // the kv head's V scale for E4M3 caches
@@ -232,7 +269,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     bool ok_lo = false, ok_hi = false;
     size_t orow_lo = 0, orow_hi = 0;
     int32_t lim_lo = 0, lim_hi = 0;
-    float acc[NTD][AR];
+    float acc[ACC_N][ACC_R];
 
     while (true) {
         if (cj == cc.jbeg) {  // new piece: load its query rows as A fragments
@@ -242,11 +279,11 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const QRows qr = query_rows(P, cc.s, cc.len);
             if (qr.clamped && cc.p == 0 && lane == 0) flag_error(PA_DEVERR_SEQ_LEN);
             const int rows_used = g * qr.n;
-            const int tok_lo = r_lo / g, tok_hi = (r_lo + 8) / g;
-            ok_lo = r_lo < rows_used;
-            ok_hi = HI && (r_lo + 8 < rows_used);
-            orow_lo = (static_cast<size_t>(qr.base) + tok_lo) * P.num_q_heads + cc.h * g + r_lo % g;
-            orow_hi = (static_cast<size_t>(qr.base) + tok_hi) * P.num_q_heads + cc.h * g + (r_lo + 8) % g;
+            const int tok_lo = row_a / g, tok_hi = row_b / g;
+            ok_lo = row_a < rows_used;
+            ok_hi = (HI || TR) && (row_b < rows_used);
+            orow_lo = (static_cast<size_t>(qr.base) + tok_lo) * P.num_q_heads + cc.h * g + row_a % g;
+            orow_hi = (static_cast<size_t>(qr.base) + tok_hi) * P.num_q_heads + cc.h * g + row_b % g;
             lim_lo = cc.len - qr.n + tok_lo;
             lim_hi = cc.len - qr.n + tok_hi;
             const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(P.q);
@@ -254,12 +291,17 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 // k-step ks covers dims 16ks..16ks+15; the K fragments hold
                 // dims 16ks+2tq..+3 (b0: first pair, b1: second), so the A
                 // fragment takes the same dims: a0/a1 the first pair, a2/a3
-                // the second.  Widened to f16 (exact for |q| in 2^-14..65504).
-                const uint2* q_lo = reinterpret_cast<const uint2*>(qb + (ok_lo ? orow_lo : 0) * D + 2 * tq);
+                // the second.  Transposed, the same registers are the B
+                // fragment of Q^T (row r_lo, the same dims).  Widened to f16
+                // (exact for |q| in 2^-14..65504).
+                const bool ok_q = r_lo < rows_used;
+                const size_t orow_q =
+                    (static_cast<size_t>(qr.base) + r_lo / g) * P.num_q_heads + cc.h * g + r_lo % g;
+                const uint2* q_lo = reinterpret_cast<const uint2*>(qb + (ok_q ? orow_q : 0) * D + 2 * tq);
                 const uint2* q_hi = reinterpret_cast<const uint2*>(qb + (ok_hi ? orow_hi : 0) * D + 2 * tq);
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ++ks) {
-                    const uint2 lo = ok_lo ? __ldg(q_lo + 4 * ks) : make_uint2(0u, 0u);
+                    const uint2 lo = ok_q ? __ldg(q_lo + 4 * ks) : make_uint2(0u, 0u);
                     if constexpr (HI) {
                         const uint2 hi = ok_hi ? __ldg(q_hi + 4 * ks) : make_uint2(0u, 0u);
                         qa[ks][0] = bf16x2_to_f16x2(lo.x);
@@ -292,9 +334,9 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             m_lo = m_hi = -INFINITY;
             l_lo = l_hi = 0.f;
 #pragma unroll
-            for (int n = 0; n < NTD; ++n)
+            for (int n = 0; n < ACC_N; ++n)
 #pragma unroll
-                for (int r = 0; r < AR; ++r) acc[n][r] = 0.f;
+                for (int r = 0; r < ACC_R; ++r) acc[n][r] = 0.f;
         }
 
         // ---- this step: BPS blocks (fewer at the end of the piece); wait for
@@ -344,146 +386,224 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
 
-        // ---- S = Q K^T per block: two n-tiles of 8 tokens, each with two
-        // accumulators (even / odd k-steps) so that the dependent MMA chains
-        // are KSTEPS/2 long
-        float sc[BPS][2][AR];
-#pragma unroll
-        for (int b = 0; b < BPS; ++b) {
-#pragma unroll
-            for (int r = 0; r < AR; ++r) sc[b][0][r] = sc[b][1][r] = 0.f;
-            if (b >= nb) continue;
-            float s0[AR], s1[AR], t0[AR], t1[AR];
-#pragma unroll
-            for (int r = 0; r < AR; ++r) s0[r] = s1[r] = t0[r] = t1[r] = 0.f;
-            const uint32_t kbase = kb[b];
-            if constexpr (FP8) {
-                // E4M3 K: ldmatrix on the codes seen as b16 gives each lane dims
-                // 4(lane%4)..+3 of one token per 16-dim chunk; matrices: (tokens
-                // 0-7, chunk j), (8-15, j), (0-7, j+1), (8-15, j+1)
+        if constexpr (TR) {
+            // ---- S^T = K Q^T: M = the block's 16 tokens, N = the query
+            // rows, K = head dims.  ldmatrix on the codes seen as 16-bit
+            // pairs gives each lane dims 4(lane%4)..+3 of token lane/4 (and of
+            // token 8 + lane/4) per 16-dim chunk: widened, those are the A
+            // fragment, and Q^T takes the same dims (qa).
+            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+            {
                 const int tok = (lane & 7) + 8 * ((lane >> 3) & 1);
 #pragma unroll
                 for (int j = 0; j < KSTEPS; j += 2) {
                     const uint32_t ch = static_cast<uint32_t>(j + (lane >> 4));
-                    uint32_t r0, r1, r2, r3, b0, b1;
-                    ldsm_x4(kbase + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
-                    e4m3x4_to_f16x2x2(r0, b0, b1);
-                    mma_frag_t<true>(s0, qa[j], b0, b1);
-                    e4m3x4_to_f16x2x2(r1, b0, b1);
-                    mma_frag_t<true>(s1, qa[j], b0, b1);
-                    e4m3x4_to_f16x2x2(r2, b0, b1);
-                    mma_frag_t<true>(t0, qa[j + 1], b0, b1);
-                    e4m3x4_to_f16x2x2(r3, b0, b1);
-                    mma_frag_t<true>(t1, qa[j + 1], b0, b1);
-                }
-            } else {
-#pragma unroll
-                for (int kp = 0; kp < KSTEPS / 2; ++kp) {
-                    const int cg = 4 * kp + (lane >> 3);  // 8-element column chunk 0 .. D/8-1
-                    const uint32_t col = (cg >> 3) * Cfg::kRegionBytes + ((((uint32_t)cg & 7u) ^ sw) << 4);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(kbase + col + (lane & 7) * 128, b0, b1, b2, b3);
-                    mma_frag(s0, qa[2 * kp], b0, b1);
-                    mma_frag(t0, qa[2 * kp + 1], b2, b3);
-                    ldsm_x4(kbase + col + (8 + (lane & 7)) * 128, b0, b1, b2, b3);
-                    mma_frag(s1, qa[2 * kp], b0, b1);
-                    mma_frag(t1, qa[2 * kp + 1], b2, b3);
+                    uint32_t r0, r1, r2, r3, l0, h0, l1, h1;
+                    ldsm_x4(kb[0] + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
+                    e4m3x4_to_f16x2x2(r0, l0, h0);  // tokens 0-7, chunk j
+                    e4m3x4_to_f16x2x2(r1, l1, h1);  // tokens 8-15, chunk j
+                    mma_f16(s0, l0, l1, h0, h1, qa[j][0], qa[j][1]);
+                    e4m3x4_to_f16x2x2(r2, l0, h0);  // chunk j + 1
+                    e4m3x4_to_f16x2x2(r3, l1, h1);
+                    mma_f16(s1, l0, l1, h0, h1, qa[j + 1][0], qa[j + 1][1]);
                 }
             }
+            // ---- online softmax: this lane holds tokens r_lo and r_lo + 8
+            // of rows tq (s[0], s[2]) and tq + 1 (s[1], s[3]); a row's 16
+            // tokens sit in the 8 lanes of equal lane % 4
+            const int vis_a = min(valid[0] - 1, lim_lo - cj * kBlockTokens);
+            const int vis_b = min(valid[0] - 1, lim_hi - cj * kBlockTokens);
+            uint32_t pk_a, pk_b;  // f16 pairs (token r_lo, token r_lo + 8) of rows tq, tq + 1
+            const float alpha_lo = softmax_update_col(m_lo, l_lo, r_lo <= vis_a ? (s0[0] + s1[0]) * sl2 : -INFINITY,
+                                          r_lo + 8 <= vis_a ? (s0[2] + s1[2]) * sl2 : -INFINITY, pk_a);
+            const float alpha_hi = softmax_update_col(m_hi, l_hi, r_lo <= vis_b ? (s0[1] + s1[1]) * sl2 : -INFINITY,
+                                          r_lo + 8 <= vis_b ? (s0[3] + s1[3]) * sl2 : -INFINITY, pk_b);
+            if (__any_sync(kFullMask, alpha_lo != 1.f || alpha_hi != 1.f)) {
 #pragma unroll
-            for (int r = 0; r < AR; ++r) {
-                sc[b][0][r] += s0[r] + t0[r];
-                sc[b][1][r] += s1[r] + t1[r];
-            }
-        }
-
-        // ---- online softmax over the step's keys (rows r_lo and r_lo + 8);
-        // key t of block b is visible to a row iff t < valid[b] and
-        // (cj + b)*16 + t <= the row's limit
-        uint32_t plo[BPS][2], phi[BPS][2];  // P as bf16 / f16 pairs: [block][tokens tq.. / 8+tq..]
-        float alpha_lo, alpha_hi = 1.f;
-        {
-            float x[4 * BPS];
-#pragma unroll
-            for (int b = 0; b < BPS; ++b) {
-                const int vis = min(valid[b] - 1, lim_lo - (cj + b) * kBlockTokens);  // last visible key
-                x[4 * b + 0] = tq <= vis ? sc[b][0][0] * sl2 : -INFINITY;
-                x[4 * b + 1] = tq + 1 <= vis ? sc[b][0][1] * sl2 : -INFINITY;
-                x[4 * b + 2] = tq + 8 <= vis ? sc[b][1][0] * sl2 : -INFINITY;
-                x[4 * b + 3] = tq + 9 <= vis ? sc[b][1][1] * sl2 : -INFINITY;
-            }
-            alpha_lo = softmax_update<FP8, BPS>(m_lo, l_lo, x, plo);
-        }
-        if constexpr (HI) {
-            float x[4 * BPS];
-#pragma unroll
-            for (int b = 0; b < BPS; ++b) {
-                const int vis = min(valid[b] - 1, lim_hi - (cj + b) * kBlockTokens);
-                x[4 * b + 0] = tq <= vis ? sc[b][0][2] * sl2 : -INFINITY;
-                x[4 * b + 1] = tq + 1 <= vis ? sc[b][0][3] * sl2 : -INFINITY;
-                x[4 * b + 2] = tq + 8 <= vis ? sc[b][1][2] * sl2 : -INFINITY;
-                x[4 * b + 3] = tq + 9 <= vis ? sc[b][1][3] * sl2 : -INFINITY;
-            }
-            alpha_hi = softmax_update<FP8, BPS>(m_hi, l_hi, x, phi);
-        }
-        // rescale the accumulators only when some row's max moved (alpha is
-        // exactly 1 otherwise): after the first blocks of a sequence it rarely does
-        if (__any_sync(kFullMask, alpha_lo != 1.f || alpha_hi != 1.f)) {
-#pragma unroll
-            for (int n = 0; n < NTD; ++n) {
-                acc[n][0] *= alpha_lo;
-                acc[n][1] *= alpha_lo;
-                if constexpr (HI) {
-                    acc[n][2] *= alpha_hi;
-                    acc[n][3] *= alpha_hi;
+                for (int c = 0; c < ACC_N; ++c) {
+                    acc[c][0] *= alpha_lo;
+                    acc[c][2] *= alpha_lo;
+                    acc[c][1] *= alpha_hi;
+                    acc[c][3] *= alpha_hi;
                 }
             }
-        }
-
-        // ---- O += P V : n-tiles of 8 head dims, K = the 16 tokens of a block
-#pragma unroll
-        for (int b = 0; b < BPS; ++b) {
-            if (b >= nb) continue;
-            uint32_t pa[AR];  // P as an A fragment
-            if constexpr (HI) {
-                pa[0] = plo[b][0]; pa[1] = phi[b][0]; pa[2] = plo[b][1]; pa[3] = phi[b][1];
-            } else {
-                pa[0] = plo[b][0]; pa[1] = plo[b][1];
+            // ---- P^T as the B fragment: lane l takes row r_lo, tokens tq,
+            // tq + 1 and 8 + tq, 9 + tq; token t < 8 of row n sits in lane
+            // 4t + n/2 (the low half of pk_a for even n, of pk_b for odd n),
+            // token 8 + t in the high half of the same register
+            uint32_t pb0, pb1;
+            {
+                const int src = 8 * (lane & 3) + (r_lo >> 1);  // holds token tq; src + 4 token tq + 1
+                const uint32_t xa = __shfl_sync(kFullMask, pk_a, src), ya = __shfl_sync(kFullMask, pk_b, src);
+                const uint32_t xb = __shfl_sync(kFullMask, pk_a, src + 4),
+                               yb = __shfl_sync(kFullMask, pk_b, src + 4);
+                const uint32_t wa = (r_lo & 1) ? ya : xa, wb = (r_lo & 1) ? yb : xb;
+                pb0 = __byte_perm(wa, wb, 0x5410);  // tokens tq, tq + 1
+                pb1 = __byte_perm(wa, wb, 0x7632);  // tokens 8 + tq, 9 + tq
             }
-            const uint32_t vbase = vb[b];
-            if constexpr (FP8) {
-                // E4M3 V: ldmatrix.trans on the codes seen as b16 gives each lane
-                // tokens 2(lane%4), +1 of the dim pair 2(lane/4), +1 of a 16-dim
-                // chunk; one byte permute splits it into the even and the odd
-                // dim's token pair.  n-tile 2c of the accumulators holds the even
-                // dims 16c + 2n of chunk c, n-tile 2c+1 the odd dims.
+            // ---- O^T += V^T P^T: M = 16 head dims of a chunk (rows 0-7 the
+            // even dims 16c + 2(lane/4), rows 8-15 the odd ones), K = tokens.
+            // ldmatrix.trans gives each lane tokens tq, tq + 1 of the dim pair
+            // 2(lane/4), +1; one byte permute splits it into the even and the
+            // odd dim's token pair: exactly the A fragment.
+            {
                 const int tok = (lane & 7) + 8 * ((lane >> 3) & 1);
 #pragma unroll
                 for (int c = 0; c < D / 16; c += 2) {
                     const uint32_t ch = static_cast<uint32_t>(c + (lane >> 4));
-                    uint32_t r0, r1, r2, r3;
-                    ldsm_x4_trans(vbase + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
-                    uint32_t e0, o0, e1, o1;
-                    e4m3x4_to_f16x2x2(byte_perm(r0, 0x3120), e0, o0);  // tokens 2(lane%4), +1
-                    e4m3x4_to_f16x2x2(byte_perm(r1, 0x3120), e1, o1);  // tokens 8 + 2(lane%4), +1
-                    mma_frag_t<true>(acc[2 * c], pa, e0, e1);
-                    mma_frag_t<true>(acc[2 * c + 1], pa, o0, o1);
-                    e4m3x4_to_f16x2x2(byte_perm(r2, 0x3120), e0, o0);
+                    uint32_t r0, r1, r2, r3, e0, o0, e1, o1;
+                    ldsm_x4_trans(vb[0] + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
+                    e4m3x4_to_f16x2x2(byte_perm(r0, 0x3120), e0, o0);  // tokens tq, tq + 1
+                    e4m3x4_to_f16x2x2(byte_perm(r1, 0x3120), e1, o1);  // tokens 8 + tq, 9 + tq
+                    mma_f16(acc[c], e0, o0, e1, o1, pb0, pb1);
+                    e4m3x4_to_f16x2x2(byte_perm(r2, 0x3120), e0, o0);  // chunk c + 1
                     e4m3x4_to_f16x2x2(byte_perm(r3, 0x3120), e1, o1);
-                    mma_frag_t<true>(acc[2 * c + 2], pa, e0, e1);
-                    mma_frag_t<true>(acc[2 * c + 3], pa, o0, o1);
+                    mma_f16(acc[c + 1], e0, o0, e1, o1, pb0, pb1);
                 }
-            } else {
-#pragma unroll
-                for (int dp = 0; dp < D / 16; ++dp) {
-                    const int cg = 2 * dp + (lane >> 4);
-                    const int t = 8 * ((lane >> 3) & 1) + (lane & 7);
-                    const uint32_t addr = vbase + (cg >> 3) * Cfg::kRegionBytes + t * 128 +
-                                          ((((uint32_t)cg & 7u) ^ sw) << 4);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_trans(addr, b0, b1, b2, b3);
-                    mma_frag(acc[2 * dp], pa, b0, b1);
-                    mma_frag(acc[2 * dp + 1], pa, b2, b3);
+            }
+        }
+        if constexpr (!TR) {
+            // ---- S = Q K^T per block: two n-tiles of 8 tokens, each with two
+            // accumulators (even / odd k-steps) so that the dependent MMA chains
+            // are KSTEPS/2 long
+            float sc[BPS][2][AR];
+    #pragma unroll
+            for (int b = 0; b < BPS; ++b) {
+    #pragma unroll
+                for (int r = 0; r < AR; ++r) sc[b][0][r] = sc[b][1][r] = 0.f;
+                if (b >= nb) continue;
+                float s0[AR], s1[AR], t0[AR], t1[AR];
+    #pragma unroll
+                for (int r = 0; r < AR; ++r) s0[r] = s1[r] = t0[r] = t1[r] = 0.f;
+                const uint32_t kbase = kb[b];
+                if constexpr (FP8) {
+                    // E4M3 K: ldmatrix on the codes seen as b16 gives each lane dims
+                    // 4(lane%4)..+3 of one token per 16-dim chunk; matrices: (tokens
+                    // 0-7, chunk j), (8-15, j), (0-7, j+1), (8-15, j+1)
+                    const int tok = (lane & 7) + 8 * ((lane >> 3) & 1);
+    #pragma unroll
+                    for (int j = 0; j < KSTEPS; j += 2) {
+                        const uint32_t ch = static_cast<uint32_t>(j + (lane >> 4));
+                        uint32_t r0, r1, r2, r3, b0, b1;
+                        ldsm_x4(kbase + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
+                        e4m3x4_to_f16x2x2(r0, b0, b1);
+                        mma_frag_t<true>(s0, qa[j], b0, b1);
+                        e4m3x4_to_f16x2x2(r1, b0, b1);
+                        mma_frag_t<true>(s1, qa[j], b0, b1);
+                        e4m3x4_to_f16x2x2(r2, b0, b1);
+                        mma_frag_t<true>(t0, qa[j + 1], b0, b1);
+                        e4m3x4_to_f16x2x2(r3, b0, b1);
+                        mma_frag_t<true>(t1, qa[j + 1], b0, b1);
+                    }
+                } else {
+    #pragma unroll
+                    for (int kp = 0; kp < KSTEPS / 2; ++kp) {
+                        const int cg = 4 * kp + (lane >> 3);  // 8-element column chunk 0 .. D/8-1
+                        const uint32_t col = (cg >> 3) * Cfg::kRegionBytes + ((((uint32_t)cg & 7u) ^ sw) << 4);
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(kbase + col + (lane & 7) * 128, b0, b1, b2, b3);
+                        mma_frag(s0, qa[2 * kp], b0, b1);
+                        mma_frag(t0, qa[2 * kp + 1], b2, b3);
+                        ldsm_x4(kbase + col + (8 + (lane & 7)) * 128, b0, b1, b2, b3);
+                        mma_frag(s1, qa[2 * kp], b0, b1);
+                        mma_frag(t1, qa[2 * kp + 1], b2, b3);
+                    }
+                }
+    #pragma unroll
+                for (int r = 0; r < AR; ++r) {
+                    sc[b][0][r] += s0[r] + t0[r];
+                    sc[b][1][r] += s1[r] + t1[r];
+                }
+            }
+
+            // ---- online softmax over the step's keys (rows r_lo and r_lo + 8);
+            // key t of block b is visible to a row iff t < valid[b] and
+            // (cj + b)*16 + t <= the row's limit
+            uint32_t plo[BPS][2], phi[BPS][2];  // P as bf16 / f16 pairs: [block][tokens tq.. / 8+tq..]
+            float alpha_lo, alpha_hi = 1.f;
+            {
+                float x[4 * BPS];
+    #pragma unroll
+                for (int b = 0; b < BPS; ++b) {
+                    const int vis = min(valid[b] - 1, lim_lo - (cj + b) * kBlockTokens);  // last visible key
+                    x[4 * b + 0] = tq <= vis ? sc[b][0][0] * sl2 : -INFINITY;
+                    x[4 * b + 1] = tq + 1 <= vis ? sc[b][0][1] * sl2 : -INFINITY;
+                    x[4 * b + 2] = tq + 8 <= vis ? sc[b][1][0] * sl2 : -INFINITY;
+                    x[4 * b + 3] = tq + 9 <= vis ? sc[b][1][1] * sl2 : -INFINITY;
+                }
+                alpha_lo = softmax_update<FP8, BPS>(m_lo, l_lo, x, plo);
+            }
+            if constexpr (HI) {
+                float x[4 * BPS];
+    #pragma unroll
+                for (int b = 0; b < BPS; ++b) {
+                    const int vis = min(valid[b] - 1, lim_hi - (cj + b) * kBlockTokens);
+                    x[4 * b + 0] = tq <= vis ? sc[b][0][2] * sl2 : -INFINITY;
+                    x[4 * b + 1] = tq + 1 <= vis ? sc[b][0][3] * sl2 : -INFINITY;
+                    x[4 * b + 2] = tq + 8 <= vis ? sc[b][1][2] * sl2 : -INFINITY;
+                    x[4 * b + 3] = tq + 9 <= vis ? sc[b][1][3] * sl2 : -INFINITY;
+                }
+                alpha_hi = softmax_update<FP8, BPS>(m_hi, l_hi, x, phi);
+            }
+            // rescale the accumulators only when some row's max moved (alpha is
+            // exactly 1 otherwise): after the first blocks of a sequence it rarely does
+            if (__any_sync(kFullMask, alpha_lo != 1.f || alpha_hi != 1.f)) {
+    #pragma unroll
+                for (int n = 0; n < NTD; ++n) {
+                    acc[n][0] *= alpha_lo;
+                    acc[n][1] *= alpha_lo;
+                    if constexpr (HI) {
+                        acc[n][2] *= alpha_hi;
+                        acc[n][3] *= alpha_hi;
+                    }
+                }
+            }
+
+            // ---- O += P V : n-tiles of 8 head dims, K = the 16 tokens of a block
+    #pragma unroll
+            for (int b = 0; b < BPS; ++b) {
+                if (b >= nb) continue;
+                uint32_t pa[AR];  // P as an A fragment
+                if constexpr (HI) {
+                    pa[0] = plo[b][0]; pa[1] = phi[b][0]; pa[2] = plo[b][1]; pa[3] = phi[b][1];
+                } else {
+                    pa[0] = plo[b][0]; pa[1] = plo[b][1];
+                }
+                const uint32_t vbase = vb[b];
+                if constexpr (FP8) {
+                    // E4M3 V: ldmatrix.trans on the codes seen as b16 gives each lane
+                    // tokens 2(lane%4), +1 of the dim pair 2(lane/4), +1 of a 16-dim
+                    // chunk; one byte permute splits it into the even and the odd
+                    // dim's token pair.  n-tile 2c of the accumulators holds the even
+                    // dims 16c + 2n of chunk c, n-tile 2c+1 the odd dims.
+                    const int tok = (lane & 7) + 8 * ((lane >> 3) & 1);
+    #pragma unroll
+                    for (int c = 0; c < D / 16; c += 2) {
+                        const uint32_t ch = static_cast<uint32_t>(c + (lane >> 4));
+                        uint32_t r0, r1, r2, r3;
+                        ldsm_x4_trans(vbase + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
+                        uint32_t e0, o0, e1, o1;
+                        e4m3x4_to_f16x2x2(byte_perm(r0, 0x3120), e0, o0);  // tokens 2(lane%4), +1
+                        e4m3x4_to_f16x2x2(byte_perm(r1, 0x3120), e1, o1);  // tokens 8 + 2(lane%4), +1
+                        mma_frag_t<true>(acc[2 * c], pa, e0, e1);
+                        mma_frag_t<true>(acc[2 * c + 1], pa, o0, o1);
+                        e4m3x4_to_f16x2x2(byte_perm(r2, 0x3120), e0, o0);
+                        e4m3x4_to_f16x2x2(byte_perm(r3, 0x3120), e1, o1);
+                        mma_frag_t<true>(acc[2 * c + 2], pa, e0, e1);
+                        mma_frag_t<true>(acc[2 * c + 3], pa, o0, o1);
+                    }
+                } else {
+    #pragma unroll
+                    for (int dp = 0; dp < D / 16; ++dp) {
+                        const int cg = 2 * dp + (lane >> 4);
+                        const int t = 8 * ((lane >> 3) & 1) + (lane & 7);
+                        const uint32_t addr = vbase + (cg >> 3) * Cfg::kRegionBytes + t * 128 +
+                                              ((((uint32_t)cg & 7u) ^ sw) << 4);
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4_trans(addr, b0, b1, b2, b3);
+                        mma_frag(acc[2 * dp], pa, b0, b1);
+                        mma_frag(acc[2 * dp + 1], pa, b2, b3);
+                    }
                 }
             }
         }
@@ -506,23 +626,31 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         // ---- item done: final row or partition partials
         if constexpr (FP8) {  // the sums of P V used the V codes: apply the V scale once
 #pragma unroll
-            for (int n = 0; n < NTD; ++n)
+            for (int n = 0; n < ACC_N; ++n)
 #pragma unroll
-                for (int r = 0; r < AR; ++r) acc[n][r] *= vscale;
+                for (int r = 0; r < ACC_R; ++r) acc[n][r] *= vscale;
         }
-        float lt_lo = l_lo + __shfl_xor_sync(kFullMask, l_lo, 1);
-        lt_lo += __shfl_xor_sync(kFullMask, lt_lo, 2);
-        float lt_hi = 0.f;
-        if constexpr (HI) {
-            lt_hi = l_hi + __shfl_xor_sync(kFullMask, l_hi, 1);
-            lt_hi += __shfl_xor_sync(kFullMask, lt_hi, 2);
+        // row sums: over the 4 lanes of a row, or (transposed) the 8 lanes of a column
+        float lt_lo = l_lo, lt_hi = l_hi;
+#pragma unroll
+        for (int x = TR ? 4 : 1; x < (TR ? 32 : 4); x *= 2) {
+            lt_lo += __shfl_xor_sync(kFullMask, lt_lo, x);
+            if constexpr (HI || TR) lt_hi += __shfl_xor_sync(kFullMask, lt_hi, x);
         }
         // This lane's accumulators of a row (r = 0: row r_lo, r = 2: row
         // r_lo + 8) go to dims 8n + tq, +1 of n-tile n (bf16); for E4M3 to
         // dims 16c + 2tq .. +3 of chunk c as (even, odd, even, odd) n-tiles.
+        // Transposed (r = 0: row tq, r = 1: row tq + 1): acc[c][r] and
+        // acc[c][r + 2] are dims 16c + 2(lane/4), +1.
+        constexpr int RB = TR ? 1 : 2;  // accumulator index of the lane's second row
         auto put_out = [&](size_t orow, int r, float inv) {
             __nv_bfloat16* o = static_cast<__nv_bfloat16*>(P.out) + orow * D;
-            if constexpr (FP8) {
+            if constexpr (TR) {
+#pragma unroll
+                for (int c = 0; c < D / 16; ++c)
+                    *reinterpret_cast<__nv_bfloat162*>(o + 16 * c + 2 * r_lo) =
+                        __floats2bfloat162_rn(acc[c][r] * inv, acc[c][r + 2] * inv);
+            } else if constexpr (FP8) {
 #pragma unroll
                 for (int c = 0; c < D / 16; ++c) {
                     uint2 u;
@@ -539,7 +667,11 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         };
         auto put_partial = [&](size_t idx, int r) {
             float* a = P.ws_acc + idx * D;
-            if constexpr (FP8) {
+            if constexpr (TR) {
+#pragma unroll
+                for (int c = 0; c < D / 16; ++c)
+                    *reinterpret_cast<float2*>(a + 16 * c + 2 * r_lo) = make_float2(acc[c][r], acc[c][r + 2]);
+            } else if constexpr (FP8) {
 #pragma unroll
                 for (int c = 0; c < D / 16; ++c)
                     *reinterpret_cast<float4*>(a + 16 * c + 2 * tq) =
@@ -552,27 +684,28 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         };
         if (cc.parts == 1 && P.piece_base == 0) {
             if (ok_lo) put_out(orow_lo, 0, lt_lo > 0.f ? 1.0f / lt_lo : 0.f);
-            if constexpr (HI) {
-                if (ok_hi) put_out(orow_hi, 2, lt_hi > 0.f ? 1.0f / lt_hi : 0.f);
+            if constexpr (HI || TR) {
+                if (ok_hi) put_out(orow_hi, RB, lt_hi > 0.f ? 1.0f / lt_hi : 0.f);
             }
         } else {
             constexpr float kLn2 = 0.693147180559945309f;
+            const bool stat_lane = TR ? r_lo == 0 : (lane & 3) == 0;  // one lane per row writes m, l
             if (ok_lo) {
                 const size_t idx = orow_lo * P.max_parts + P.piece_base + cc.p;
-                if ((lane & 3) == 0) {
+                if (stat_lane) {
                     P.ws_m[idx] = m_lo * kLn2;
                     P.ws_l[idx] = lt_lo;
                 }
                 put_partial(idx, 0);
             }
-            if constexpr (HI) {
+            if constexpr (HI || TR) {
                 if (ok_hi) {
                     const size_t idx = orow_hi * P.max_parts + P.piece_base + cc.p;
-                    if ((lane & 3) == 0) {
+                    if (stat_lane) {
                         P.ws_m[idx] = m_hi * kLn2;
                         P.ws_l[idx] = lt_hi;
                     }
-                    put_partial(idx, 2);
+                    put_partial(idx, RB);
                 }
             }
         }
