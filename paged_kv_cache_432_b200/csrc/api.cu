@@ -488,6 +488,9 @@ int simt_shape(const DecodeParams& P, LaunchShape* L) {
 template <bool FP8>
 int mma_shape_for(const DecodeParams& P, LaunchShape* L) {
     const int rows = P.group * P.max_q_len;
+    if constexpr (FP8) {  // one query row: the E4M3 kernel's single-column form
+        if (rows <= 1) return P.head_dim == 128 ? mma_shape<128, 1, FP8>(P, L) : mma_shape<64, 1, FP8>(P, L);
+    }
     if (P.head_dim == 128)
         return rows <= 8 ? mma_shape<128, 8, FP8>(P, L) : mma_shape<128, 16, FP8>(P, L);
     return rows <= 8 ? mma_shape<64, 8, FP8>(P, L) : mma_shape<64, 16, FP8>(P, L);
@@ -546,6 +549,9 @@ int launch_simt(const DecodeParams& base, cudaStream_t st) {
 template <bool FP8>
 int launch_mma_for(const DecodeParams& P, cudaStream_t st) {
     const int rows = P.group * P.max_q_len;  // query rows of one (sequence, kv head) unit
+    if constexpr (FP8) {  // one query row: the E4M3 kernel's single-column form
+        if (rows <= 1) return P.head_dim == 128 ? launch_mma<128, 1, FP8>(P, st) : launch_mma<64, 1, FP8>(P, st);
+    }
     if (P.head_dim == 128)
         return rows <= 8 ? launch_mma<128, 8, FP8>(P, st) : launch_mma<128, 16, FP8>(P, st);
     return rows <= 8 ? launch_mma<64, 8, FP8>(P, st) : launch_mma<64, 16, FP8>(P, st);

@@ -151,6 +151,9 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // E4M3 with <= 8 query rows: the transposed products S^T = K Q^T and
     // O^T = V^T P^T, tokens / head dims in M and the query rows in N
     constexpr bool TR = FP8 && !HI;
+    // one query row (MHA): only the even columns of S^T / O^T are real, so
+    // each lane keeps one row's softmax instead of two
+    constexpr bool ONE = TR && ROWS == 1;
     constexpr int ACC_N = TR ? D / 16 : NTD;  // accumulator tiles
     constexpr int ACC_R = TR ? 4 : AR;        // registers held per tile
     // blocks per consumer step (one max / sum reduction and one rescale per
@@ -416,15 +419,22 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             uint32_t pk_a, pk_b;  // f16 pairs (token r_lo, token r_lo + 8) of rows tq, tq + 1
             const float alpha_lo = softmax_update_col(m_lo, l_lo, r_lo <= vis_a ? (s0[0] + s1[0]) * sl2 : -INFINITY,
                                           r_lo + 8 <= vis_a ? (s0[2] + s1[2]) * sl2 : -INFINITY, pk_a);
-            const float alpha_hi = softmax_update_col(m_hi, l_hi, r_lo <= vis_b ? (s0[1] + s1[1]) * sl2 : -INFINITY,
-                                          r_lo + 8 <= vis_b ? (s0[3] + s1[3]) * sl2 : -INFINITY, pk_b);
+            float alpha_hi = 1.f;
+            if constexpr (ONE) {
+                pk_b = pk_a;  // the odd columns only carry padding
+            } else {
+                alpha_hi = softmax_update_col(m_hi, l_hi, r_lo <= vis_b ? (s0[1] + s1[1]) * sl2 : -INFINITY,
+                                              r_lo + 8 <= vis_b ? (s0[3] + s1[3]) * sl2 : -INFINITY, pk_b);
+            }
             if (__any_sync(kFullMask, alpha_lo != 1.f || alpha_hi != 1.f)) {
 #pragma unroll
                 for (int c = 0; c < ACC_N; ++c) {
                     acc[c][0] *= alpha_lo;
                     acc[c][2] *= alpha_lo;
-                    acc[c][1] *= alpha_hi;
-                    acc[c][3] *= alpha_hi;
+                    if constexpr (!ONE) {
+                        acc[c][1] *= alpha_hi;
+                        acc[c][3] *= alpha_hi;
+                    }
                 }
             }
             // ---- P^T as the B fragment: lane l takes row r_lo, tokens tq,
@@ -434,10 +444,13 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             uint32_t pb0, pb1;
             {
                 const int src = 8 * (lane & 3) + (r_lo >> 1);  // holds token tq; src + 4 token tq + 1
-                const uint32_t xa = __shfl_sync(kFullMask, pk_a, src), ya = __shfl_sync(kFullMask, pk_b, src);
-                const uint32_t xb = __shfl_sync(kFullMask, pk_a, src + 4),
-                               yb = __shfl_sync(kFullMask, pk_b, src + 4);
-                const uint32_t wa = (r_lo & 1) ? ya : xa, wb = (r_lo & 1) ? yb : xb;
+                const uint32_t xa = __shfl_sync(kFullMask, pk_a, src), xb = __shfl_sync(kFullMask, pk_a, src + 4);
+                uint32_t wa = xa, wb = xb;
+                if constexpr (!ONE) {
+                    const uint32_t ya = __shfl_sync(kFullMask, pk_b, src), yb = __shfl_sync(kFullMask, pk_b, src + 4);
+                    wa = (r_lo & 1) ? ya : xa;
+                    wb = (r_lo & 1) ? yb : xb;
+                }
                 pb0 = __byte_perm(wa, wb, 0x5410);  // tokens tq, tq + 1
                 pb1 = __byte_perm(wa, wb, 0x7632);  // tokens 8 + tq, 9 + tq
             }
@@ -635,7 +648,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
         for (int x = TR ? 4 : 1; x < (TR ? 32 : 4); x *= 2) {
             lt_lo += __shfl_xor_sync(kFullMask, lt_lo, x);
-            if constexpr (HI || TR) lt_hi += __shfl_xor_sync(kFullMask, lt_hi, x);
+            if constexpr (HI || (TR && !ONE)) lt_hi += __shfl_xor_sync(kFullMask, lt_hi, x);
         }
         // This lane's accumulators of a row (r = 0: row r_lo, r = 2: row
         // r_lo + 8) go to dims 8n + tq, +1 of n-tile n (bf16); for E4M3 to
@@ -684,7 +697,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         };
         if (cc.parts == 1 && P.piece_base == 0) {
             if (ok_lo) put_out(orow_lo, 0, lt_lo > 0.f ? 1.0f / lt_lo : 0.f);
-            if constexpr (HI || TR) {
+            if constexpr (HI || (TR && !ONE)) {
                 if (ok_hi) put_out(orow_hi, RB, lt_hi > 0.f ? 1.0f / lt_hi : 0.f);
             }
         } else {
@@ -698,7 +711,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
                 put_partial(idx, 0);
             }
-            if constexpr (HI || TR) {
+            if constexpr (HI || (TR && !ONE)) {
                 if (ok_hi) {
                     const size_t idx = orow_hi * P.max_parts + P.piece_base + cc.p;
                     if (stat_lane) {
