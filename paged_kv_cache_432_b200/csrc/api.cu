@@ -265,7 +265,7 @@ struct PrefixKernel {
     static constexpr int kThreads = kPrefixTc ? PrefixTcCfg<D>::kThreads : PrefixCfg<D>::kThreads;
     static constexpr const char* kName = kPrefixTc ? "decode_prefix_tc_kernel" : "decode_prefix_mma_kernel";
 };
-constexpr int32_t kWideReducePieces = 32;  // rows that can have more pieces merge with 4 warps each
+constexpr int32_t kWideReducePieces = 32;  // rows that can have more pieces merge with a CTA each
 
 Plan make_prefix_plan(int32_t max_seq_len, int32_t partition_blocks, int32_t shared_blocks,
                       int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads) {
@@ -637,7 +637,7 @@ int launch_reduce(const DecodeParams& base, int32_t dtype, cudaStream_t st) {
         cudaError_t e;
         if (P.max_parts > kWideReducePieces)
             e = launch_pdl(lse_reduce_wide_kernel<OutT, D>, dim3(static_cast<unsigned>(rows)),
-                           dim3(kReduceWarps * 32), 0, st, P);
+                           dim3(kWideWarps * 32), 0, st, P);
         else
             e = launch_pdl(lse_reduce_kernel<OutT, D>,
                            dim3(static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps)),
@@ -657,9 +657,9 @@ int launch_reduce(const DecodeParams& base, int32_t dtype, cudaStream_t st) {
                            decode_warps);
         } else {
             const int64_t rows = static_cast<int64_t>(P.seq_count) * P.num_q_heads;
-            if (P.max_parts > kWideReducePieces) {  // many pieces per row: 4 warps per row
+            if (P.max_parts > kWideReducePieces) {  // many pieces per row: a CTA per row
                 e = launch_pdl(lse_reduce_wide_kernel<OutT, D>, dim3(static_cast<unsigned>(rows)),
-                               dim3(kReduceWarps * 32), 0, st, P);
+                               dim3(kWideWarps * 32), 0, st, P);
             } else {
                 const unsigned grid = static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps);
                 e = launch_pdl(lse_reduce_kernel<OutT, D>, dim3(grid), dim3(kReduceWarps * 32), 0, st, P);

@@ -117,14 +117,20 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const Dec
 }
 
 // Row-wise merge for rows with many pieces (long sequences in fixed
-// partitions): one CTA per row, the 4 warps split the pieces and their sums
-// are added in a fixed order.
+// partitions): one CTA of kWideWarps warps per row.  The pieces' weights
+// e^(m_p - M) are computed once, into shared memory, while the row sum is
+// taken; the warps then split the pieces and accumulate their acc rows with
+// eight 16-byte loads in flight per warp, and the warps' sums are added in a
+// fixed order.
+constexpr int kWideWarps = 8;
+constexpr int kWideWeights = 1024;  // pieces whose weight is kept in shared memory
 template <typename OutT, int D>
-__global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_wide_kernel(const DecodeParams P) {
+__global__ void __launch_bounds__(kWideWarps * 32) lse_reduce_wide_kernel(const DecodeParams P) {
     constexpr int DPL = D / 32;
     using Vec = typename std::conditional<DPL == 4, float4, float2>::type;
-    __shared__ float red[kReduceWarps][D];
-    __shared__ float wmax[kReduceWarps], wden[kReduceWarps];
+    __shared__ float wts[kWideWeights];
+    __shared__ float red[kWideWarps][D];
+    __shared__ float wmax[kWideWarps], wden[kWideWarps];
     grid_dependency_wait();
     RowRef R;
     if (!locate_row(P, blockIdx.x, &R)) return;
@@ -142,22 +148,29 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_wide_kernel(cons
     M = warp_max(M);
     if (lane == 0) wmax[warp] = M;
     __syncthreads();
-    M = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+    M = wmax[0];
+#pragma unroll
+    for (int w = 1; w < kWideWarps; ++w) M = fmaxf(M, wmax[w]);
     OutT* o = static_cast<OutT*>(P.out) + R.r * D;
     if (M == -INFINITY) {
         for (int d = tid; d < D; d += blockDim.x) o[d] = from_float<OutT>(0.f);
         return;
     }
     float den = 0.f;
-    for (int p = tid; p < parts; p += blockDim.x) den += expf(wm[p] - M) * wl[p];
+    for (int p = tid; p < parts; p += blockDim.x) {
+        const float w = expf(wm[p] - M);
+        if (p < kWideWeights) wts[p] = w;
+        den += w * wl[p];
+    }
     den = warp_sum(den);
     if (lane == 0) wden[warp] = den;
+    __syncthreads();  // the weights and the warps' sums
     float a[DPL];
 #pragma unroll
     for (int e = 0; e < DPL; ++e) a[e] = 0.f;
-#pragma unroll 4
-    for (int p = warp; p < parts; p += kReduceWarps) {
-        const float w = expf(wm[p] - M);
+#pragma unroll 8
+    for (int p = warp; p < parts; p += kWideWarps) {
+        const float w = p < kWideWeights ? wts[p] : expf(wm[p] - M);
         const Vec x = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(p) * D + lane * DPL);
         const float* f = reinterpret_cast<const float*>(&x);
 #pragma unroll
@@ -166,10 +179,16 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_wide_kernel(cons
 #pragma unroll
     for (int e = 0; e < DPL; ++e) red[warp][lane * DPL + e] = a[e];
     __syncthreads();
-    den = (wden[0] + wden[1]) + (wden[2] + wden[3]);
+    den = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWideWarps; ++w) den += wden[w];
     const float inv = den > 0.f ? 1.0f / den : 0.f;
-    for (int d = tid; d < D; d += blockDim.x)
-        o[d] = from_float<OutT>(((red[0][d] + red[1][d]) + (red[2][d] + red[3][d])) * inv);
+    for (int d = tid; d < D; d += blockDim.x) {
+        float x = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWideWarps; ++w) x += red[w][d];
+        o[d] = from_float<OutT>(x * inv);
+    }
 }
 
 // Balanced split: only units that cross a boundary between two decode warps'
