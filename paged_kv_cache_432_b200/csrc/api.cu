@@ -245,9 +245,9 @@ Plan make_plan(int32_t max_seq_len, int32_t partition_blocks) {
 // device (choose_prefix_splits).
 constexpr int32_t kMaxPrefixSplits = 16;
 
-// The shared-prefix kernel: tcgen05 with TMEM accumulators (two tiles of 128
-// query rows per CTA), or the mma.sync kernel (64 rows per CTA) when built
-// with PA_PREFIX_TC=0.
+// The shared-prefix kernel: tcgen05 with TMEM accumulators (128 query rows
+// per tile, PA_PREFIX_TC_TILES tiles per CTA), or the mma.sync kernel (64
+// rows per CTA) when built with PA_PREFIX_TC=0.
 #ifndef PA_PREFIX_TC
 #define PA_PREFIX_TC 1
 #endif

@@ -264,13 +264,6 @@ __device__ __forceinline__ float2 unpack2(uint32_t u) {
     else return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
 }
 
-// E4M3 pair (low byte = first value) -> f16 pair; exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
-    uint32_t r;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
-    return r;
-}
-
 // Four E4M3 codes (bytes 0..3 of x) -> two f16 pairs: lo = (byte 0, byte 1),
 // hi = (byte 2, byte 3), first value in the low half; exact.
 __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
@@ -320,10 +313,6 @@ __device__ __forceinline__ uint32_t e4m3x4_canonical_nan(uint32_t w) {
 
 __device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) {
     return *reinterpret_cast<uint32_t*>(&v);
-}
-
-__device__ __forceinline__ __nv_bfloat162 bits_bf162(uint32_t u) {
-    return *reinterpret_cast<__nv_bfloat162*>(&u);
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

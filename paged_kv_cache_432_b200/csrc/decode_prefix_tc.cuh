@@ -6,29 +6,29 @@
 // KV-Speicherzuweisung für LLMs?", slavadubrov.com, §"Gemeinsame Nutzung
 // erfordert mehr als Speicherzuweisung"; "PagedAttention et vLLM",
 // aiunderstanding.org, §"Questions fréquemment posées") attend to the prefix
-// keys, which are read once per CTA for 256 rows.  S = Q K^T and O += P V are
-// real matrix products here (M = 128 query rows, N = 64 keys or D dims), so
-// they run as tcgen05.mma with the accumulators in TMEM:
+// keys, which are read once per CTA for all of its query rows.  S = Q K^T
+// and O += P V are real matrix products here (M = 128 query rows, N = 64 keys
+// or D dims), so they run as tcgen05.mma with the accumulators in TMEM:
 //
-//  * one CTA per SM: two tiles of 128 query rows (each tile's rows are the
-//    TMEM lanes of its own columns) x one key split; 18 warps.  Both tiles use
-//    every K/V stage, so the TMA boxes per query row are halved.
-//    Warps 0-15: two threads per query row.  Warp w serves tile w / 8, reaches
-//    TMEM lanes 32 (w mod 4) .. +31 (its rows) and takes half (w / 4) mod 2 of
-//    each step's keys and of O's columns.  They load Q into shared memory,
-//    run the online softmax of their row half straight from TMEM (tcgen05.ld
-//    gives a thread its own row: the max and sum of a half need no shuffles;
-//    the two halves swap their maxima through shared memory once per step,
-//    one named barrier per tile), write P as bf16 into shared memory, rescale
-//    their half of O in TMEM when the row max moved, and finally write the
-//    split's partial (m, l, acc).
-//    Warp 16: TMA producer; 4 blocks (64 keys) of K and V per stage, a ring of
-//    PA_PREFIX_TC_STAGES stages (3 by default, 96 KB).  It starts as soon as
+//  * one CTA per SM: T tiles of 128 query rows (PA_PREFIX_TC_TILES, 1 by
+//    default; each tile's rows are the TMEM lanes of its own columns) x one
+//    key split; 8T + 2 warps.  All tiles of a CTA use every K/V stage.
+//    Softmax warps 0 .. 8T-1: two threads per query row.  Warp w serves tile
+//    w / 8, reaches TMEM lanes 32 (w mod 4) .. +31 (its rows) and takes half
+//    (w / 4) mod 2 of each step's keys and of O's columns.  They load Q into
+//    shared memory, run the online softmax of their row half straight from
+//    TMEM (tcgen05.ld gives a thread its own row: the max and sum of a half
+//    need no shuffles; the two halves swap their maxima through shared memory
+//    once per step, one named barrier per tile), write P as bf16 into shared
+//    memory, rescale their half of O in TMEM when the row max moved, and
+//    finally write the split's partial (m, l, acc).
+//    Warp 8T: TMA producer; 4 blocks (64 keys) of K and V per stage, a ring of
+//    PA_PREFIX_TC_STAGES stages (4 by default, 128 KB).  It starts as soon as
 //    the barriers exist, while the softmax warps load Q.
-//    Warp 17: allocates TMEM and issues the MMAs from one thread.
+//    Warp 8T + 1: allocates TMEM and issues the MMAs from one thread.
 //  * TMEM, per tile: S in two buffers of 64 columns (the MMA of step j+1 runs
-//    while the softmax of step j reads the other), O in D columns; 512
-//    columns in all.
+//    while the softmax of step j reads the other), O in D columns; 256
+//    columns per tile.
 //  * shared memory operands all use the 128-byte swizzle (rows of 128 bytes,
 //    16-byte chunk c of row r at c ^ (r mod 8), 1 KB atoms of 8 rows): Q and K
 //    K-major for S, P K-major and V MN-major for O.
@@ -37,6 +37,8 @@
 //    o_done (tcgen05.commit after each P V -> softmax).  Every wait is
 //    bounded; on timeout the CTA flags PA_DEVERR_TIMEOUT, drains what it
 //    issued and still frees its TMEM.
+//  * What bounds it: with one tile, the delivery of the 2 KB TMA boxes (about
+//    1.1 us per 64-key stage); with two, the softmax of 256 rows per step.
 //
 // The partial of each row goes to the workspace at piece index = split, as
 // the mma.sync kernel writes it, and the same log-sum-exp reduction merges it
@@ -162,29 +164,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-// 64 consecutive fp32 columns, as tmem_ld32.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-    uint32_t r[64];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, "
-        "%36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, "
-        "%57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-          "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]),
-          "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
-          "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
-          "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
-          "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-        : "r"(taddr));
-#pragma unroll
-    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 // Named barrier `id` (1.. : barrier 0 is __syncthreads) over `nthreads` softmax threads.
 __device__ __forceinline__ void softmax_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
