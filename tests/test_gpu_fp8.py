@@ -103,7 +103,7 @@ EDGE_LENS = [1, 15, 16, 17, 0, 511, 512, 513, 33, 1000]
 
 
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (32, 8), (16, 2), (32, 2)])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (6, 2), (8, 2), (32, 8), (16, 2), (32, 2)])
 @pytest.mark.parametrize("pb", [0, -1, 3, 32])
 def test_fp8_decode_edge_lengths(D, Hq, Hkv, pb):
     """Block and partition edges, an empty sequence, group sizes 1..16, both

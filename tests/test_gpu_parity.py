@@ -88,7 +88,7 @@ EDGE_LENS = [1, 15, 16, 17, 0, 511, 512, 513, 33, 1000]
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (32, 8), (16, 2), (32, 2)])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (6, 2), (8, 2), (32, 8), (16, 2), (32, 2)])
 @pytest.mark.parametrize("pb", [0, -1, 3, 32])
 def test_edge_lengths(dtype, D, Hq, Hkv, pb):
     """Lengths at block and partition edges (and an empty sequence), group sizes
