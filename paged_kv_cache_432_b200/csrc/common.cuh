@@ -148,6 +148,12 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// Brings the 128-byte line holding p into L2 ahead of a dependent load.  p
+// must lie inside an allocation the kernel may read.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // L2 policy for data read once (the KV stream): evict first.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;

@@ -179,17 +179,29 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
         fence_barrier_init();
     }
     // Launched with programmatic stream serialization: the CTAs become
-    // resident while the previous kernel (typically the cache write) drains,
-    // and wait here until its results are visible.  Nothing above touched
-    // global memory.
-    grid_dependency_wait();
+    // resident while the previous kernel (typically the cache write) still
+    // runs.  Until grid_dependency_wait() they read only inputs that no kernel
+    // of this library writes (lengths, block tables, query rows): the
+    // schedule, the first table window and, into L2, the first query rows are
+    // ready when the wait ends.  The pool (which the cache write fills), the
+    // output and the workspace are touched only after it.
     allow_dependents();  // the reduction may launch and wait for this grid
     const Schedule sched = make_schedule(P, prefix, lens, WARPS);  // ends with __syncthreads
-    zero_empty_sequences<__nv_bfloat16>(P, lens);
-
     const int32_t my_warp = blockIdx.x * WARPS + warp;
     Cursor pc;  // producer: the piece whose next block is loaded next
     sched.start(pc, my_warp);
+    int32_t first_tbl = 0;  // lane l: table entry jbeg + l of the first piece
+    if (pc.valid) {
+        const int32_t jj = pc.jbeg + lane;
+        first_tbl = jj < pc.jend
+                        ? __ldg(P.block_tables + static_cast<size_t>(pc.s) * P.max_blocks_per_seq + jj)
+                        : 0;
+        if (!P.q_start && lane < P.group * D / 64)  // its g query rows of D bf16: 128-byte lines
+            prefetch_l2(static_cast<const __nv_bfloat16*>(P.q) +
+                        (static_cast<size_t>(pc.s) * P.num_q_heads + pc.h * P.group) * D + 64 * lane);
+    }
+    grid_dependency_wait();
+    zero_empty_sequences<__nv_bfloat16>(P, lens);
     if (!pc.valid) return;
     Cursor cc = pc;  // consumer: the piece being computed
 
@@ -204,8 +216,8 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // ---------------- producer state (warp-uniform except `tbl`)
     int32_t pj = pc.jbeg;
     bool prod_live = true;
-    int32_t tbl = 0, tbase = 0;
-    bool tbl_fresh = false;  // tbl holds entries of the producer's current piece
+    int32_t tbl = first_tbl, tbase = pc.jbeg;
+    bool tbl_fresh = true;  // tbl holds entries of the producer's current piece
     uint32_t oob_mask = 0;   // stages whose block id was outside the pool
     uint32_t issued = 0, consumed = 0;
 

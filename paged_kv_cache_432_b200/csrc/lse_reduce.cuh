@@ -200,11 +200,13 @@ __global__ void __launch_bounds__(kWideWarps * 32) lse_reduce_wide_kernel(const 
 template <typename OutT, int D>
 __global__ void __launch_bounds__(kReduceWarps * 32)
 lse_reduce_balanced_kernel(const DecodeParams P, int32_t decode_warps) {
-    grid_dependency_wait();  // the partials of the decode launched just before
     extern __shared__ int32_t smem_i[];
     int32_t* prefix = smem_i;
     int32_t* lens = prefix + P.seq_count + 1;
+    // the lengths are input no kernel of this library writes: the prefix is
+    // built while the decode launched just before still runs
     const int32_t total = build_prefix(P, prefix, lens);  // blocks per sequence
+    grid_dependency_wait();  // the decode's partials
     const int64_t hk = P.num_kv_heads;
     const int64_t T = static_cast<int64_t>(total) * hk;
     const int64_t even = (T + decode_warps - 1) / decode_warps;
