@@ -1,6 +1,10 @@
 """Benchmark of the paged KV-cache decode path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config mha|gqa|prefix|long|tiny]
+    python bench.py --kv fp8 ...              (the step on E4M3 pools: quantising write + decode)
+    python bench.py --op multi --q-len n ...  (several query tokens per sequence)
+    python bench.py --op copy_blocks ...      (copy-on-write block copies)
+    python bench.py --config prefix --plain-decode ...  (the prefix batch without the shared-prefix path)
     python bench.py --impl reference ...      (the fp64 CPU oracle, timed on host cores)
 
 One step = one pass of the hot path over one batch: the cache write of each
