@@ -285,7 +285,8 @@ PA_API int pa_decode_reduce(const int32_t* seq_lens, int32_t max_seq_len, int32_
  * aiunderstanding.org, §"Questions fréquemment posées").  Same result as
  * pa_decode, computed in three launches: the query rows of all sequences
  * attend to the shared blocks together, so those blocks are read once per
- * kv head rather than once per sequence (tensor-core tiles of 64 query rows);
+ * tile of 128 query rows of a kv head rather than once per sequence
+ * (5th-generation tensor cores, accumulators in tensor memory);
  * each sequence's own blocks go through the decode kernel; a log-sum-exp
  * reduction merges the two.  Preconditions: every table starts with the
  * prefix blocks of table 0, and every seq_len >= shared_blocks * block_size.
