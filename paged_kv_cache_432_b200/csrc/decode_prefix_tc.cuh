@@ -217,7 +217,11 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     constexpr int kSoftmaxThreads = Cfg::kSoftmaxWarps * 32;
     static_assert(T == 1 || T == 2, "one or two query tiles");
 
-    grid_dependency_wait();
+    // Launched with programmatic stream serialization: the CTA starts while
+    // the previous kernel (the cache write) may still run.  Setup, Q and the
+    // table windows are inputs no kernel of this library writes; the pool is
+    // read (producer) and the workspace written (softmax epilogue) only after
+    // grid_dependency_wait().
     allow_dependents();
 
     extern __shared__ uint8_t smem_raw[];
@@ -325,6 +329,7 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         };
         int32_t win_cur = table_entry(jbeg + lane);
         int32_t win_next = table_entry(jbeg + 32 + lane);
+        grid_dependency_wait();  // the pool: the cache write has finished
         for (int j = 0; j < nsteps; ++j) {
             const int st = j % S;
             const int fill = j / S;
@@ -521,6 +526,7 @@ decode_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 mbar_arrive(pfull_of(tl));
             }
         }
+        grid_dependency_wait();  // before the workspace writes below
         // the row sum over both halves (its own buffer: the partner may still
         // read the last step's maximum)
         xchg[4 * Cfg::kTileRows + hf * Cfg::kTileRows + row] = l;
