@@ -1,11 +1,15 @@
 """Benchmark of the paged KV-cache decode path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config mha|gqa|prefix|long|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config long|mha|gqa|prefix|tiny]
     python bench.py --kv fp8 ...              (the step on E4M3 pools: quantising write + decode)
     python bench.py --op multi --q-len n ...  (several query tokens per sequence)
     python bench.py --op copy_blocks ...      (copy-on-write block copies)
     python bench.py --config prefix --plain-decode ...  (the prefix batch without the shared-prefix path)
     python bench.py --impl reference ...      (the fp64 CPU oracle, timed on host cores)
+
+The default workload is the long-context one (8 sequences of 32k-128k tokens,
+64 query heads over 8 kv heads, 32-block partitions), the largest that fits one
+GPU; --config picks another.
 
 One step = one pass of the hot path over one batch: the cache write of each
 sequence's newest token (pa_cache_write), then the decode (the block-table
@@ -72,7 +76,16 @@ def algorithmic_bytes(w: wl.Workload, kv_bytes=None) -> dict:
                 kv_logical=kv_logical, q_out=q_out, meta=meta)
 
 
-def workload_config(w: wl.Workload, pb: int) -> dict:
+def resolve_partition_blocks(pb: int) -> int:
+    """The partition setting the decode runs with (as pa_decode_partition_blocks
+    resolves it): > 0 fixed partitions, -1 never split (1 << 24), 0 balanced."""
+    return pb if pb > 0 else ((1 << 24) if pb == -1 else 0)
+
+
+def workload_config(w: wl.Workload, pb: int, kv: str = "bf16") -> dict:
+    """The workload a line measures; both arms (the GPU path and the oracle)
+    report the same dict for the same arguments."""
+    by = algorithmic_bytes(w, kv_bytes=1 if kv == "fp8" else None)
     return {
         "workload": w.name,
         "desc": w.desc,
@@ -91,8 +104,11 @@ def workload_config(w: wl.Workload, pb: int) -> dict:
         "new_tokens": int(w.slot_mapping.numel()),
         "shared_prefix_blocks": w.shared_prefix_blocks,
         "slot_utilisation": round(sum(w.lens_host) / (16 * sum(len(t) for t in w.tables_host)), 5),
-        "l2": "flushed before every step (512 MiB write + 512 MiB read, outside the timed "
-              "events); KV footprint exceeds L2",
+        "kv": "e4m3 codes, per-head fp32 scales" if kv == "fp8" else (
+            "bf16" if w.dtype == torch.bfloat16 else "f32"),
+        "l2": f"inputs larger than L2 (distinct KV read per step {by['kv_unique'] / 1e6:.0f} MB vs 126 MB "
+              "of L2) and L2 flushed before every GPU step (512 MiB write + 512 MiB read, outside "
+              "the timed events)",
     }
 
 
@@ -338,35 +354,72 @@ def cpu_baseline_all_cores(w: wl.Workload, h: dict, seqs: list, budget_s: float)
                       f"decode tasks, {wall:.1f} s wall on {cores} threads"}
 
 
+def oracle_unit_sample(w: wl.Workload, h: dict, units: list) -> tuple:
+    """Runs the oracle on (sequence, kv head) units: the cache write of each
+    touched sequence's newest token (all heads), then the decode of every
+    query head of each unit.  Returns (seconds, algorithmic bytes)."""
+    import numpy as np
+
+    import oracle
+
+    g = w.num_q_heads // w.num_kv_heads
+    seqs = sorted({s for s, _ in units})
+    sel = np.array(seqs)
+    rows = [(s, kh * g + i) for s, kh in units for i in range(g)]
+    t0 = time.perf_counter()
+    oracle.cache_write(h["nk"][sel], h["nv"][sel], h["sm"][sel], h["kc"], h["vc"], inplace=True)
+    oracle.paged_decode(h["q"], h["kc"], h["vc"], h["bt"], h["sl"], w.scale, rows=rows)
+    dt = time.perf_counter() - t0
+    e, D = w.elem_bytes, w.head_dim
+    by = sum(2 * w.lens_host[s] * D * e + 2 * g * D * e + 4 * len(w.tables_host[s]) for s, _ in units)
+    by += len(seqs) * 2 * (2 * w.num_kv_heads * D * e)
+    return dt, by
+
+
 def run_reference(args) -> None:
-    ws, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    """The reference arm: the fp64 oracle on host cores, on the same workload
+    and metric as the GPU arm.  Each step is a bounded sample of the batch:
+    a fixed number of (sequence, kv head) units, rotating over the batch,
+    sized from one calibration unit so that warm-up and timed steps together
+    take about --ref-budget-s seconds."""
+    ws, rank = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = wl.make(args.config, seed=args.seed, device="cpu")
+    w = wl.make(args.config, seed=args.seed, device="cpu", max_seqs=args.max_seqs)
     h = host_arrays(w)
-    per_step = max(1, args.ref_seqs_per_step)
-    times, nbytes, nseq = [], [], []
-    s = 0
+    Hkv = w.num_kv_heads
+    all_units = [(s, kh) for s in range(w.num_seqs) if w.lens_host[s] > 0 for kh in range(Hkv)]
+    t_unit, _ = oracle_unit_sample(w, h, [max(all_units, key=lambda u: w.lens_host[u[0]])])
+    per_step = max(1, int(args.ref_budget_s / (args.warmup + args.steps) / max(t_unit, 1e-6)))
+    per_step = min(per_step, len(all_units))
+    times, nbytes, nunits = [], [], []
+    cur = 0
     for i in range(args.warmup + args.steps):
-        seqs = [(s + k) % w.num_seqs for k in range(per_step)]
-        s = (s + per_step) % w.num_seqs
-        dt, by = oracle_step_sample(w, h, seqs)
+        units = [all_units[(cur + k) % len(all_units)] for k in range(per_step)]
+        cur = (cur + per_step) % len(all_units)
+        dt, by = oracle_unit_sample(w, h, units)
         if i >= args.warmup:
             times.append(dt)
             nbytes.append(by)
-            nseq.append(len(seqs))
+            nunits.append(len(units))
     T = sum(times)
     value = sum(nbytes) / T / 1e9
+    sample = (f"{per_step} (sequence, kv head) unit(s) per step (each: all {w.num_q_heads // Hkv} query "
+              f"heads of the unit, plus the cache write of its sequence's new token), rotating over "
+              f"the batch's {len(all_units)} units; single-threaded fp64")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(1e3 * T / len(times), 3), "higher_is_better": True,
+        "ms_per_step": round(1e3 * T / len(times), 3),
+        "step_ms": {"mean": round(1e3 * T / len(times), 3), "median": round(1e3 * statistics.median(times), 3),
+                    "min": round(1e3 * min(times), 3)},
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": dict(workload_config(w, 0), l2="n/a (host)"),
-        "tokens_per_s": round(sum(nseq) / T, 3),
+        "config": workload_config(w, resolve_partition_blocks(w.partition_blocks if args.partition_blocks is None
+                                                              else args.partition_blocks), args.kv),
+        "tokens_per_s": round(sum(nunits) / Hkv / T, 3),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{per_step} whole sequence(s) per step (all {w.num_q_heads} q "
-                                   f"heads, cache write + decode), rotating over the batch"},
+                         "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -383,7 +436,7 @@ def run_ours(args) -> None:
         pa_build.build()
     barrier(ws)
     dev = torch.device("cuda", local)
-    w = wl.make(args.config, seed=replica_seed(args.seed, rank), device=dev)
+    w = wl.make(args.config, seed=replica_seed(args.seed, rank), device=dev, max_seqs=args.max_seqs)
     pb = w.partition_blocks if args.partition_blocks is None else args.partition_blocks
     msl = w.max_seq_len
     resolved_pb = pa.partition_blocks(w.num_seqs, w.num_kv_heads, msl, pb)
@@ -480,17 +533,22 @@ def run_ours(args) -> None:
                 step(ev_k[k])
             torch.cuda.synchronize(dev)
         barrier(ws)
-        tot = sum(a.elapsed_time(b) for a, b in ev_step)
+        per_step = [a.elapsed_time(b) for a, b in ev_step]
         dec = sum(e[1].elapsed_time(e[2]) for e in ev_k)
         red = sum(e[2].elapsed_time(e[3]) for e in ev_k)
         wr = sum(e[0].elapsed_time(e[1]) for e in ev_k)
-        return tot, dec, red, wr, cs.summary()
+        return per_step, dec, red, wr, cs.summary()
 
-    tot, dec, red, wr, clocks = timed()
+    per_step, dec, red, wr, clocks = timed()
     if set(clocks.get("reasons", [])) & _BAD:  # re-measure once
-        tot, dec, red, wr, clocks = timed()
+        per_step, dec, red, wr, clocks = timed()
         clocks["remeasured"] = True
     K = args.steps
+    tot = sum(per_step)
+    step_stats = {"mean": round(max_over_ranks(tot / K, ws), 5),
+                  "median": round(max_over_ranks(statistics.median(per_step), ws), 5),
+                  "min": round(max_over_ranks(min(per_step), ws), 5),
+                  "how": "CUDA events at step boundaries; each statistic is the max over ranks"}
     agg = aggregate(tot / K, by["step"], w.num_seqs, ws)
     step_ms, total_bytes, total_seqs, value = agg["step_ms"], agg["bytes"], agg["seqs"], agg["gbs"]
     dec_ms = max_over_ranks(dec / K, ws)
@@ -588,13 +646,13 @@ def run_ours(args) -> None:
         "steps": K,
         "warmup": args.warmup,
         "ms_per_step": round(step_ms, 5),
+        "step_ms": step_stats,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": ("e4m3 KV, f16 MMA" if fp8 else "bf16") if w.dtype == torch.bfloat16 else "f32",
         "data": "synthetic",
-        "config": dict(workload_config(w, resolved_pb), kv="e4m3 codes, per-head fp32 scales" if fp8 else
-                       ("bf16" if w.dtype == torch.bfloat16 else "f32")),
+        "config": workload_config(w, resolved_pb, args.kv),
         "tokens_per_s": round(total_seqs / (step_ms * 1e-3), 1),
         "kernel_ms": {"cache_write": round(wr_ms, 5), "decode_partitions": round(dec_ms, 5),
                       "lse_reduce": round(red_ms, 5),
@@ -746,7 +804,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="mha", choices=list(wl.CONFIGS))
+    ap.add_argument("--config", default="long", choices=list(wl.CONFIGS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--op", default="step", choices=["step", "copy_blocks", "multi"],
@@ -756,12 +814,16 @@ def main():
     ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
                     help="KV pool element type for --op step (fp8: E4M3 codes with per-head scales)")
     ap.add_argument("--partition-blocks", type=int, default=None)
+    ap.add_argument("--max-seqs", type=int, default=None,
+                    help="keep only the first N sequences of the workload (a smaller case of the same "
+                         "shape, for profiler captures; not a bench line)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--plain-decode", action="store_true",
                     help="decode a shared-prefix batch with pa_decode instead of pa_decode_shared_prefix")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
-    ap.add_argument("--ref-seqs-per-step", type=int, default=2)
+    ap.add_argument("--ref-budget-s", type=float, default=90.0,
+                    help="--impl reference: host seconds the warm-up and timed steps take together")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":

@@ -30,7 +30,23 @@
  * Ownership and execution: every pointer argument is device memory owned by
  * the caller (the library allocates no device memory and keeps no pointer).
  * Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
- * default stream) and return once the work is enqueued.  Host-side validation
+ * default stream) and return once the work is enqueued.
+ *
+ * Early start of the decode kernels: every decode entry point (pa_decode,
+ * pa_decode_partitions, pa_decode_reduce, pa_decode_fp8, pa_decode_multi,
+ * pa_decode_shared_prefix, pa_decode_noalloc) launches its kernels with
+ * programmatic stream serialization, so they may start before the previous
+ * kernel in the stream has finished.  Before waiting for that kernel they
+ * already read seq_lens, block_tables, q_start and q (they never touch the
+ * caches, out or the workspace before the wait).  This is safe whenever the
+ * previous kernel in the stream did not trigger its dependents early (a kernel
+ * that never executes griddepcontrol.launch_dependents /
+ * cudaTriggerProgrammaticLaunchCompletion lets dependents start only when it
+ * completes), and whenever those four arrays were written before such a
+ * trigger.  A caller whose previous kernel writes them after an early trigger
+ * must separate the two launches (an event, or any kernel without an early
+ * trigger in between).  The library's own cache writes trigger early, but
+ * they write only the caches, which the decode reads after the wait.  Host-side validation
  * never reads device memory.  Pointers to q, k, v, caches and out must be
  * 16-byte aligned; tables, lengths and slots naturally aligned.  The caches
  * and tables may be shared between sequences but must not overlap `out` or the
@@ -74,6 +90,9 @@ extern "C" {
 #define PA_DEVERR_TIMEOUT 8u   /* a bounded wait on an async copy gave up                  */
 #define PA_DEVERR_PREFIX 16u   /* shared-prefix decode: a table does not start with the
                                   shared blocks, or a sequence is shorter than them      */
+#define PA_DEVERR_Q_RANGE 32u  /* E4M3 decode: a query value outside the f16 range the
+                                  kernel rounds q to (|q| > 65504, inf, NaN); the rows
+                                  of that (sequence, kv head) are not meaningful        */
 
 /*
  * Cache write (the scatter of newly computed K/V into the paged pool).
@@ -206,7 +225,10 @@ PA_API int32_t pa_decode_partition_blocks(int32_t num_seqs, int32_t num_kv_heads
 
 /*
  * Bytes of workspace pa_decode needs for these sizes (0 when no sequence of up
- * to max_seq_len tokens can be split).  Workspace layout: P is the number of
+ * to max_seq_len tokens can be split).  Interface plumbing: the pages describe
+ * no workspace (the split-K partials are this library's design).  It takes
+ * num_kv_heads because the workspace ends with one piece count per
+ * (sequence, kv head).  Workspace layout: P is the number of
  * pieces a unit can have at max_seq_len (fixed: ceil(nb / partition_blocks);
  * balanced: ceil(nb / 16) + 1, with nb = ceil(max_seq_len / 16)), and rows
  * r = seq * num_q_heads + q_head:
@@ -363,7 +385,10 @@ PA_API int pa_bm_export_tables(pa_block_manager* m, const int32_t* seq_ids, int3
 
 /*
  * Reads the sticky device error word of the current device (PA_DEVERR_* bits)
- * after synchronising `stream`; clears it when `clear` is non-zero.
+ * after synchronising `stream`; clears it when `clear` is non-zero (so that a
+ * caller can check one call at a time).  Interface plumbing: the pages have no
+ * passage on error reporting.  Returns PA_ERR_INVALID_ARG for a null `bits`,
+ * PA_ERR_CUDA if the synchronisation or the read fails.
  */
 PA_API int pa_get_device_error(uint32_t* bits, int32_t clear, void* stream);
 
@@ -385,8 +410,11 @@ PA_API int pa_get_device_error(uint32_t* bits, int32_t clear, void* stream);
  * with your own workspace instead.
  *
  * The first call on a device looks up the buffer's device address (a
- * one-time set-up per device, done with that device current).  Make that
- * first call before any stream capture.  All calls share the one buffer and
+ * one-time set-up per device, done with that device current) and keeps it for
+ * the life of the process.  Make that first call before any stream capture.
+ * Call it with the device's primary context current (the CUDA runtime's
+ * default); after cudaDeviceReset, or from another context on the same device,
+ * the kept address is no longer valid, so neither is supported.  All calls share the one buffer and
  * it keeps the last call's contents.  Nothing in it needs to start at zero,
  * since each partial is written before it is read.  Calls that overlap on the
  * GPU race on that buffer (two streams, or two threads), so serialise them.
@@ -402,7 +430,8 @@ PA_API int pa_decode_noalloc(const void* q, const void* k_cache, const void* v_c
 #define PA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 
 /* Human-readable text for a return code (for PA_ERR_CUDA: the last CUDA error
- * seen by the calling thread). */
+ * seen by the calling thread).  Interface plumbing: no passage of the pages.
+ * The string is static (or thread-local for PA_ERR_CUDA); do not free it. */
 PA_API const char* pa_status_string(int status);
 
 #ifdef __cplusplus

@@ -296,9 +296,11 @@ __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) {
 }
 
 // A bf16 pair -> an f16 pair (round to nearest; exact for magnitudes in
-// 2^-14 .. 65504).
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
+// 2^-14 .. 65504).  `bad` is set when a value lies outside the f16 range
+// (magnitude above 65504, infinity or NaN).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_checked(uint32_t u, bool& bad) {
     const float2 f = unpack2<false>(u);
+    bad |= !(fabsf(f.x) <= 65504.f && fabsf(f.y) <= 65504.f);
     return pack2<true>(f.x, f.y);
 }
 

@@ -156,14 +156,6 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     constexpr bool ONE = TR && ROWS == 1;
     constexpr int ACC_N = TR ? D / 16 : NTD;  // accumulator tiles
     constexpr int ACC_R = TR ? 4 : AR;        // registers held per tile
-    // blocks per consumer step (one max / sum reduction and one rescale per
-    // step); one measured fastest for both element types
-#ifndef PA_FP8_BLOCKS_PER_STEP
-#define PA_FP8_BLOCKS_PER_STEP 1
-#endif
-    constexpr int BPS = (FP8 && !TR) ? PA_FP8_BLOCKS_PER_STEP : 1;
-    static_assert(STAGES >= 2 * BPS, "a step's stages plus as many in flight");
-
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
@@ -314,20 +306,22 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     (static_cast<size_t>(qr.base) + r_lo / g) * P.num_q_heads + cc.h * g + r_lo % g;
                 const uint2* q_lo = reinterpret_cast<const uint2*>(qb + (ok_q ? orow_q : 0) * D + 2 * tq);
                 const uint2* q_hi = reinterpret_cast<const uint2*>(qb + (ok_hi ? orow_hi : 0) * D + 2 * tq);
+                bool q_out_of_range = false;  // a value f16 cannot hold (|q| > 65504, inf, NaN)
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ++ks) {
                     const uint2 lo = ok_q ? __ldg(q_lo + 4 * ks) : make_uint2(0u, 0u);
                     if constexpr (HI) {
                         const uint2 hi = ok_hi ? __ldg(q_hi + 4 * ks) : make_uint2(0u, 0u);
-                        qa[ks][0] = bf16x2_to_f16x2(lo.x);
-                        qa[ks][1] = bf16x2_to_f16x2(hi.x);
-                        qa[ks][2] = bf16x2_to_f16x2(lo.y);
-                        qa[ks][3] = bf16x2_to_f16x2(hi.y);
+                        qa[ks][0] = bf16x2_to_f16x2_checked(lo.x, q_out_of_range);
+                        qa[ks][1] = bf16x2_to_f16x2_checked(hi.x, q_out_of_range);
+                        qa[ks][2] = bf16x2_to_f16x2_checked(lo.y, q_out_of_range);
+                        qa[ks][3] = bf16x2_to_f16x2_checked(hi.y, q_out_of_range);
                     } else {
-                        qa[ks][0] = bf16x2_to_f16x2(lo.x);
-                        qa[ks][1] = bf16x2_to_f16x2(lo.y);
+                        qa[ks][0] = bf16x2_to_f16x2_checked(lo.x, q_out_of_range);
+                        qa[ks][1] = bf16x2_to_f16x2_checked(lo.y, q_out_of_range);
                     }
                 }
+                if (__any_sync(kFullMask, q_out_of_range) && lane == 0) flag_error(PA_DEVERR_Q_RANGE);
                 sl2 = P.scale_log2 * __ldg(P.k_scale + cc.h);
                 vscale = __ldg(P.v_scale + cc.h);
             } else {
@@ -354,51 +348,37 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 for (int r = 0; r < ACC_R; ++r) acc[n][r] = 0.f;
         }
 
-        // ---- this step: BPS blocks (fewer at the end of the piece); wait for
-        // their stages and mask what they hold
-        const int nb = BPS == 1 ? 1 : min(BPS, cc.jend - cj);
-        uint32_t kb[BPS], vb[BPS];
-        int valid[BPS];
-#pragma unroll
-        for (int b = 0; b < BPS; ++b) {
-            valid[b] = 0;
-            kb[b] = vb[b] = 0;
-            if (b >= nb) continue;
-            int sb = stage + b;
+        // ---- this step's block: wait for its stage and mask what it holds
+        if (!mbar_wait_bounded(bar_u32 + stage * 8, phase)) {
+            if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
+            // drain: wait (bounded) for the copies still in flight, then leave
+            int sb = stage;
             uint32_t pb = phase;
-            if (sb >= STAGES) {
-                sb -= STAGES;
-                pb ^= 1u;
+            for (uint32_t k = 1; k < issued - consumed; ++k) {
+                if (++sb == STAGES) { sb = 0; pb ^= 1u; }
+                mbar_wait_bounded(bar_u32 + sb * 8, pb);
             }
-            if (!mbar_wait_bounded(bar_u32 + sb * 8, pb)) {
-                if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
-                // drain: wait (bounded) for the copies still in flight, then leave
-                for (uint32_t k = 1; k < issued - consumed; ++k) {
-                    if (++sb == STAGES) { sb = 0; pb ^= 1u; }
-                    mbar_wait_bounded(bar_u32 + sb * 8, pb);
-                }
-                return;
+            return;
+        }
+        ++consumed;
+        const int valid = ((oob_mask >> stage) & 1u) ? 0 : min(kBlockTokens, cc.len - cj * kBlockTokens);
+        const uint32_t kb = ring_u32 + stage * Cfg::kStageBytes;
+        const uint32_t vb = kb + Cfg::kTileBytes;
+        if (valid < kBlockTokens) {
+            // zero V rows [valid, 16) so that 0 * (stale or NaN) never enters P V
+            uint8_t* vs = ring + stage * Cfg::kStageBytes + Cfg::kTileBytes;
+            constexpr int kRowChunks = Cfg::kRegions * Cfg::kRowBytes / 16;  // 16-byte chunks per row
+            constexpr int kSlabChunks = Cfg::kRowBytes / 16;
+            const int chunks = (kBlockTokens - valid) * kRowChunks;
+            for (int c = lane; c < chunks; c += 32) {
+                const int row = valid + c / kRowChunks;
+                const int rem = c % kRowChunks;
+                *reinterpret_cast<uint4*>(vs + (rem / kSlabChunks) * Cfg::kRegionBytes +
+                                          row * Cfg::kRowBytes + (rem % kSlabChunks) * 16) =
+                    make_uint4(0, 0, 0, 0);
             }
-            ++consumed;
-            valid[b] = ((oob_mask >> sb) & 1u) ? 0 : min(kBlockTokens, cc.len - (cj + b) * kBlockTokens);
-            kb[b] = ring_u32 + sb * Cfg::kStageBytes;
-            vb[b] = kb[b] + Cfg::kTileBytes;
-            if (valid[b] < kBlockTokens) {
-                // zero V rows [valid, 16) so that 0 * (stale or NaN) never enters P V
-                uint8_t* vs = ring + sb * Cfg::kStageBytes + Cfg::kTileBytes;
-                constexpr int kRowChunks = Cfg::kRegions * Cfg::kRowBytes / 16;  // 16-byte chunks per row
-                constexpr int kSlabChunks = Cfg::kRowBytes / 16;
-                const int chunks = (kBlockTokens - valid[b]) * kRowChunks;
-                for (int c = lane; c < chunks; c += 32) {
-                    const int row = valid[b] + c / kRowChunks;
-                    const int rem = c % kRowChunks;
-                    *reinterpret_cast<uint4*>(vs + (rem / kSlabChunks) * Cfg::kRegionBytes +
-                                              row * Cfg::kRowBytes + (rem % kSlabChunks) * 16) =
-                        make_uint4(0, 0, 0, 0);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
+            fence_proxy_async_smem();
+            __syncwarp();
         }
 
         if constexpr (TR) {
@@ -414,7 +394,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 for (int j = 0; j < KSTEPS; j += 2) {
                     const uint32_t ch = static_cast<uint32_t>(j + (lane >> 4));
                     uint32_t r0, r1, r2, r3, l0, h0, l1, h1;
-                    ldsm_x4(kb[0] + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
+                    ldsm_x4(kb + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
                     e4m3x4_to_f16x2x2(r0, l0, h0);  // tokens 0-7, chunk j
                     e4m3x4_to_f16x2x2(r1, l1, h1);  // tokens 8-15, chunk j
                     mma_f16(s0, l0, l1, h0, h1, qa[j][0], qa[j][1]);
@@ -426,8 +406,8 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             // ---- online softmax: this lane holds tokens r_lo and r_lo + 8
             // of rows tq (s[0], s[2]) and tq + 1 (s[1], s[3]); a row's 16
             // tokens sit in the 8 lanes of equal lane % 4
-            const int vis_a = min(valid[0] - 1, lim_lo - cj * kBlockTokens);
-            const int vis_b = min(valid[0] - 1, lim_hi - cj * kBlockTokens);
+            const int vis_a = min(valid - 1, lim_lo - cj * kBlockTokens);
+            const int vis_b = min(valid - 1, lim_hi - cj * kBlockTokens);
             uint32_t pk_a, pk_b;  // f16 pairs (token r_lo, token r_lo + 8) of rows tq, tq + 1
             const float alpha_lo = softmax_update_col(m_lo, l_lo, r_lo <= vis_a ? (s0[0] + s1[0]) * sl2 : -INFINITY,
                                           r_lo + 8 <= vis_a ? (s0[2] + s1[2]) * sl2 : -INFINITY, pk_a);
@@ -477,7 +457,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 for (int c = 0; c < D / 16; c += 2) {
                     const uint32_t ch = static_cast<uint32_t>(c + (lane >> 4));
                     uint32_t r0, r1, r2, r3, e0, o0, e1, o1;
-                    ldsm_x4_trans(vb[0] + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
+                    ldsm_x4_trans(vb + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
                     e4m3x4_to_f16x2x2(byte_perm(r0, 0x3120), e0, o0);  // tokens tq, tq + 1
                     e4m3x4_to_f16x2x2(byte_perm(r1, 0x3120), e1, o1);  // tokens 8 + tq, 9 + tq
                     mma_f16(acc[c], e0, o0, e1, o1, pb0, pb1);
@@ -488,29 +468,24 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
         if constexpr (!TR) {
-            // ---- S = Q K^T per block: two n-tiles of 8 tokens, each with two
-            // accumulators (even / odd k-steps) so that the dependent MMA chains
-            // are KSTEPS/2 long
-            float sc[BPS][2][AR];
-    #pragma unroll
-            for (int b = 0; b < BPS; ++b) {
-    #pragma unroll
-                for (int r = 0; r < AR; ++r) sc[b][0][r] = sc[b][1][r] = 0.f;
-                if (b >= nb) continue;
+            // ---- S = Q K^T of the block: two n-tiles of 8 tokens, each with
+            // two accumulators (even / odd k-steps) so that the dependent MMA
+            // chains are KSTEPS/2 long
+            float sc[2][AR];
+            {
                 float s0[AR], s1[AR], t0[AR], t1[AR];
-    #pragma unroll
+#pragma unroll
                 for (int r = 0; r < AR; ++r) s0[r] = s1[r] = t0[r] = t1[r] = 0.f;
-                const uint32_t kbase = kb[b];
                 if constexpr (FP8) {
                     // E4M3 K: ldmatrix on the codes seen as b16 gives each lane dims
                     // 4(lane%4)..+3 of one token per 16-dim chunk; matrices: (tokens
                     // 0-7, chunk j), (8-15, j), (0-7, j+1), (8-15, j+1)
                     const int tok = (lane & 7) + 8 * ((lane >> 3) & 1);
-    #pragma unroll
+#pragma unroll
                     for (int j = 0; j < KSTEPS; j += 2) {
                         const uint32_t ch = static_cast<uint32_t>(j + (lane >> 4));
                         uint32_t r0, r1, r2, r3, b0, b1;
-                        ldsm_x4(kbase + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
+                        ldsm_x4(kb + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
                         e4m3x4_to_f16x2x2(r0, b0, b1);
                         mma_frag_t<true>(s0, qa[j], b0, b1);
                         e4m3x4_to_f16x2x2(r1, b0, b1);
@@ -521,59 +496,51 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         mma_frag_t<true>(t1, qa[j + 1], b0, b1);
                     }
                 } else {
-    #pragma unroll
+#pragma unroll
                     for (int kp = 0; kp < KSTEPS / 2; ++kp) {
                         const int cg = 4 * kp + (lane >> 3);  // 8-element column chunk 0 .. D/8-1
                         const uint32_t col = (cg >> 3) * Cfg::kRegionBytes + ((((uint32_t)cg & 7u) ^ sw) << 4);
                         uint32_t b0, b1, b2, b3;
-                        ldsm_x4(kbase + col + (lane & 7) * 128, b0, b1, b2, b3);
+                        ldsm_x4(kb + col + (lane & 7) * 128, b0, b1, b2, b3);
                         mma_frag(s0, qa[2 * kp], b0, b1);
                         mma_frag(t0, qa[2 * kp + 1], b2, b3);
-                        ldsm_x4(kbase + col + (8 + (lane & 7)) * 128, b0, b1, b2, b3);
+                        ldsm_x4(kb + col + (8 + (lane & 7)) * 128, b0, b1, b2, b3);
                         mma_frag(s1, qa[2 * kp], b0, b1);
                         mma_frag(t1, qa[2 * kp + 1], b2, b3);
                     }
                 }
-    #pragma unroll
+#pragma unroll
                 for (int r = 0; r < AR; ++r) {
-                    sc[b][0][r] += s0[r] + t0[r];
-                    sc[b][1][r] += s1[r] + t1[r];
+                    sc[0][r] = s0[r] + t0[r];
+                    sc[1][r] = s1[r] + t1[r];
                 }
             }
 
-            // ---- online softmax over the step's keys (rows r_lo and r_lo + 8);
-            // key t of block b is visible to a row iff t < valid[b] and
-            // (cj + b)*16 + t <= the row's limit
-            uint32_t plo[BPS][2], phi[BPS][2];  // P as bf16 / f16 pairs: [block][tokens tq.. / 8+tq..]
+            // ---- online softmax over the block's keys (rows r_lo and r_lo + 8);
+            // key t is visible to a row iff t < valid and cj*16 + t <= the
+            // row's limit
+            uint32_t plo[1][2], phi[1][2];  // P as bf16 / f16 pairs: tokens tq.. / 8+tq..
             float alpha_lo, alpha_hi = 1.f;
             {
-                float x[4 * BPS];
-    #pragma unroll
-                for (int b = 0; b < BPS; ++b) {
-                    const int vis = min(valid[b] - 1, lim_lo - (cj + b) * kBlockTokens);  // last visible key
-                    x[4 * b + 0] = tq <= vis ? sc[b][0][0] * sl2 : -INFINITY;
-                    x[4 * b + 1] = tq + 1 <= vis ? sc[b][0][1] * sl2 : -INFINITY;
-                    x[4 * b + 2] = tq + 8 <= vis ? sc[b][1][0] * sl2 : -INFINITY;
-                    x[4 * b + 3] = tq + 9 <= vis ? sc[b][1][1] * sl2 : -INFINITY;
-                }
-                alpha_lo = softmax_update<FP8, BPS>(m_lo, l_lo, x, plo);
+                const int vis = min(valid - 1, lim_lo - cj * kBlockTokens);  // last visible key
+                const float x[4] = {tq <= vis ? sc[0][0] * sl2 : -INFINITY,
+                                    tq + 1 <= vis ? sc[0][1] * sl2 : -INFINITY,
+                                    tq + 8 <= vis ? sc[1][0] * sl2 : -INFINITY,
+                                    tq + 9 <= vis ? sc[1][1] * sl2 : -INFINITY};
+                alpha_lo = softmax_update<FP8, 1>(m_lo, l_lo, x, plo);
             }
             if constexpr (HI) {
-                float x[4 * BPS];
-    #pragma unroll
-                for (int b = 0; b < BPS; ++b) {
-                    const int vis = min(valid[b] - 1, lim_hi - (cj + b) * kBlockTokens);
-                    x[4 * b + 0] = tq <= vis ? sc[b][0][2] * sl2 : -INFINITY;
-                    x[4 * b + 1] = tq + 1 <= vis ? sc[b][0][3] * sl2 : -INFINITY;
-                    x[4 * b + 2] = tq + 8 <= vis ? sc[b][1][2] * sl2 : -INFINITY;
-                    x[4 * b + 3] = tq + 9 <= vis ? sc[b][1][3] * sl2 : -INFINITY;
-                }
-                alpha_hi = softmax_update<FP8, BPS>(m_hi, l_hi, x, phi);
+                const int vis = min(valid - 1, lim_hi - cj * kBlockTokens);
+                const float x[4] = {tq <= vis ? sc[0][2] * sl2 : -INFINITY,
+                                    tq + 1 <= vis ? sc[0][3] * sl2 : -INFINITY,
+                                    tq + 8 <= vis ? sc[1][2] * sl2 : -INFINITY,
+                                    tq + 9 <= vis ? sc[1][3] * sl2 : -INFINITY};
+                alpha_hi = softmax_update<FP8, 1>(m_hi, l_hi, x, phi);
             }
             // rescale the accumulators only when some row's max moved (alpha is
             // exactly 1 otherwise): after the first blocks of a sequence it rarely does
             if (__any_sync(kFullMask, alpha_lo != 1.f || alpha_hi != 1.f)) {
-    #pragma unroll
+#pragma unroll
                 for (int n = 0; n < NTD; ++n) {
                     acc[n][0] *= alpha_lo;
                     acc[n][1] *= alpha_lo;
@@ -584,69 +551,59 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
             }
 
-            // ---- O += P V : n-tiles of 8 head dims, K = the 16 tokens of a block
-    #pragma unroll
-            for (int b = 0; b < BPS; ++b) {
-                if (b >= nb) continue;
-                uint32_t pa[AR];  // P as an A fragment
-                if constexpr (HI) {
-                    pa[0] = plo[b][0]; pa[1] = phi[b][0]; pa[2] = plo[b][1]; pa[3] = phi[b][1];
-                } else {
-                    pa[0] = plo[b][0]; pa[1] = plo[b][1];
+            // ---- O += P V : n-tiles of 8 head dims, K = the 16 tokens of the block
+            uint32_t pa[AR];  // P as an A fragment
+            if constexpr (HI) {
+                pa[0] = plo[0][0]; pa[1] = phi[0][0]; pa[2] = plo[0][1]; pa[3] = phi[0][1];
+            } else {
+                pa[0] = plo[0][0]; pa[1] = plo[0][1];
+            }
+            if constexpr (FP8) {
+                // E4M3 V: ldmatrix.trans on the codes seen as b16 gives each lane
+                // tokens 2(lane%4), +1 of the dim pair 2(lane/4), +1 of a 16-dim
+                // chunk; one byte permute splits it into the even and the odd
+                // dim's token pair.  n-tile 2c of the accumulators holds the even
+                // dims 16c + 2n of chunk c, n-tile 2c+1 the odd dims.
+                const int tok = (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+                for (int c = 0; c < D / 16; c += 2) {
+                    const uint32_t ch = static_cast<uint32_t>(c + (lane >> 4));
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4_trans(vb + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
+                    uint32_t e0, o0, e1, o1;
+                    e4m3x4_to_f16x2x2(byte_perm(r0, 0x3120), e0, o0);  // tokens 2(lane%4), +1
+                    e4m3x4_to_f16x2x2(byte_perm(r1, 0x3120), e1, o1);  // tokens 8 + 2(lane%4), +1
+                    mma_frag_t<true>(acc[2 * c], pa, e0, e1);
+                    mma_frag_t<true>(acc[2 * c + 1], pa, o0, o1);
+                    e4m3x4_to_f16x2x2(byte_perm(r2, 0x3120), e0, o0);
+                    e4m3x4_to_f16x2x2(byte_perm(r3, 0x3120), e1, o1);
+                    mma_frag_t<true>(acc[2 * c + 2], pa, e0, e1);
+                    mma_frag_t<true>(acc[2 * c + 3], pa, o0, o1);
                 }
-                const uint32_t vbase = vb[b];
-                if constexpr (FP8) {
-                    // E4M3 V: ldmatrix.trans on the codes seen as b16 gives each lane
-                    // tokens 2(lane%4), +1 of the dim pair 2(lane/4), +1 of a 16-dim
-                    // chunk; one byte permute splits it into the even and the odd
-                    // dim's token pair.  n-tile 2c of the accumulators holds the even
-                    // dims 16c + 2n of chunk c, n-tile 2c+1 the odd dims.
-                    const int tok = (lane & 7) + 8 * ((lane >> 3) & 1);
-    #pragma unroll
-                    for (int c = 0; c < D / 16; c += 2) {
-                        const uint32_t ch = static_cast<uint32_t>(c + (lane >> 4));
-                        uint32_t r0, r1, r2, r3;
-                        ldsm_x4_trans(vbase + tok * Cfg::kRowBytes + ((ch ^ Cfg::swz(tok)) << 4), r0, r1, r2, r3);
-                        uint32_t e0, o0, e1, o1;
-                        e4m3x4_to_f16x2x2(byte_perm(r0, 0x3120), e0, o0);  // tokens 2(lane%4), +1
-                        e4m3x4_to_f16x2x2(byte_perm(r1, 0x3120), e1, o1);  // tokens 8 + 2(lane%4), +1
-                        mma_frag_t<true>(acc[2 * c], pa, e0, e1);
-                        mma_frag_t<true>(acc[2 * c + 1], pa, o0, o1);
-                        e4m3x4_to_f16x2x2(byte_perm(r2, 0x3120), e0, o0);
-                        e4m3x4_to_f16x2x2(byte_perm(r3, 0x3120), e1, o1);
-                        mma_frag_t<true>(acc[2 * c + 2], pa, e0, e1);
-                        mma_frag_t<true>(acc[2 * c + 3], pa, o0, o1);
-                    }
-                } else {
-    #pragma unroll
-                    for (int dp = 0; dp < D / 16; ++dp) {
-                        const int cg = 2 * dp + (lane >> 4);
-                        const int t = 8 * ((lane >> 3) & 1) + (lane & 7);
-                        const uint32_t addr = vbase + (cg >> 3) * Cfg::kRegionBytes + t * 128 +
-                                              ((((uint32_t)cg & 7u) ^ sw) << 4);
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4_trans(addr, b0, b1, b2, b3);
-                        mma_frag(acc[2 * dp], pa, b0, b1);
-                        mma_frag(acc[2 * dp + 1], pa, b2, b3);
-                    }
+            } else {
+#pragma unroll
+                for (int dp = 0; dp < D / 16; ++dp) {
+                    const int cg = 2 * dp + (lane >> 4);
+                    const int t = 8 * ((lane >> 3) & 1) + (lane & 7);
+                    const uint32_t addr = vb + (cg >> 3) * Cfg::kRegionBytes + t * 128 +
+                                          ((((uint32_t)cg & 7u) ^ sw) << 4);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_trans(addr, b0, b1, b2, b3);
+                    mma_frag(acc[2 * dp], pa, b0, b1);
+                    mma_frag(acc[2 * dp + 1], pa, b2, b3);
                 }
             }
         }
         __syncwarp();
 
-        // ---- hand the stages back to the producer
-#pragma unroll
-        for (int b = 0; b < BPS; ++b) {
-            if (b >= nb) continue;
-            if (prod_live) produce(stage);
-            if (++stage == STAGES) {
-                stage = 0;
-                phase ^= 1;
-            }
+        // ---- hand the stage back to the producer
+        if (prod_live) produce(stage);
+        if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
         }
 
-        cj += nb;
-        if (cj < cc.jend) continue;
+        if (++cj < cc.jend) continue;
 
         // ---- item done: final row or partition partials
         if constexpr (FP8) {  // the sums of P V used the V codes: apply the V scale once

@@ -33,6 +33,7 @@ PA_DEVERR_BLOCK_OOB = 2
 PA_DEVERR_SEQ_LEN = 4
 PA_DEVERR_TIMEOUT = 8
 PA_DEVERR_PREFIX = 16
+PA_DEVERR_Q_RANGE = 32
 
 # every symbol the header declares, with (restype, argtypes)
 _P, _I32, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float

@@ -386,10 +386,16 @@ def config_plan(name: str, seed: int = 0) -> Plan:
     return plan(lens, seed=seed, num_blocks=16 if name == "tiny" else None, prefix_len=prefix)
 
 
-def make(name: str, seed: int = 0, device="cpu", poison_unused: bool = False, **kw) -> Workload:
-    """One of the five named workloads (see CONFIGS)."""
+def make(name: str, seed: int = 0, device="cpu", poison_unused: bool = False,
+         max_seqs: Optional[int] = None, **kw) -> Workload:
+    """One of the five named workloads (see CONFIGS).  ``max_seqs`` keeps only
+    the first sequences of the batch (a smaller case of the same shape, for
+    profiler captures)."""
     desc = CONFIGS[name]["desc"]
     lens, prefix = config_lens(name, seed)
+    if max_seqs is not None:
+        lens = lens[:max_seqs]
+        desc += f" (first {len(lens)} sequences only)"
     common = dict(seed=seed, device=device, poison_unused=poison_unused, name=name, desc=desc)
     if name == "tiny":
         return build(lens, 2, 1, 64, torch.float32, num_blocks=16, **common, **kw)

@@ -1,5 +1,8 @@
 """Shared test helpers: run the CUDA path and the oracle on the same seeded
 inputs and compare them with the stated tolerances."""
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import torch
 
@@ -50,3 +53,65 @@ def gpu_decode(w: wl.Workload, partition_blocks=None, max_seq_len=None, q=None, 
 def oracle_decode(w: wl.Workload, h=None, rows=None):
     h = h or host(w)
     return oracle.paged_decode(h["q"], h["kc"], h["vc"], h["bt"], h["sl"], w.scale, rows=rows)
+
+
+def host_threads() -> int:
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_decode_all_rows(w: wl.Workload, h=None) -> np.ndarray:
+    """Every (sequence, query head) row of the oracle's decode, [N, Hq, D].
+    The same plain oracle as oracle_decode, run as one task per (sequence, kv
+    head) on host threads (the C oracle releases the interpreter lock), longest
+    sequences first, so that full-size batches are compared in seconds."""
+    h = h or host(w)
+    N, Hq, D = h["q"].shape
+    Hkv = h["kc"].shape[1]
+    g = Hq // Hkv
+    out = np.zeros((N, Hq, D), dtype=np.float64)
+    units = sorted(((s, kh) for s in range(N) for kh in range(Hkv)), key=lambda u: -int(h["sl"][u[0]]))
+
+    def run(u):
+        s, kh = u
+        rows = [(s, kh * g + i) for i in range(g)]
+        out[s, kh * g:(kh + 1) * g] = oracle.paged_decode(h["q"], h["kc"], h["vc"], h["bt"], h["sl"], w.scale,
+                                                          rows=rows)
+
+    with ThreadPoolExecutor(max_workers=host_threads()) as ex:
+        list(ex.map(run, units))
+    return out
+
+
+def oracle_decode_fp8_all_rows(q, kc, vc, bt, sl, ks, vs, scale) -> np.ndarray:
+    """oracle.paged_decode_fp8 over a whole batch, one task per sequence on
+    host threads (each task sees its own sequence's query rows, table and
+    length, and the whole pools)."""
+    N, Hq, D = q.shape
+    out = np.zeros((N, Hq, D), dtype=np.float64)
+    order = sorted(range(N), key=lambda s: -int(sl[s]))
+
+    def run(s):
+        out[s:s + 1] = oracle.paged_decode_fp8(q[s:s + 1], kc, vc, bt[s:s + 1], sl[s:s + 1], ks, vs, scale)
+
+    with ThreadPoolExecutor(max_workers=host_threads()) as ex:
+        list(ex.map(run, order))
+    return out
+
+
+def oracle_decode_multi_all_rows(q, kc, vc, bt, sl, qs, scale) -> np.ndarray:
+    """oracle.paged_decode_multi over a whole batch, one task per sequence on
+    host threads (q_start rebased to each sequence's rows)."""
+    T, Hq, D = q.shape
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    N = len(sl)
+    order = sorted(range(N), key=lambda s: -int(sl[s]) * int(qs[s + 1] - qs[s]))
+
+    def run(s):
+        a, b = int(qs[s]), int(qs[s + 1])
+        if b > a:
+            out[a:b] = oracle.paged_decode_multi(q[a:b], kc, vc, bt[s:s + 1], sl[s:s + 1],
+                                                 np.array([0, b - a], dtype=np.int32), scale)
+
+    with ThreadPoolExecutor(max_workers=host_threads()) as ex:
+        list(ex.map(run, order))
+    return out

@@ -194,3 +194,21 @@ def test_fp8_entry_points_reject_bad_arguments_on_the_host(lib):
 
 def test_get_device_error_rejects_null(lib):
     assert lib.pa_get_device_error(None, 0, None) == pa.PA_ERR_INVALID_ARG
+
+
+def _comment_before(name: str) -> str:
+    """The comment block that directly precedes the declaration of `name`."""
+    src = open(HEADER).read()
+    i = re.search(r"PA_API[^;]*?\b" + name + r"\s*\(", src).start()
+    j = src.rfind("*/", 0, i)
+    return src[src.rfind("/*", 0, j):j]
+
+
+@pytest.mark.parametrize("name", ["pa_cache_write", "pa_decode", "pa_decode_workspace_size",
+                                  "pa_get_device_error", "pa_status_string"])
+def test_boundary_calls_cite_a_passage_or_say_plumbing(name):
+    """Each call of the boundary names the page passage that defines it, or
+    says that it is interface plumbing with no passage."""
+    c = _comment_before(name)
+    pages = ("slavadubrov.com", "aiunderstanding.org", "de.news.hada.io", "artificials.ru")
+    assert any(p in c for p in pages) or "Interface plumbing" in c, name

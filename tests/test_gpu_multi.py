@@ -59,27 +59,6 @@ def test_one_query_token_each_is_bitwise_the_decode():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-def test_speculative_check_on_the_gqa_workload_sampled_rows():
-    """The GQA workload at full size with 4 query tokens per sequence (the
-    check of 3 drafted tokens + 1)."""
-    w = wl.make("gqa", device=DEV)
-    nq = [4] * w.num_seqs
-    q, qs = _queries(nq, w.num_q_heads, w.head_dim, seed=9)
-    out = pa.decode_multi(q, qs, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, 4,
-                          max_seq_len=w.max_seq_len)
-    torch.cuda.synchronize()
-    rng = np.random.default_rng(1)
-    seqs = sorted(set(int(x) for x in rng.integers(0, w.num_seqs, 12)) | {int(np.argmax(w.lens_host))})
-    # oracle on the sampled sequences only (their tables and lengths)
-    h = host(w)
-    sel_q = np.concatenate([wl.as_numpy(q)[4 * s:4 * s + 4] for s in seqs])
-    ref = oracle.paged_decode_multi(sel_q, h["kc"], h["vc"], h["bt"][seqs], h["sl"][seqs],
-                                    np.arange(0, 4 * len(seqs) + 1, 4, dtype=np.int32), w.scale)
-    got = np.concatenate([to_f64(out)[4 * s:4 * s + 4] for s in seqs])
-    assert_close(got, ref, torch.bfloat16, "gqa speculative check")
-    assert pa.device_error() == 0
-
-
 def test_too_many_query_tokens_are_flagged():
     w = wl.build([40, 40], 8, 2, 128, torch.bfloat16, seed=4, device=DEV)
     q, qs = _queries([2, 5], 8, 128, seed=4)  # the second sequence has 5 > max_q_len = 4

@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import assert_close, gpu_decode, host, oracle_decode, to_f64
+from helpers import assert_close, gpu_decode, host, oracle_decode, oracle_decode_all_rows, to_f64
 from paged_kv_cache_432_b200 import pagedattn as pa
 from paged_kv_cache_432_b200 import workload as wl
 
@@ -113,34 +113,6 @@ def test_config_shapes_reduced_lengths(name, Hq, Hkv):
     assert_close(to_f64(out), oracle_decode(w), torch.bfloat16, name)
 
 
-# ------------------------------------------------------------------ full-size configs, sampled rows
-def _sample_rows(w, n, seed):
-    rng = np.random.default_rng(seed)
-    rows = {(int(rng.integers(w.num_seqs)), int(rng.integers(w.num_q_heads))) for _ in range(n)}
-    longest = int(np.argmax(w.lens_host))
-    rows |= {(longest, 0), (longest, w.num_q_heads - 1), (0, 0)}
-    return sorted(rows)
-
-
-@pytest.mark.parametrize("name,nrows", [("mha", 48), ("gqa", 48), ("prefix", 32), ("long", 12)])
-def test_full_size_config_sampled_rows(name, nrows):
-    """The config at full size, in the launch configuration the benchmark times
-    (cache write of the newest token, then decode with the config's partition
-    setting); sampled (sequence, head) rows against the oracle."""
-    w = wl.make(name, device=DEV)
-    h = host(w)  # pre-write pools
-    pa.cache_write(w.new_k, w.new_v, w.slot_mapping, w.k_cache, w.v_cache)
-    out = gpu_decode(w)
-    h["kc"], h["vc"], _ = oracle.cache_write(h["nk"], h["nv"], h["sm"], h["kc"], h["vc"])
-    rows = _sample_rows(w, nrows, seed=len(name))
-    ref = oracle_decode(w, h, rows=rows)
-    g = to_f64(out)
-    got = np.stack([g[s, qh] for s, qh in rows])
-    assert_close(got, ref, torch.bfloat16, name)
-    assert np.isfinite(g).all()
-    assert pa.device_error() == 0
-
-
 # ------------------------------------------------------------------ invariances (bitwise on the GPU)
 def test_physical_permutation_is_bitwise_invariant():
     w = wl.build([35, 1, 16, 17, 700, 1500, 96], 32, 8, 128, torch.bfloat16, seed=21, device=DEV)
@@ -172,10 +144,7 @@ def test_shared_prefix_matches_private_copies_bitwise(prefix_len):
         i += len(t)
     private = gpu_decode(w, k_cache=kc, v_cache=vc, block_tables=bt)
     assert torch.equal(shared.view(torch.int16), private.view(torch.int16))
-    rows = _sample_rows(w, 16, seed=prefix_len)
-    ref = oracle_decode(w, rows=rows)
-    g = to_f64(shared)
-    assert_close(np.stack([g[s, qh] for s, qh in rows]), ref, torch.bfloat16, "prefix")
+    assert_close(to_f64(shared), oracle_decode_all_rows(w), torch.bfloat16, "prefix, every row")
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
@@ -233,23 +202,6 @@ def test_shared_prefix_decode_matches_oracle(prefix_len, suffixes, Hq, Hkv, D, p
     assert w.shared_prefix_blocks == prefix_len // 16
     out = _shared_prefix_decode(w, pb)
     assert_close(to_f64(out), oracle_decode(w), torch.bfloat16, f"shared prefix {prefix_len}")
-    assert pa.device_error() == 0
-
-
-def test_shared_prefix_full_size_workload_sampled_rows():
-    """The prefix-sharing workload at full size through the shared-prefix path,
-    after the cache write of each sequence's newest token."""
-    w = wl.make("prefix", device=DEV)
-    h = host(w)
-    pa.cache_write(w.new_k, w.new_v, w.slot_mapping, w.k_cache, w.v_cache)
-    out = _shared_prefix_decode(w)
-    h["kc"], h["vc"], _ = oracle.cache_write(h["nk"], h["nv"], h["sm"], h["kc"], h["vc"])
-    rows = _sample_rows(w, 40, seed=7)
-    ref = oracle_decode(w, h, rows=rows)
-    g = to_f64(out)
-    assert_close(np.stack([g[s, qh] for s, qh in rows]), ref, torch.bfloat16, "prefix full size")
-    plain = to_f64(gpu_decode(w))
-    assert_close(g, plain, torch.bfloat16, "shared-prefix vs plain decode")
     assert pa.device_error() == 0
 
 
