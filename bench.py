@@ -29,8 +29,9 @@ the cache write's reads and writes.  Decode tokens/s = sequences / step time.
 from __future__ import annotations
 
 import argparse
-import hashlib
 import glob
+import hashlib
+import itertools
 import json
 import math
 import os
@@ -48,6 +49,7 @@ from paged_kv_cache_432_b200 import workload as wl  # noqa: E402
 
 FLUSH_BYTES = 512 << 20
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 METRIC = "paged decode attention KV GB/s and decode tokens/s on 1 B200 vs 8 TB/s HBM roofline"
 
 
@@ -126,6 +128,28 @@ def load_peaks() -> tuple:
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_tensor_peak() -> tuple:
+    """Dense bf16 tensor peak in TFLOP/s: the measured burst figure (a kernel
+    timed alone), else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def causal_flops(lens, n_per_seq, num_q_heads, head_dim) -> int:
+    """Algorithmic FLOPs of several query tokens per sequence: token k of n
+    sees L - n + k + 1 keys; per (token, head, key) 2 D for q . k and 2 D for
+    p . v."""
+    tot = 0
+    for L, n in zip(lens, n_per_seq):
+        n = min(n, L)
+        tot += n * (L - n) + n * (n + 1) // 2
+    return 4 * head_dim * num_q_heads * tot
 
 
 def load_traffic(tag: str):
@@ -385,7 +409,9 @@ def run_reference(args) -> None:
     ws, rank = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = wl.make(args.config, seed=args.seed, device="cpu", max_seqs=args.max_seqs)
+    ng = getattr(args, "prompt_groups", 1)
+    extra = {"prompt_groups": ng} if ng > 1 else {}
+    w = wl.make(args.config, seed=args.seed, device="cpu", max_seqs=args.max_seqs, **extra)
     h = host_arrays(w)
     Hkv = w.num_kv_heads
     all_units = [(s, kh) for s in range(w.num_seqs) if w.lens_host[s] > 0 for kh in range(Hkv)]
@@ -436,7 +462,8 @@ def run_ours(args) -> None:
         pa_build.build()
     barrier(ws)
     dev = torch.device("cuda", local)
-    w = wl.make(args.config, seed=replica_seed(args.seed, rank), device=dev, max_seqs=args.max_seqs)
+    extra = {"prompt_groups": args.prompt_groups} if args.prompt_groups > 1 else {}
+    w = wl.make(args.config, seed=replica_seed(args.seed, rank), device=dev, max_seqs=args.max_seqs, **extra)
     pb = w.partition_blocks if args.partition_blocks is None else args.partition_blocks
     msl = w.max_seq_len
     resolved_pb = pa.partition_blocks(w.num_seqs, w.num_kv_heads, msl, pb)
@@ -448,8 +475,15 @@ def run_ours(args) -> None:
         k_inv, v_inv = (1.0 / k_scale).float(), (1.0 / v_scale).float()
         torch.cuda.empty_cache()
     # a batch sharing a prompt prefix goes through the shared-prefix decode
-    use_sp = w.shared_prefix_blocks > 0 and not args.plain_decode and not fp8
-    if use_sp:
+    # (several prompts: the prompt-group form)
+    groups = len(w.group_blocks_host) > 1 and max(w.group_blocks_host) > 0
+    use_sp = (w.shared_prefix_blocks > 0 or groups) and not args.plain_decode and not fp8
+    maxs = max(w.group_blocks_host) if groups else 0
+    if use_sp and groups:
+        n = pa.shared_prefix_groups_workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, msl,
+                                                   maxs, len(w.group_blocks_host), pb)
+        wsp = torch.empty(n, dtype=torch.uint8, device=dev)
+    elif use_sp:
         n = pa.shared_prefix_workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, msl,
                                             w.shared_prefix_blocks, pb)
         wsp = torch.empty(n, dtype=torch.uint8, device=dev)
@@ -471,6 +505,16 @@ def run_ours(args) -> None:
     chunks = math.ceil(w.num_seqs / 2048)
     launches_per_step = 1 + chunks + (chunks if split else 0) + (1 if use_sp else 0)
 
+    def shared_prefix_call(q, block_tables, seq_lens):
+        if groups:
+            pa.decode_shared_prefix_groups(q, w.k_cache, w.v_cache, block_tables, seq_lens, w.scale, w.group_start,
+                                           w.group_blocks, maxs, out=out, max_seq_len=msl, partition_blocks=pb,
+                                           workspace=wsp, stream=stream)
+        else:
+            pa.decode_shared_prefix(q, w.k_cache, w.v_cache, block_tables, seq_lens, w.scale,
+                                    w.shared_prefix_blocks, out=out, max_seq_len=msl, partition_blocks=pb,
+                                    workspace=wsp, stream=stream)
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
@@ -488,9 +532,7 @@ def run_ours(args) -> None:
         if ev is not None:
             ev[1].record(stream)
         if use_sp:  # prefix kernel + private-part decode + merge, one call
-            pa.decode_shared_prefix(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale,
-                                    w.shared_prefix_blocks, out=out, max_seq_len=msl, partition_blocks=pb,
-                                    workspace=wsp, stream=stream)
+            shared_prefix_call(w.q, w.block_tables, w.seq_lens)
             if ev is not None:
                 ev[2].record(stream)
                 ev[3].record(stream)
@@ -590,9 +632,7 @@ def run_ours(args) -> None:
                 return
             pa.cache_write(dev_in["new_k"], dev_in["new_v"], dev_in["slot_mapping"], w.k_cache, w.v_cache, stream)
             if use_sp:
-                pa.decode_shared_prefix(dev_in["q"], w.k_cache, w.v_cache, dev_in["block_tables"],
-                                        dev_in["seq_lens"], w.scale, w.shared_prefix_blocks, out=out,
-                                        max_seq_len=msl, partition_blocks=pb, workspace=wsp, stream=stream)
+                shared_prefix_call(dev_in["q"], dev_in["block_tables"], dev_in["seq_lens"])
             else:
                 pa.decode(dev_in["q"], w.k_cache, w.v_cache, dev_in["block_tables"], dev_in["seq_lens"], w.scale,
                           out=out, max_seq_len=msl, partition_blocks=pb, workspace=wsp, stream=stream)
@@ -624,7 +664,8 @@ def run_ours(args) -> None:
     achieved = by["decode"] / (dec_ms * 1e-3) / 1e9
     kname = "decode_bf16_mma_kernel" if w.dtype == torch.bfloat16 else "decode_f32_simt_kernel"
     if use_sp:
-        kname = "pa_decode_shared_prefix (prefix kernel + decode_bf16_mma_kernel + reduce, timed together)"
+        kname = ("pa_decode_shared_prefix_groups" if groups else "pa_decode_shared_prefix") + \
+            " (attn_tiles_tc_kernel + decode_bf16_mma_kernel + reduce, timed together)"
     if fp8:
         kname = "pa_decode_fp8 (decode_bf16_mma_kernel<E4M3> + reduce, timed together)"
     roof = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1), "peak": peak,
@@ -732,8 +773,10 @@ def run_copy_blocks(args) -> None:
 
 def run_multi(args) -> None:
     """Several query tokens per sequence (pa_decode_multi): the check step of
-    speculative decoding with q_len - 1 drafted tokens.  The KV of every
-    sequence is read once for all its query tokens."""
+    speculative decoding with q_len - 1 drafted tokens, or (group x q_len > 16)
+    a prefill chunk of q_len tokens on the tensor-memory tile kernel.  A
+    sequence shorter than q_len takes all its positions as query tokens.  The
+    KV of every sequence is read once for all its query tokens (per tile)."""
     from paged_kv_cache_432_b200 import build as pa_build
     from paged_kv_cache_432_b200 import pagedattn as pa
 
@@ -744,9 +787,10 @@ def run_multi(args) -> None:
     dev = torch.device("cuda", local)
     w = wl.make(args.config, seed=replica_seed(args.seed, rank), device=dev)
     nq = args.q_len
+    n_per = [min(nq, L) for L in w.lens_host]
     gen = torch.Generator(device=dev).manual_seed(args.seed + 7)
-    q = torch.randn((w.num_seqs * nq, w.num_q_heads, w.head_dim), generator=gen, device=dev).to(w.dtype)
-    qs = torch.arange(0, w.num_seqs * nq + 1, nq, dtype=torch.int32, device=dev)
+    q = torch.randn((sum(n_per), w.num_q_heads, w.head_dim), generator=gen, device=dev).to(w.dtype)
+    qs = torch.tensor([0] + list(itertools.accumulate(n_per)), dtype=torch.int32, device=dev)
     out = torch.empty_like(q)
     pb = w.partition_blocks if args.partition_blocks is None else args.partition_blocks
     msl = w.max_seq_len
@@ -776,10 +820,24 @@ def run_multi(args) -> None:
             e[1].record(stream)
         torch.cuda.synchronize(dev)
     barrier(ws)
-    agg = aggregate(sum(a.elapsed_time(b) for a, b in evs) / args.steps, step_bytes, w.num_seqs * nq, ws)
+    step_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    agg = aggregate(step_ms, step_bytes, sum(n_per), ws)
     peak, peak_kind = load_peaks()
     if pa.device_error() != 0:
         raise RuntimeError("device error flagged")
+    tiles = w.group * nq > 16  # more rows per (sequence, kv head) than one warp-level MMA holds
+    flops = causal_flops(w.lens_host, n_per, w.num_q_heads, w.head_dim)
+    if tiles:  # a prefill chunk: tensor-core bound
+        tpeak, tkind = load_tensor_peak()
+        ach = flops / (max_over_ranks(step_ms, ws) * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "attn_tiles_tc_kernel (+ merge when the keys are cut)",
+                "achieved": round(ach, 1), "peak": tpeak, "unit": "TFLOP/s", "frac": round(ach / tpeak, 4),
+                "peak_source": f"{tkind} (MEASURED_PEAKS.json bf16_tflops, burst)" if tkind == "measured"
+                else "fallback 1590 TFLOP/s", "algorithmic_flops_per_step": flops, "traffic": None}
+    else:
+        roof = {"bound": "hbm", "kernel": "decode_bf16_mma_kernel + reduce", "achieved": round(agg["gbs"] / ws, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(agg["gbs"] / ws / peak, 4),
+                "peak_source": peak_kind, "traffic": None}
     line = {"metric": f"multi-token paged decode KV GB/s ({nq} query tokens per sequence)",
             "value": round(agg["gbs"], 1), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(agg["step_ms"], 5), "higher_is_better": True,
@@ -787,9 +845,8 @@ def run_multi(args) -> None:
             "config": dict(workload_config(w, pa.partition_blocks(w.num_seqs, w.num_kv_heads, msl, pb)),
                            op="pa_decode_multi", q_len=nq),
             "query_tokens_per_s": round(agg["tokens_per_s"], 1),
-            "roofline": {"bound": "hbm", "kernel": "decode_bf16_mma_kernel + reduce", "achieved": round(agg["gbs"] / ws, 1),
-                         "peak": peak, "unit": "GB/s", "frac": round(agg["gbs"] / ws / peak, 4),
-                         "peak_source": peak_kind, "traffic": None},
+            "tflops": round(flops * ws / (agg["step_ms"] * 1e-3) / 1e12, 2),
+            "roofline": roof,
             "clocks": cs.summary(), "gpu_launches": 2 * args.steps}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -814,6 +871,8 @@ def main():
     ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
                     help="KV pool element type for --op step (fp8: E4M3 codes with per-head scales)")
     ap.add_argument("--partition-blocks", type=int, default=None)
+    ap.add_argument("--prompt-groups", type=int, default=1,
+                    help="--config prefix: that many prompts, each shared by a consecutive share of the batch")
     ap.add_argument("--max-seqs", type=int, default=None,
                     help="keep only the first N sequences of the workload (a smaller case of the same "
                          "shape, for profiler captures; not a bench line)")

@@ -37,7 +37,7 @@
  * pa_decode_shared_prefix, pa_decode_noalloc) launches its kernels with
  * programmatic stream serialization, so they may start before the previous
  * kernel in the stream has finished.  Before waiting for that kernel they
- * already read seq_lens, block_tables, q_start and q (they never touch the
+ * already read seq_lens, block_tables, q_start, the prefix groups and q (they never touch the
  * caches, out or the workspace before the wait).  This is safe whenever the
  * previous kernel in the stream did not trigger its dependents early (a kernel
  * that never executes griddepcontrol.launch_dependents /
@@ -168,10 +168,16 @@ PA_API int pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache
  * (int32 [num_seqs+1], q_start[num_seqs] = num_q_rows) of q and out, both
  * [num_q_rows][num_q_heads][head_dim].  They are the sequence's last n
  * positions (their K/V already in the cache), so token k attends to keys
- * 0 .. seq_lens[s] - n + k (causal among the new tokens).  Needs PA_DTYPE_BF16
- * and group * max_q_len <= 16; a sequence with more than max_q_len or more
- * than seq_lens[s] query tokens has the excess ignored (its rows are not
- * written) and PA_DEVERR_SEQ_LEN set.  Workspace from
+ * 0 .. seq_lens[s] - n + k (causal among the new tokens).  Needs PA_DTYPE_BF16.
+ * With group * max_q_len <= 16 the (token, head) rows of a (sequence, kv head)
+ * fit one warp-level MMA tile and run in the decode kernel (the check of a few
+ * drafted tokens); with more (prefill chunks of any length), tiles of up to
+ * 128 rows (floor(128 / group) tokens x group heads) of one sequence run on
+ * the tensor-memory kernel, reading each K/V block once per tile, with the
+ * keys cut into at most 16 chunks (merged by a log-sum-exp reduction) only
+ * when there are too few tiles to fill the device.  A sequence with more than
+ * max_q_len or more than seq_lens[s] query tokens has the excess ignored (its
+ * rows are not written) and PA_DEVERR_SEQ_LEN set.  Workspace from
  * pa_decode_multi_workspace_size (rows are query-token rows); other arguments
  * as for pa_decode.  With one query token per sequence this is pa_decode.
  */
@@ -185,7 +191,9 @@ PA_API int pa_decode_multi(const void* q, const int32_t* q_start, int32_t num_q_
                            void* out, int32_t dtype, void* stream);
 
 /* Workspace bytes pa_decode_multi needs: the pa_decode layout with
- * num_q_rows * num_q_heads rows. */
+ * num_q_rows * num_q_heads rows and as many pieces per row as either path can
+ * write (the tile path's key chunks depend on the current device's SM count:
+ * query the size on the device that runs the call). */
 PA_API size_t pa_decode_multi_workspace_size(int32_t num_seqs, int32_t num_q_rows,
                                              int32_t num_q_heads, int32_t num_kv_heads,
                                              int32_t head_dim, int32_t max_seq_len,
@@ -338,6 +346,55 @@ PA_API size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t n
                                                      int32_t max_seq_len, int32_t shared_blocks,
                                                      int32_t block_size,
                                                      int32_t partition_blocks);
+
+/*
+ * Decode for a batch that holds several prompt groups, each stored once: the
+ * sequences of group i are seq group_start[i] .. group_start[i+1]-1 (groups
+ * are consecutive ranges of the batch, group_start[0] = 0 and
+ * group_start[num_groups] = num_seqs), and the first group_shared_blocks[i]
+ * entries of every table of group i are the same physical blocks (those of
+ * the group's first sequence).  This is the general form of
+ * pa_decode_shared_prefix: several system prompts in one batch, or branches
+ * of a request (parallel samples, beams) that share its prompt, each group
+ * with its own prefix length; a group with 0 shared blocks is decoded as by
+ * pa_decode ("Was ändert PagedAttention an der KV-Speicherzuweisung für
+ * LLMs?", slavadubrov.com, §"Gemeinsame Nutzung erfordert mehr als
+ * Speicherzuweisung": parallel sampling and beam search share blocks;
+ * "PagedAttention et vLLM", aiunderstanding.org, §"Mise en œuvre dans le monde
+ * réel" and §"Questions fréquemment posées": many requests with a common
+ * system prompt).  Each group's shared blocks are read once per tile of up to
+ * 128 query rows of its sequences (tensor-memory kernel); each sequence's own
+ * blocks go through the decode kernel; a log-sum-exp reduction merges both.
+ * group_start (int32 [num_groups + 1]) and group_shared_blocks (int32
+ * [num_groups]) are device arrays read like the block tables;
+ * max_shared_blocks is a host bound on group_shared_blocks that sizes the
+ * workspace (pa_decode_shared_prefix_groups_workspace_size).  Device checks
+ * (PA_DEVERR_PREFIX, the rows of an offending group are then meaningless): the
+ * groups are ordered ranges of the batch, no count exceeds max_shared_blocks,
+ * every table of a group starts with its shared blocks and no sequence of a
+ * group is shorter than them.  Only PA_DTYPE_BF16 (max_shared_blocks = 0:
+ * plain pa_decode, any dtype).  Other arguments and errors as pa_decode.
+ */
+PA_API int pa_decode_shared_prefix_groups(const void* q, const void* k_cache, const void* v_cache,
+                                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                          const int32_t* seq_lens, int32_t max_seq_len,
+                                          const int32_t* group_start, const int32_t* group_shared_blocks,
+                                          int32_t num_groups, int32_t max_shared_blocks, int32_t num_seqs,
+                                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                          int32_t num_blocks, int32_t block_size, float scale,
+                                          int32_t partition_blocks, void* workspace, size_t workspace_bytes,
+                                          void* out, int32_t dtype, void* stream);
+
+/*
+ * Workspace bytes pa_decode_shared_prefix_groups needs: the pa_decode layout
+ * with P = min(16, max_shared_blocks) slots for the prefix chunks + the pieces
+ * a whole sequence of max_seq_len tokens can have (a group may share nothing).
+ */
+PA_API size_t pa_decode_shared_prefix_groups_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                                            int32_t num_kv_heads, int32_t head_dim,
+                                                            int32_t max_seq_len, int32_t max_shared_blocks,
+                                                            int32_t num_groups, int32_t block_size,
+                                                            int32_t partition_blocks);
 
 /*
  * Host-side block manager: the bookkeeping that hands out physical blocks.

@@ -20,9 +20,8 @@
 
 #include "cache_write.cuh"
 #include "common.cuh"
+#include "attn_tiles_tc.cuh"
 #include "decode_mma.cuh"
-#include "decode_prefix.cuh"
-#include "decode_prefix_tc.cuh"
 #include "decode_simt.cuh"
 #include "items.cuh"
 #include "lse_reduce.cuh"
@@ -237,48 +236,47 @@ Plan make_plan(int32_t max_seq_len, int32_t partition_blocks) {
     return p;
 }
 
-// Shared-prefix decode: the prefix kernel's key splits are pieces 0..splits-1
-// of every row; the private part of each sequence (blocks from shared_blocks
-// on) is cut as pa_decode would cut a sequence of the remaining length, and
-// its pieces follow.  The workspace reserves kMaxPrefixSplits slots; the launch
-// picks the split count that fills one wave of the prefix kernel on the
-// device (choose_prefix_splits).
-constexpr int32_t kMaxPrefixSplits = 16;
-
-// The shared-prefix kernel: tcgen05 with TMEM accumulators (128 query rows
-// per tile, PA_PREFIX_TC_TILES tiles per CTA), or the mma.sync kernel (64
-// rows per CTA) when built with PA_PREFIX_TC=0.
-#ifndef PA_PREFIX_TC
-#define PA_PREFIX_TC 1
-#endif
-constexpr bool kPrefixTc = PA_PREFIX_TC != 0;
-constexpr int kPrefixTileRows = kPrefixTc ? PrefixTcCfg<128>::kRows : kPrefixRows;  // query rows per CTA
-
-template <int D>
-struct PrefixKernel {
-    using Fn = void (*)(CUtensorMap, CUtensorMap, PrefixParams);
-    static Fn fn() {
-        if constexpr (kPrefixTc) return decode_prefix_tc_kernel<D>;
-        else return decode_prefix_mma_kernel<D>;
-    }
-    static constexpr size_t kSmem = kPrefixTc ? PrefixTcCfg<D>::kSmem : PrefixCfg<D>::kSmem;
-    static constexpr int kThreads = kPrefixTc ? PrefixTcCfg<D>::kThreads : PrefixCfg<D>::kThreads;
-    static constexpr const char* kName = kPrefixTc ? "decode_prefix_tc_kernel" : "decode_prefix_mma_kernel";
-};
+// Shared-prefix decode: the tile kernel's key chunks of the prefix are pieces
+// 0..splits-1 of every row; the private part of each sequence (blocks from
+// shared_blocks on) is cut as pa_decode would cut a sequence of the remaining
+// length, and its pieces follow.  The workspace reserves kMaxTileSplits slots;
+// the launch picks the chunking that fills the device (choose_tile_split).
+constexpr int32_t kMaxTileSplits = 16;
 constexpr int32_t kWideReducePieces = 32;  // rows that can have more pieces merge with a CTA each
+
+// Query tokens (or sequences) per 128-row tile of the tile kernel.
+int32_t tile_tokens(int32_t group) { return 128 / group; }
 
 Plan make_prefix_plan(int32_t max_seq_len, int32_t partition_blocks, int32_t shared_blocks,
                       int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads) {
     const int32_t rest = max_seq_len - shared_blocks * kBlockTokens;
     Plan p = make_plan(rest > 0 ? rest : 0, partition_blocks);
     p.max_len = max_seq_len;
-    const int64_t rows = static_cast<int64_t>(num_seqs) * (num_q_heads / num_kv_heads);
-    p.prefix_row_tiles = static_cast<int32_t>((rows + kPrefixTileRows - 1) / kPrefixTileRows);
+    const int32_t tt = tile_tokens(num_q_heads / num_kv_heads);
+    p.prefix_row_tiles = (num_seqs + tt - 1) / tt;
     if (p.prefix_row_tiles < 1) p.prefix_row_tiles = 1;
     p.shared_blocks = shared_blocks;
-    const int32_t slots = shared_blocks < kMaxPrefixSplits ? shared_blocks : kMaxPrefixSplits;
+    const int32_t slots = shared_blocks < kMaxTileSplits ? shared_blocks : kMaxTileSplits;
     p.prefix_splits = slots;  // reserved; narrowed at launch
     p.prefix_split_blocks = (shared_blocks + slots - 1) / slots;
+    p.max_parts += slots;
+    p.split = true;
+    return p;
+}
+
+// Several prompt groups: every sequence's private part can be as long as the
+// whole sequence (a group may share nothing), and up to kMaxTileSplits
+// prefix chunks come first.  prefix_row_tiles bounds the tiles over all
+// groups.
+Plan make_group_plan(int32_t max_seq_len, int32_t partition_blocks, int32_t max_shared_blocks,
+                     int32_t num_groups, int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads) {
+    Plan p = make_plan(max_seq_len, partition_blocks);
+    const int32_t tt = tile_tokens(num_q_heads / num_kv_heads);
+    p.prefix_row_tiles = (num_seqs + tt - 1) / tt + num_groups;
+    p.shared_blocks = max_shared_blocks;
+    const int32_t slots = max_shared_blocks < kMaxTileSplits ? max_shared_blocks : kMaxTileSplits;
+    p.prefix_splits = slots;
+    p.prefix_split_blocks = (max_shared_blocks + slots - 1) / slots;
     p.max_parts += slots;
     p.split = true;
     return p;
@@ -340,7 +338,7 @@ int check_shapes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, in
 // Validates and fills the kernel parameter block (workspace pointers included).
 // shared_blocks > 0: the shared-prefix decode (plan from make_prefix_plan).
 int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan* plan,
-                   int32_t shared_blocks = 0) {
+                   int32_t shared_blocks = 0, int32_t num_groups = 0) {
     int rc = check_shapes(a.num_seqs, a.num_q_heads, a.num_kv_heads, a.head_dim, a.block_size,
                           a.dtype);
     if (rc != PA_OK) return rc;
@@ -372,8 +370,10 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
         if (shared_blocks > a.max_blocks_per_seq ||
             static_cast<int64_t>(shared_blocks) * kBlockTokens > max_len)
             return PA_ERR_INVALID_ARG;
-        *plan = make_prefix_plan(max_len, a.partition_blocks, shared_blocks, a.num_seqs,
-                                 a.num_q_heads, a.num_kv_heads);
+        *plan = num_groups > 0 ? make_group_plan(max_len, a.partition_blocks, shared_blocks, num_groups,
+                                                 a.num_seqs, a.num_q_heads, a.num_kv_heads)
+                               : make_prefix_plan(max_len, a.partition_blocks, shared_blocks, a.num_seqs,
+                                                  a.num_q_heads, a.num_kv_heads);
     } else {
         *plan = make_plan(max_len, a.partition_blocks);
     }
@@ -413,8 +413,9 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
     P->min_chunk = kMinChunk;
     P->max_parts = plan->max_parts;
     P->len_cap = static_cast<int32_t>(max_len < table_tokens ? max_len : table_tokens);
-    P->skip_blocks = plan->shared_blocks;
+    P->skip_blocks = num_groups > 0 ? 0 : plan->shared_blocks;
     P->piece_base = plan->prefix_splits;
+    P->max_shared = plan->shared_blocks;
     P->scale = a.scale;
     P->scale_log2 = a.scale * 1.4426950408889634f;
     return PA_OK;
@@ -481,7 +482,7 @@ int mma_shape(const DecodeParams& P, LaunchShape* L) {
 
 template <int D, int MAXG>
 int simt_shape(const DecodeParams& P, LaunchShape* L) {
-    return shape_of(decode_f32_simt_kernel<D, MAXG>, kSimtWarps, 8 * static_cast<size_t>(P.seq_count + 1),
+    return shape_of(decode_f32_simt_kernel<D, MAXG>, kSimtWarps, 12 * static_cast<size_t>(P.seq_count + 1),
                     P, L);
 }
 
@@ -565,63 +566,116 @@ int run_partitions(const DecodeParams& P, int32_t dtype, cudaStream_t st) {
     return P.group <= 4 ? launch_simt<64, 4>(P, st) : launch_simt<64, 16>(P, st);
 }
 
-// Key splits of the shared prefix: as many as fill one wave of the prefix
-// kernel (resident CTAs on the device / CTAs per split), within the slots the
-// workspace reserves.  Sets plan->prefix_splits / prefix_split_blocks.
-template <int D>
-int choose_prefix_splits(const DecodeParams& P, Plan* plan) {
-    using K = PrefixKernel<D>;
-    auto kernel = K::fn();
-    int rc = ensure_smem_attr(kernel, K::kSmem);
+// ------------------------------------------------------------ tile kernel (tcgen05)
+// q seen as a 3-D tensor [rows][num_q_heads][head_dim], loaded in boxes of 64
+// columns x `group` heads x `tile_tokens` rows: one box lands as the tile's
+// tile_tokens * group query rows of 128 bytes (one 64-column slab), in the
+// 128-byte swizzle the tensor-core descriptors expect.
+int encode_q_map(CUtensorMap* map, const void* q, int64_t rows, int32_t num_q_heads, int head_dim,
+                 int32_t group) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    int rc = get_encoder(&enc);
     if (rc != PA_OK) return rc;
-    DeviceInfo di;
-    if ((rc = device_info(&di)) != PA_OK) return rc;
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, K::kThreads, K::kSmem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
-    const int64_t wave = static_cast<int64_t>(di.sms) * (per_sm > 0 ? per_sm : 1);
-    const int64_t per_split = static_cast<int64_t>(P.num_kv_heads) * plan->prefix_row_tiles;
-    int64_t splits = wave / per_split;
-    const int32_t slots = plan->prefix_splits;
-    if (splits > slots) splits = slots;
-    if (splits < 1) splits = 1;
-    plan->prefix_split_blocks = static_cast<int32_t>((plan->shared_blocks + splits - 1) / splits);
-    plan->prefix_splits = (plan->shared_blocks + plan->prefix_split_blocks - 1) / plan->prefix_split_blocks;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                          static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                             static_cast<cuuint64_t>(num_q_heads) * head_dim * 2};
+    cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(tile_tokens(group))};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
+                      "cuTensorMapEncodeTiled (q) failed (CUresult %d)", static_cast<int>(r));
+        return PA_ERR_CUDA;
+    }
     return PA_OK;
 }
 
+struct TileSplit {
+    int32_t splits;        // key chunks of the longest unit
+    int32_t chunk_blocks;  // blocks per chunk, a multiple of the 4-block step
+};
+
+// Key chunking for `work_tiles` (tile, kv head) pairs over units of at most
+// nb_max key blocks: as many chunks as fill the device's SMs (one tile-kernel
+// CTA each), at most kMaxTileSplits; one chunk when the tiles alone fill it.
+TileSplit choose_tile_split(int sms, int64_t work_tiles, int32_t nb_max) {
+    int64_t want = work_tiles > 0 ? sms / work_tiles : 1;
+    if (want < 1) want = 1;
+    if (want > kMaxTileSplits) want = kMaxTileSplits;
+    if (nb_max < 1) nb_max = 1;
+    int32_t ch = static_cast<int32_t>((nb_max + want - 1) / want);
+    ch = (ch + kTileStepBlocks - 1) / kTileStepBlocks * kTileStepBlocks;
+    return TileSplit{(nb_max + ch - 1) / ch, ch};
+}
+
 template <int D>
-int launch_prefix(const DecodeParams& P, const Plan& plan, cudaStream_t st) {
-    using K = PrefixKernel<D>;
-    auto kernel = K::fn();
-    int rc = ensure_smem_attr(kernel, K::kSmem);
+int launch_tiles(const TileParams& base, const void* q, int64_t q_rows, const void* k_cache,
+                 const void* v_cache, int64_t items_bound, cudaStream_t st) {
+    auto kernel = attn_tiles_tc_kernel<D>;
+    int rc = ensure_smem_attr(kernel, TileCfg<D>::kSmem);
     if (rc != PA_OK) return rc;
-    const int64_t rows = static_cast<int64_t>(P.num_blocks) * P.num_kv_heads * kBlockTokens;
-    alignas(64) CUtensorMap mk, mv;
-    if ((rc = encode_pool_map(&mk, P.k_cache, rows, D)) != PA_OK) return rc;
-    if ((rc = encode_pool_map(&mv, P.v_cache, rows, D)) != PA_OK) return rc;
-    PrefixParams PP;
-    PP.q = P.q;
-    PP.block_tables = P.block_tables;
-    PP.seq_lens = P.seq_lens;
-    PP.ws_m = P.ws_m;
-    PP.ws_l = P.ws_l;
-    PP.ws_acc = P.ws_acc;
-    PP.num_seqs = P.num_seqs;
-    PP.num_q_heads = P.num_q_heads;
-    PP.num_kv_heads = P.num_kv_heads;
-    PP.group = P.group;
-    PP.max_blocks_per_seq = P.max_blocks_per_seq;
-    PP.num_blocks = P.num_blocks;
-    PP.shared_blocks = plan.shared_blocks;
-    PP.split_blocks = plan.prefix_split_blocks;
-    PP.row_tiles = plan.prefix_row_tiles;
-    PP.max_parts = P.max_parts;
-    PP.scale_log2 = P.scale_log2;
-    const dim3 grid(static_cast<unsigned>(plan.prefix_row_tiles) * plan.prefix_splits,
-                    static_cast<unsigned>(P.num_kv_heads));
-    cudaError_t e = launch_pdl(kernel, grid, dim3(K::kThreads), K::kSmem, st, mk, mv, PP);
-    return e == cudaSuccess ? PA_OK : cuda_fail(e, K::kName);
+    const int64_t rows = static_cast<int64_t>(base.num_blocks) * base.num_kv_heads * kBlockTokens;
+    alignas(64) CUtensorMap mk, mv, mq;
+    if ((rc = encode_pool_map(&mk, k_cache, rows, D)) != PA_OK) return rc;
+    if ((rc = encode_pool_map(&mv, v_cache, rows, D)) != PA_OK) return rc;
+    if ((rc = encode_q_map(&mq, q, q_rows > 0 ? q_rows : 1, base.num_q_heads, D, base.group)) != PA_OK) return rc;
+    DeviceInfo di;
+    if ((rc = device_info(&di)) != PA_OK) return rc;
+    const int32_t units = base.num_units;
+    for (int32_t b = 0; b < units; b += TileCfg<D>::kMaxUnits) {
+        TileParams P = base;
+        P.unit_begin = base.unit_begin + b;
+        P.num_units = units - b < TileCfg<D>::kMaxUnits ? units - b : TileCfg<D>::kMaxUnits;
+        int64_t grid = items_bound < di.sms ? items_bound : di.sms;
+        if (grid < 1) grid = 1;
+        cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(TileCfg<D>::kThreads),
+                                   TileCfg<D>::kSmem, st, mk, mv, mq, P);
+        if (e != cudaSuccess) return cuda_fail(e, "attn_tiles_tc_kernel launch");
+    }
+    return PA_OK;
+}
+
+// The shared prefixes' key chunks through the tile kernel (prefix mode: one
+// group of every sequence, or P.num_groups groups from P.group_start /
+// P.group_blocks); sets plan->prefix_splits / prefix_split_blocks.
+int launch_prefix_tiles(const DecodeParams& P, Plan* plan, cudaStream_t st) {
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc != PA_OK) return rc;
+    const TileSplit sp = choose_tile_split(di.sms, static_cast<int64_t>(plan->prefix_row_tiles) * P.num_kv_heads,
+                                           plan->shared_blocks);
+    plan->prefix_splits = sp.splits;
+    plan->prefix_split_blocks = sp.chunk_blocks;
+    TileParams T;
+    std::memset(&T, 0, sizeof T);
+    T.block_tables = P.block_tables;
+    T.seq_lens = P.seq_lens;
+    T.ws_m = P.ws_m;
+    T.ws_l = P.ws_l;
+    T.ws_acc = P.ws_acc;
+    T.mode = kTileModePrefix;
+    T.unit_begin = 0;
+    T.num_units = P.group_start ? P.num_groups : 1;
+    T.group_start = P.group_start;
+    T.group_blocks = P.group_blocks;
+    T.num_seqs = P.num_seqs;
+    T.num_q_heads = P.num_q_heads;
+    T.num_kv_heads = P.num_kv_heads;
+    T.group = P.group;
+    T.tile_tokens = tile_tokens(P.group);
+    T.max_blocks_per_seq = P.max_blocks_per_seq;
+    T.num_blocks = P.num_blocks;
+    T.chunk_blocks = sp.chunk_blocks;
+    T.max_parts = P.max_parts;
+    T.len_cap = P.len_cap;
+    T.shared_blocks = plan->shared_blocks;
+    T.scale_log2 = P.scale_log2;
+    const int64_t items = static_cast<int64_t>(plan->prefix_row_tiles) * P.num_kv_heads * sp.splits;
+    return P.head_dim == 128 ? launch_tiles<128>(T, P.q, P.num_seqs, P.k_cache, P.v_cache, items, st)
+                             : launch_tiles<64>(T, P.q, P.num_seqs, P.k_cache, P.v_cache, items, st);
 }
 
 template <typename OutT, int D>
@@ -653,7 +707,7 @@ int launch_reduce(const DecodeParams& base, int32_t dtype, cudaStream_t st) {
             const int decode_warps = L.grid * (L.threads / 32);
             if (decode_warps < 2) return PA_OK;  // one warp range: nothing was cut
             e = launch_pdl(lse_reduce_balanced_kernel<OutT, D>, dim3(decode_warps - 1),
-                           dim3(kReduceWarps * 32), 8 * static_cast<size_t>(P.seq_count + 1), st, P,
+                           dim3(kReduceWarps * 32), 12 * static_cast<size_t>(P.seq_count + 1), st, P,
                            decode_warps);
         } else {
             const int64_t rows = static_cast<int64_t>(P.seq_count) * P.num_q_heads;
@@ -676,6 +730,119 @@ int run_reduce(const DecodeParams& P, const Plan& plan, int32_t dtype, cudaStrea
                                  : launch_reduce<__nv_bfloat16, 64>(P, dtype, st);
     return P.head_dim == 128 ? launch_reduce<float, 128>(P, dtype, st)
                              : launch_reduce<float, 64>(P, dtype, st);
+}
+
+// Several query tokens per sequence with group * max_q_len > 16 (prefill
+// chunks): the tile kernel in prefill mode, then, when the keys were cut into
+// chunks, the row-wise merge of each row's chunks.
+struct PrefillPlan {
+    TileSplit split;
+    int64_t tiles_bound;  // tiles over all sequences, at most
+    WsLayout ws;
+};
+
+PrefillPlan make_prefill_plan(int sms, int32_t num_seqs, int32_t num_q_rows, int32_t num_q_heads,
+                              int32_t num_kv_heads, int32_t head_dim, int32_t max_len) {
+    PrefillPlan pp;
+    const int32_t tt = tile_tokens(num_q_heads / num_kv_heads);
+    pp.tiles_bound = (static_cast<int64_t>(num_q_rows) + tt - 1) / tt + num_seqs;
+    pp.split = choose_tile_split(sms, pp.tiles_bound * num_kv_heads, (max_len + kBlockTokens - 1) / kBlockTokens);
+    pp.ws = ws_layout(num_seqs, num_q_heads, num_kv_heads, pp.split.splits, head_dim, pp.split.splits > 1,
+                      num_q_rows);
+    return pp;
+}
+
+int run_prefill_tiles(const DecodeArgs& a) {
+    int rc = check_shapes(a.num_seqs, a.num_q_heads, a.num_kv_heads, a.head_dim, a.block_size, a.dtype);
+    if (rc != PA_OK) return rc;
+    if (a.dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
+    if (a.max_blocks_per_seq <= 0 || a.partition_blocks < -1 || a.num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    if (!a.q || !a.k_cache || !a.v_cache || !a.block_tables || !a.seq_lens || !a.out || !a.q_start)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(a.q, 16) || !aligned(a.k_cache, 16) || !aligned(a.v_cache, 16) || !aligned(a.out, 16) ||
+        !aligned(a.block_tables, 4) || !aligned(a.seq_lens, 4) || !aligned(a.q_start, 4))
+        return PA_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(a.num_blocks) * a.num_kv_heads * kBlockTokens > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    if (!std::isfinite(a.scale)) return PA_ERR_INVALID_ARG;
+    if (a.num_seqs == 0 || a.num_q_rows == 0) return PA_OK;
+    const int64_t table_tokens = static_cast<int64_t>(a.max_blocks_per_seq) * kBlockTokens;
+    const int32_t max_len = a.max_seq_len > 0
+                                ? a.max_seq_len
+                                : static_cast<int32_t>(table_tokens > INT32_MAX ? INT32_MAX : table_tokens);
+    DeviceInfo di;
+    if ((rc = device_info(&di)) != PA_OK) return rc;
+    const PrefillPlan pp = make_prefill_plan(di.sms, a.num_seqs, a.num_q_rows, a.num_q_heads, a.num_kv_heads,
+                                             a.head_dim, max_len);
+    const bool direct = pp.split.splits == 1;
+    float* ws_m = nullptr;
+    float* ws_l = nullptr;
+    float* ws_acc = nullptr;
+    if (!direct) {
+        if (!a.workspace || !aligned(a.workspace, 256) || a.workspace_bytes < pp.ws.bytes) return PA_ERR_WORKSPACE;
+        char* w = static_cast<char*>(a.workspace);
+        ws_m = reinterpret_cast<float*>(w + pp.ws.off_m);
+        ws_l = reinterpret_cast<float*>(w + pp.ws.off_l);
+        ws_acc = reinterpret_cast<float*>(w + pp.ws.off_acc);
+    }
+    TileParams T;
+    std::memset(&T, 0, sizeof T);
+    T.block_tables = a.block_tables;
+    T.seq_lens = a.seq_lens;
+    T.q_start = a.q_start;
+    T.out = a.out;
+    T.ws_m = ws_m;
+    T.ws_l = ws_l;
+    T.ws_acc = ws_acc;
+    T.mode = kTileModePrefill;
+    T.unit_begin = 0;
+    T.num_units = a.num_seqs;
+    T.num_seqs = a.num_seqs;
+    T.num_q_heads = a.num_q_heads;
+    T.num_kv_heads = a.num_kv_heads;
+    T.group = a.num_q_heads / a.num_kv_heads;
+    T.tile_tokens = tile_tokens(T.group);
+    T.max_blocks_per_seq = a.max_blocks_per_seq;
+    T.num_blocks = a.num_blocks;
+    T.chunk_blocks = pp.split.chunk_blocks;
+    T.max_parts = pp.split.splits;
+    T.len_cap = static_cast<int32_t>(max_len < table_tokens ? max_len : table_tokens);
+    T.max_q_len = a.max_q_len;
+    T.direct = direct ? 1 : 0;
+    T.scale_log2 = a.scale * 1.4426950408889634f;
+    const int64_t items = pp.tiles_bound * a.num_kv_heads * pp.split.splits;
+    rc = a.head_dim == 128 ? launch_tiles<128>(T, a.q, a.num_q_rows, a.k_cache, a.v_cache, items, a.stream)
+                           : launch_tiles<64>(T, a.q, a.num_q_rows, a.k_cache, a.v_cache, items, a.stream);
+    if (rc != PA_OK || direct) return rc;
+    // the row-wise merge of each row's chunks (their number follows from the row's tile)
+    DecodeParams R;
+    std::memset(&R, 0, sizeof R);
+    R.seq_lens = a.seq_lens;
+    R.q_start = a.q_start;
+    R.out = a.out;
+    R.ws_m = ws_m;
+    R.ws_l = ws_l;
+    R.ws_acc = ws_acc;
+    R.max_q_len = a.max_q_len;
+    R.num_q_rows = a.num_q_rows;
+    R.num_seqs = a.num_seqs;
+    R.seq_count = a.num_seqs;
+    R.num_q_heads = a.num_q_heads;
+    R.num_kv_heads = a.num_kv_heads;
+    R.head_dim = a.head_dim;
+    R.group = T.group;
+    R.max_parts = pp.split.splits;
+    R.len_cap = T.len_cap;
+    R.part_blocks = kNoSplit;
+    R.tile_tokens = T.tile_tokens;
+    R.tile_chunk = pp.split.chunk_blocks;
+    const int64_t rows = static_cast<int64_t>(a.num_q_rows) * a.num_q_heads;
+    const unsigned grid = static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps);
+    cudaError_t e = a.head_dim == 128
+                        ? launch_pdl(lse_reduce_kernel<__nv_bfloat16, 128>, dim3(grid), dim3(kReduceWarps * 32), 0,
+                                     a.stream, R)
+                        : launch_pdl(lse_reduce_kernel<__nv_bfloat16, 64>, dim3(grid), dim3(kReduceWarps * 32), 0,
+                                     a.stream, R);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "lse_reduce_kernel launch");
 }
 
 DecodeArgs make_args(const void* q, const void* k_cache, const void* v_cache,
@@ -957,14 +1124,64 @@ int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_ca
     int rc = prepare_decode(a, true, &P, &plan, shared_blocks);
     if (rc != PA_OK) return rc;
     if (num_seqs == 0) return PA_OK;
-    rc = head_dim == 128 ? choose_prefix_splits<128>(P, &plan) : choose_prefix_splits<64>(P, &plan);
+    rc = launch_prefix_tiles(P, &plan, a.stream);
     if (rc != PA_OK) return rc;
-    P.piece_base = plan.prefix_splits;  // the private pieces follow the splits actually used
-    rc = head_dim == 128 ? launch_prefix<128>(P, plan, a.stream) : launch_prefix<64>(P, plan, a.stream);
-    if (rc != PA_OK) return rc;
+    P.piece_base = plan.prefix_splits;  // the private pieces follow the chunks actually used
     rc = run_partitions(P, dtype, a.stream);
     if (rc != PA_OK) return rc;
     return run_reduce(P, plan, dtype, a.stream);
+}
+
+int pa_decode_shared_prefix_groups(const void* q, const void* k_cache, const void* v_cache,
+                                   const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   const int32_t* seq_lens, int32_t max_seq_len, const int32_t* group_start,
+                                   const int32_t* group_shared_blocks, int32_t num_groups,
+                                   int32_t max_shared_blocks, int32_t num_seqs, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks, int32_t block_size,
+                                   float scale, int32_t partition_blocks, void* workspace, size_t workspace_bytes,
+                                   void* out, int32_t dtype, void* stream) {
+    if (!group_start || !group_shared_blocks || !aligned(group_start, 4) || !aligned(group_shared_blocks, 4) ||
+        num_groups < 1 || max_shared_blocks < 0)
+        return PA_ERR_INVALID_ARG;
+    if (max_shared_blocks == 0)
+        return pa_decode(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, max_seq_len, num_seqs,
+                         num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale, partition_blocks,
+                         workspace, workspace_bytes, out, dtype, stream);
+    const DecodeArgs a = make_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                                   max_seq_len, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                   num_blocks, block_size, scale, partition_blocks, workspace,
+                                   workspace_bytes, out, dtype, stream);
+    DecodeParams P;
+    Plan plan;
+    int rc = prepare_decode(a, true, &P, &plan, max_shared_blocks, num_groups);
+    if (rc != PA_OK) return rc;
+    if (num_seqs == 0) return PA_OK;
+    P.group_start = group_start;
+    P.group_blocks = group_shared_blocks;
+    P.num_groups = num_groups;
+    rc = launch_prefix_tiles(P, &plan, a.stream);
+    if (rc != PA_OK) return rc;
+    P.piece_base = plan.prefix_splits;  // the private pieces follow the most chunks a group has
+    P.group_chunk = plan.prefix_split_blocks;
+    rc = run_partitions(P, dtype, a.stream);
+    if (rc != PA_OK) return rc;
+    return run_reduce(P, plan, dtype, a.stream);
+}
+
+size_t pa_decode_shared_prefix_groups_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                                     int32_t head_dim, int32_t max_seq_len,
+                                                     int32_t max_shared_blocks, int32_t num_groups,
+                                                     int32_t block_size, int32_t partition_blocks) {
+    if (max_shared_blocks == 0)
+        return pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len,
+                                        block_size, partition_blocks);
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_seq_len < 0 ||
+        block_size != kBlockTokens || partition_blocks < -1 || max_shared_blocks < 0 || num_groups < 1 ||
+        num_q_heads % num_kv_heads != 0 || static_cast<int64_t>(max_shared_blocks) * kBlockTokens > max_seq_len)
+        return 0;
+    const Plan plan = make_group_plan(max_seq_len, partition_blocks, max_shared_blocks, num_groups, num_seqs,
+                                      num_q_heads, num_kv_heads);
+    return ws_layout(num_seqs, num_q_heads, num_kv_heads, plan.max_parts, head_dim, plan.split).bytes;
 }
 
 int pa_decode_multi(const void* q, const int32_t* q_start, int32_t num_q_rows, int32_t max_q_len,
@@ -977,7 +1194,6 @@ int pa_decode_multi(const void* q, const int32_t* q_start, int32_t num_q_rows, i
     if (!q_start || !aligned(q_start, 4) || num_q_rows < 0 || max_q_len < 1) return PA_ERR_INVALID_ARG;
     if (dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
     if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
-    if (static_cast<int64_t>(num_q_heads / num_kv_heads) * max_q_len > 16) return PA_ERR_UNSUPPORTED;
     DecodeArgs a = make_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
                              max_seq_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
                              block_size, scale, partition_blocks, workspace, workspace_bytes, out,
@@ -985,6 +1201,9 @@ int pa_decode_multi(const void* q, const int32_t* q_start, int32_t num_q_rows, i
     a.q_start = q_start;
     a.max_q_len = max_q_len;
     a.num_q_rows = num_q_rows;
+    // more rows per (sequence, kv head) than one warp-level MMA tile holds: the
+    // tensor-memory tile kernel (prefill chunks)
+    if (static_cast<int64_t>(num_q_heads / num_kv_heads) * max_q_len > 16) return run_prefill_tiles(a);
     DecodeParams P;
     Plan plan;
     int rc = prepare_decode(a, true, &P, &plan);
@@ -1000,10 +1219,17 @@ size_t pa_decode_multi_workspace_size(int32_t num_seqs, int32_t num_q_rows, int3
     if (num_seqs < 0 || num_q_rows < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         max_seq_len < 0 || block_size != kBlockTokens || partition_blocks < -1)
         return 0;
+    if (num_q_heads % num_kv_heads != 0) return 0;
     const Plan plan = make_plan(max_seq_len, partition_blocks);
-    return ws_layout(num_seqs, num_q_heads, num_kv_heads, plan.max_parts, head_dim, plan.split,
-                     num_q_rows)
-        .bytes;
+    const size_t dec = ws_layout(num_seqs, num_q_heads, num_kv_heads, plan.max_parts, head_dim, plan.split,
+                                 num_q_rows).bytes;
+    // the tile path (group * max_q_len > 16) keeps its chunks' partials; its
+    // chunking follows the device's SM count (the most chunks if unknown)
+    DeviceInfo di;
+    const int sms = device_info(&di) == PA_OK ? di.sms : (1 << 30);
+    const size_t til = make_prefill_plan(sms, num_seqs, num_q_rows, num_q_heads, num_kv_heads, head_dim,
+                                         max_seq_len).ws.bytes;
+    return dec > til ? dec : til;
 }
 
 size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads,

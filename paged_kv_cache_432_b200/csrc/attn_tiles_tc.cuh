@@ -1,0 +1,702 @@
+// attn_tiles_tc.cuh -- attention of query tiles of up to 128 rows to paged
+// keys on the 5th-generation tensor cores (tcgen05: S = Q K^T and O += P V
+// accumulate in tensor memory).
+//
+// Two jobs are real matrix products over paged K/V and share this kernel:
+//  * prefix mode.  The sequences of a group start with the same prompt, whose
+//    blocks every table of the group names ("Was ändert PagedAttention an der
+//    KV-Speicherzuweisung für LLMs?", slavadubrov.com, §"Gemeinsame Nutzung
+//    erfordert mehr als Speicherzuweisung": several requests reference one
+//    cache block; "PagedAttention et vLLM", aiunderstanding.org, §"Questions
+//    fréquemment posées": identical prefixes refer to the same physical
+//    pages).  For kv head h, the g query heads of all sequences of the group
+//    are the rows of S = Q K^T against the shared prefix keys, so a prefix
+//    block is read once per tile of rows instead of once per sequence.  The
+//    tile writes each row's partial (m, l, acc); the private suffix goes
+//    through the decode kernel and the log-sum-exp merge joins both.
+//  * prefill mode.  The n new query tokens of one sequence (a prefill chunk,
+//    "vLLM PagedAttention: eine Revolution für den Durchsatz bei der
+//    LLM-Inferenz", de.news.hada.io, list of advanced features: chunked
+//    prefill; "Внутреннее устройство vLLM", artificials.ru, paragraph on
+//    chunked prefill) attend causally to the sequence's own blocks: token k
+//    sits at position L - n + k and sees keys 0 .. L - n + k.
+//
+// Work: a unit is a group (prefix) or a sequence (prefill).  Its tokens (the
+// group's sequences, or the new query tokens) are cut into tiles of
+// T = floor(128 / g) tokens; row r of a tile is token r / g, query head
+// h*g + r % g, one TMEM lane.  The unit's key blocks are cut into chunks of
+// chunk_blocks blocks (one chunk when the device is full without a split).
+// An item is (chunk c, kv head h, tile t), numbered with t fastest, so that
+// the tiles reading the same keys run side by side and share them in L2.  The
+// grid is persistent, one CTA per SM: CTA b takes items b, b + grid, ...; each
+// CTA builds the per-unit item prefix once in shared memory and finds any
+// item by binary search.  An item whose chunk lies wholly past its tile's last
+// visible key is empty: every role skips it.
+//
+// Roles (320 threads): warps 0-7 softmax (two threads per query row: warp w
+// reaches TMEM lanes 32 (w mod 4) .. +31 and takes half w / 4 of a step's 64
+// keys and of O's columns), warp 8 TMA producer, warp 9 MMA issue (one
+// thread).  Per item, the producer loads the tile's Q rows with one 3-D TMA
+// box per 64-column slab (tokens x heads x columns, the 128-byte swizzle) into
+// one of two Q buffers, then 64-key steps of K and V (4 blocks, 64 x 16
+// boxes) into a 4-stage ring.  The MMA thread issues S of step j + 1 before
+// P V of step j (two S buffers in TMEM), so the tensor cores run while the
+// softmax works, also across item boundaries.  The softmax threads read their
+// half of a row of S straight from TMEM, swap their maxima through shared
+// memory, write P (bf16) to shared memory, rescale O in TMEM when the row max
+// moved, and at the item's end write the row: a partial (m, l, acc) at piece
+// c, or the final bf16 row when the units have one chunk (prefill).
+// All step counters run on across items, so every mbarrier's phase follows
+// from a per-CTA global step or item count.  Every wait is bounded; a role
+// that gives up flags PA_DEVERR_TIMEOUT and stops issuing, the other roles'
+// waits then run out too, and TMEM is freed on every path.
+#pragma once
+
+#include "items.cuh"
+#include "tcgen05.cuh"
+
+namespace pa {
+
+constexpr int kTileModePrefix = 0;
+constexpr int kTileModePrefill = 1;
+constexpr int kTileStepBlocks = 4;  // 64 keys per step
+
+struct TileParams {
+    const int32_t* block_tables;  // [num_seqs][max_blocks_per_seq]
+    const int32_t* seq_lens;      // [num_seqs]
+    const int32_t* q_start;       // prefill: [num_seqs + 1] query-token rows of each sequence
+    const int32_t* group_start;   // prefix: [groups + 1] sequences of each group (contiguous;
+                                  //   null: one group of every sequence)
+    const int32_t* group_blocks;  // prefix: [groups] shared blocks of each group (null: shared_blocks)
+    void* out;                    // direct: final rows, bf16 [rows][Hq][D]
+    float* ws_m;                  // partials (layout of the decode workspace)
+    float* ws_l;
+    float* ws_acc;
+    int32_t mode;            // kTileModePrefix or kTileModePrefill
+    int32_t unit_begin;      // first unit of this launch
+    int32_t num_units;       // units of this launch
+    int32_t num_seqs;
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t group;           // query heads per kv head
+    int32_t tile_tokens;     // tokens (prefill) or sequences (prefix) per tile: floor(128 / group)
+    int32_t max_blocks_per_seq;
+    int32_t num_blocks;
+    int32_t chunk_blocks;    // key blocks per item (a multiple of 4)
+    int32_t max_parts;       // workspace pieces per row
+    int32_t len_cap;         // sequences longer than this are clamped
+    int32_t max_q_len;       // prefill: query tokens per sequence handled
+    int32_t shared_blocks;   // prefix: blocks of every group when group_blocks is null, else
+                             //   the bound on group_blocks
+    int32_t direct;          // 1: one chunk per unit, rows written to out as final bf16
+    float scale_log2;        // softmax scale * log2(e)
+};
+
+template <int D>
+struct TileCfg {
+    static constexpr int kTileRows = 128;      // TMEM lanes
+    static constexpr int kKeys = 64;           // keys per step
+    static constexpr int kStepBlocks = kKeys / kBlockTokens;
+    static_assert(kStepBlocks == kTileStepBlocks, "steps of 64 keys");
+    static constexpr int kSlabs = D / 64;      // 64-column slabs (128-byte rows)
+    static constexpr int kQBytes = kSlabs * kTileRows * 128;
+    static constexpr int kKVSlab = kKeys * 128;               // one slab of K (or V) for a step
+    static constexpr int kStageBytes = 2 * kSlabs * kKVSlab;  // K slabs, then V slabs
+    static constexpr int kStages = 4;
+    static constexpr int kPBytes = kTileRows * 128;            // P: 64 bf16 keys per row
+    static constexpr int kSoftmaxWarps = 8;
+    static constexpr int kProducerWarp = 8, kMmaWarp = 9;
+    static constexpr int kThreads = 10 * 32;
+    static constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
+    static constexpr uint32_t kTmemCols = 256;  // S0 | S1 | O
+    static constexpr uint32_t kColS = 0, kColO = 2 * kKeys;
+    // full, empty per stage; s_full x2, p_full, o_done, o_free, q_full x2, q_empty x2, drain
+    static constexpr int kBars = 2 * kStages + 10;
+    // halves of a row exchange: [2 step parities][2 halves][128] maxima, [2 halves][128] sums
+    static constexpr int kXBytes = 3 * 2 * kTileRows * 4;
+    static constexpr int kMaxUnits = 2048;  // units whose item prefix one CTA holds
+    static constexpr int kPrefixBytes = (4 * (kMaxUnits + 1) + 15) / 16 * 16;
+    static constexpr size_t kSmem = 1024 + 2 * kQBytes + kStages * kStageBytes + kPBytes + kXBytes +
+                                    kPrefixBytes + 8 * kBars + 16 + 4 * kStages;
+    static_assert(kColO + D <= kTmemCols, "TMEM columns");
+    static_assert(kSmem <= 227u * 1024u, "shared memory per CTA");
+};
+
+// What one unit holds.
+struct TileUnit {
+    int32_t n;        // tokens: new query tokens (prefill) or sequences (prefix)
+    int32_t q_base;   // q row of token 0
+    int32_t table;    // block-table row the keys are read through
+    int32_t len;      // key positions 0 .. len-1 exist (prefill: the sequence length)
+    int32_t kblocks;  // key blocks of the unit
+    int32_t tiles;
+    int32_t chunks;   // 0 when the unit has no work
+    bool clamped;     // prefill: more query tokens than max_q_len or the length allow
+};
+
+__device__ __forceinline__ TileUnit tile_unit(const TileParams& P, int32_t u) {
+    TileUnit U;
+    U.clamped = false;
+    if (P.mode == kTileModePrefix) {
+        // (out-of-range group bounds are clamped here and flagged by check_group_tables)
+        const int32_t s0 = P.group_start ? min(max(__ldg(P.group_start + u), 0), P.num_seqs) : 0;
+        const int32_t s1 = P.group_start ? min(max(__ldg(P.group_start + u + 1), s0), P.num_seqs) : P.num_seqs;
+        U.n = s1 - s0;
+        U.q_base = s0;
+        U.table = s0;
+        const int32_t kb = P.group_blocks ? __ldg(P.group_blocks + u) : P.shared_blocks;
+        U.kblocks = max(0, min(kb, min(P.shared_blocks, P.max_blocks_per_seq)));
+        U.len = U.kblocks * kBlockTokens;
+    } else {
+        int32_t L = __ldg(P.seq_lens + u);
+        L = max(0, min(L, P.len_cap));
+        const int32_t q0 = __ldg(P.q_start + u);
+        int32_t n = __ldg(P.q_start + u + 1) - q0;
+        const int32_t cap = min(P.max_q_len, L);
+        if (n > cap || n < 0) {
+            U.clamped = true;
+            n = n < 0 ? 0 : cap;
+        }
+        U.n = n;
+        U.q_base = q0;
+        U.table = u;
+        U.len = L;
+        U.kblocks = (L + kBlockTokens - 1) / kBlockTokens;
+    }
+    U.tiles = (U.n + P.tile_tokens - 1) / P.tile_tokens;
+    U.chunks = (U.n == 0 || U.kblocks == 0) ? 0 : (U.kblocks + P.chunk_blocks - 1) / P.chunk_blocks;
+    return U;
+}
+
+struct TileItem {
+    TileUnit U;
+    int32_t u, t, c, h;
+    int32_t tok0, ntok;  // tokens of the tile
+    int32_t kb0, kb1;    // key blocks [kb0, kb1) of the item
+    int32_t nsteps;      // 0: empty item
+};
+
+// Item `it` of the launch (prefix[] holds the units' exclusive item sums).
+__device__ __forceinline__ TileItem tile_item(const TileParams& P, const int32_t* prefix, int32_t it) {
+    TileItem I;
+    const int i = upper_index(P.num_units, it, [&](int k) { return static_cast<int64_t>(prefix[k]); });
+    I.u = P.unit_begin + i;
+    I.U = tile_unit(P, I.u);
+    const int32_t j = it - prefix[i];
+    const int32_t th = I.U.tiles * P.num_kv_heads;
+    I.c = j / th;
+    const int32_t r = j - I.c * th;
+    I.h = r / I.U.tiles;
+    I.t = r - I.h * I.U.tiles;
+    I.tok0 = I.t * P.tile_tokens;
+    I.ntok = min(P.tile_tokens, I.U.n - I.tok0);
+    int32_t kend = I.U.kblocks;
+    if (P.mode == kTileModePrefill) {  // blocks up to the tile's last visible key
+        const int32_t last = I.U.len - I.U.n + I.tok0 + I.ntok - 1;
+        kend = min(kend, last / kBlockTokens + 1);
+    }
+    I.kb0 = I.c * P.chunk_blocks;
+    I.kb1 = min(I.kb0 + P.chunk_blocks, kend);
+    I.nsteps = I.kb1 > I.kb0 ? (I.kb1 - I.kb0 + kTileStepBlocks - 1) / kTileStepBlocks : 0;
+    return I;
+}
+
+// Exclusive sums of the units' item counts into prefix[0..num_units]; all
+// threads of the CTA call it.  Returns the total.  Reports clamped query
+// counts (CTA 0 only, so each is counted once).
+__device__ __forceinline__ int32_t build_unit_prefix(const TileParams& P, int32_t* prefix) {
+    __shared__ int32_t warp_tot[32];
+    const int n = P.num_units;
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int per = (n + nthr - 1) / nthr;
+    const int beg = min(n, tid * per), end = min(n, beg + per);
+    int32_t local = 0;
+    for (int i = beg; i < end; ++i) {
+        const TileUnit U = tile_unit(P, P.unit_begin + i);
+        if (U.clamped && blockIdx.x == 0) flag_error(PA_DEVERR_SEQ_LEN);
+        local += U.tiles * U.chunks * P.num_kv_heads;
+    }
+    const int lane = tid & 31, warp = tid >> 5, nwarps = (nthr + 31) >> 5;
+    int32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t v = __shfl_up_sync(kFullMask, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int32_t t = lane < nwarps ? warp_tot[lane] : 0;
+        int32_t ti = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t v = __shfl_up_sync(kFullMask, ti, o);
+            if (lane >= o) ti += v;
+        }
+        warp_tot[lane] = ti - t;
+    }
+    __syncthreads();
+    int32_t run = warp_tot[warp] + incl - local;
+    for (int i = beg; i < end; ++i) {
+        prefix[i] = run;
+        const TileUnit U = tile_unit(P, P.unit_begin + i);
+        run += U.tiles * U.chunks * P.num_kv_heads;
+    }
+    if (tid == nthr - 1) prefix[n] = run;
+    __syncthreads();
+    return prefix[n];
+}
+
+// Prefix mode precondition, checked by the producer and MMA warps of the grid
+// after their main work: the groups are ordered ranges of the batch with
+// shared block counts within the bound, every table of a group starts with the
+// group's shared blocks (those of its first sequence), and no sequence of the
+// group is shorter than them.  Violations set PA_DEVERR_PREFIX.  `me` of
+// `nthreads`.
+__device__ __forceinline__ void check_group_tables(const TileParams& P, int64_t me, int64_t nthreads) {
+    for (int32_t g = P.unit_begin; g < P.unit_begin + P.num_units; ++g) {
+        if (me == 0 && P.group_start) {  // the group list itself: ordered, inside the batch, within the bound
+            const int32_t s0 = P.group_start[g], s1 = P.group_start[g + 1], kb = P.group_blocks[g];
+            if (s0 < 0 || s1 < s0 || s1 > P.num_seqs || kb < 0 || kb > P.shared_blocks) flag_error(PA_DEVERR_PREFIX);
+        }
+        const TileUnit U = tile_unit(P, g);
+        const int64_t entries = static_cast<int64_t>(U.n) * U.kblocks;
+        const int32_t* lead = P.block_tables + static_cast<size_t>(U.table) * P.max_blocks_per_seq;
+        for (int64_t e = me; e < entries; e += nthreads) {
+            const int64_t s = U.q_base + e / U.kblocks, j = e % U.kblocks;
+            if (P.block_tables[s * P.max_blocks_per_seq + j] != lead[j]) flag_error(PA_DEVERR_PREFIX);
+        }
+        for (int64_t s = me; s < U.n; s += nthreads)
+            if (P.seq_lens[U.q_base + s] < U.len) flag_error(PA_DEVERR_PREFIX);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(TileCfg<D>::kThreads, 1)
+attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                     const __grid_constant__ CUtensorMap tmap_q, const TileParams P) {
+    using Cfg = TileCfg<D>;
+    constexpr int S = Cfg::kStages;
+    constexpr int kHalfKeys = Cfg::kKeys / 2;  // keys of a step per softmax thread
+    constexpr int kHalfD = D / 2;              // O columns per softmax thread
+
+    // Launched with programmatic stream serialization: until
+    // grid_dependency_wait() the CTA reads only the lengths, q_start, the
+    // groups and block tables and q (inputs no kernel of this library
+    // writes); the pool is read (producer) and out / the workspace written
+    // (softmax) only after the wait.
+    allow_dependents();
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+    // layout: Q[2] | ring[S] | P | exchange | unit prefix | barriers | TMEM slot | stage masks
+    const uint32_t q_u32 = smem_u32(smem);
+    const uint32_t ring_u32 = q_u32 + 2 * Cfg::kQBytes;
+    const uint32_t p_u32 = ring_u32 + S * Cfg::kStageBytes;
+    uint8_t* ring_smem = smem + 2 * Cfg::kQBytes;
+    uint8_t* p_smem = ring_smem + S * Cfg::kStageBytes;
+    float* xchg = reinterpret_cast<float*>(p_smem + Cfg::kPBytes);
+    int32_t* prefix = reinterpret_cast<int32_t*>(p_smem + Cfg::kPBytes + Cfg::kXBytes);
+    const uint32_t bars_u32 = p_u32 + Cfg::kPBytes + Cfg::kXBytes + Cfg::kPrefixBytes;
+    const uint32_t full_u32 = bars_u32;           // [S]
+    const uint32_t empty_u32 = bars_u32 + 8 * S;  // [S]
+    const uint32_t sfull_u32 = bars_u32 + 16 * S;  // [2]
+    const uint32_t pfull_u32 = sfull_u32 + 16;
+    const uint32_t odone_u32 = pfull_u32 + 8;
+    const uint32_t ofree_u32 = odone_u32 + 8;
+    const uint32_t qfull_u32 = ofree_u32 + 8;     // [2]
+    const uint32_t qempty_u32 = qfull_u32 + 16;   // [2]
+    const uint32_t drain_u32 = qempty_u32 + 16;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (drain_u32 + 8 - q_u32));
+    uint32_t* stage_present = tmem_slot + 4;  // [S]: blocks of the stage that were loaded
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = P.group;
+    const int tile_rows = P.tile_tokens * g;  // rows the Q box fills
+    const bool prefill = P.mode == kTileModePrefill;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < S; ++st) {
+            mbar_init(full_u32 + 8 * st, 1);
+            mbar_init(empty_u32 + 8 * st, 1);
+        }
+        mbar_init(sfull_u32, 1);
+        mbar_init(sfull_u32 + 8, 1);
+        mbar_init(pfull_u32, Cfg::kSoftmaxThreads);
+        mbar_init(odone_u32, 1);
+        mbar_init(ofree_u32, Cfg::kSoftmaxThreads);
+        mbar_init(qfull_u32, 1);
+        mbar_init(qfull_u32 + 8, 1);
+        mbar_init(qempty_u32, 1);
+        mbar_init(qempty_u32 + 8, 1);
+        mbar_init(drain_u32, 1);
+        fence_barrier_init();
+    }
+    // the rows past the Q box (128 mod g of them) are never loaded: zero them
+    // in both buffers once, so that their S and P stay finite
+    for (int e = threadIdx.x; e < 2 * Cfg::kSlabs * (Cfg::kTileRows - tile_rows) * 8; e += blockDim.x) {
+        const int chunk = e & 7, rest = e >> 3;
+        const int row = tile_rows + rest % (Cfg::kTileRows - tile_rows);
+        const int buf_slab = rest / (Cfg::kTileRows - tile_rows);
+        *reinterpret_cast<uint4*>(smem + buf_slab * Cfg::kTileRows * 128 + row * 128 + chunk * 16) =
+            make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+    if (warp == Cfg::kMmaWarp) tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    const int32_t total = build_unit_prefix(P, prefix);  // ends with __syncthreads
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int64_t check_me = static_cast<int64_t>(blockIdx.x) * 64 + threadIdx.x - Cfg::kProducerWarp * 32;
+    const int64_t check_n = static_cast<int64_t>(gridDim.x) * 64;
+
+    if (warp == Cfg::kProducerWarp) {
+        // ---------------- producer: Q of each item, then its steps of K and V
+        const uint64_t keep = l2_policy_evict_last();  // K/V and Q are read by several tiles
+        bool ok = true;
+        uint32_t iq = 0, gs = 0;  // items with work, global steps
+        grid_dependency_wait();    // the pool: a cache write launched before has finished
+        for (int32_t it = blockIdx.x; it < total && ok; it += gridDim.x) {
+            const TileItem I = tile_item(P, prefix, it);
+            if (I.nsteps == 0) continue;
+            const uint32_t b = iq & 1u;
+            if (iq >= 2 && !mbar_wait_bounded(qempty_u32 + 8 * b, ((iq >> 1) - 1) & 1u)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(qfull_u32 + 8 * b, Cfg::kSlabs * tile_rows * 128);
+#pragma unroll
+                for (int sl = 0; sl < Cfg::kSlabs; ++sl)
+                    tma_load_3d(q_u32 + b * Cfg::kQBytes + sl * Cfg::kTileRows * 128, &tmap_q, sl * 64, I.h * g,
+                                I.U.q_base + I.tok0, qfull_u32 + 8 * b, keep);
+            }
+            ++iq;
+            // table entries of the item's blocks, 32 at a time: lane l holds
+            // block win + l (-1 where past the item or outside the pool)
+            const int32_t* trow = P.block_tables + static_cast<size_t>(I.U.table) * P.max_blocks_per_seq;
+            auto table_entry = [&](int jb) -> int32_t {
+                if (jb >= I.kb1) return -1;
+                const int32_t pb = __ldg(trow + jb);
+                if (static_cast<uint32_t>(pb) >= static_cast<uint32_t>(P.num_blocks)) {
+                    flag_error(PA_DEVERR_BLOCK_OOB);
+                    return -1;
+                }
+                return pb;
+            };
+            int32_t win = table_entry(I.kb0 + lane);
+            for (int j = 0; j < I.nsteps; ++j, ++gs) {
+                const int st = gs % S;
+                if (gs >= static_cast<uint32_t>(S) && !mbar_wait_bounded(empty_u32 + 8 * st, ((gs / S) - 1) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                const int first = j * Cfg::kStepBlocks;  // block of the item at this step's start
+                if (first > 0 && (first & 31) == 0) win = table_entry(I.kb0 + first + lane);
+                const int32_t pb = __shfl_sync(kFullMask, win, (first & 31) + (lane & (Cfg::kStepBlocks - 1)));
+                const uint32_t present =
+                    __ballot_sync(kFullMask, lane < Cfg::kStepBlocks && pb >= 0) & ((1u << Cfg::kStepBlocks) - 1u);
+                const uint32_t sbase = ring_u32 + st * Cfg::kStageBytes;
+                if (present != (1u << Cfg::kStepBlocks) - 1u) {
+                    // blocks past the item or outside the pool: zero their V rows
+                    // so that P = 0 times them stays 0
+                    for (int c = lane; c < Cfg::kStepBlocks * Cfg::kSlabs * kBlockTokens * 8; c += 32) {
+                        const int bb = c / (Cfg::kSlabs * kBlockTokens * 8);
+                        if ((present >> bb) & 1u) continue;
+                        const int rem = c % (Cfg::kSlabs * kBlockTokens * 8);
+                        const int sl = rem / (kBlockTokens * 8), rr = rem % (kBlockTokens * 8);
+                        const int t = bb * kBlockTokens + rr / 8;
+                        *reinterpret_cast<uint4*>(ring_smem + st * Cfg::kStageBytes + (Cfg::kSlabs + sl) * Cfg::kKVSlab +
+                                                  t * 128 + (rr % 8) * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    stage_present[st] = present;  // read by the softmax after this barrier's phase
+                    mbar_arrive_expect_tx(full_u32 + 8 * st, __popc(present) * 2 * Cfg::kSlabs * 2048);
+                }
+#pragma unroll
+                for (int bb = 0; bb < Cfg::kStepBlocks; ++bb) {
+                    const int32_t pbb = __shfl_sync(kFullMask, pb, bb);
+                    if (lane == 0 && pbb >= 0) {
+                        const int32_t row = (pbb * P.num_kv_heads + I.h) * kBlockTokens;
+#pragma unroll
+                        for (int sl = 0; sl < Cfg::kSlabs; ++sl) {
+                            tma_load_2d(sbase + sl * Cfg::kKVSlab + bb * kBlockTokens * 128, &tmap_k, sl * 64, row,
+                                        full_u32 + 8 * st, keep);
+                            tma_load_2d(sbase + (Cfg::kSlabs + sl) * Cfg::kKVSlab + bb * kBlockTokens * 128, &tmap_v,
+                                        sl * 64, row, full_u32 + 8 * st, keep);
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        if (!ok && lane == 0) flag_error(PA_DEVERR_TIMEOUT);
+        // this warp's last copies into every stage and Q buffer have landed before leaving
+        for (uint32_t k = 0; k < static_cast<uint32_t>(S) && k < gs; ++k) {
+            const uint32_t last = gs - 1 - k;  // one of the last S steps
+            mbar_wait_bounded(full_u32 + 8 * (last % S), (last / S) & 1u);
+        }
+        for (uint32_t k = 0; k < 2 && k < iq; ++k) {
+            const uint32_t last = iq - 1 - k;
+            mbar_wait_bounded(qfull_u32 + 8 * (last & 1u), (last >> 1) & 1u);
+        }
+    } else if (warp == Cfg::kMmaWarp) {
+        // ---------------- MMA issue (one thread): S of step j + 1, then P V of step j
+        if (lane == 0) {
+            constexpr uint32_t kIdescS = umma_idesc_bf16(Cfg::kTileRows, Cfg::kKeys, 0);
+            constexpr uint32_t kIdescO = umma_idesc_bf16(Cfg::kTileRows, D, 1);
+            // the step sequence of this CTA: (item, step j within it)
+            struct Cur {
+                int32_t it;      // item index
+                int32_t j;       // step within the item
+                int32_t nsteps;  // steps of the item
+                uint32_t iq;     // items with work before this one
+                uint32_t gs;     // global step
+            };
+            auto first_step = [&](int32_t it, uint32_t iq, uint32_t gs, Cur& c) -> bool {
+                for (; it < total; it += gridDim.x) {
+                    const TileItem I = tile_item(P, prefix, it);
+                    if (I.nsteps == 0) continue;
+                    c = Cur{it, 0, I.nsteps, iq, gs};
+                    return true;
+                }
+                return false;
+            };
+            auto next_step = [&](const Cur& c, Cur& n) -> bool {
+                if (c.j + 1 < c.nsteps) {
+                    n = c;
+                    ++n.j;
+                    ++n.gs;
+                    return true;
+                }
+                return first_step(c.it + gridDim.x, c.iq + 1, c.gs + 1, n);
+            };
+            auto issue_s = [&](const Cur& c) -> bool {
+                const uint32_t b = c.iq & 1u;
+                if (c.j == 0) {
+                    if (!mbar_wait_bounded_thread(qfull_u32 + 8 * b, (c.iq >> 1) & 1u)) return false;
+                }
+                const int st = c.gs % S;
+                if (!mbar_wait_bounded_thread(full_u32 + 8 * st, (c.gs / S) & 1u)) return false;
+                tc_fence_after();
+                const uint32_t kb = ring_u32 + st * Cfg::kStageBytes;
+                const uint32_t qb = q_u32 + b * Cfg::kQBytes;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t off = (ks % 4) * 32u;  // k-step within the 128-byte row
+                    const uint64_t a = umma_desc_sw128(qb + (ks / 4) * Cfg::kTileRows * 128 + off, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(kb + (ks / 4) * Cfg::kKVSlab + off, 16, 1024);
+                    umma_bf16(tmem + Cfg::kColS + (c.gs & 1u) * Cfg::kKeys, a, bd, kIdescS, ks > 0);
+                }
+                umma_commit(sfull_u32 + 8 * (c.gs & 1u));
+                if (c.j + 1 == c.nsteps) umma_commit(qempty_u32 + 8 * b);  // the item's last read of Q
+                return true;
+            };
+            bool ok = true;
+            Cur cur;
+            bool have = first_step(blockIdx.x, 0, 0, cur);
+            if (have) ok = issue_s(cur);
+            while (have && ok) {
+                Cur nxt;
+                const bool more = next_step(cur, nxt);
+                if (more && !(ok = issue_s(nxt))) break;
+                // P V of the current step; the first step of an item overwrites O,
+                // which the softmax must have read out for the previous item
+                if (cur.j == 0 && cur.iq > 0 &&
+                    !(ok = mbar_wait_bounded_thread(ofree_u32, (cur.iq - 1) & 1u)))
+                    break;
+                if (!(ok = mbar_wait_bounded_thread(pfull_u32, cur.gs & 1u))) break;
+                tc_fence_after();
+                const uint32_t vb = ring_u32 + (cur.gs % S) * Cfg::kStageBytes + Cfg::kSlabs * Cfg::kKVSlab;
+#pragma unroll
+                for (int ks = 0; ks < Cfg::kKeys / 16; ++ks) {
+                    const uint64_t a = umma_desc_sw128(p_u32 + ks * 32u, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(vb + ks * 16 * 128, Cfg::kKVSlab, 1024);
+                    umma_bf16(tmem + Cfg::kColO, a, bd, kIdescO, cur.j > 0 || ks > 0);
+                }
+                umma_commit(odone_u32);
+                umma_commit(empty_u32 + 8 * (cur.gs % S));
+                if (!more) break;
+                cur = nxt;
+            }
+            if (!ok) flag_error(PA_DEVERR_TIMEOUT);
+            // every MMA this thread issued has completed before TMEM goes away
+            umma_commit(drain_u32);
+            mbar_wait_bounded_thread(drain_u32, 0);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- softmax: two threads per query row
+        const int row = 32 * (warp & 3) + lane;  // TMEM lane = row of the tile
+        const int hf = (warp >> 2) & 1;          // half of the keys and of O
+        const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp & 3) * 32u) << 16);
+        const float sl2 = P.scale_log2;
+        bool ok = true;  // warp-uniform: a wait that gave up stops TMEM work and arrivals
+        uint32_t iq = 0, gs = 0;
+        bool waited = false;  // grid_dependency_wait done (before the first output write)
+        for (int32_t it = blockIdx.x; it < total; it += gridDim.x) {
+            const TileItem I = tile_item(P, prefix, it);
+            if (I.nsteps == 0) continue;
+            const int tok = row / g;  // token of the tile (a sequence in prefix mode)
+            const bool row_ok = row < tile_rows && tok < I.ntok;
+            const int32_t ktok = I.tok0 + tok;  // token within the unit
+            // last key this row sees (prefill: causal; prefix: every prefix key)
+            const int32_t lim = !row_ok ? -1 : prefill ? I.U.len - I.U.n + ktok : I.U.len - 1;
+            const size_t orow = row_ok ? static_cast<size_t>(I.U.q_base + ktok) * P.num_q_heads + I.h * g + row % g : 0;
+            float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
+            for (int j = 0; j < I.nsteps; ++j, ++gs) {
+                const int st = gs % S;
+                ok = ok && mbar_wait_bounded(sfull_u32 + 8 * (gs & 1u), (gs >> 1) & 1u);
+                ok = ok && mbar_wait_bounded(full_u32 + 8 * st, (gs / S) & 1u);
+                tc_fence_after();
+                const int32_t key0 = (I.kb0 + j * Cfg::kStepBlocks) * kBlockTokens;  // first key of the step
+                float x[kHalfKeys];
+                float mx = -INFINITY;
+                if (ok) {
+                    const uint32_t present = stage_present[st] >> (hf * kHalfKeys / kBlockTokens);
+                    tmem_ld32(lane_base + Cfg::kColS + (gs & 1u) * Cfg::kKeys + hf * kHalfKeys, x);
+                    // keys key0 + 32 hf + i; visible iff their block was loaded and key <= lim
+                    const int32_t vis = lim - key0 - hf * kHalfKeys;  // last visible i
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int i = 0; i < kHalfKeys; ++i) {
+                        x[i] = (((present >> (i / kBlockTokens)) & 1u) && i <= vis) ? x[i] * sl2 : -INFINITY;
+                        m4[i & 3] = fmaxf(m4[i & 3], x[i]);
+                    }
+                    mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kHalfKeys; ++i) x[i] = -INFINITY;
+                }
+                // the row max over both halves
+                float* xs = xchg + (gs & 1u) * 2 * Cfg::kTileRows;
+                xs[hf * Cfg::kTileRows + row] = mx;
+                softmax_bar_sync(1, Cfg::kSoftmaxThreads);
+                mx = fmaxf(mx, xs[(1 - hf) * Cfg::kTileRows + row]);
+                const float mn = fmaxf(m, mx);
+                const float mu = mn == -INFINITY ? 0.0f : mn;
+                const float alpha = fast_exp2(m - mu);
+                m = mn;
+                uint32_t pw[kHalfKeys / 2];
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int i = 0; i < kHalfKeys / 2; ++i) {
+                    pw[i] = pack2<false>(fast_exp2(x[2 * i] - mu), fast_exp2(x[2 * i + 1] - mu));
+                    s4[i & 3] += __uint_as_float(pw[i] << 16) + __uint_as_float(pw[i] & 0xffff0000u);
+                }
+                l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+                if (j > 0) {
+                    // P V of the previous step is done: the P buffer is free, O holds the sum up to it
+                    ok = ok && mbar_wait_bounded(odone_u32, (gs - 1) & 1u);
+                    tc_fence_after();
+                    if (ok && __any_sync(kFullMask, alpha != 1.f)) {
+#pragma unroll
+                        for (int c = 0; c < kHalfD / 32; ++c) {
+                            float v[32];
+                            tmem_ld32(lane_base + Cfg::kColO + hf * kHalfD + 32 * c, v);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                            tmem_st32(lane_base + Cfg::kColO + hf * kHalfD + 32 * c, v);
+                        }
+                    }
+                }
+                if (ok) {
+                    // keys 32 hf .. 32 hf + 31 of the row: 16-byte chunks 4 hf .. 4 hf + 3
+                    // of its 128-byte P row, K-major, 128-byte swizzle
+#pragma unroll
+                    for (int c = 0; c < kHalfKeys / 8; ++c) {
+                        const int cc = hf * (kHalfKeys / 8) + c;
+                        *reinterpret_cast<uint4*>(p_smem + row * 128 + ((cc ^ (row & 7)) << 4)) =
+                            make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+                    }
+                    // key slots at or past the sequence's length hold stale data
+                    // (weight 0, but 0 * NaN is NaN): zero their V rows in the stage
+                    const int32_t zero_from = I.U.len - key0;
+                    if (zero_from < Cfg::kKeys) {
+                        const int zrows = Cfg::kKeys - max(0, zero_from);
+                        for (int e = threadIdx.x; e < zrows * Cfg::kSlabs * 8; e += Cfg::kSoftmaxThreads) {
+                            const int zr = Cfg::kKeys - zrows + e / (Cfg::kSlabs * 8);
+                            const int sl = (e / 8) % Cfg::kSlabs;
+                            *reinterpret_cast<uint4*>(ring_smem + st * Cfg::kStageBytes + (Cfg::kSlabs + sl) * Cfg::kKVSlab +
+                                                      zr * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(pfull_u32);
+                }
+            }
+            // ---- the item's rows
+            if (!waited) {
+                grid_dependency_wait();  // before the first write of out or the workspace
+                waited = true;
+            }
+            xchg[4 * Cfg::kTileRows + hf * Cfg::kTileRows + row] = l;
+            softmax_bar_sync(1, Cfg::kSoftmaxThreads);
+            l += xchg[4 * Cfg::kTileRows + (1 - hf) * Cfg::kTileRows + row];
+            ok = ok && mbar_wait_bounded(odone_u32, (gs - 1) & 1u);  // the item's last P V
+            tc_fence_after();
+            if (ok) {
+                constexpr float kLn2 = 0.693147180559945309f;
+                if (P.direct) {
+                    const float inv = l > 0.f ? 1.0f / l : 0.f;
+                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(P.out) + orow * D + hf * kHalfD;
+#pragma unroll
+                    for (int c = 0; c < kHalfD / 32; ++c) {
+                        float v[32];
+                        tmem_ld32(lane_base + Cfg::kColO + hf * kHalfD + 32 * c, v);
+                        if (row_ok) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                uint4 u;
+                                u.x = pack2<false>(v[8 * i] * inv, v[8 * i + 1] * inv);
+                                u.y = pack2<false>(v[8 * i + 2] * inv, v[8 * i + 3] * inv);
+                                u.z = pack2<false>(v[8 * i + 4] * inv, v[8 * i + 5] * inv);
+                                u.w = pack2<false>(v[8 * i + 6] * inv, v[8 * i + 7] * inv);
+                                *reinterpret_cast<uint4*>(o + 32 * c + 8 * i) = u;
+                            }
+                        }
+                    }
+                } else {
+                    const size_t idx = orow * P.max_parts + I.c;
+                    if (row_ok && hf == 0) {
+                        P.ws_m[idx] = m * kLn2;
+                        P.ws_l[idx] = l;
+                    }
+                    float* a = P.ws_acc + idx * D + hf * kHalfD;
+#pragma unroll
+                    for (int c = 0; c < kHalfD / 32; ++c) {
+                        float v[32];
+                        tmem_ld32(lane_base + Cfg::kColO + hf * kHalfD + 32 * c, v);
+                        if (row_ok) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                *reinterpret_cast<float4*>(a + 32 * c + 4 * i) =
+                                    make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(ofree_u32);  // O may be overwritten by the next item
+            }
+            ++iq;
+        }
+        if (!ok && lane == 0) flag_error(PA_DEVERR_TIMEOUT);
+        (void)iq;
+    }
+
+    if (P.mode == kTileModePrefix && warp >= Cfg::kProducerWarp) check_group_tables(P, check_me, check_n);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == Cfg::kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
+}
+
+}  // namespace pa

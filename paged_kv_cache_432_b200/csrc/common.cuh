@@ -60,6 +60,14 @@ struct DecodeParams {
     int32_t skip_blocks;         // pieces cover blocks [skip_blocks, nb) of each sequence
     int32_t piece_base;          // > 0: pieces are written as partials at index piece_base + p
                                  //      (the first piece_base partials come from elsewhere)
+    const int32_t* group_start;  // several prompt groups: sequences of group i are
+                                 //   group_start[i] .. group_start[i+1]-1 (null: one or no prefix)
+    const int32_t* group_blocks; //   and group i shares its first group_blocks[i] blocks
+    int32_t num_groups;
+    int32_t max_shared;          //   bound on group_blocks
+    int32_t group_chunk;         //   key blocks per prefix chunk of the tile kernel
+    int32_t tile_tokens;         // merge of tile-kernel prefill rows: query tokens per tile
+    int32_t tile_chunk;          //   and key blocks per chunk (0: not a tile-kernel merge)
     int32_t seq_begin;           // first sequence of this launch
     int32_t seq_count;           // sequences in this launch
     float scale;                 // softmax scale (natural units)
@@ -145,6 +153,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+// 3-D tile load global -> shared (innermost coordinate first).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint32_t bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy)
         : "memory");
 }
 

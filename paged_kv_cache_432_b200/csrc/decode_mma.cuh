@@ -81,8 +81,8 @@ struct MmaCfg {
     static constexpr int kRingBytes = WARPS * STAGES * kStageBytes;
     static constexpr int kBarBytes = WARPS * STAGES * 8;
     static constexpr int kThreads = WARPS * 32;
-    static size_t smem_bytes(int seq_count) {
-        return 1024 + kRingBytes + kBarBytes + 8 * static_cast<size_t>(seq_count + 1);
+    static size_t smem_bytes(int seq_count) {  // + prefix, lengths and skips of the launch's sequences
+        return 1024 + kRingBytes + kBarBytes + 12 * static_cast<size_t>(seq_count + 1);
     }
     // 16-byte chunk c of row t sits at chunk c ^ swz(t) (the TMA swizzle pattern)
     static __device__ __forceinline__ uint32_t swz(int t) {
@@ -178,7 +178,7 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // ready when the wait ends.  The pool (which the cache write fills), the
     // output and the workspace are touched only after it.
     allow_dependents();  // the reduction may launch and wait for this grid
-    const Schedule sched = make_schedule(P, prefix, lens, WARPS);  // ends with __syncthreads
+    const Schedule sched = make_schedule(P, prefix, WARPS);  // ends with __syncthreads
     const int32_t my_warp = blockIdx.x * WARPS + warp;
     Cursor pc;  // producer: the piece whose next block is loaded next
     sched.start(pc, my_warp);

@@ -29,7 +29,7 @@ decode_f32_simt_kernel(const DecodeParams P) {
     int32_t* lens = prefix + P.seq_count + 1;
     grid_dependency_wait();  // global memory only once the previous kernel is done
     allow_dependents();
-    const Schedule sched = make_schedule(P, prefix, lens, kSimtWarps);
+    const Schedule sched = make_schedule(P, prefix, kSimtWarps);
     zero_empty_sequences<float>(P, lens);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

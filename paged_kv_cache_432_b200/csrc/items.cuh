@@ -35,24 +35,56 @@ struct SeqGeom {
     int32_t parts;  // fixed mode: ceil(work / part_blocks); 0 when there is no work
 };
 
-__device__ __forceinline__ SeqGeom seq_geometry(const DecodeParams& P, int32_t len) {
+// `skip`: the leading blocks of the sequence that other kernels cover (a
+// shared prefix), from seq_skip.
+__device__ __forceinline__ SeqGeom seq_geometry(const DecodeParams& P, int32_t len, int32_t skip) {
     SeqGeom g;
     if (len < 0) len = 0;
     if (len > P.len_cap) len = P.len_cap;
     g.len = len;
     g.nb = (len + kBlockTokens - 1) / kBlockTokens;
-    g.first = min(P.skip_blocks, g.nb);
+    g.first = min(skip, g.nb);
     g.work = g.nb - g.first;
     g.parts = g.work == 0 ? 0 : 1 + (g.work - 1) / P.part_blocks;
     return g;
 }
 
+// Largest s in [0, n) with key(s) <= x, where key is non-decreasing and
+// key(0) <= x < key(n).
+template <typename Key>
+__device__ __forceinline__ int upper_index(int n, int64_t x, Key key) {
+    int lo = 0, hi = n;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (key(mid) <= x) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+// Prefix group of sequence s (several prompt groups: group i is sequences
+// group_start[i] .. group_start[i+1]-1).
+__device__ __forceinline__ int32_t seq_group(const DecodeParams& P, int32_t s) {
+    return upper_index(P.num_groups, s, [&](int k) { return static_cast<int64_t>(__ldg(P.group_start + k)); });
+}
+
+// Shared blocks of a group, within [0, max_shared] (larger values are clamped;
+// the tile kernel flags them).
+__device__ __forceinline__ int32_t group_shared(const DecodeParams& P, int32_t grp) {
+    return max(0, min(__ldg(P.group_blocks + grp), P.max_shared));
+}
+
+// Leading blocks of sequence s that a shared-prefix kernel covers.
+__device__ __forceinline__ int32_t seq_skip(const DecodeParams& P, int32_t s) {
+    return P.group_start ? group_shared(P, seq_group(P, s)) : P.skip_blocks;
+}
+
 // Builds prefix[0..n] (exclusive sums of the per-sequence quantity: blocks in
-// balanced mode, pieces x kv heads in fixed mode; prefix[n] = total) and
-// lens[0..n) (clamped lengths) in shared memory.  All threads of the CTA must
-// call it.  Returns the total.
+// balanced mode, pieces x kv heads in fixed mode; prefix[n] = total), lens[0..n)
+// (clamped lengths) and skips[0..n) (leading blocks covered elsewhere) in
+// shared memory.  All threads of the CTA must call it.  Returns the total.
 __device__ __forceinline__ int32_t build_prefix(const DecodeParams& P, int32_t* prefix,
-                                                int32_t* lens) {
+                                                int32_t* lens, int32_t* skips) {
     __shared__ int32_t warp_tot[32];
     const int n = P.seq_count;
     const int tid = threadIdx.x, nthr = blockDim.x;
@@ -64,7 +96,8 @@ __device__ __forceinline__ int32_t build_prefix(const DecodeParams& P, int32_t* 
     for (int i = beg; i < end; ++i) {
         const int32_t raw = P.seq_lens[P.seq_begin + i];
         if (report && (raw < 0 || raw > P.len_cap)) flag_error(PA_DEVERR_SEQ_LEN);
-        const SeqGeom g = seq_geometry(P, raw);
+        skips[i] = seq_skip(P, P.seq_begin + i);
+        const SeqGeom g = seq_geometry(P, raw, skips[i]);
         lens[i] = g.len;
         local += P.balanced ? g.work : g.parts * P.num_kv_heads;
     }
@@ -91,25 +124,12 @@ __device__ __forceinline__ int32_t build_prefix(const DecodeParams& P, int32_t* 
     int32_t run = warp_tot[warp] + incl - local;
     for (int i = beg; i < end; ++i) {
         prefix[i] = run;
-        const SeqGeom g = seq_geometry(P, lens[i]);
+        const SeqGeom g = seq_geometry(P, lens[i], skips[i]);
         run += P.balanced ? g.work : g.parts * P.num_kv_heads;
     }
     if (tid == nthr - 1) prefix[n] = run;  // the last thread ends on the grand total
     __syncthreads();
     return prefix[n];
-}
-
-// Largest s in [0, n) with key(s) <= x, where key is non-decreasing and
-// key(0) <= x < key(n).
-template <typename Key>
-__device__ __forceinline__ int upper_index(int n, int64_t x, Key key) {
-    int lo = 0, hi = n;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (key(mid) <= x) lo = mid;
-        else hi = mid;
-    }
-    return lo;
 }
 
 // Iterates the pieces one warp owns.  Warp-uniform.
@@ -134,6 +154,7 @@ struct Schedule {
     const DecodeParams* P;
     const int32_t* prefix;
     const int32_t* lens;
+    const int32_t* skips;
     int32_t total;  // blocks (balanced) or pieces (fixed)
     int64_t chunk;  // balanced: blocks per warp range
     int32_t nw;     // warps in the grid
@@ -145,7 +166,7 @@ struct Schedule {
         c.p = r / P->num_kv_heads;
         c.h = r - c.p * P->num_kv_heads;
         c.s = P->seq_begin + i;
-        const SeqGeom g = seq_geometry(*P, lens[i]);
+        const SeqGeom g = seq_geometry(*P, lens[i], skips[i]);
         c.len = g.len;
         c.parts = g.parts;
         c.jbeg = g.first + c.p * P->part_blocks;
@@ -156,7 +177,7 @@ struct Schedule {
         const int n = P->seq_count;
         const int64_t hk = P->num_kv_heads;
         const int i = upper_index(n, c.pos, [&](int k) { return hk * prefix[k]; });
-        const SeqGeom g = seq_geometry(*P, lens[i]);
+        const SeqGeom g = seq_geometry(*P, lens[i], skips[i]);
         const int64_t off = c.pos - hk * prefix[i];
         c.h = static_cast<int32_t>(off / g.work);
         const int64_t jrel = off - static_cast<int64_t>(c.h) * g.work;
@@ -199,13 +220,18 @@ struct Schedule {
 };
 
 // Sets up the schedule of a launch (all threads of the CTA call it).
-__device__ __forceinline__ Schedule make_schedule(const DecodeParams& P, int32_t* prefix,
-                                                  int32_t* lens, int warps_per_cta) {
+// `smem_seqs` holds 3 * seq_count + 1 ints: the prefix, the lengths, the skips.
+__device__ __forceinline__ Schedule make_schedule(const DecodeParams& P, int32_t* smem_seqs,
+                                                  int warps_per_cta) {
     Schedule sc;
     sc.P = &P;
+    int32_t* prefix = smem_seqs;
+    int32_t* lens = prefix + P.seq_count + 1;
+    int32_t* skips = lens + P.seq_count;
     sc.prefix = prefix;
     sc.lens = lens;
-    sc.total = build_prefix(P, prefix, lens);
+    sc.skips = skips;
+    sc.total = build_prefix(P, prefix, lens, skips);
     sc.nw = gridDim.x * warps_per_cta;
     if (P.balanced) {
         const int64_t blocks = static_cast<int64_t>(sc.total) * P.num_kv_heads;
@@ -260,6 +286,17 @@ __device__ __forceinline__ QRows query_rows(const DecodeParams& P, int32_t s, in
         q.n = q.n < 0 ? 0 : cap;
     }
     return q;
+}
+
+// Pieces a prefill row's tile wrote (for the merge): the chunks of key blocks
+// up to the tile's last visible key.  Token k of a sequence of length len with
+// n new tokens.
+__device__ __forceinline__ int32_t prefill_row_pieces(int32_t len, int32_t n, int32_t k, int32_t tile_tokens,
+                                                      int32_t chunk_blocks) {
+    const int32_t t = k / tile_tokens;
+    const int32_t last = min((t + 1) * tile_tokens, n) - 1;
+    const int32_t kend = (len - n + last) / kBlockTokens + 1;
+    return (kend + chunk_blocks - 1) / chunk_blocks;
 }
 
 // Records how many pieces unit (s, h) has (written by the warp holding piece 0;

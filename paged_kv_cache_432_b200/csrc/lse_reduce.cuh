@@ -32,32 +32,43 @@ __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) {
     return __float2bfloat16_rn(x);
 }
 
-// One warp merges one row (sequence, query head) from its `parts` pieces
-// starting at partial index `base`; lanes hold D/32 consecutive head dims.
+// The pieces of a row: `n1` partials at indices 0 .. n1-1 (after `base`),
+// then `n2` at off2 .. off2+n2-1 (a shared prefix's key chunks, then the
+// decode's pieces of the private part, which start at a fixed index).
+struct RowPieces {
+    int n1, off2, n2;
+    __device__ __forceinline__ int count() const { return n1 + n2; }
+    __device__ __forceinline__ int index(int p) const { return p < n1 ? p : off2 + (p - n1); }
+};
+
+// One warp merges one row (sequence, query head) from its pieces (partial
+// indices after `base`); lanes hold D/32 consecutive head dims.
 template <typename OutT, int D>
-__device__ __forceinline__ void merge_row_warp(const DecodeParams& P, size_t base, int parts,
+__device__ __forceinline__ void merge_row_warp(const DecodeParams& P, size_t base, RowPieces pcs,
                                                OutT* o, int lane) {
     constexpr int DPL = D / 32;
     using Vec = typename std::conditional<DPL == 4, float4, float2>::type;
     const float* wm = P.ws_m + base;
     const float* wl = P.ws_l + base;
     const float* wa = P.ws_acc + base * D + lane * DPL;
+    const int parts = pcs.count();
     float M = -INFINITY;
-    for (int p = lane; p < parts; p += 32) M = fmaxf(M, wm[p]);
+    for (int p = lane; p < parts; p += 32) M = fmaxf(M, wm[pcs.index(p)]);
     M = warp_max(M);
-    if (M == -INFINITY) {  // every piece fully masked
+    if (M == -INFINITY) {  // every piece fully masked, or none
 #pragma unroll
         for (int e = 0; e < DPL; ++e) o[lane * DPL + e] = from_float<OutT>(0.f);
         return;
     }
     float den = 0.f;
-    for (int p = lane; p < parts; p += 32) den += expf(wm[p] - M) * wl[p];
+    for (int p = lane; p < parts; p += 32) den += expf(wm[pcs.index(p)] - M) * wl[pcs.index(p)];
     den = warp_sum(den);
     float a[DPL];
 #pragma unroll
     for (int e = 0; e < DPL; ++e) a[e] = 0.f;
 #pragma unroll 8
-    for (int p = 0; p < parts; ++p) {
+    for (int q = 0; q < parts; ++q) {
+        const int p = pcs.index(q);
         const float w = expf(wm[p] - M);
         const Vec x = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(p) * D);
         const float* f = reinterpret_cast<const float*>(&x);
@@ -75,7 +86,10 @@ __device__ __forceinline__ void merge_row_warp(const DecodeParams& P, size_t bas
 // when the row was not computed (a token beyond the clamped count).
 struct RowRef {
     int32_t s, qh;
-    size_t r;  // output row (query token row * Hq + qh)
+    size_t r;     // output row (query token row * Hq + qh)
+    int32_t len;  // the sequence's (clamped) length
+    int32_t tok;  // query token within the sequence, of
+    int32_t n;    // its query tokens
 };
 
 __device__ __forceinline__ bool locate_row(const DecodeParams& P, int64_t row, RowRef* R) {
@@ -83,15 +97,39 @@ __device__ __forceinline__ bool locate_row(const DecodeParams& P, int64_t row, R
         R->s = P.seq_begin + static_cast<int32_t>(row / P.num_q_heads);
         R->qh = static_cast<int32_t>(row % P.num_q_heads);
         R->r = static_cast<size_t>(R->s) * P.num_q_heads + R->qh;
+        R->len = 0;
+        R->tok = 0;
+        R->n = 1;
         return true;
     }
     const int32_t t = static_cast<int32_t>(row / P.num_q_heads);
     R->qh = static_cast<int32_t>(row % P.num_q_heads);
     R->s = upper_index(P.num_seqs, t, [&](int k) { return static_cast<int64_t>(__ldg(P.q_start + k)); });
     R->r = static_cast<size_t>(row);
-    const int32_t len = seq_geometry(P, P.seq_lens[R->s]).len;
-    const QRows qr = query_rows(P, R->s, len);
-    return t - qr.base < qr.n;
+    R->len = seq_geometry(P, P.seq_lens[R->s], 0).len;
+    const QRows qr = query_rows(P, R->s, R->len);
+    R->tok = t - qr.base;
+    R->n = qr.n;
+    return R->tok < qr.n;
+}
+
+// Which partials row R merges; false when the row needs no merge (its one
+// piece was written as the final row by the decode).
+__device__ __forceinline__ bool row_pieces(const DecodeParams& P, const RowRef& R, RowPieces* pcs) {
+    if (P.tile_chunk > 0) {  // a prefill row of the tile kernel: its tile's key chunks
+        *pcs = RowPieces{prefill_row_pieces(R.len, R.n, R.tok, P.tile_tokens, P.tile_chunk), 0, 0};
+        return true;
+    }
+    const int32_t skip = seq_skip(P, R.s);
+    const SeqGeom geo = seq_geometry(P, P.seq_lens[R.s], skip);
+    const int own = geo.work > 0 ? P.ws_parts[static_cast<size_t>(R.s) * P.num_kv_heads + R.qh / P.group] : 0;
+    if (P.group_start) {  // several prompt groups: this group's prefix chunks, then the own pieces
+        const int pre = (skip + P.group_chunk - 1) / P.group_chunk;
+        *pcs = RowPieces{pre, P.piece_base, own};
+        return true;
+    }
+    *pcs = RowPieces{P.piece_base + own, 0, 0};
+    return !(P.piece_base == 0 && own <= 1);
 }
 
 // Row-wise merge (fixed partitions, or a shared prefix): one warp per
@@ -109,11 +147,9 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const Dec
     if (row >= rows) return;
     RowRef R;
     if (!locate_row(P, row, &R)) return;
-    const SeqGeom geo = seq_geometry(P, P.seq_lens[R.s]);
-    const int own = geo.work > 0 ? P.ws_parts[static_cast<size_t>(R.s) * P.num_kv_heads + R.qh / P.group] : 0;
-    const int parts = P.piece_base + own;
-    if (P.piece_base == 0 && parts <= 1) return;
-    merge_row_warp<OutT, D>(P, R.r * P.max_parts, parts, static_cast<OutT*>(P.out) + R.r * D, lane);
+    RowPieces pcs;
+    if (!row_pieces(P, R, &pcs)) return;
+    merge_row_warp<OutT, D>(P, R.r * P.max_parts, pcs, static_cast<OutT*>(P.out) + R.r * D, lane);
 }
 
 // Row-wise merge for rows with many pieces (long sequences in fixed
@@ -134,17 +170,16 @@ __global__ void __launch_bounds__(kWideWarps * 32) lse_reduce_wide_kernel(const 
     grid_dependency_wait();
     RowRef R;
     if (!locate_row(P, blockIdx.x, &R)) return;
-    const SeqGeom geo = seq_geometry(P, P.seq_lens[R.s]);
-    const int own = geo.work > 0 ? P.ws_parts[static_cast<size_t>(R.s) * P.num_kv_heads + R.qh / P.group] : 0;
-    const int parts = P.piece_base + own;
-    if (P.piece_base == 0 && parts <= 1) return;
+    RowPieces pcs;
+    if (!row_pieces(P, R, &pcs)) return;
+    const int parts = pcs.count();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t base = R.r * P.max_parts;
     const float* wm = P.ws_m + base;
     const float* wl = P.ws_l + base;
     const float* wa = P.ws_acc + base * D;
     float M = -INFINITY;
-    for (int p = tid; p < parts; p += blockDim.x) M = fmaxf(M, wm[p]);
+    for (int p = tid; p < parts; p += blockDim.x) M = fmaxf(M, wm[pcs.index(p)]);
     M = warp_max(M);
     if (lane == 0) wmax[warp] = M;
     __syncthreads();
@@ -158,9 +193,9 @@ __global__ void __launch_bounds__(kWideWarps * 32) lse_reduce_wide_kernel(const 
     }
     float den = 0.f;
     for (int p = tid; p < parts; p += blockDim.x) {
-        const float w = expf(wm[p] - M);
+        const float w = expf(wm[pcs.index(p)] - M);
         if (p < kWideWeights) wts[p] = w;
-        den += w * wl[p];
+        den += w * wl[pcs.index(p)];
     }
     den = warp_sum(den);
     if (lane == 0) wden[warp] = den;
@@ -170,8 +205,8 @@ __global__ void __launch_bounds__(kWideWarps * 32) lse_reduce_wide_kernel(const 
     for (int e = 0; e < DPL; ++e) a[e] = 0.f;
 #pragma unroll 8
     for (int p = warp; p < parts; p += kWideWarps) {
-        const float w = p < kWideWeights ? wts[p] : expf(wm[p] - M);
-        const Vec x = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(p) * D + lane * DPL);
+        const float w = p < kWideWeights ? wts[p] : expf(wm[pcs.index(p)] - M);
+        const Vec x = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(pcs.index(p)) * D + lane * DPL);
         const float* f = reinterpret_cast<const float*>(&x);
 #pragma unroll
         for (int e = 0; e < DPL; ++e) a[e] = fmaf(w, f[e], a[e]);
@@ -203,9 +238,10 @@ lse_reduce_balanced_kernel(const DecodeParams P, int32_t decode_warps) {
     extern __shared__ int32_t smem_i[];
     int32_t* prefix = smem_i;
     int32_t* lens = prefix + P.seq_count + 1;
+    int32_t* skips = lens + P.seq_count;
     // the lengths are input no kernel of this library writes: the prefix is
     // built while the decode launched just before still runs
-    const int32_t total = build_prefix(P, prefix, lens);  // blocks per sequence
+    const int32_t total = build_prefix(P, prefix, lens, skips);  // blocks per sequence
     grid_dependency_wait();  // the decode's partials
     const int64_t hk = P.num_kv_heads;
     const int64_t T = static_cast<int64_t>(total) * hk;
@@ -214,7 +250,7 @@ lse_reduce_balanced_kernel(const DecodeParams P, int32_t decode_warps) {
     const int64_t b = (static_cast<int64_t>(blockIdx.x) + 1) * C;
     if (b >= T) return;
     const int i = upper_index(P.seq_count, b, [&](int k) { return hk * prefix[k]; });
-    const SeqGeom geo = seq_geometry(P, lens[i]);
+    const SeqGeom geo = seq_geometry(P, lens[i], skips[i]);
     const int64_t off = b - hk * prefix[i];
     const int32_t h = static_cast<int32_t>(off / geo.work);
     const int64_t j = off - static_cast<int64_t>(h) * geo.work;
@@ -229,7 +265,7 @@ lse_reduce_balanced_kernel(const DecodeParams P, int32_t decode_warps) {
     for (int r = warp; r < P.group * qr.n; r += kReduceWarps) {  // (query token, head) rows
         const size_t row = (static_cast<size_t>(qr.base) + r / P.group) * P.num_q_heads +
                            h * P.group + r % P.group;
-        merge_row_warp<OutT, D>(P, row * P.max_parts, parts, static_cast<OutT*>(P.out) + row * D,
+        merge_row_warp<OutT, D>(P, row * P.max_parts, RowPieces{parts, 0, 0}, static_cast<OutT*>(P.out) + row * D,
                                 lane);
     }
 }

@@ -53,6 +53,10 @@ SIGNATURES = {
     "pa_decode_shared_prefix": (ctypes.c_int, [_P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32,
                                                _I32, _F, _I32, _P, _SZ, _P, _I32, _P]),
     "pa_decode_shared_prefix_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32]),
+    "pa_decode_shared_prefix_groups": (ctypes.c_int, [_P, _P, _P, _P, _I32, _P, _I32, _P, _P, _I32, _I32, _I32,
+                                                      _I32, _I32, _I32, _I32, _I32, _F, _I32, _P, _SZ, _P, _I32,
+                                                      _P]),
+    "pa_decode_shared_prefix_groups_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "pa_decode_multi": (ctypes.c_int, [_P, _P, _I32, _I32, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
                                        _I32, _I32, _F, _I32, _P, _SZ, _P, _I32, _P]),
     "pa_decode_multi_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32]),
@@ -231,6 +235,37 @@ def decode_shared_prefix(q, k_cache, v_cache, block_tables, seq_lens, scale, sha
         max_seq_len, shared_blocks, N, Hq, Hkv, D, NB, B, float(scale), partition_blocks, _ptr(workspace),
         ws_bytes, _ptr(out), dtype_code(q.dtype), _stream(stream))
     _check("pa_decode_shared_prefix", rc)
+    return out
+
+
+def shared_prefix_groups_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len,
+                                        max_shared_blocks, num_groups, partition_blocks=0, block_size=16) -> int:
+    return int(lib().pa_decode_shared_prefix_groups_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                                   max_seq_len, max_shared_blocks, num_groups,
+                                                                   block_size, partition_blocks))
+
+
+def decode_shared_prefix_groups(q, k_cache, v_cache, block_tables, seq_lens, scale, group_start,
+                                group_shared_blocks, max_shared_blocks, out=None, max_seq_len=0, partition_blocks=0,
+                                workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode_shared_prefix_groups: group i = sequences group_start[i] ..
+    group_start[i+1]-1 (int32 device tensors), sharing their first
+    group_shared_blocks[i] blocks; max_shared_blocks bounds those counts."""
+    N, Hq, D = q.shape
+    NB, Hkv, B, _ = k_cache.shape
+    G = group_start.numel() - 1
+    msl = max_seq_len if max_seq_len > 0 else block_tables.shape[1] * 16
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        n = shared_prefix_groups_workspace_size(N, Hq, Hkv, D, msl, max_shared_blocks, G, partition_blocks)
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().pa_decode_shared_prefix_groups(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens),
+        max_seq_len, _ptr(group_start), _ptr(group_shared_blocks), G, max_shared_blocks, N, Hq, Hkv, D, NB, B,
+        float(scale), partition_blocks, _ptr(workspace), ws_bytes, _ptr(out), dtype_code(q.dtype), _stream(stream))
+    _check("pa_decode_shared_prefix_groups", rc)
     return out
 
 

@@ -87,6 +87,12 @@ class Workload:
     shared_blocks: list = field(default_factory=list)  # physical ids referenced by >1 seq
     shared_prefix_blocks: int = 0  # leading table entries every sequence shares (whole blocks)
     desc: str = ""
+    # several prompt groups: group i = sequences group_start_host[i] .. [i+1]-1,
+    # sharing their first group_blocks_host[i] table entries (whole blocks)
+    group_start_host: list = field(default_factory=list)
+    group_blocks_host: list = field(default_factory=list)
+    group_start: Optional[torch.Tensor] = None  # int32 [G + 1] on the device
+    group_blocks: Optional[torch.Tensor] = None  # int32 [G]
 
     @property
     def num_seqs(self) -> int:
@@ -156,13 +162,15 @@ class Plan:
     lens: list
     tables: list
     num_blocks: int
-    shared: list  # physical ids referenced by every sequence (shared prefix)
-    cow_pairs: list  # (shared source block, private copy) for a prefix ending mid-block
-    prefix_len: int = 0
+    shared: list  # physical ids of the full shared prefix blocks (all groups)
+    cow_pairs: list  # (shared source block, private copy, tokens copied) for a prefix ending mid-block
+    prefix_len: int = 0  # one prompt shared by every sequence (0 with several groups)
+    group_start: list = field(default_factory=list)  # sequences of group i: [start[i], start[i+1])
+    group_blocks: list = field(default_factory=list)  # full blocks group i shares
 
     @property
     def needed_blocks(self) -> int:
-        ids = set(b for t in self.tables for b in t) | set(src for src, _ in self.cow_pairs)
+        ids = set(b for t in self.tables for b in t) | set(src for src, _, _ in self.cow_pairs)
         return len(ids)
 
 
@@ -172,29 +180,35 @@ def plan(
     num_blocks: Optional[int] = None,
     pool_factor: float = 1.25,
     prefix_len: int = 0,
+    groups: Optional[Sequence[tuple]] = None,
 ) -> Plan:
     """Allocate physical blocks for sequences of the given total lengths.
 
     The pool holds ``ceil(pool_factor * needed)`` blocks unless ``num_blocks`` is
     given; blocks are taken in order from a seeded random permutation of the pool
-    (a shuffled free list).  With ``prefix_len > 0`` every sequence starts with the
-    same ``prefix_len`` tokens: the full prefix blocks are allocated once and every
-    table points at them; if the prefix ends inside a block, that block is kept
-    once as a shared source and each sequence gets a private copy of it
-    (copy-on-write) into which its own suffix continues.
+    (a shuffled free list).  ``groups`` = [(count, prefix_len), ...] splits the
+    sequences, in order, into prompt groups: the ``count`` sequences of a group
+    start with the same ``prefix_len`` tokens, whose full blocks are allocated
+    once and named by every table of the group; if the prefix ends inside a
+    block, that block is kept once as a shared source and each sequence of the
+    group gets a private copy of it (copy-on-write) into which its own suffix
+    continues.  ``prefix_len > 0`` without ``groups`` is one group of every
+    sequence.
     """
     B = BLOCK_SIZE
     lens = [int(x) for x in lens]
+    if groups is None:
+        groups = [(len(lens), prefix_len)]
+    assert sum(c for c, _ in groups) == len(lens), "the groups must cover every sequence"
     gen = torch.Generator(device="cpu")
     gen.manual_seed(seed)
-    n_full_prefix = prefix_len // B
-    prefix_rem = prefix_len % B
-    if prefix_len:
-        assert all(L >= prefix_len for L in lens), "every sequence must hold the prefix"
-    # tokens of a sequence that live in its private blocks
-    private_tokens = [L - n_full_prefix * B for L in lens]
-    needed = n_full_prefix + (1 if prefix_rem else 0)
-    needed += sum(_blocks_for(n, B) for n in private_tokens)
+    needed = 0
+    start = 0
+    for count, pl in groups:
+        assert all(L >= pl for L in lens[start:start + count]), "every sequence must hold its prefix"
+        needed += pl // B + (1 if pl % B else 0)
+        needed += sum(_blocks_for(L - (pl // B) * B, B) for L in lens[start:start + count])
+        start += count
     if num_blocks is None:
         num_blocks = max(1, math.ceil(pool_factor * needed))
     assert num_blocks >= needed, (num_blocks, needed)
@@ -208,19 +222,26 @@ def plan(
         cursor += 1
         return b
 
-    shared = [take() for _ in range(n_full_prefix)]
-    cow_source = take() if prefix_rem else None
-    tables = []
-    cow_pairs = []
-    for rest in private_tokens:
-        t = list(shared)
-        for j in range(_blocks_for(rest, B)):
-            b = take()
-            if j == 0 and prefix_rem:
-                cow_pairs.append((cow_source, b))
-            t.append(b)
-        tables.append(t)
-    return Plan(lens, tables, num_blocks, shared, cow_pairs, prefix_len)
+    tables, cow_pairs, shared_all, gstart, gblocks = [], [], [], [0], []
+    start = 0
+    for count, pl in groups:
+        n_full, rem = pl // B, pl % B
+        shared = [take() for _ in range(n_full)]
+        shared_all += shared
+        cow_source = take() if rem else None
+        for L in lens[start:start + count]:
+            t = list(shared)
+            for j in range(_blocks_for(L - n_full * B, B)):
+                b = take()
+                if j == 0 and rem:
+                    cow_pairs.append((cow_source, b, rem))
+                t.append(b)
+            tables.append(t)
+        start += count
+        gstart.append(start)
+        gblocks.append(n_full)
+    one = len(groups) == 1
+    return Plan(lens, tables, num_blocks, shared_all, cow_pairs, groups[0][1] if one else 0, gstart, gblocks)
 
 
 def build(
@@ -239,6 +260,7 @@ def build(
     name: str = "custom",
     desc: str = "",
     table_width: Optional[int] = None,
+    groups: Optional[Sequence[tuple]] = None,
 ) -> Workload:
     """Build a workload from explicit per-sequence total lengths (see ``plan``).
 
@@ -248,9 +270,8 @@ def build(
     """
     B = BLOCK_SIZE
     assert num_q_heads % num_kv_heads == 0
-    p = plan(lens, seed=seed, num_blocks=num_blocks, pool_factor=pool_factor, prefix_len=prefix_len)
+    p = plan(lens, seed=seed, num_blocks=num_blocks, pool_factor=pool_factor, prefix_len=prefix_len, groups=groups)
     lens, tables, num_blocks = p.lens, p.tables, p.num_blocks
-    prefix_rem = prefix_len % B
 
     width = max([len(t) for t in tables] + [1])
     if table_width is not None:
@@ -271,9 +292,9 @@ def build(
     new_v = _randn((N, num_kv_heads, head_dim), vgen, device, dtype)
 
     # copy-on-write of the partial last prefix block into each private copy
-    for src, dst in p.cow_pairs:
-        k_cache[dst, :, :prefix_rem] = k_cache[src, :, :prefix_rem]
-        v_cache[dst, :, :prefix_rem] = v_cache[src, :, :prefix_rem]
+    for src, dst, rem in p.cow_pairs:
+        k_cache[dst, :, :rem] = k_cache[src, :, :rem]
+        v_cache[dst, :, :rem] = v_cache[src, :, :rem]
 
     slot_mapping = torch.tensor(new_token_slots(p), dtype=torch.int64)
 
@@ -304,9 +325,13 @@ def build(
         new_v=new_v,
         slot_mapping=slot_mapping.to(device),
         partition_blocks=partition_blocks,
-        shared_blocks=sorted(p.shared + [src for src, _ in p.cow_pairs[:1]]),
-        shared_prefix_blocks=len(p.shared),
+        shared_blocks=sorted(set(p.shared + [src for src, _, _ in p.cow_pairs])),
+        shared_prefix_blocks=p.prefix_len // B if groups is None else 0,
         desc=desc,
+        group_start_host=list(p.group_start),
+        group_blocks_host=list(p.group_blocks),
+        group_start=torch.tensor(p.group_start, dtype=torch.int32).to(device),
+        group_blocks=torch.tensor(p.group_blocks, dtype=torch.int32).to(device),
     )
 
 
@@ -407,6 +432,12 @@ def make(name: str, seed: int = 0, device="cpu", poison_unused: bool = False,
         prefix = kw.pop("prefix_len", prefix)
         if prefix != 4096:  # variant with a different prefix length, same suffixes
             lens = [L - 4096 + prefix for L in lens]
+        ng = kw.pop("prompt_groups", 1)
+        if ng > 1:  # variant: ng prompts of the same length, each shared by a consecutive share of the batch
+            n = len(lens)
+            groups = [(n * (i + 1) // ng - n * i // ng, prefix) for i in range(ng)]
+            common["desc"] = desc + f" (variant: {ng} prompts, each shared by {n // ng} sequences)"
+            return build(lens, 32, 8, 128, torch.bfloat16, groups=groups, **common, **kw)
         return build(lens, 32, 8, 128, torch.bfloat16, prefix_len=prefix, **common, **kw)
     if name == "long":
         kw.setdefault("partition_blocks", 32)

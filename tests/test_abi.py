@@ -96,16 +96,31 @@ def test_shared_prefix_workspace_size(lib):
     assert lib.pa_decode_shared_prefix_workspace_size(N, Hq, Hkv, D, 1000, 256, 16, 0) == 0
 
 
+def _tile_splits(sms, work_tiles, nb_max):
+    """The key chunking the tile kernel picks (as documented in the header):
+    as many chunks as fill the SMs, at most 16, in multiples of 4 blocks."""
+    want = max(1, min(16, sms // work_tiles if work_tiles else 1))
+    ch = -(-nb_max // want)
+    ch = -(-ch // 4) * 4
+    return -(-nb_max // ch)
+
+
 def test_multi_query_workspace_and_limits(lib):
+    import torch
+
     a256 = lambda x: (x + 255) // 256 * 256
     N, T, Hq, Hkv, D, L = 4, 13, 8, 2, 128, 3000
-    P = -(-(-(-L // 16)) // 16) + 1  # balanced bound
-    rows = T * Hq
-    assert lib.pa_decode_multi_workspace_size(N, T, Hq, Hkv, D, L, 16, 0) == \
-        2 * a256(rows * P * 4) + a256(rows * P * D * 4) + a256(N * Hkv * 4)
-    # group 4 x 5 query tokens = 20 rows > 16: unsupported; fp32: unsupported
+    layout = lambda P: 2 * a256(T * Hq * P * 4) + a256(T * Hq * P * D * 4) + a256(N * Hkv * 4)
+    P = -(-(-(-L // 16)) // 16) + 1  # balanced bound of the warp-level path
+    # the tile path (group x query tokens > 16) keeps one partial per key chunk
+    sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 1 << 30
+    tiles = -(-T // (128 // (Hq // Hkv))) + N
+    C = _tile_splits(sms, tiles * Hkv, -(-L // 16))
+    want = max(layout(P), layout(C) if C > 1 else 0)
+    assert lib.pa_decode_multi_workspace_size(N, T, Hq, Hkv, D, L, 16, 0) == want
+    # fp32 or a missing q_start are refused before anything is launched
     assert lib.pa_decode_multi(16, 16, T, 5, 16, 16, 16, 64, 16, L, N, 8, 2, D, 64, 16, 0.1, 0, None, 0, 16,
-                               pa.PA_DTYPE_BF16, None) == pa.PA_ERR_UNSUPPORTED
+                               pa.PA_DTYPE_F32, None) == pa.PA_ERR_UNSUPPORTED
     assert lib.pa_decode_multi(16, 16, T, 2, 16, 16, 16, 64, 16, L, N, 8, 2, D, 64, 16, 0.1, 0, None, 0, 16,
                                pa.PA_DTYPE_F32, None) == pa.PA_ERR_UNSUPPORTED
     assert lib.pa_decode_multi(16, None, T, 2, 16, 16, 16, 64, 16, L, N, 8, 2, D, 64, 16, 0.1, 0, None, 0, 16,

@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import assert_close, host, to_f64
+from helpers import assert_close, host, oracle_decode_multi_all_rows, to_f64
 from paged_kv_cache_432_b200 import build as pa_build
 from paged_kv_cache_432_b200 import pagedattn as pa
 from paged_kv_cache_432_b200 import workload as wl
@@ -64,3 +64,67 @@ def test_too_many_query_tokens_are_flagged():
     q, qs = _queries([2, 5], 8, 128, seed=4)  # the second sequence has 5 > max_q_len = 4
     pa.decode_multi(q, qs, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, 4, max_seq_len=40)
     assert pa.device_error() & pa.PA_DEVERR_SEQ_LEN
+
+
+# ------------------------------------------------------------------ prefill chunks (tile kernel)
+PREFILL_CASES = [
+    # lens, new tokens per sequence: chunks of 64..512, chunks that start
+    # mid-block, a whole sequence (n = L), an empty sequence
+    ([700, 513, 64, 1000, 300, 0], [64, 100, 64, 512, 300, 0]),
+    ([4100, 77, 2049], [257, 77, 129]),
+]
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (64, 8), (6, 1), (16, 16)])
+@pytest.mark.parametrize("D", [128, 64])
+@pytest.mark.parametrize("case", [0, 1])
+def test_prefill_chunks_match_oracle(Hq, Hkv, D, case):
+    """More (query token, head) rows per sequence than one MMA fragment: the
+    tensor-memory tile kernel, causal among the new tokens; unused slots hold
+    NaN (a slot past a sequence's length must not reach the output)."""
+    lens, nq = PREFILL_CASES[case]
+    w = wl.build(lens, Hq, Hkv, D, torch.bfloat16, seed=Hq + D + case, device=DEV, poison_unused=True)
+    q, qs = _queries(nq, Hq, D, seed=Hq + case)
+    out = pa.decode_multi(q, qs, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, max(nq),
+                          max_seq_len=w.max_seq_len)
+    torch.cuda.synchronize()
+    assert pa.device_error() == 0
+    assert_close(to_f64(out), _oracle(w, q, qs), torch.bfloat16, f"prefill {Hq}/{Hkv} D={D} case {case}")
+
+
+def test_prefill_many_sequences_without_key_chunks():
+    """Enough tiles to fill the device without cutting the keys: every row is
+    written by its tile directly (no merge)."""
+    rng = np.random.default_rng(4)
+    lens = [int(x) for x in rng.integers(300, 2500, size=24)]
+    nq = [min(L, int(x)) for L, x in zip(lens, rng.integers(64, 400, size=24))]
+    w = wl.build(lens, 32, 8, 128, torch.bfloat16, seed=77, device=DEV, poison_unused=True)
+    q, qs = _queries(nq, 32, 128, seed=5)
+    assert pa.multi_workspace_size(w.num_seqs, q.shape[0], 32, 8, 128, w.max_seq_len) >= 0
+    out = pa.decode_multi(q, qs, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, max(nq),
+                          max_seq_len=w.max_seq_len)
+    torch.cuda.synchronize()
+    assert pa.device_error() == 0
+    h = host(w)
+    ref = oracle_decode_multi_all_rows(wl.as_numpy(q), h["kc"], h["vc"], h["bt"], h["sl"], qs.cpu().numpy(), w.scale)
+    assert_close(to_f64(out), ref, torch.bfloat16, "prefill, 24 sequences")
+
+
+def test_prefill_more_tokens_than_max_q_len_are_flagged():
+    w = wl.build([300, 300], 32, 8, 128, torch.bfloat16, seed=6, device=DEV)
+    q, qs = _queries([64, 100], 32, 128, seed=6)  # 100 > max_q_len = 80
+    out = torch.full_like(q, float("nan"))
+    pa.decode_multi(q, qs, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, 80, out=out,
+                    max_seq_len=300)
+    torch.cuda.synchronize()
+    assert pa.device_error() & pa.PA_DEVERR_SEQ_LEN
+    # the rows within the bound are exact: sequence 0 whole, and sequence 1's
+    # first 80 query rows as its last 80 positions; its excess rows are not written
+    assert torch.isnan(out[144:164].float()).all()
+    h = host(w)
+    ref0 = oracle.paged_decode_multi(wl.as_numpy(q)[:64], h["kc"], h["vc"], h["bt"][:1], h["sl"][:1],
+                                     np.array([0, 64], np.int32), w.scale)
+    assert_close(to_f64(out)[:64], ref0, torch.bfloat16, "prefill seq 0")
+    ref1 = oracle.paged_decode_multi(wl.as_numpy(q)[64:144], h["kc"], h["vc"], h["bt"][1:2],
+                                     np.array([300], np.int32), np.array([0, 80], np.int32), w.scale)
+    assert_close(to_f64(out)[64:144], ref1, torch.bfloat16, "prefill seq 1, clamped")

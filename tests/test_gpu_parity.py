@@ -345,3 +345,68 @@ def test_sequence_longer_than_bound_is_clamped_and_flagged():
     h["sl"] = np.array([100, 300], np.int32)
     ref = oracle.paged_decode(h["q"], h["kc"], h["vc"], h["bt"], h["sl"], w.scale)
     assert_close(to_f64(out), ref, torch.bfloat16, "clamped")
+
+
+# ------------------------------------------------------------------ several prompt groups
+GROUP_CASES = [
+    # (count, prefix tokens) per group, suffix lengths
+    ([(3, 4096), (2, 0), (5, 1600), (1, 64)], [64, 1, 300, 512, 16, 5, 40, 700, 33, 0, 90]),
+    ([(20, 512), (20, 4090)], [int(x) for x in np.random.default_rng(1).integers(1, 400, 40)]),
+]
+
+
+@pytest.mark.parametrize("case", [0, 1])
+@pytest.mark.parametrize("Hq,Hkv,D", [(32, 8, 128), (16, 2, 64), (8, 8, 128)])
+@pytest.mark.parametrize("pb", [0, 4])
+def test_shared_prefix_groups_match_oracle(case, Hq, Hkv, D, pb):
+    """Several prompt groups in one batch (a group that shares nothing, a
+    prompt ending mid-block with copy-on-write, a one-sequence group), each
+    group's shared blocks read once per tile of its query rows."""
+    groups, suffixes = GROUP_CASES[case]
+    lens, i = [], 0
+    for count, pl in groups:
+        lens += [pl + suffixes[i + k] for k in range(count)]
+        i += count
+    w = wl.build(lens, Hq, Hkv, D, torch.bfloat16, seed=case + Hq, device=DEV, groups=groups, poison_unused=True)
+    maxs = max(w.group_blocks_host)
+    out = pa.decode_shared_prefix_groups(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale,
+                                         w.group_start, w.group_blocks, maxs, max_seq_len=w.max_seq_len,
+                                         partition_blocks=pb)
+    torch.cuda.synchronize()
+    assert pa.device_error() == 0
+    assert_close(to_f64(out), oracle_decode(w), torch.bfloat16, f"groups case {case} {Hq}/{Hkv} D={D} pb={pb}")
+
+
+def test_shared_prefix_groups_four_prompts_full_size():
+    """The prefix-sharing workload with four prompts of 4096 tokens, each shared
+    by 32 sequences, after the cache write; every row against the oracle."""
+    w = wl.make("prefix", device=DEV, prompt_groups=4)
+    h = host(w)
+    pa.cache_write(w.new_k, w.new_v, w.slot_mapping, w.k_cache, w.v_cache)
+    oracle.cache_write(h["nk"], h["nv"], h["sm"], h["kc"], h["vc"], inplace=True)
+    out = pa.decode_shared_prefix_groups(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale,
+                                         w.group_start, w.group_blocks, max(w.group_blocks_host),
+                                         max_seq_len=w.max_seq_len)
+    torch.cuda.synchronize()
+    assert pa.device_error() == 0
+    assert_close(to_f64(out), oracle_decode_all_rows(w, h), torch.bfloat16, "four prompts, every row")
+
+
+def test_shared_prefix_groups_bad_group_list_is_flagged():
+    w = wl.build([600, 700, 300], 8, 2, 128, torch.bfloat16, seed=5, device=DEV, groups=[(2, 512), (1, 0)])
+    # a count above the bound
+    gb = torch.tensor([40, 0], dtype=torch.int32, device=DEV)
+    pa.decode_shared_prefix_groups(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale,
+                                   w.group_start, gb, 32, max_seq_len=700)
+    assert pa.device_error() & pa.PA_DEVERR_PREFIX
+    # groups out of order
+    gs = torch.tensor([0, 3, 2], dtype=torch.int32, device=DEV)
+    pa.decode_shared_prefix_groups(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale,
+                                   gs, w.group_blocks, 32, max_seq_len=700)
+    assert pa.device_error() & pa.PA_DEVERR_PREFIX
+    # a table of group 0 that does not start with the group's blocks
+    bt = w.block_tables.clone()
+    bt[1, 2] = w.tables_host[2][0]
+    pa.decode_shared_prefix_groups(w.q, w.k_cache, w.v_cache, bt, w.seq_lens, w.scale,
+                                   w.group_start, w.group_blocks, 32, max_seq_len=700)
+    assert pa.device_error() & pa.PA_DEVERR_PREFIX

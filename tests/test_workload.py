@@ -63,7 +63,8 @@ def test_copy_on_write_of_partial_prefix_block():
     w = wl.build([4090 + 5, 4090 + 40], 2, 1, 16, torch.bfloat16, seed=3, prefix_len=4090)
     p = wl.plan(w.lens_host, seed=3, prefix_len=4090)
     assert len(p.cow_pairs) == 2
-    for src, dst in p.cow_pairs:
+    for src, dst, rem in p.cow_pairs:
+        assert rem == 10
         assert torch.equal(w.k_cache[dst, :, :10], w.k_cache[src, :, :10])
         assert not torch.equal(w.k_cache[dst, :, 10:], w.k_cache[src, :, 10:])
     # the copies are private: different tables, same logical prefix
@@ -97,3 +98,29 @@ def test_fp8_pools_draw_no_nan_code_and_poison_only_unreachable_slots():
         for t in range(L):
             assert not nan[w.tables_host[s][t // 16], t % 16]
     assert int(nan.sum()) == w.num_blocks * 16 - sum(w.lens_host)
+
+
+def test_prompt_groups_share_their_own_prefix_blocks():
+    """Several prompt groups: the tables of a group start with the same full
+    blocks (its own prompt), different groups share nothing, and a prompt
+    ending mid-block gives each sequence of its group a private copy."""
+    groups = [(3, 64), (2, 0), (4, 37)]
+    lens = [64 + 5, 64 + 40, 64 + 16, 9, 300, 37 + 1, 37 + 20, 37 + 100, 37]
+    w = wl.build(lens, 4, 2, 16, torch.bfloat16, seed=8, groups=groups)
+    assert w.group_start_host == [0, 3, 5, 9] and w.group_blocks_host == [4, 0, 2]
+    assert w.group_start.tolist() == [0, 3, 5, 9] and w.group_blocks.tolist() == [4, 0, 2]
+    assert w.shared_prefix_blocks == 0
+    t = w.tables_host
+    assert t[0][:4] == t[1][:4] == t[2][:4]
+    assert t[5][:2] == t[6][:2] == t[7][:2] == t[8][:2]
+    assert t[5][2] != t[6][2]                     # the partial third block: private copies
+    assert not set(t[0][:4]) & set(t[5][:2])      # the groups share nothing
+    assert not set(t[3]) & set(t[4])
+    p = wl.plan(lens, seed=8, groups=groups)
+    assert sorted(rem for _, _, rem in p.cow_pairs) == [5] * 4
+    for src, dst, rem in p.cow_pairs:
+        assert torch.equal(w.k_cache[dst, :, :rem], w.k_cache[src, :, :rem])
+    # one group of every sequence gives the same tables as the single-prefix form
+    a = wl.plan(lens[:3], seed=2, prefix_len=64)
+    b = wl.plan(lens[:3], seed=2, groups=[(3, 64)])
+    assert a.tables == b.tables and a.num_blocks == b.num_blocks
