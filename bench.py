@@ -114,10 +114,15 @@ def workload_config(w: wl.Workload, pb: int, kv: str = "bf16") -> dict:
     }
 
 
-def source_digest() -> str:
+# the device sources of the decode kernel (decode_bf16_mma_kernel, bf16 and
+# E4M3): a committed traffic figure counts only while these are unchanged
+DECODE_SOURCES = ("common.cuh", "items.cuh", "decode_mma.cuh")
+
+
+def source_digest(files=DECODE_SOURCES) -> str:
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "paged_kv_cache_432_b200", "csrc", "*"))):
-        h.update(open(p, "rb").read())
+    for name in files:
+        h.update(open(os.path.join(ROOT, "paged_kv_cache_432_b200", "csrc", name), "rb").read())
     return h.hexdigest()[:16]
 
 
