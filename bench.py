@@ -790,7 +790,7 @@ def run_multi(args) -> None:
         pa_build.build()
     barrier(ws)
     dev = torch.device("cuda", local)
-    w = wl.make(args.config, seed=replica_seed(args.seed, rank), device=dev)
+    w = wl.make(args.config, seed=replica_seed(args.seed, rank), device=dev, max_seqs=args.max_seqs)
     nq = args.q_len
     n_per = [min(nq, L) for L in w.lens_host]
     gen = torch.Generator(device=dev).manual_seed(args.seed + 7)

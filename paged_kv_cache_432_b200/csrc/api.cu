@@ -244,8 +244,10 @@ Plan make_plan(int32_t max_seq_len, int32_t partition_blocks) {
 constexpr int32_t kMaxTileSplits = 16;
 constexpr int32_t kWideReducePieces = 32;  // rows that can have more pieces merge with a CTA each
 
-// Query tokens (or sequences) per 128-row tile of the tile kernel.
-int32_t tile_tokens(int32_t group) { return 128 / group; }
+// Query tokens (or sequences) per 128-row half of a tile of the tile kernel,
+// and per tile (two halves).
+int32_t half_tokens(int32_t group) { return 128 / group; }
+int32_t tile_tokens(int32_t group) { return kTileHalves * half_tokens(group); }
 
 Plan make_prefix_plan(int32_t max_seq_len, int32_t partition_blocks, int32_t shared_blocks,
                       int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads) {
@@ -568,8 +570,8 @@ int run_partitions(const DecodeParams& P, int32_t dtype, cudaStream_t st) {
 
 // ------------------------------------------------------------ tile kernel (tcgen05)
 // q seen as a 3-D tensor [rows][num_q_heads][head_dim], loaded in boxes of 64
-// columns x `group` heads x `tile_tokens` rows: one box lands as the tile's
-// tile_tokens * group query rows of 128 bytes (one 64-column slab), in the
+// columns x `group` heads x half_tokens rows: one box lands as a half tile's
+// half_tokens * group query rows of 128 bytes (one 64-column slab), in the
 // 128-byte swizzle the tensor-core descriptors expect.
 int encode_q_map(CUtensorMap* map, const void* q, int64_t rows, int32_t num_q_heads, int head_dim,
                  int32_t group) {
@@ -580,7 +582,7 @@ int encode_q_map(CUtensorMap* map, const void* q, int64_t rows, int32_t num_q_he
                           static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
                              static_cast<cuuint64_t>(num_q_heads) * head_dim * 2};
-    cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(tile_tokens(group))};
+    cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(half_tokens(group))};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -665,7 +667,7 @@ int launch_prefix_tiles(const DecodeParams& P, Plan* plan, cudaStream_t st) {
     T.num_q_heads = P.num_q_heads;
     T.num_kv_heads = P.num_kv_heads;
     T.group = P.group;
-    T.tile_tokens = tile_tokens(P.group);
+    T.half_tokens = half_tokens(P.group);
     T.max_blocks_per_seq = P.max_blocks_per_seq;
     T.num_blocks = P.num_blocks;
     T.chunk_blocks = sp.chunk_blocks;
@@ -800,7 +802,7 @@ int run_prefill_tiles(const DecodeArgs& a) {
     T.num_q_heads = a.num_q_heads;
     T.num_kv_heads = a.num_kv_heads;
     T.group = a.num_q_heads / a.num_kv_heads;
-    T.tile_tokens = tile_tokens(T.group);
+    T.half_tokens = half_tokens(T.group);
     T.max_blocks_per_seq = a.max_blocks_per_seq;
     T.num_blocks = a.num_blocks;
     T.chunk_blocks = pp.split.chunk_blocks;
@@ -833,7 +835,7 @@ int run_prefill_tiles(const DecodeArgs& a) {
     R.max_parts = pp.split.splits;
     R.len_cap = T.len_cap;
     R.part_blocks = kNoSplit;
-    R.tile_tokens = T.tile_tokens;
+    R.tile_tokens = tile_tokens(T.group);
     R.tile_chunk = pp.split.chunk_blocks;
     const int64_t rows = static_cast<int64_t>(a.num_q_rows) * a.num_q_heads;
     const unsigned grid = static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps);

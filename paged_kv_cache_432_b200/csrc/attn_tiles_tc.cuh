@@ -1,4 +1,4 @@
-// attn_tiles_tc.cuh -- attention of query tiles of up to 128 rows to paged
+// attn_tiles_tc.cuh -- attention of query tiles of up to 256 rows to paged
 // keys on the 5th-generation tensor cores (tcgen05: S = Q K^T and O += P V
 // accumulate in tensor memory).
 //
@@ -22,30 +22,35 @@
 //    sits at position L - n + k and sees keys 0 .. L - n + k.
 //
 // Work: a unit is a group (prefix) or a sequence (prefill).  Its tokens (the
-// group's sequences, or the new query tokens) are cut into tiles of
-// T = floor(128 / g) tokens; row r of a tile is token r / g, query head
-// h*g + r % g, one TMEM lane.  The unit's key blocks are cut into chunks of
-// chunk_blocks blocks (one chunk when the device is full without a split).
-// An item is (chunk c, kv head h, tile t), numbered with t fastest, so that
-// the tiles reading the same keys run side by side and share them in L2.  The
-// grid is persistent, one CTA per SM: CTA b takes items b, b + grid, ...; each
-// CTA builds the per-unit item prefix once in shared memory and finds any
-// item by binary search.  An item whose chunk lies wholly past its tile's last
-// visible key is empty: every role skips it.
+// group's sequences, or the new query tokens) are cut into tiles of two
+// halves of T = floor(128 / g) tokens; row r of a half is token r / g, query
+// head h*g + r % g, one TMEM lane, and the two halves are two accumulator
+// sets in tensor memory that share every K/V stage (so a K/V block is fetched
+// once per 2T tokens: the SM's TMA engine, which bounds a one-half tile, then
+// delivers half the boxes per row).  The unit's key blocks are cut into
+// chunks of chunk_blocks blocks (one chunk when the device is full without a
+// split).  An item is (chunk c, kv head h, tile t), numbered with t fastest,
+// so that the tiles reading the same keys run side by side and share them in
+// L2.  The grid is persistent, one CTA per SM: CTA b takes items b, b + grid,
+// ...; each CTA builds the per-unit item prefix once in shared memory and finds
+// any item by binary search.  An item whose chunk lies wholly past its tile's
+// last visible key is empty: every role skips it.
 //
-// Roles (320 threads): warps 0-7 softmax (two threads per query row: warp w
-// reaches TMEM lanes 32 (w mod 4) .. +31 and takes half w / 4 of a step's 64
-// keys and of O's columns), warp 8 TMA producer, warp 9 MMA issue (one
-// thread).  Per item, the producer loads the tile's Q rows with one 3-D TMA
-// box per 64-column slab (tokens x heads x columns, the 128-byte swizzle) into
-// one of two Q buffers, then 64-key steps of K and V (4 blocks, 64 x 16
-// boxes) into a 4-stage ring.  The MMA thread issues S of step j + 1 before
-// P V of step j (two S buffers in TMEM), so the tensor cores run while the
-// softmax works, also across item boundaries.  The softmax threads read their
-// half of a row of S straight from TMEM, swap their maxima through shared
-// memory, write P (bf16) to shared memory, rescale O in TMEM when the row max
-// moved, and at the item's end write the row: a partial (m, l, acc) at piece
-// c, or the final bf16 row when the units have one chunk (prefill).
+// Roles (320 threads): warps 0-7 softmax, one thread per query row (warp w:
+// half w / 4, TMEM lanes 32 (w mod 4) .. +31), warp 8 TMA producer, warp 9
+// MMA issue (one thread).  Per item, the producer loads the tile's Q rows with
+// one 3-D TMA box per half and 64-column slab (tokens x heads x columns, the
+// 128-byte swizzle), then 64-key steps of K and V (4 blocks, 64 x 16 boxes)
+// into a 3-stage ring.  The MMA thread issues S of step j + 1 (both halves)
+// before P V of step j (two S buffers per half in TMEM), so the tensor cores
+// run while the softmax works, also across item boundaries.  A softmax thread
+// reads its row of S straight from TMEM, takes the running max with the scale
+// folded into one multiply-add per key (a step that is wholly visible needs
+// no masking), writes P (bf16) to shared memory, rescales its O row in TMEM
+// when the max moved, and at the item's end writes the row: a partial (m, l,
+// acc) at piece c, or the final bf16 row when the units have one chunk
+// (prefill), staged through shared memory so that every store writes whole
+// 128-byte lines.
 // All step counters run on across items, so every mbarrier's phase follows
 // from a per-CTA global step or item count.  Every wait is bounded; a role
 // that gives up flags PA_DEVERR_TIMEOUT and stops issuing, the other roles'
@@ -60,6 +65,7 @@ namespace pa {
 constexpr int kTileModePrefix = 0;
 constexpr int kTileModePrefill = 1;
 constexpr int kTileStepBlocks = 4;  // 64 keys per step
+constexpr int kTileHalves = 2;      // accumulator sets of 128 rows per tile
 
 struct TileParams {
     const int32_t* block_tables;  // [num_seqs][max_blocks_per_seq]
@@ -79,7 +85,7 @@ struct TileParams {
     int32_t num_q_heads;
     int32_t num_kv_heads;
     int32_t group;           // query heads per kv head
-    int32_t tile_tokens;     // tokens (prefill) or sequences (prefix) per tile: floor(128 / group)
+    int32_t half_tokens;     // tokens (prefill) or sequences (prefix) per 128-row half: floor(128 / group)
     int32_t max_blocks_per_seq;
     int32_t num_blocks;
     int32_t chunk_blocks;    // key blocks per item (a multiple of 4)
@@ -94,31 +100,33 @@ struct TileParams {
 
 template <int D>
 struct TileCfg {
-    static constexpr int kTileRows = 128;      // TMEM lanes
+    static constexpr int kHalfRows = 128;      // TMEM lanes: rows of one half
     static constexpr int kKeys = 64;           // keys per step
     static constexpr int kStepBlocks = kKeys / kBlockTokens;
     static_assert(kStepBlocks == kTileStepBlocks, "steps of 64 keys");
     static constexpr int kSlabs = D / 64;      // 64-column slabs (128-byte rows)
-    static constexpr int kQBytes = kSlabs * kTileRows * 128;
+    static constexpr int kQHalfBytes = kSlabs * kHalfRows * 128;
+    static constexpr int kQBytes = kTileHalves * kQHalfBytes;
     static constexpr int kKVSlab = kKeys * 128;               // one slab of K (or V) for a step
     static constexpr int kStageBytes = 2 * kSlabs * kKVSlab;  // K slabs, then V slabs
-    static constexpr int kStages = 4;
-    static constexpr int kPBytes = kTileRows * 128;            // P: 64 bf16 keys per row
-    static constexpr int kSoftmaxWarps = 8;
-    static constexpr int kProducerWarp = 8, kMmaWarp = 9;
-    static constexpr int kThreads = 10 * 32;
+    static constexpr int kStages = 3;
+    static constexpr int kPHalfBytes = kHalfRows * 128;       // P: 64 bf16 keys per row
+    static constexpr int kPBytes = kTileHalves * kPHalfBytes;
+    static constexpr int kSoftmaxWarps = 4 * kTileHalves;
+    static constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
+    static constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
     static constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
-    static constexpr uint32_t kTmemCols = 256;  // S0 | S1 | O
+    static constexpr uint32_t kHalfCols = 256;  // per half: S0 | S1 | O
+    static constexpr uint32_t kTmemCols = kTileHalves * kHalfCols;
     static constexpr uint32_t kColS = 0, kColO = 2 * kKeys;
-    // full, empty per stage; s_full x2, p_full, o_done, o_free, q_full x2, q_empty x2, drain
-    static constexpr int kBars = 2 * kStages + 10;
-    // halves of a row exchange: [2 step parities][2 halves][128] maxima, [2 halves][128] sums
-    static constexpr int kXBytes = 3 * 2 * kTileRows * 4;
+    // full, empty per stage; s_full x2, p_full, o_done, o_free, q_full, q_empty, drain
+    static constexpr int kBars = 2 * kStages + 8;
     static constexpr int kMaxUnits = 2048;  // units whose item prefix one CTA holds
     static constexpr int kPrefixBytes = (4 * (kMaxUnits + 1) + 15) / 16 * 16;
-    static constexpr size_t kSmem = 1024 + 2 * kQBytes + kStages * kStageBytes + kPBytes + kXBytes +
-                                    kPrefixBytes + 8 * kBars + 16 + 4 * kStages;
-    static_assert(kColO + D <= kTmemCols, "TMEM columns");
+    static constexpr size_t kSmem = 1024 + kQBytes + kStages * kStageBytes + kPBytes + kPrefixBytes +
+                                    8 * kBars + 16 + 4 * kStages;
+    static_assert(kColO + D <= kHalfCols, "TMEM columns");
+    static_assert(kTmemCols <= 512, "TMEM columns");
     static_assert(kSmem <= 227u * 1024u, "shared memory per CTA");
 };
 
@@ -163,7 +171,8 @@ __device__ __forceinline__ TileUnit tile_unit(const TileParams& P, int32_t u) {
         U.len = L;
         U.kblocks = (L + kBlockTokens - 1) / kBlockTokens;
     }
-    U.tiles = (U.n + P.tile_tokens - 1) / P.tile_tokens;
+    const int32_t tile_tokens = kTileHalves * P.half_tokens;
+    U.tiles = (U.n + tile_tokens - 1) / tile_tokens;
     U.chunks = (U.n == 0 || U.kblocks == 0) ? 0 : (U.kblocks + P.chunk_blocks - 1) / P.chunk_blocks;
     return U;
 }
@@ -171,7 +180,7 @@ __device__ __forceinline__ TileUnit tile_unit(const TileParams& P, int32_t u) {
 struct TileItem {
     TileUnit U;
     int32_t u, t, c, h;
-    int32_t tok0, ntok;  // tokens of the tile
+    int32_t tok0, ntok;  // tokens of the tile (both halves)
     int32_t kb0, kb1;    // key blocks [kb0, kb1) of the item
     int32_t nsteps;      // 0: empty item
 };
@@ -188,8 +197,9 @@ __device__ __forceinline__ TileItem tile_item(const TileParams& P, const int32_t
     const int32_t r = j - I.c * th;
     I.h = r / I.U.tiles;
     I.t = r - I.h * I.U.tiles;
-    I.tok0 = I.t * P.tile_tokens;
-    I.ntok = min(P.tile_tokens, I.U.n - I.tok0);
+    const int32_t tile_tokens = kTileHalves * P.half_tokens;
+    I.tok0 = I.t * tile_tokens;
+    I.ntok = min(tile_tokens, I.U.n - I.tok0);
     int32_t kend = I.U.kblocks;
     if (P.mode == kTileModePrefill) {  // blocks up to the tile's last visible key
         const int32_t last = I.U.len - I.U.n + I.tok0 + I.ntok - 1;
@@ -277,8 +287,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                      const __grid_constant__ CUtensorMap tmap_q, const TileParams P) {
     using Cfg = TileCfg<D>;
     constexpr int S = Cfg::kStages;
-    constexpr int kHalfKeys = Cfg::kKeys / 2;  // keys of a step per softmax thread
-    constexpr int kHalfD = D / 2;              // O columns per softmax thread
+    constexpr int K = Cfg::kKeys;
 
     // Launched with programmatic stream serialization: until
     // grid_dependency_wait() the CTA reads only the lengths, q_start, the
@@ -290,30 +299,29 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
-    // layout: Q[2] | ring[S] | P | exchange | unit prefix | barriers | TMEM slot | stage masks
+    // layout: Q[half][slab] | ring[S] | P[half] | unit prefix | barriers | TMEM slot | stage masks
     const uint32_t q_u32 = smem_u32(smem);
-    const uint32_t ring_u32 = q_u32 + 2 * Cfg::kQBytes;
+    const uint32_t ring_u32 = q_u32 + Cfg::kQBytes;
     const uint32_t p_u32 = ring_u32 + S * Cfg::kStageBytes;
-    uint8_t* ring_smem = smem + 2 * Cfg::kQBytes;
+    uint8_t* ring_smem = smem + Cfg::kQBytes;
     uint8_t* p_smem = ring_smem + S * Cfg::kStageBytes;
-    float* xchg = reinterpret_cast<float*>(p_smem + Cfg::kPBytes);
-    int32_t* prefix = reinterpret_cast<int32_t*>(p_smem + Cfg::kPBytes + Cfg::kXBytes);
-    const uint32_t bars_u32 = p_u32 + Cfg::kPBytes + Cfg::kXBytes + Cfg::kPrefixBytes;
-    const uint32_t full_u32 = bars_u32;           // [S]
-    const uint32_t empty_u32 = bars_u32 + 8 * S;  // [S]
+    int32_t* prefix = reinterpret_cast<int32_t*>(p_smem + Cfg::kPBytes);
+    const uint32_t bars_u32 = p_u32 + Cfg::kPBytes + Cfg::kPrefixBytes;
+    const uint32_t full_u32 = bars_u32;            // [S]
+    const uint32_t empty_u32 = bars_u32 + 8 * S;   // [S]
     const uint32_t sfull_u32 = bars_u32 + 16 * S;  // [2]
     const uint32_t pfull_u32 = sfull_u32 + 16;
     const uint32_t odone_u32 = pfull_u32 + 8;
     const uint32_t ofree_u32 = odone_u32 + 8;
-    const uint32_t qfull_u32 = ofree_u32 + 8;     // [2]
-    const uint32_t qempty_u32 = qfull_u32 + 16;   // [2]
-    const uint32_t drain_u32 = qempty_u32 + 16;
+    const uint32_t qfull_u32 = ofree_u32 + 8;
+    const uint32_t qempty_u32 = qfull_u32 + 8;
+    const uint32_t drain_u32 = qempty_u32 + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (drain_u32 + 8 - q_u32));
     uint32_t* stage_present = tmem_slot + 4;  // [S]: blocks of the stage that were loaded
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = P.group;
-    const int tile_rows = P.tile_tokens * g;  // rows the Q box fills
+    const int half_rows = P.half_tokens * g;  // rows a half's Q box fills
     const bool prefill = P.mode == kTileModePrefill;
 
     if (threadIdx.x == 0) {
@@ -327,19 +335,17 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         mbar_init(odone_u32, 1);
         mbar_init(ofree_u32, Cfg::kSoftmaxThreads);
         mbar_init(qfull_u32, 1);
-        mbar_init(qfull_u32 + 8, 1);
         mbar_init(qempty_u32, 1);
-        mbar_init(qempty_u32 + 8, 1);
         mbar_init(drain_u32, 1);
         fence_barrier_init();
     }
-    // the rows past the Q box (128 mod g of them) are never loaded: zero them
-    // in both buffers once, so that their S and P stay finite
-    for (int e = threadIdx.x; e < 2 * Cfg::kSlabs * (Cfg::kTileRows - tile_rows) * 8; e += blockDim.x) {
+    // the rows past the Q boxes (128 mod g of each half) are never loaded:
+    // zero them once, so that their S and P stay finite
+    for (int e = threadIdx.x; e < kTileHalves * Cfg::kSlabs * (Cfg::kHalfRows - half_rows) * 8; e += blockDim.x) {
         const int chunk = e & 7, rest = e >> 3;
-        const int row = tile_rows + rest % (Cfg::kTileRows - tile_rows);
-        const int buf_slab = rest / (Cfg::kTileRows - tile_rows);
-        *reinterpret_cast<uint4*>(smem + buf_slab * Cfg::kTileRows * 128 + row * 128 + chunk * 16) =
+        const int row = half_rows + rest % (Cfg::kHalfRows - half_rows);
+        const int half_slab = rest / (Cfg::kHalfRows - half_rows);
+        *reinterpret_cast<uint4*>(smem + half_slab * Cfg::kHalfRows * 128 + row * 128 + chunk * 16) =
             make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
@@ -361,17 +367,19 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         for (int32_t it = blockIdx.x; it < total && ok; it += gridDim.x) {
             const TileItem I = tile_item(P, prefix, it);
             if (I.nsteps == 0) continue;
-            const uint32_t b = iq & 1u;
-            if (iq >= 2 && !mbar_wait_bounded(qempty_u32 + 8 * b, ((iq >> 1) - 1) & 1u)) {
+            // Q of both halves, once the previous item's S products are done with the buffer
+            if (iq >= 1 && !mbar_wait_bounded(qempty_u32, (iq - 1) & 1u)) {
                 ok = false;
                 break;
             }
             if (lane == 0) {
-                mbar_arrive_expect_tx(qfull_u32 + 8 * b, Cfg::kSlabs * tile_rows * 128);
+                mbar_arrive_expect_tx(qfull_u32, kTileHalves * Cfg::kSlabs * half_rows * 128);
 #pragma unroll
-                for (int sl = 0; sl < Cfg::kSlabs; ++sl)
-                    tma_load_3d(q_u32 + b * Cfg::kQBytes + sl * Cfg::kTileRows * 128, &tmap_q, sl * 64, I.h * g,
-                                I.U.q_base + I.tok0, qfull_u32 + 8 * b, keep);
+                for (int hh = 0; hh < kTileHalves; ++hh)
+#pragma unroll
+                    for (int sl = 0; sl < Cfg::kSlabs; ++sl)
+                        tma_load_3d(q_u32 + hh * Cfg::kQHalfBytes + sl * Cfg::kHalfRows * 128, &tmap_q, sl * 64,
+                                    I.h * g, I.U.q_base + I.tok0 + hh * P.half_tokens, qfull_u32, keep);
             }
             ++iq;
             // table entries of the item's blocks, 32 at a time: lane l holds
@@ -436,20 +444,17 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             }
         }
         if (!ok && lane == 0) flag_error(PA_DEVERR_TIMEOUT);
-        // this warp's last copies into every stage and Q buffer have landed before leaving
+        // this warp's last copies into every stage and into Q have landed before leaving
         for (uint32_t k = 0; k < static_cast<uint32_t>(S) && k < gs; ++k) {
             const uint32_t last = gs - 1 - k;  // one of the last S steps
             mbar_wait_bounded(full_u32 + 8 * (last % S), (last / S) & 1u);
         }
-        for (uint32_t k = 0; k < 2 && k < iq; ++k) {
-            const uint32_t last = iq - 1 - k;
-            mbar_wait_bounded(qfull_u32 + 8 * (last & 1u), (last >> 1) & 1u);
-        }
+        if (iq > 0) mbar_wait_bounded(qfull_u32, (iq - 1) & 1u);
     } else if (warp == Cfg::kMmaWarp) {
         // ---------------- MMA issue (one thread): S of step j + 1, then P V of step j
         if (lane == 0) {
-            constexpr uint32_t kIdescS = umma_idesc_bf16(Cfg::kTileRows, Cfg::kKeys, 0);
-            constexpr uint32_t kIdescO = umma_idesc_bf16(Cfg::kTileRows, D, 1);
+            constexpr uint32_t kIdescS = umma_idesc_bf16(Cfg::kHalfRows, K, 0);
+            constexpr uint32_t kIdescO = umma_idesc_bf16(Cfg::kHalfRows, D, 1);
             // the step sequence of this CTA: (item, step j within it)
             struct Cur {
                 int32_t it;      // item index
@@ -477,24 +482,24 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 return first_step(c.it + gridDim.x, c.iq + 1, c.gs + 1, n);
             };
             auto issue_s = [&](const Cur& c) -> bool {
-                const uint32_t b = c.iq & 1u;
-                if (c.j == 0) {
-                    if (!mbar_wait_bounded_thread(qfull_u32 + 8 * b, (c.iq >> 1) & 1u)) return false;
-                }
+                if (c.j == 0 && !mbar_wait_bounded_thread(qfull_u32, c.iq & 1u)) return false;
                 const int st = c.gs % S;
                 if (!mbar_wait_bounded_thread(full_u32 + 8 * st, (c.gs / S) & 1u)) return false;
                 tc_fence_after();
                 const uint32_t kb = ring_u32 + st * Cfg::kStageBytes;
-                const uint32_t qb = q_u32 + b * Cfg::kQBytes;
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks % 4) * 32u;  // k-step within the 128-byte row
-                    const uint64_t a = umma_desc_sw128(qb + (ks / 4) * Cfg::kTileRows * 128 + off, 16, 1024);
-                    const uint64_t bd = umma_desc_sw128(kb + (ks / 4) * Cfg::kKVSlab + off, 16, 1024);
-                    umma_bf16(tmem + Cfg::kColS + (c.gs & 1u) * Cfg::kKeys, a, bd, kIdescS, ks > 0);
+                for (int hh = 0; hh < kTileHalves; ++hh) {
+                    const uint32_t qb = q_u32 + hh * Cfg::kQHalfBytes;
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t off = (ks % 4) * 32u;  // k-step within the 128-byte row
+                        const uint64_t a = umma_desc_sw128(qb + (ks / 4) * Cfg::kHalfRows * 128 + off, 16, 1024);
+                        const uint64_t bd = umma_desc_sw128(kb + (ks / 4) * Cfg::kKVSlab + off, 16, 1024);
+                        umma_bf16(tmem + hh * Cfg::kHalfCols + Cfg::kColS + (c.gs & 1u) * K, a, bd, kIdescS, ks > 0);
+                    }
                 }
                 umma_commit(sfull_u32 + 8 * (c.gs & 1u));
-                if (c.j + 1 == c.nsteps) umma_commit(qempty_u32 + 8 * b);  // the item's last read of Q
+                if (c.j + 1 == c.nsteps) umma_commit(qempty_u32);  // the item's last read of Q
                 return true;
             };
             bool ok = true;
@@ -507,17 +512,19 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 if (more && !(ok = issue_s(nxt))) break;
                 // P V of the current step; the first step of an item overwrites O,
                 // which the softmax must have read out for the previous item
-                if (cur.j == 0 && cur.iq > 0 &&
-                    !(ok = mbar_wait_bounded_thread(ofree_u32, (cur.iq - 1) & 1u)))
+                if (cur.j == 0 && cur.iq > 0 && !(ok = mbar_wait_bounded_thread(ofree_u32, (cur.iq - 1) & 1u)))
                     break;
                 if (!(ok = mbar_wait_bounded_thread(pfull_u32, cur.gs & 1u))) break;
                 tc_fence_after();
                 const uint32_t vb = ring_u32 + (cur.gs % S) * Cfg::kStageBytes + Cfg::kSlabs * Cfg::kKVSlab;
 #pragma unroll
-                for (int ks = 0; ks < Cfg::kKeys / 16; ++ks) {
-                    const uint64_t a = umma_desc_sw128(p_u32 + ks * 32u, 16, 1024);
-                    const uint64_t bd = umma_desc_sw128(vb + ks * 16 * 128, Cfg::kKVSlab, 1024);
-                    umma_bf16(tmem + Cfg::kColO, a, bd, kIdescO, cur.j > 0 || ks > 0);
+                for (int hh = 0; hh < kTileHalves; ++hh) {
+#pragma unroll
+                    for (int ks = 0; ks < K / 16; ++ks) {
+                        const uint64_t a = umma_desc_sw128(p_u32 + hh * Cfg::kPHalfBytes + ks * 32u, 16, 1024);
+                        const uint64_t bd = umma_desc_sw128(vb + ks * 16 * 128, Cfg::kKVSlab, 1024);
+                        umma_bf16(tmem + hh * Cfg::kHalfCols + Cfg::kColO, a, bd, kIdescO, cur.j > 0 || ks > 0);
+                    }
                 }
                 umma_commit(odone_u32);
                 umma_commit(empty_u32 + 8 * (cur.gs % S));
@@ -531,96 +538,113 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         }
         __syncwarp();
     } else {
-        // ---------------- softmax: two threads per query row
-        const int row = 32 * (warp & 3) + lane;  // TMEM lane = row of the tile
-        const int hf = (warp >> 2) & 1;          // half of the keys and of O
-        const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp & 3) * 32u) << 16);
+        // ---------------- softmax: one thread per query row
+        const int hh = warp >> 2;                // half of the tile
+        const int row = 32 * (warp & 3) + lane;  // TMEM lane = row of the half
+        const uint32_t lane_base = tmem + hh * Cfg::kHalfCols + ((static_cast<uint32_t>(warp & 3) * 32u) << 16);
+        uint8_t* p_half = p_smem + hh * Cfg::kPHalfBytes;
         const float sl2 = P.scale_log2;
         bool ok = true;  // warp-uniform: a wait that gave up stops TMEM work and arrivals
-        uint32_t iq = 0, gs = 0;
+        uint32_t gs = 0;
         bool waited = false;  // grid_dependency_wait done (before the first output write)
         for (int32_t it = blockIdx.x; it < total; it += gridDim.x) {
             const TileItem I = tile_item(P, prefix, it);
             if (I.nsteps == 0) continue;
-            const int tok = row / g;  // token of the tile (a sequence in prefix mode)
-            const bool row_ok = row < tile_rows && tok < I.ntok;
+            const int tok = hh * P.half_tokens + row / g;  // token of the tile (a sequence in prefix mode)
+            const bool row_ok = row < half_rows && tok < I.ntok;
             const int32_t ktok = I.tok0 + tok;  // token within the unit
             // last key this row sees (prefill: causal; prefix: every prefix key)
             const int32_t lim = !row_ok ? -1 : prefill ? I.U.len - I.U.n + ktok : I.U.len - 1;
             const size_t orow = row_ok ? static_cast<size_t>(I.U.q_base + ktok) * P.num_q_heads + I.h * g + row % g : 0;
-            float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
+            float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of the row
             for (int j = 0; j < I.nsteps; ++j, ++gs) {
                 const int st = gs % S;
                 ok = ok && mbar_wait_bounded(sfull_u32 + 8 * (gs & 1u), (gs >> 1) & 1u);
                 ok = ok && mbar_wait_bounded(full_u32 + 8 * st, (gs / S) & 1u);
                 tc_fence_after();
                 const int32_t key0 = (I.kb0 + j * Cfg::kStepBlocks) * kBlockTokens;  // first key of the step
-                float x[kHalfKeys];
-                float mx = -INFINITY;
+                float x[K];
+                float mu = 0.f, alpha = 1.f;
                 if (ok) {
-                    const uint32_t present = stage_present[st] >> (hf * kHalfKeys / kBlockTokens);
-                    tmem_ld32(lane_base + Cfg::kColS + (gs & 1u) * Cfg::kKeys + hf * kHalfKeys, x);
-                    // keys key0 + 32 hf + i; visible iff their block was loaded and key <= lim
-                    const int32_t vis = lim - key0 - hf * kHalfKeys;  // last visible i
-                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    tmem_ld32(lane_base + Cfg::kColS + (gs & 1u) * K, *reinterpret_cast<float(*)[32]>(x));
+                    tmem_ld32(lane_base + Cfg::kColS + (gs & 1u) * K + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+                    const uint32_t present = stage_present[st];
+                    float mx;
+                    // a wholly visible step (every block loaded, every key within
+                    // the row's limit) with a positive scale takes the plain max of
+                    // the raw scores; otherwise mask and scale first
+                    const bool plain = present == 0xFu && key0 + K - 1 <= lim && sl2 > 0.f;
+                    if (plain) {
+                        float m4[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-                    for (int i = 0; i < kHalfKeys; ++i) {
-                        x[i] = (((present >> (i / kBlockTokens)) & 1u) && i <= vis) ? x[i] * sl2 : -INFINITY;
-                        m4[i & 3] = fmaxf(m4[i & 3], x[i]);
+                        for (int i = 4; i < K; ++i) m4[i & 3] = fmaxf(m4[i & 3], x[i]);
+                        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+                    } else {
+                        const int32_t vis = lim - key0;  // last visible key of the step
+                        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                        for (int i = 0; i < K; ++i) {
+                            x[i] = (((present >> (i / kBlockTokens)) & 1u) && i <= vis) ? x[i] * sl2 : -INFINITY;
+                            m4[i & 3] = fmaxf(m4[i & 3], x[i]);
+                        }
+                        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                     }
-                    mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-                } else {
+                    const float mn = fmaxf(m, mx);
+                    mu = mn == -INFINITY ? 0.0f : mn;
+                    alpha = fast_exp2(m - mu);
+                    m = mn;
+                    // P = 2^(s - mu) as bf16, the row sum in fp32
+                    uint32_t pw[K / 2];
+                    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (plain) {
 #pragma unroll
-                    for (int i = 0; i < kHalfKeys; ++i) x[i] = -INFINITY;
-                }
-                // the row max over both halves
-                float* xs = xchg + (gs & 1u) * 2 * Cfg::kTileRows;
-                xs[hf * Cfg::kTileRows + row] = mx;
-                softmax_bar_sync(1, Cfg::kSoftmaxThreads);
-                mx = fmaxf(mx, xs[(1 - hf) * Cfg::kTileRows + row]);
-                const float mn = fmaxf(m, mx);
-                const float mu = mn == -INFINITY ? 0.0f : mn;
-                const float alpha = fast_exp2(m - mu);
-                m = mn;
-                uint32_t pw[kHalfKeys / 2];
-                float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                        for (int i = 0; i < K / 2; ++i) {
+                            const float p0 = fast_exp2(fmaf(x[2 * i], sl2, -mu));
+                            const float p1 = fast_exp2(fmaf(x[2 * i + 1], sl2, -mu));
+                            s4[i & 3] += p0 + p1;
+                            pw[i] = pack2<false>(p0, p1);
+                        }
+                    } else {
 #pragma unroll
-                for (int i = 0; i < kHalfKeys / 2; ++i) {
-                    pw[i] = pack2<false>(fast_exp2(x[2 * i] - mu), fast_exp2(x[2 * i + 1] - mu));
-                    s4[i & 3] += __uint_as_float(pw[i] << 16) + __uint_as_float(pw[i] & 0xffff0000u);
-                }
-                l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-                if (j > 0) {
-                    // P V of the previous step is done: the P buffer is free, O holds the sum up to it
-                    ok = ok && mbar_wait_bounded(odone_u32, (gs - 1) & 1u);
-                    tc_fence_after();
-                    if (ok && __any_sync(kFullMask, alpha != 1.f)) {
-#pragma unroll
-                        for (int c = 0; c < kHalfD / 32; ++c) {
-                            float v[32];
-                            tmem_ld32(lane_base + Cfg::kColO + hf * kHalfD + 32 * c, v);
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                            tmem_st32(lane_base + Cfg::kColO + hf * kHalfD + 32 * c, v);
+                        for (int i = 0; i < K / 2; ++i) {
+                            const float p0 = fast_exp2(x[2 * i] - mu);
+                            const float p1 = fast_exp2(x[2 * i + 1] - mu);
+                            s4[i & 3] += p0 + p1;
+                            pw[i] = pack2<false>(p0, p1);
                         }
                     }
+                    l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+                    if (j > 0) {
+                        // P V of the previous step is done: the P buffer is free, O holds the sum up to it
+                        ok = mbar_wait_bounded(odone_u32, (gs - 1) & 1u);
+                        tc_fence_after();
+                    }
+                    if (ok) {
+                        if (j > 0 && __any_sync(kFullMask, alpha != 1.f)) {
+#pragma unroll
+                            for (int c = 0; c < D / 32; ++c) {
+                                float v[32];
+                                tmem_ld32(lane_base + Cfg::kColO + 32 * c, v);
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                                tmem_st32(lane_base + Cfg::kColO + 32 * c, v);
+                            }
+                        }
+                        // the row's 64 keys: its 128-byte P row, K-major, 128-byte swizzle
+#pragma unroll
+                        for (int c = 0; c < K / 8; ++c)
+                            *reinterpret_cast<uint4*>(p_half + row * 128 + ((c ^ (row & 7)) << 4)) =
+                                make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+                    }
                 }
                 if (ok) {
-                    // keys 32 hf .. 32 hf + 31 of the row: 16-byte chunks 4 hf .. 4 hf + 3
-                    // of its 128-byte P row, K-major, 128-byte swizzle
-#pragma unroll
-                    for (int c = 0; c < kHalfKeys / 8; ++c) {
-                        const int cc = hf * (kHalfKeys / 8) + c;
-                        *reinterpret_cast<uint4*>(p_smem + row * 128 + ((cc ^ (row & 7)) << 4)) =
-                            make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-                    }
                     // key slots at or past the sequence's length hold stale data
                     // (weight 0, but 0 * NaN is NaN): zero their V rows in the stage
                     const int32_t zero_from = I.U.len - key0;
-                    if (zero_from < Cfg::kKeys) {
-                        const int zrows = Cfg::kKeys - max(0, zero_from);
+                    if (zero_from < K) {
+                        const int zrows = K - max(0, zero_from);
                         for (int e = threadIdx.x; e < zrows * Cfg::kSlabs * 8; e += Cfg::kSoftmaxThreads) {
-                            const int zr = Cfg::kKeys - zrows + e / (Cfg::kSlabs * 8);
+                            const int zr = K - zrows + e / (Cfg::kSlabs * 8);
                             const int sl = (e / 8) % Cfg::kSlabs;
                             *reinterpret_cast<uint4*>(ring_smem + st * Cfg::kStageBytes + (Cfg::kSlabs + sl) * Cfg::kKVSlab +
                                                       zr * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
@@ -631,63 +655,72 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                     mbar_arrive(pfull_u32);
                 }
             }
-            // ---- the item's rows
+            // ---- the item's rows (the P buffers are free once the last P V is done,
+            // and serve as staging: each warp's 32 rows, 128 bytes of each at a time)
             if (!waited) {
                 grid_dependency_wait();  // before the first write of out or the workspace
                 waited = true;
             }
-            xchg[4 * Cfg::kTileRows + hf * Cfg::kTileRows + row] = l;
-            softmax_bar_sync(1, Cfg::kSoftmaxThreads);
-            l += xchg[4 * Cfg::kTileRows + (1 - hf) * Cfg::kTileRows + row];
             ok = ok && mbar_wait_bounded(odone_u32, (gs - 1) & 1u);  // the item's last P V
             tc_fence_after();
             if (ok) {
                 constexpr float kLn2 = 0.693147180559945309f;
-                if (P.direct) {
-                    const float inv = l > 0.f ? 1.0f / l : 0.f;
-                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(P.out) + orow * D + hf * kHalfD;
-#pragma unroll
-                    for (int c = 0; c < kHalfD / 32; ++c) {
-                        float v[32];
-                        tmem_ld32(lane_base + Cfg::kColO + hf * kHalfD + 32 * c, v);
-                        if (row_ok) {
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                uint4 u;
-                                u.x = pack2<false>(v[8 * i] * inv, v[8 * i + 1] * inv);
-                                u.y = pack2<false>(v[8 * i + 2] * inv, v[8 * i + 3] * inv);
-                                u.z = pack2<false>(v[8 * i + 4] * inv, v[8 * i + 5] * inv);
-                                u.w = pack2<false>(v[8 * i + 6] * inv, v[8 * i + 7] * inv);
-                                *reinterpret_cast<uint4*>(o + 32 * c + 8 * i) = u;
-                            }
-                        }
-                    }
-                } else {
+                uint8_t* stage = p_smem + warp * 32 * 128;  // this warp's 4 KB
+                const bool direct = P.direct != 0;
+                const float inv = direct ? (l > 0.f ? 1.0f / l : 0.f) : 1.f;
+                if (!direct && row_ok) {
                     const size_t idx = orow * P.max_parts + I.c;
-                    if (row_ok && hf == 0) {
-                        P.ws_m[idx] = m * kLn2;
-                        P.ws_l[idx] = l;
-                    }
-                    float* a = P.ws_acc + idx * D + hf * kHalfD;
+                    P.ws_m[idx] = m * kLn2;
+                    P.ws_l[idx] = l;
+                }
+                // 128 bytes of a row per round: 32 fp32 (partial) or 64 bf16 (final)
+                constexpr int kRounds = D / 32;
+                for (int rd = 0; rd < (direct ? kRounds / 2 : kRounds); ++rd) {
+                    uint32_t w[32];
+                    if (direct) {
+                        float v[32], u[32];
+                        tmem_ld32(lane_base + Cfg::kColO + 64 * rd, v);
+                        tmem_ld32(lane_base + Cfg::kColO + 64 * rd + 32, u);
 #pragma unroll
-                    for (int c = 0; c < kHalfD / 32; ++c) {
+                        for (int i = 0; i < 16; ++i) {
+                            w[i] = pack2<false>(v[2 * i] * inv, v[2 * i + 1] * inv);
+                            w[16 + i] = pack2<false>(u[2 * i] * inv, u[2 * i + 1] * inv);
+                        }
+                    } else {
                         float v[32];
-                        tmem_ld32(lane_base + Cfg::kColO + hf * kHalfD + 32 * c, v);
-                        if (row_ok) {
+                        tmem_ld32(lane_base + Cfg::kColO + 32 * rd, v);
 #pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                *reinterpret_cast<float4*>(a + 32 * c + 4 * i) =
-                                    make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                        for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
+                    }
+                    // lane's 128 bytes -> its staging row, 16-byte chunk c at c ^ (lane mod 8)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4*>(stage + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                    __syncwarp();
+                    // 4 rows per store: lanes 8 r' .. 8 r' + 7 write row 4 k + r' (128 contiguous bytes)
+                    for (int k = 0; k < 8; ++k) {
+                        const int rr = 4 * k + (lane >> 3), c = lane & 7;
+                        const unsigned long long dst_row =
+                            __shfl_sync(kFullMask, static_cast<unsigned long long>(orow), rr);
+                        const bool rok = __shfl_sync(kFullMask, row_ok ? 1 : 0, rr) != 0;
+                        const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((c ^ (rr & 7)) << 4));
+                        if (rok) {
+                            if (direct)
+                                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.out) + dst_row * D + 64 * rd +
+                                                          8 * c) = val;
+                            else
+                                *reinterpret_cast<uint4*>(P.ws_acc + (dst_row * P.max_parts + I.c) * D + 32 * rd +
+                                                          4 * c) = val;
                         }
                     }
+                    __syncwarp();
                 }
                 tc_fence_before();
                 mbar_arrive(ofree_u32);  // O may be overwritten by the next item
             }
-            ++iq;
         }
         if (!ok && lane == 0) flag_error(PA_DEVERR_TIMEOUT);
-        (void)iq;
     }
 
     if (P.mode == kTileModePrefix && warp >= Cfg::kProducerWarp) check_group_tables(P, check_me, check_n);

@@ -114,7 +114,7 @@ def test_multi_query_workspace_and_limits(lib):
     P = -(-(-(-L // 16)) // 16) + 1  # balanced bound of the warp-level path
     # the tile path (group x query tokens > 16) keeps one partial per key chunk
     sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 1 << 30
-    tiles = -(-T // (128 // (Hq // Hkv))) + N
+    tiles = -(-T // (2 * (128 // (Hq // Hkv)))) + N  # tiles of two 128-row halves
     C = _tile_splits(sms, tiles * Hkv, -(-L // 16))
     want = max(layout(P), layout(C) if C > 1 else 0)
     assert lib.pa_decode_multi_workspace_size(N, T, Hq, Hkv, D, L, 16, 0) == want
