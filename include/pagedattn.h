@@ -193,7 +193,9 @@ PA_API int pa_decode_multi(const void* q, const int32_t* q_start, int32_t num_q_
 /* Workspace bytes pa_decode_multi needs: the pa_decode layout with
  * num_q_rows * num_q_heads rows and as many pieces per row as either path can
  * write (the tile path's key chunks depend on the current device's SM count:
- * query the size on the device that runs the call). */
+ * query the size on the device that runs the call), and for the tile path 256
+ * bytes at the end for its work counter (zeroed by every call), so the size is
+ * never 0. */
 PA_API size_t pa_decode_multi_workspace_size(int32_t num_seqs, int32_t num_q_rows,
                                              int32_t num_q_heads, int32_t num_kv_heads,
                                              int32_t head_dim, int32_t max_seq_len,
@@ -336,10 +338,12 @@ PA_API int pa_decode_shared_prefix(const void* q, const void* k_cache, const voi
 
 /*
  * Workspace bytes pa_decode_shared_prefix needs.  Layout as for pa_decode, with
- * P = min(16, shared_blocks) slots for the prefix's key splits + the pieces the
- * private part of a sequence can have; pieces 0 .. splits-1 of every row hold
- * the shared prefix's partials (the split count, at most 16, is chosen at
- * launch to fill one wave of the device) and the private pieces follow.
+ * P = min(16, shared_blocks) slots for the prefix's key chunks + the pieces the
+ * private part of a sequence can have; pieces 0 .. chunks-1 of every row hold
+ * the shared prefix's partials (the chunk count, at most 16, is chosen at
+ * launch to fill the device) and the private pieces follow.  256 more bytes at
+ * the end hold the tile kernel's work counter, which every call sets to zero
+ * on its stream before the kernel runs.
  */
 PA_API size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                                      int32_t num_kv_heads, int32_t head_dim,
@@ -388,7 +392,9 @@ PA_API int pa_decode_shared_prefix_groups(const void* q, const void* k_cache, co
 /*
  * Workspace bytes pa_decode_shared_prefix_groups needs: the pa_decode layout
  * with P = min(16, max_shared_blocks) slots for the prefix chunks + the pieces
- * a whole sequence of max_seq_len tokens can have (a group may share nothing).
+ * a whole sequence of max_seq_len tokens can have (a group may share nothing),
+ * and 256 bytes at the end for the tile kernel's work counter (zeroed by every
+ * call).
  */
 PA_API size_t pa_decode_shared_prefix_groups_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                                             int32_t num_kv_heads, int32_t head_dim,

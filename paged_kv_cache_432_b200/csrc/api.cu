@@ -285,21 +285,29 @@ Plan make_group_plan(int32_t max_seq_len, int32_t partition_blocks, int32_t max_
 }
 
 struct WsLayout {
-    size_t off_m, off_l, off_acc, off_parts, bytes;
+    size_t off_m, off_l, off_acc, off_parts, off_ctr, bytes;
 };
 
+constexpr size_t kCounterBytes = 256;  // the tile kernel's item counter (zeroed by each call)
+
 // q_rows: query-token rows (num_seqs with one query token per sequence).
+// counter: the tile kernel runs in the call and needs its item counter (last).
 WsLayout ws_layout(int64_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_parts,
-                   int32_t head_dim, bool split, int64_t q_rows = -1) {
-    WsLayout w{0, 0, 0, 0, 0};
-    if (!split) return w;
-    const int64_t rows = (q_rows >= 0 ? q_rows : num_seqs) * num_q_heads;
-    const size_t ml = align256(static_cast<size_t>(rows) * max_parts * sizeof(float));
-    w.off_m = 0;
-    w.off_l = ml;
-    w.off_acc = 2 * ml;
-    w.off_parts = w.off_acc + align256(static_cast<size_t>(rows) * max_parts * head_dim * sizeof(float));
-    w.bytes = w.off_parts + align256(static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int32_t));
+                   int32_t head_dim, bool split, int64_t q_rows = -1, bool counter = false) {
+    WsLayout w{0, 0, 0, 0, 0, 0};
+    if (split) {
+        const int64_t rows = (q_rows >= 0 ? q_rows : num_seqs) * num_q_heads;
+        const size_t ml = align256(static_cast<size_t>(rows) * max_parts * sizeof(float));
+        w.off_m = 0;
+        w.off_l = ml;
+        w.off_acc = 2 * ml;
+        w.off_parts = w.off_acc + align256(static_cast<size_t>(rows) * max_parts * head_dim * sizeof(float));
+        w.bytes = w.off_parts + align256(static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int32_t));
+    }
+    if (counter) {
+        w.off_ctr = w.bytes;
+        w.bytes += kCounterBytes;
+    }
     return w;
 }
 
@@ -381,7 +389,7 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
     }
     const int64_t q_rows = a.q_start ? a.num_q_rows : a.num_seqs;
     const WsLayout ws = ws_layout(a.num_seqs, a.num_q_heads, a.num_kv_heads, plan->max_parts,
-                                  a.head_dim, plan->split, q_rows);
+                                  a.head_dim, plan->split, q_rows, shared_blocks > 0);
     std::memset(P, 0, sizeof *P);
     if (plan->split) {
         if (!a.workspace || !aligned(a.workspace, 256)) return PA_ERR_WORKSPACE;
@@ -391,6 +399,7 @@ int prepare_decode(const DecodeArgs& a, bool need_inputs, DecodeParams* P, Plan*
         P->ws_l = reinterpret_cast<float*>(w + ws.off_l);
         P->ws_acc = reinterpret_cast<float*>(w + ws.off_acc);
         P->ws_parts = reinterpret_cast<int32_t*>(w + ws.off_parts);
+        if (shared_blocks > 0) P->tile_counter = reinterpret_cast<int32_t*>(w + ws.off_ctr);
     }
     P->q = a.q;
     P->q_start = a.q_start;
@@ -633,7 +642,15 @@ int launch_tiles(const TileParams& base, const void* q, int64_t q_rows, const vo
         P.num_units = units - b < TileCfg<D>::kMaxUnits ? units - b : TileCfg<D>::kMaxUnits;
         int64_t grid = items_bound < di.sms ? items_bound : di.sms;
         if (grid < 1) grid = 1;
-        cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(TileCfg<D>::kThreads),
+        cudaError_t e;
+        if (items_bound > grid) {
+            // more items than CTAs: they are claimed from a counter, which starts at zero
+            e = cudaMemsetAsync(P.item_counter, 0, sizeof(int32_t), st);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (tile item counter)");
+        } else {
+            P.item_counter = nullptr;  // at most one item per CTA: no counter
+        }
+        e = launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(TileCfg<D>::kThreads),
                                    TileCfg<D>::kSmem, st, mk, mv, mq, P);
         if (e != cudaSuccess) return cuda_fail(e, "attn_tiles_tc_kernel launch");
     }
@@ -658,6 +675,7 @@ int launch_prefix_tiles(const DecodeParams& P, Plan* plan, cudaStream_t st) {
     T.ws_m = P.ws_m;
     T.ws_l = P.ws_l;
     T.ws_acc = P.ws_acc;
+    T.item_counter = P.tile_counter;
     T.mode = kTileModePrefix;
     T.unit_begin = 0;
     T.num_units = P.group_start ? P.num_groups : 1;
@@ -750,7 +768,7 @@ PrefillPlan make_prefill_plan(int sms, int32_t num_seqs, int32_t num_q_rows, int
     pp.tiles_bound = (static_cast<int64_t>(num_q_rows) + tt - 1) / tt + num_seqs;
     pp.split = choose_tile_split(sms, pp.tiles_bound * num_kv_heads, (max_len + kBlockTokens - 1) / kBlockTokens);
     pp.ws = ws_layout(num_seqs, num_q_heads, num_kv_heads, pp.split.splits, head_dim, pp.split.splits > 1,
-                      num_q_rows);
+                      num_q_rows, true);
     return pp;
 }
 
@@ -779,9 +797,9 @@ int run_prefill_tiles(const DecodeArgs& a) {
     float* ws_m = nullptr;
     float* ws_l = nullptr;
     float* ws_acc = nullptr;
+    if (!a.workspace || !aligned(a.workspace, 256) || a.workspace_bytes < pp.ws.bytes) return PA_ERR_WORKSPACE;
+    char* w = static_cast<char*>(a.workspace);
     if (!direct) {
-        if (!a.workspace || !aligned(a.workspace, 256) || a.workspace_bytes < pp.ws.bytes) return PA_ERR_WORKSPACE;
-        char* w = static_cast<char*>(a.workspace);
         ws_m = reinterpret_cast<float*>(w + pp.ws.off_m);
         ws_l = reinterpret_cast<float*>(w + pp.ws.off_l);
         ws_acc = reinterpret_cast<float*>(w + pp.ws.off_acc);
@@ -795,6 +813,7 @@ int run_prefill_tiles(const DecodeArgs& a) {
     T.ws_m = ws_m;
     T.ws_l = ws_l;
     T.ws_acc = ws_acc;
+    T.item_counter = reinterpret_cast<int32_t*>(w + pp.ws.off_ctr);
     T.mode = kTileModePrefill;
     T.unit_begin = 0;
     T.num_units = a.num_seqs;
@@ -1183,7 +1202,7 @@ size_t pa_decode_shared_prefix_groups_workspace_size(int32_t num_seqs, int32_t n
         return 0;
     const Plan plan = make_group_plan(max_seq_len, partition_blocks, max_shared_blocks, num_groups, num_seqs,
                                       num_q_heads, num_kv_heads);
-    return ws_layout(num_seqs, num_q_heads, num_kv_heads, plan.max_parts, head_dim, plan.split).bytes;
+    return ws_layout(num_seqs, num_q_heads, num_kv_heads, plan.max_parts, head_dim, plan.split, -1, true).bytes;
 }
 
 int pa_decode_multi(const void* q, const int32_t* q_start, int32_t num_q_rows, int32_t max_q_len,
@@ -1248,7 +1267,7 @@ size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_he
         return 0;
     const Plan plan = make_prefix_plan(max_seq_len, partition_blocks, shared_blocks, num_seqs,
                                        num_q_heads, num_kv_heads);
-    return ws_layout(num_seqs, num_q_heads, num_kv_heads, plan.max_parts, head_dim, plan.split).bytes;
+    return ws_layout(num_seqs, num_q_heads, num_kv_heads, plan.max_parts, head_dim, plan.split, -1, true).bytes;
 }
 
 int pa_get_device_error(uint32_t* bits, int32_t clear, void* stream) {

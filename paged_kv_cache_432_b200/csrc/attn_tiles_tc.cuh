@@ -31,10 +31,13 @@
 // chunks of chunk_blocks blocks (one chunk when the device is full without a
 // split).  An item is (chunk c, kv head h, tile t), numbered with t fastest,
 // so that the tiles reading the same keys run side by side and share them in
-// L2.  The grid is persistent, one CTA per SM: CTA b takes items b, b + grid,
-// ...; each CTA builds the per-unit item prefix once in shared memory and finds
-// any item by binary search.  An item whose chunk lies wholly past its tile's
-// last visible key is empty: every role skips it.
+// L2.  The grid is persistent, one CTA per SM: CTA b starts with item b and
+// then takes the next unclaimed item from a counter in global memory (one
+// atomic add per item, so the CTAs finish together whatever the length mix);
+// the producer warp claims items and passes them to the other roles through a
+// small queue in shared memory.  Each CTA builds the per-unit item prefix once
+// in shared memory and finds any item by binary search.  An item whose chunk
+// lies wholly past its tile's last visible key is empty and is skipped.
 //
 // Roles (320 threads): warps 0-7 softmax, one thread per query row (warp w:
 // half w / 4, TMEM lanes 32 (w mod 4) .. +31), warp 8 TMA producer, warp 9
@@ -66,6 +69,7 @@ constexpr int kTileModePrefix = 0;
 constexpr int kTileModePrefill = 1;
 constexpr int kTileStepBlocks = 4;  // 64 keys per step
 constexpr int kTileHalves = 2;      // accumulator sets of 128 rows per tile
+constexpr float kLazyRescale = 8.f;  // log2 units: the reference max lags the true max by at most this
 
 struct TileParams {
     const int32_t* block_tables;  // [num_seqs][max_blocks_per_seq]
@@ -78,6 +82,8 @@ struct TileParams {
     float* ws_m;                  // partials (layout of the decode workspace)
     float* ws_l;
     float* ws_acc;
+    int32_t* item_counter;        // items handed out after each CTA's first (zero at launch);
+                                  //   null: CTA b takes items b, b + grid, b + 2 grid, ...
     int32_t mode;            // kTileModePrefix or kTileModePrefill
     int32_t unit_begin;      // first unit of this launch
     int32_t num_units;       // units of this launch
@@ -109,7 +115,7 @@ struct TileCfg {
     static constexpr int kQBytes = kTileHalves * kQHalfBytes;
     static constexpr int kKVSlab = kKeys * 128;               // one slab of K (or V) for a step
     static constexpr int kStageBytes = 2 * kSlabs * kKVSlab;  // K slabs, then V slabs
-    static constexpr int kStages = 3;
+    static constexpr int kStages = 4;
     static constexpr int kPHalfBytes = kHalfRows * 128;       // P: 64 bf16 keys per row
     static constexpr int kPBytes = kTileHalves * kPHalfBytes;
     static constexpr int kSoftmaxWarps = 4 * kTileHalves;
@@ -119,12 +125,14 @@ struct TileCfg {
     static constexpr uint32_t kHalfCols = 256;  // per half: S0 | S1 | O
     static constexpr uint32_t kTmemCols = kTileHalves * kHalfCols;
     static constexpr uint32_t kColS = 0, kColO = 2 * kKeys;
-    // full, empty per stage; s_full x2, p_full, o_done, o_free, q_full, q_empty, drain
-    static constexpr int kBars = 2 * kStages + 8;
-    static constexpr int kMaxUnits = 2048;  // units whose item prefix one CTA holds
+    // full, empty per stage; s_full x2, p_full, o_done, o_free, q_full, q_empty, drain;
+    // item queue full / empty x kItemSlots
+    static constexpr int kItemSlots = 4;
+    static constexpr int kBars = 2 * kStages + 8 + 2 * kItemSlots;
+    static constexpr int kMaxUnits = 256;  // units whose item prefix one CTA holds (more: several launches)
     static constexpr int kPrefixBytes = (4 * (kMaxUnits + 1) + 15) / 16 * 16;
     static constexpr size_t kSmem = 1024 + kQBytes + kStages * kStageBytes + kPBytes + kPrefixBytes +
-                                    8 * kBars + 16 + 4 * kStages;
+                                    8 * kBars + 16 + 4 * kStages + 4 * kItemSlots;
     static_assert(kColO + D <= kHalfCols, "TMEM columns");
     static_assert(kTmemCols <= 512, "TMEM columns");
     static_assert(kSmem <= 227u * 1024u, "shared memory per CTA");
@@ -316,8 +324,11 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     const uint32_t qfull_u32 = ofree_u32 + 8;
     const uint32_t qempty_u32 = qfull_u32 + 8;
     const uint32_t drain_u32 = qempty_u32 + 8;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (drain_u32 + 8 - q_u32));
+    const uint32_t iqfull_u32 = drain_u32 + 8;                        // [kItemSlots]
+    const uint32_t iqempty_u32 = iqfull_u32 + 8 * Cfg::kItemSlots;  // [kItemSlots]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (iqempty_u32 + 8 * Cfg::kItemSlots - q_u32));
     uint32_t* stage_present = tmem_slot + 4;  // [S]: blocks of the stage that were loaded
+    volatile int32_t* item_q = reinterpret_cast<volatile int32_t*>(stage_present + S);  // [kItemSlots]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = P.group;
@@ -337,6 +348,10 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         mbar_init(qfull_u32, 1);
         mbar_init(qempty_u32, 1);
         mbar_init(drain_u32, 1);
+        for (int i = 0; i < Cfg::kItemSlots; ++i) {
+            mbar_init(iqfull_u32 + 8 * i, 1);
+            mbar_init(iqempty_u32 + 8 * i, 1 + Cfg::kSoftmaxThreads);
+        }
         fence_barrier_init();
     }
     // the rows past the Q boxes (128 mod g of each half) are never loaded:
@@ -363,11 +378,50 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         const uint64_t keep = l2_policy_evict_last();  // K/V and Q are read by several tiles
         bool ok = true;
         uint32_t iq = 0, gs = 0;  // items with work, global steps
-        grid_dependency_wait();    // the pool: a cache write launched before has finished
-        for (int32_t it = blockIdx.x; it < total && ok; it += gridDim.x) {
-            const TileItem I = tile_item(P, prefix, it);
-            if (I.nsteps == 0) continue;
+        bool waited = false;       // grid_dependency_wait done
+        bool first = true;         // the CTA's first item is item blockIdx.x
+        int32_t cand = blockIdx.x;
+        while (ok) {
+            // the next item with work; it goes into the item queue the other roles read
+            // (-1: none left)
+            int32_t it = -1;
+            TileItem I;
+            while (true) {
+                if (first) {
+                    first = false;
+                } else if (P.item_counter) {
+                    if (!waited) {
+                        grid_dependency_wait();  // (the counter was set to zero before this launch)
+                        waited = true;
+                    }
+                    cand = 0;
+                    if (lane == 0) cand = static_cast<int32_t>(gridDim.x) + atomicAdd(P.item_counter, 1);
+                    cand = __shfl_sync(kFullMask, cand, 0);
+                } else {
+                    cand += gridDim.x;
+                }
+                if (cand >= total) break;
+                I = tile_item(P, prefix, cand);
+                if (I.nsteps > 0) {
+                    it = cand;
+                    break;
+                }
+            }
+            const uint32_t slot = iq % Cfg::kItemSlots;
+            if (iq >= static_cast<uint32_t>(Cfg::kItemSlots) &&
+                !mbar_wait_bounded(iqempty_u32 + 8 * slot, ((iq / Cfg::kItemSlots) - 1) & 1u)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
+                item_q[slot] = it;
+                mbar_arrive(iqfull_u32 + 8 * slot);
+            }
+            __syncwarp();
+            if (it < 0) break;
             // Q of both halves, once the previous item's S products are done with the buffer
+            // (the first item's Q, an input no kernel of this library writes, before the
+            // dependency wait)
             if (iq >= 1 && !mbar_wait_bounded(qempty_u32, (iq - 1) & 1u)) {
                 ok = false;
                 break;
@@ -382,6 +436,10 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                                     I.h * g, I.U.q_base + I.tok0 + hh * P.half_tokens, qfull_u32, keep);
             }
             ++iq;
+            if (!waited) {
+                grid_dependency_wait();  // the pool: a cache write launched before has finished
+                waited = true;
+            }
             // table entries of the item's blocks, 32 at a time: lane l holds
             // block win + l (-1 where past the item or outside the pool)
             const int32_t* trow = P.block_tables + static_cast<size_t>(I.U.table) * P.max_blocks_per_seq;
@@ -463,14 +521,20 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 uint32_t iq;     // items with work before this one
                 uint32_t gs;     // global step
             };
-            auto first_step = [&](int32_t it, uint32_t iq, uint32_t gs, Cur& c) -> bool {
-                for (; it < total; it += gridDim.x) {
-                    const TileItem I = tile_item(P, prefix, it);
-                    if (I.nsteps == 0) continue;
-                    c = Cur{it, 0, I.nsteps, iq, gs};
-                    return true;
+            bool ok = true;
+            // the iq-th item of the queue (false: none left, or the wait gave up)
+            auto first_step = [&](uint32_t iq, uint32_t gs, Cur& c) -> bool {
+                const uint32_t slot = iq % Cfg::kItemSlots;
+                if (!mbar_wait_bounded_thread(iqfull_u32 + 8 * slot, (iq / Cfg::kItemSlots) & 1u)) {
+                    ok = false;
+                    return false;
                 }
-                return false;
+                const int32_t it = item_q[slot];
+                mbar_arrive(iqempty_u32 + 8 * slot);
+                if (it < 0) return false;
+                const TileItem I = tile_item(P, prefix, it);
+                c = Cur{it, 0, I.nsteps, iq, gs};
+                return true;
             };
             auto next_step = [&](const Cur& c, Cur& n) -> bool {
                 if (c.j + 1 < c.nsteps) {
@@ -479,7 +543,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                     ++n.gs;
                     return true;
                 }
-                return first_step(c.it + gridDim.x, c.iq + 1, c.gs + 1, n);
+                return first_step(c.iq + 1, c.gs + 1, n);
             };
             auto issue_s = [&](const Cur& c) -> bool {
                 if (c.j == 0 && !mbar_wait_bounded_thread(qfull_u32, c.iq & 1u)) return false;
@@ -502,9 +566,8 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 if (c.j + 1 == c.nsteps) umma_commit(qempty_u32);  // the item's last read of Q
                 return true;
             };
-            bool ok = true;
             Cur cur;
-            bool have = first_step(blockIdx.x, 0, 0, cur);
+            bool have = first_step(0, 0, cur);
             if (have) ok = issue_s(cur);
             while (have && ok) {
                 Cur nxt;
@@ -547,16 +610,21 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         bool ok = true;  // warp-uniform: a wait that gave up stops TMEM work and arrivals
         uint32_t gs = 0;
         bool waited = false;  // grid_dependency_wait done (before the first output write)
-        for (int32_t it = blockIdx.x; it < total; it += gridDim.x) {
+        for (uint32_t iq = 0; ok; ++iq) {
+            const uint32_t slot = iq % Cfg::kItemSlots;
+            ok = mbar_wait_bounded(iqfull_u32 + 8 * slot, (iq / Cfg::kItemSlots) & 1u);
+            if (!ok) break;
+            const int32_t it = item_q[slot];
+            mbar_arrive(iqempty_u32 + 8 * slot);
+            if (it < 0) break;
             const TileItem I = tile_item(P, prefix, it);
-            if (I.nsteps == 0) continue;
             const int tok = hh * P.half_tokens + row / g;  // token of the tile (a sequence in prefix mode)
             const bool row_ok = row < half_rows && tok < I.ntok;
             const int32_t ktok = I.tok0 + tok;  // token within the unit
             // last key this row sees (prefill: causal; prefix: every prefix key)
             const int32_t lim = !row_ok ? -1 : prefill ? I.U.len - I.U.n + ktok : I.U.len - 1;
             const size_t orow = row_ok ? static_cast<size_t>(I.U.q_base + ktok) * P.num_q_heads + I.h * g + row % g : 0;
-            float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of the row
+            float m = -INFINITY, l = 0.f;  // reference max (log2 units) and sum of the row
             for (int j = 0; j < I.nsteps; ++j, ++gs) {
                 const int st = gs % S;
                 ok = ok && mbar_wait_bounded(sfull_u32 + 8 * (gs & 1u), (gs >> 1) & 1u);
@@ -566,8 +634,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 float x[K];
                 float mu = 0.f, alpha = 1.f;
                 if (ok) {
-                    tmem_ld32(lane_base + Cfg::kColS + (gs & 1u) * K, *reinterpret_cast<float(*)[32]>(x));
-                    tmem_ld32(lane_base + Cfg::kColS + (gs & 1u) * K + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+                    tmem_ld64(lane_base + Cfg::kColS + (gs & 1u) * K, x);
                     const uint32_t present = stage_present[st];
                     float mx;
                     // a wholly visible step (every block loaded, every key within
@@ -589,7 +656,11 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                         }
                         mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                     }
-                    const float mn = fmaxf(m, mx);
+                    // the reference max m (the exponents' offset) moves only when
+                    // the step's max exceeds it by more than kLazyRescale: weights
+                    // up to 2^kLazyRescale are exact enough in bf16 and fp32, and
+                    // O and l then need no rescale (alpha = 1)
+                    const float mn = mx > m + kLazyRescale ? mx : m;
                     mu = mn == -INFINITY ? 0.0f : mn;
                     alpha = fast_exp2(m - mu);
                     m = mn;

@@ -41,6 +41,7 @@ struct DecodeParams {
     float* ws_l;    // [num_seqs*num_q_heads][max_parts]
     float* ws_acc;  // [num_seqs*num_q_heads][max_parts][head_dim]
     int32_t* ws_parts;  // [num_seqs*num_kv_heads] pieces of each unit (split only)
+    int32_t* tile_counter;  // shared-prefix calls: the tile kernel's item counter (host use only)
     const int32_t* q_start;  // several query tokens per sequence: rows q_start[s] .. q_start[s+1]-1
                              // (null: one query token per sequence, row = sequence)
     int32_t max_q_len;       // bound on query tokens per sequence (1 without q_start)

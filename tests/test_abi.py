@@ -87,8 +87,14 @@ def test_shared_prefix_workspace_size(lib):
     # (4604 - 4096) tokens -> 32 blocks -> balanced bound ceil(32/16)+1 = 3 pieces
     P = 16 + 3
     rows = N * Hq
-    expect = 2 * a256(rows * P * 4) + a256(rows * P * D * 4) + a256(N * Hkv * 4)
+    # + 256 bytes: the tile kernel's item counter
+    expect = 2 * a256(rows * P * 4) + a256(rows * P * D * 4) + a256(N * Hkv * 4) + 256
     assert lib.pa_decode_shared_prefix_workspace_size(N, Hq, Hkv, D, 4604, 256, 16, 0) == expect
+    # several prompt groups: the private part can be a whole sequence (4604 tokens -> 288 blocks ->
+    # ceil(288/16)+1 = 19 pieces) after the 16 slots
+    P = 16 + 19
+    expect = 2 * a256(rows * P * 4) + a256(rows * P * D * 4) + a256(N * Hkv * 4) + 256
+    assert lib.pa_decode_shared_prefix_groups_workspace_size(N, Hq, Hkv, D, 4604, 256, 4, 16, 0) == expect
     # no shared blocks: the plain decode's size
     assert lib.pa_decode_shared_prefix_workspace_size(N, Hq, Hkv, D, 4604, 0, 16, 0) == \
         lib.pa_decode_workspace_size(N, Hq, Hkv, D, 4604, 16, 0)
@@ -116,7 +122,7 @@ def test_multi_query_workspace_and_limits(lib):
     sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 1 << 30
     tiles = -(-T // (2 * (128 // (Hq // Hkv)))) + N  # tiles of two 128-row halves
     C = _tile_splits(sms, tiles * Hkv, -(-L // 16))
-    want = max(layout(P), layout(C) if C > 1 else 0)
+    want = max(layout(P), (layout(C) if C > 1 else 0) + 256)  # + the tile kernel's item counter
     assert lib.pa_decode_multi_workspace_size(N, T, Hq, Hkv, D, L, 16, 0) == want
     # fp32 or a missing q_start are refused before anything is launched
     assert lib.pa_decode_multi(16, 16, T, 5, 16, 16, 16, 64, 16, L, N, 8, 2, D, 64, 16, 0.1, 0, None, 0, 16,

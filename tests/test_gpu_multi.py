@@ -128,3 +128,20 @@ def test_prefill_more_tokens_than_max_q_len_are_flagged():
     ref1 = oracle.paged_decode_multi(wl.as_numpy(q)[64:144], h["kc"], h["vc"], h["bt"][1:2],
                                      np.array([300], np.int32), np.array([0, 80], np.int32), w.scale)
     assert_close(to_f64(out)[64:144], ref1, torch.bfloat16, "prefill seq 1, clamped")
+
+
+def test_prefill_more_sequences_than_one_launch_holds():
+    """More sequences than one tile-kernel launch takes (256): several launches
+    over consecutive ranges of sequences, each with its own work counter."""
+    rng = np.random.default_rng(9)
+    lens = [int(x) for x in rng.integers(20, 300, size=300)]
+    nq = [min(L, int(x)) for L, x in zip(lens, rng.integers(5, 40, size=300))]
+    w = wl.build(lens, 16, 4, 64, torch.bfloat16, seed=12, device=DEV, poison_unused=True)
+    q, qs = _queries(nq, 16, 64, seed=12)
+    out = pa.decode_multi(q, qs, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, max(nq),
+                          max_seq_len=w.max_seq_len)
+    torch.cuda.synchronize()
+    assert pa.device_error() == 0
+    h = host(w)
+    ref = oracle_decode_multi_all_rows(wl.as_numpy(q), h["kc"], h["vc"], h["bt"], h["sl"], qs.cpu().numpy(), w.scale)
+    assert_close(to_f64(out), ref, torch.bfloat16, "prefill, 300 sequences")
