@@ -789,6 +789,8 @@ int run_prefill_tiles(const DecodeArgs& a) {
     const int32_t max_len = a.max_seq_len > 0
                                 ? a.max_seq_len
                                 : static_cast<int32_t>(table_tokens > INT32_MAX ? INT32_MAX : table_tokens);
+    // the workspace holds at least the item counter (checked before any CUDA call)
+    if (!a.workspace || !aligned(a.workspace, 256) || a.workspace_bytes < kCounterBytes) return PA_ERR_WORKSPACE;
     DeviceInfo di;
     if ((rc = device_info(&di)) != PA_OK) return rc;
     const PrefillPlan pp = make_prefill_plan(di.sms, a.num_seqs, a.num_q_rows, a.num_q_heads, a.num_kv_heads,

@@ -233,3 +233,35 @@ def test_boundary_calls_cite_a_passage_or_say_plumbing(name):
     c = _comment_before(name)
     pages = ("slavadubrov.com", "aiunderstanding.org", "de.news.hada.io", "artificials.ru")
     assert any(p in c for p in pages) or "Interface plumbing" in c, name
+
+
+def test_prompt_groups_and_prefill_reject_bad_arguments_on_the_host(lib):
+    """The prompt-group decode and the prefill path validate on the host
+    before any CUDA call (fake, never dereferenced addresses)."""
+    g = lib.pa_decode_shared_prefix_groups
+
+    def grc(**over):
+        a = dict(q=16, k=16, v=16, bt=16, mb=64, sl=16, msl=1000, gs=16, gb=16, G=2, maxs=32, N=4, Hq=8, Hkv=2,
+                 D=128, NB=64, B=16, scale=0.1, pb=0, ws=256, wsb=1 << 30, out=16, dt=pa.PA_DTYPE_BF16)
+        a.update(over)
+        return g(a["q"], a["k"], a["v"], a["bt"], a["mb"], a["sl"], a["msl"], a["gs"], a["gb"], a["G"], a["maxs"],
+                 a["N"], a["Hq"], a["Hkv"], a["D"], a["NB"], a["B"], a["scale"], a["pb"], a["ws"], a["wsb"],
+                 a["out"], a["dt"], None)
+
+    assert grc(gs=None) == pa.PA_ERR_INVALID_ARG
+    assert grc(gb=None) == pa.PA_ERR_INVALID_ARG
+    assert grc(gs=18) == pa.PA_ERR_INVALID_ARG          # misaligned
+    assert grc(G=0) == pa.PA_ERR_INVALID_ARG
+    assert grc(maxs=-1) == pa.PA_ERR_INVALID_ARG
+    assert grc(maxs=100) == pa.PA_ERR_INVALID_ARG       # more shared blocks than max_seq_len holds
+    assert grc(dt=pa.PA_DTYPE_F32) == pa.PA_ERR_UNSUPPORTED
+    need = lib.pa_decode_shared_prefix_groups_workspace_size(4, 8, 2, 128, 1000, 32, 2, 16, 0)
+    assert need > 0
+    assert grc(wsb=need - 1) == pa.PA_ERR_WORKSPACE
+    assert grc(ws=None) == pa.PA_ERR_WORKSPACE
+    # the prefill path (group 4 x 64 query tokens > 16 rows): the workspace holds at least its counter
+    m = lib.pa_decode_multi
+    assert m(16, 16, 64, 64, 16, 16, 16, 64, 16, 1000, 1, 8, 2, 128, 64, 16, 0.1, 0, None, 0, 16,
+             pa.PA_DTYPE_BF16, None) == pa.PA_ERR_WORKSPACE
+    assert m(16, 16, 64, 64, 16, 16, 16, 64, 16, 1000, 1, 8, 2, 96, 64, 16, 0.1, 0, 256, 1 << 20, 16,
+             pa.PA_DTYPE_BF16, None) == pa.PA_ERR_UNSUPPORTED  # head_dim 96
