@@ -125,10 +125,10 @@ struct TileCfg {
     static constexpr uint32_t kHalfCols = 256;  // per half: S0 | S1 | O
     static constexpr uint32_t kTmemCols = kTileHalves * kHalfCols;
     static constexpr uint32_t kColS = 0, kColO = 2 * kKeys;
-    // K full / empty, V full / empty per stage; s_full x2, p_full, o_done, o_free, q_full,
-    // q_empty, drain; item queue full / empty x kItemSlots
+    // full, empty per stage; s_full x2, p_full, o_done, o_free, q_full, q_empty, drain;
+    // item queue full / empty x kItemSlots
     static constexpr int kItemSlots = 4;
-    static constexpr int kBars = 4 * kStages + 8 + 2 * kItemSlots;
+    static constexpr int kBars = 2 * kStages + 8 + 2 * kItemSlots;
     static constexpr int kMaxUnits = 256;  // units whose item prefix one CTA holds (more: several launches)
     static constexpr int kPrefixBytes = (4 * (kMaxUnits + 1) + 15) / 16 * 16;
     static constexpr size_t kSmem = 1024 + kQBytes + kStages * kStageBytes + kPBytes + kPrefixBytes +
@@ -315,13 +315,9 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     uint8_t* p_smem = ring_smem + S * Cfg::kStageBytes;
     int32_t* prefix = reinterpret_cast<int32_t*>(p_smem + Cfg::kPBytes);
     const uint32_t bars_u32 = p_u32 + Cfg::kPBytes + Cfg::kPrefixBytes;
-    // a stage's K and V land and are released separately: the scores need
-    // only K, and K is free again once they are computed
-    const uint32_t kfull_u32 = bars_u32;            // [S]
-    const uint32_t kempty_u32 = bars_u32 + 8 * S;   // [S]
-    const uint32_t vfull_u32 = bars_u32 + 16 * S;   // [S]
-    const uint32_t vempty_u32 = bars_u32 + 24 * S;  // [S]
-    const uint32_t sfull_u32 = bars_u32 + 32 * S;   // [2]
+    const uint32_t full_u32 = bars_u32;            // [S]
+    const uint32_t empty_u32 = bars_u32 + 8 * S;   // [S]
+    const uint32_t sfull_u32 = bars_u32 + 16 * S;  // [2]
     const uint32_t pfull_u32 = sfull_u32 + 16;
     const uint32_t odone_u32 = pfull_u32 + 8;
     const uint32_t ofree_u32 = odone_u32 + 8;
@@ -341,10 +337,8 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < S; ++st) {
-            mbar_init(kfull_u32 + 8 * st, 1);
-            mbar_init(kempty_u32 + 8 * st, 1);
-            mbar_init(vfull_u32 + 8 * st, 1);
-            mbar_init(vempty_u32 + 8 * st, 1);
+            mbar_init(full_u32 + 8 * st, 1);
+            mbar_init(empty_u32 + 8 * st, 1);
         }
         mbar_init(sfull_u32, 1);
         mbar_init(sfull_u32 + 8, 1);
@@ -386,48 +380,6 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         uint32_t iq = 0, gs = 0;  // items with work, global steps
         bool waited = false;       // grid_dependency_wait done
         bool first = true;         // the CTA's first item is item blockIdx.x
-        // The V boxes of a step go out after the next step's K boxes (the
-        // scores never wait behind V; an item's last V right after its last
-        // K): the step whose V is pending.
-        bool v_pending = false;
-        int v_st = 0, v_h = 0;
-        uint32_t v_gs = 0, v_present = 0;
-        int32_t v_pb = -1;  // lane b < 4: block b of that step
-        auto issue_v = [&]() -> bool {
-            if (v_gs >= static_cast<uint32_t>(S) && !mbar_wait_bounded(vempty_u32 + 8 * v_st, ((v_gs / S) - 1) & 1u))
-                return false;
-            if (v_present != (1u << Cfg::kStepBlocks) - 1u) {
-                // blocks past the item or outside the pool: zero their V rows
-                // so that P = 0 times them stays 0
-                for (int c = lane; c < Cfg::kStepBlocks * Cfg::kSlabs * kBlockTokens * 8; c += 32) {
-                    const int bb = c / (Cfg::kSlabs * kBlockTokens * 8);
-                    if ((v_present >> bb) & 1u) continue;
-                    const int rem = c % (Cfg::kSlabs * kBlockTokens * 8);
-                    const int sl = rem / (kBlockTokens * 8), rr = rem % (kBlockTokens * 8);
-                    const int t = bb * kBlockTokens + rr / 8;
-                    *reinterpret_cast<uint4*>(ring_smem + v_st * Cfg::kStageBytes + (Cfg::kSlabs + sl) * Cfg::kKVSlab +
-                                              t * 128 + (rr % 8) * 16) = make_uint4(0, 0, 0, 0);
-                }
-                fence_proxy_async_smem();
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive_expect_tx(vfull_u32 + 8 * v_st, __popc(v_present) * Cfg::kSlabs * 2048);
-            const uint32_t vbase = ring_u32 + v_st * Cfg::kStageBytes + Cfg::kSlabs * Cfg::kKVSlab;
-#pragma unroll
-            for (int bb = 0; bb < Cfg::kStepBlocks; ++bb) {
-                const int32_t pbb = __shfl_sync(kFullMask, v_pb, bb);
-                if (lane == 0 && pbb >= 0) {
-                    const int32_t row = (pbb * P.num_kv_heads + v_h) * kBlockTokens;
-#pragma unroll
-                    for (int sl = 0; sl < Cfg::kSlabs; ++sl)
-                        tma_load_2d(vbase + sl * Cfg::kKVSlab + bb * kBlockTokens * 128, &tmap_v, sl * 64, row,
-                                    vfull_u32 + 8 * v_st, keep);
-                }
-            }
-            __syncwarp();
-            v_pending = false;
-            return true;
-        };
         int32_t cand = blockIdx.x;
         while (ok) {
             // the next item with work; it goes into the item queue the other roles read
@@ -503,7 +455,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             int32_t win = table_entry(I.kb0 + lane);
             for (int j = 0; j < I.nsteps; ++j, ++gs) {
                 const int st = gs % S;
-                if (gs >= static_cast<uint32_t>(S) && !mbar_wait_bounded(kempty_u32 + 8 * st, ((gs / S) - 1) & 1u)) {
+                if (gs >= static_cast<uint32_t>(S) && !mbar_wait_bounded(empty_u32 + 8 * st, ((gs / S) - 1) & 1u)) {
                     ok = false;
                     break;
                 }
@@ -512,10 +464,25 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 const int32_t pb = __shfl_sync(kFullMask, win, (first & 31) + (lane & (Cfg::kStepBlocks - 1)));
                 const uint32_t present =
                     __ballot_sync(kFullMask, lane < Cfg::kStepBlocks && pb >= 0) & ((1u << Cfg::kStepBlocks) - 1u);
-                const uint32_t kbase = ring_u32 + st * Cfg::kStageBytes;
+                const uint32_t sbase = ring_u32 + st * Cfg::kStageBytes;
+                if (present != (1u << Cfg::kStepBlocks) - 1u) {
+                    // blocks past the item or outside the pool: zero their V rows
+                    // so that P = 0 times them stays 0
+                    for (int c = lane; c < Cfg::kStepBlocks * Cfg::kSlabs * kBlockTokens * 8; c += 32) {
+                        const int bb = c / (Cfg::kSlabs * kBlockTokens * 8);
+                        if ((present >> bb) & 1u) continue;
+                        const int rem = c % (Cfg::kSlabs * kBlockTokens * 8);
+                        const int sl = rem / (kBlockTokens * 8), rr = rem % (kBlockTokens * 8);
+                        const int t = bb * kBlockTokens + rr / 8;
+                        *reinterpret_cast<uint4*>(ring_smem + st * Cfg::kStageBytes + (Cfg::kSlabs + sl) * Cfg::kKVSlab +
+                                                  t * 128 + (rr % 8) * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
                 if (lane == 0) {
                     stage_present[st] = present;  // read by the softmax after this barrier's phase
-                    mbar_arrive_expect_tx(kfull_u32 + 8 * st, __popc(present) * Cfg::kSlabs * 2048);
+                    mbar_arrive_expect_tx(full_u32 + 8 * st, __popc(present) * 2 * Cfg::kSlabs * 2048);
                 }
 #pragma unroll
                 for (int bb = 0; bb < Cfg::kStepBlocks; ++bb) {
@@ -523,28 +490,22 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                     if (lane == 0 && pbb >= 0) {
                         const int32_t row = (pbb * P.num_kv_heads + I.h) * kBlockTokens;
 #pragma unroll
-                        for (int sl = 0; sl < Cfg::kSlabs; ++sl)
-                            tma_load_2d(kbase + sl * Cfg::kKVSlab + bb * kBlockTokens * 128, &tmap_k, sl * 64, row,
-                                        kfull_u32 + 8 * st, keep);
+                        for (int sl = 0; sl < Cfg::kSlabs; ++sl) {
+                            tma_load_2d(sbase + sl * Cfg::kKVSlab + bb * kBlockTokens * 128, &tmap_k, sl * 64, row,
+                                        full_u32 + 8 * st, keep);
+                            tma_load_2d(sbase + (Cfg::kSlabs + sl) * Cfg::kKVSlab + bb * kBlockTokens * 128, &tmap_v,
+                                        sl * 64, row, full_u32 + 8 * st, keep);
+                        }
                     }
                 }
                 __syncwarp();
-                if (v_pending && !(ok = issue_v())) break;  // the previous step's V
-                v_pending = true;
-                v_st = st;
-                v_gs = gs;
-                v_present = present;
-                v_pb = pb;
-                v_h = I.h;
             }
-            if (ok && v_pending) ok = issue_v();  // the item's last V
         }
         if (!ok && lane == 0) flag_error(PA_DEVERR_TIMEOUT);
         // this warp's last copies into every stage and into Q have landed before leaving
         for (uint32_t k = 0; k < static_cast<uint32_t>(S) && k < gs; ++k) {
             const uint32_t last = gs - 1 - k;  // one of the last S steps
-            mbar_wait_bounded(kfull_u32 + 8 * (last % S), (last / S) & 1u);
-            if (ok) mbar_wait_bounded(vfull_u32 + 8 * (last % S), (last / S) & 1u);
+            mbar_wait_bounded(full_u32 + 8 * (last % S), (last / S) & 1u);
         }
         if (iq > 0) mbar_wait_bounded(qfull_u32, (iq - 1) & 1u);
     } else if (warp == Cfg::kMmaWarp) {
@@ -587,7 +548,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             auto issue_s = [&](const Cur& c) -> bool {
                 if (c.j == 0 && !mbar_wait_bounded_thread(qfull_u32, c.iq & 1u)) return false;
                 const int st = c.gs % S;
-                if (!mbar_wait_bounded_thread(kfull_u32 + 8 * st, (c.gs / S) & 1u)) return false;
+                if (!mbar_wait_bounded_thread(full_u32 + 8 * st, (c.gs / S) & 1u)) return false;
                 tc_fence_after();
                 const uint32_t kb = ring_u32 + st * Cfg::kStageBytes;
 #pragma unroll
@@ -602,7 +563,6 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                     }
                 }
                 umma_commit(sfull_u32 + 8 * (c.gs & 1u));
-                umma_commit(kempty_u32 + 8 * st);  // K of the stage is free once the scores are done
                 if (c.j + 1 == c.nsteps) umma_commit(qempty_u32);  // the item's last read of Q
                 return true;
             };
@@ -618,7 +578,6 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 if (cur.j == 0 && cur.iq > 0 && !(ok = mbar_wait_bounded_thread(ofree_u32, (cur.iq - 1) & 1u)))
                     break;
                 if (!(ok = mbar_wait_bounded_thread(pfull_u32, cur.gs & 1u))) break;
-                if (!(ok = mbar_wait_bounded_thread(vfull_u32 + 8 * (cur.gs % S), (cur.gs / S) & 1u))) break;
                 tc_fence_after();
                 const uint32_t vb = ring_u32 + (cur.gs % S) * Cfg::kStageBytes + Cfg::kSlabs * Cfg::kKVSlab;
 #pragma unroll
@@ -631,7 +590,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                     }
                 }
                 umma_commit(odone_u32);
-                umma_commit(vempty_u32 + 8 * (cur.gs % S));
+                umma_commit(empty_u32 + 8 * (cur.gs % S));
                 if (!more) break;
                 cur = nxt;
             }
@@ -669,7 +628,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             for (int j = 0; j < I.nsteps; ++j, ++gs) {
                 const int st = gs % S;
                 ok = ok && mbar_wait_bounded(sfull_u32 + 8 * (gs & 1u), (gs >> 1) & 1u);
-                ok = ok && mbar_wait_bounded(kfull_u32 + 8 * st, (gs / S) & 1u);
+                ok = ok && mbar_wait_bounded(full_u32 + 8 * st, (gs / S) & 1u);
                 tc_fence_after();
                 const int32_t key0 = (I.kb0 + j * Cfg::kStepBlocks) * kBlockTokens;  // first key of the step
                 float x[K];
@@ -753,7 +712,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                     // key slots at or past the sequence's length hold stale data
                     // (weight 0, but 0 * NaN is NaN): zero their V rows in the stage
                     const int32_t zero_from = I.U.len - key0;
-                    if (zero_from < K && (ok = mbar_wait_bounded(vfull_u32 + 8 * st, (gs / S) & 1u))) {
+                    if (zero_from < K) {
                         const int zrows = K - max(0, zero_from);
                         for (int e = threadIdx.x; e < zrows * Cfg::kSlabs * 8; e += Cfg::kSoftmaxThreads) {
                             const int zr = K - zrows + e / (Cfg::kSlabs * 8);
