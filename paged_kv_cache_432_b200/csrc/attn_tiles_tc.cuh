@@ -130,7 +130,9 @@ struct TileCfg {
     static constexpr int kItemSlots = 4;
     static constexpr int kBars = 2 * kStages + 8 + 2 * kItemSlots;
     static constexpr int kMaxUnits = 256;  // units whose item prefix one CTA holds (more: several launches)
-    static constexpr int kPrefixBytes = (4 * (kMaxUnits + 1) + 15) / 16 * 16;
+    static_assert(kMaxUnits <= 256 && kMaxUnits <= kThreads, "unit positions in a byte, one thread per unit");
+    // item prefix (int32 [kMaxUnits + 1]) and the units' order (uint8 [kMaxUnits])
+    static constexpr int kPrefixBytes = (4 * (kMaxUnits + 1) + kMaxUnits + 15) / 16 * 16;
     static constexpr size_t kSmem = 1024 + kQBytes + kStages * kStageBytes + kPBytes + kPrefixBytes +
                                     8 * kBars + 16 + 4 * kStages + 4 * kItemSlots;
     static_assert(kColO + D <= kHalfCols, "TMEM columns");
@@ -193,11 +195,13 @@ struct TileItem {
     int32_t nsteps;      // 0: empty item
 };
 
-// Item `it` of the launch (prefix[] holds the units' exclusive item sums).
-__device__ __forceinline__ TileItem tile_item(const TileParams& P, const int32_t* prefix, int32_t it) {
+// Item `it` of the launch: prefix[] holds the exclusive item sums of the
+// units in the order ord[] (heaviest unit first).
+__device__ __forceinline__ TileItem tile_item(const TileParams& P, const int32_t* prefix, const uint8_t* ord,
+                                              int32_t it) {
     TileItem I;
     const int i = upper_index(P.num_units, it, [&](int k) { return static_cast<int64_t>(prefix[k]); });
-    I.u = P.unit_begin + i;
+    I.u = P.unit_begin + ord[i];
     I.U = tile_unit(P, I.u);
     const int32_t j = it - prefix[i];
     const int32_t th = I.U.tiles * P.num_kv_heads;
@@ -219,21 +223,41 @@ __device__ __forceinline__ TileItem tile_item(const TileParams& P, const int32_t
     return I;
 }
 
-// Exclusive sums of the units' item counts into prefix[0..num_units]; all
-// threads of the CTA call it.  Returns the total.  Reports clamped query
-// counts (CTA 0 only, so each is counted once).
-__device__ __forceinline__ int32_t build_unit_prefix(const TileParams& P, int32_t* prefix) {
+// The launch's units in order of decreasing work (items x key blocks, ties by
+// index) into ord[0..num_units), and the exclusive sums of their item counts
+// in that order into prefix[0..num_units]: items of the heaviest units are
+// claimed first, so the last items to be claimed are short and the CTAs finish
+// together.  `scratch` holds 2 * num_units words (free during the prologue).
+// All threads of the CTA call it (num_units <= kMaxUnits <= blockDim.x).
+// Returns the total.  Reports clamped query counts (CTA 0 only, so each is
+// counted once).
+__device__ __forceinline__ int32_t build_unit_prefix(const TileParams& P, int32_t* prefix, uint8_t* ord,
+                                                     uint32_t* scratch) {
     __shared__ int32_t warp_tot[32];
     const int n = P.num_units;
     const int tid = threadIdx.x, nthr = blockDim.x;
-    const int per = (n + nthr - 1) / nthr;
-    const int beg = min(n, tid * per), end = min(n, beg + per);
-    int32_t local = 0;
-    for (int i = beg; i < end; ++i) {
-        const TileUnit U = tile_unit(P, P.unit_begin + i);
+    uint32_t* cost = scratch;
+    int32_t* items = reinterpret_cast<int32_t*>(scratch + n);
+    uint32_t my_cost = 0;
+    if (tid < n) {
+        const TileUnit U = tile_unit(P, P.unit_begin + tid);
         if (U.clamped && blockIdx.x == 0) flag_error(PA_DEVERR_SEQ_LEN);
-        local += U.tiles * U.chunks * P.num_kv_heads;
+        const int32_t it = U.tiles * U.chunks * P.num_kv_heads;
+        my_cost = static_cast<uint32_t>(min(static_cast<int64_t>(it) * max(U.kblocks, 1), int64_t{0xffffffff}));
+        cost[tid] = my_cost;
+        items[tid] = it;
     }
+    __syncthreads();
+    if (tid < n) {
+        int rank = 0;
+        for (int u = 0; u < n; ++u) {
+            const uint32_t c = cost[u];
+            rank += (c > my_cost) || (c == my_cost && u < tid);
+        }
+        ord[rank] = static_cast<uint8_t>(tid);
+    }
+    __syncthreads();
+    const int32_t local = tid < n ? items[ord[tid]] : 0;
     const int lane = tid & 31, warp = tid >> 5, nwarps = (nthr + 31) >> 5;
     int32_t incl = local;
 #pragma unroll
@@ -254,13 +278,10 @@ __device__ __forceinline__ int32_t build_unit_prefix(const TileParams& P, int32_
         warp_tot[lane] = ti - t;
     }
     __syncthreads();
-    int32_t run = warp_tot[warp] + incl - local;
-    for (int i = beg; i < end; ++i) {
-        prefix[i] = run;
-        const TileUnit U = tile_unit(P, P.unit_begin + i);
-        run += U.tiles * U.chunks * P.num_kv_heads;
-    }
-    if (tid == nthr - 1) prefix[n] = run;
+    const int32_t excl = warp_tot[warp] + incl - local;
+    if (tid < n) prefix[tid] = excl;
+    if (tid == n - 1) prefix[n] = excl + local;
+    if (n == 0 && tid == 0) prefix[0] = 0;
     __syncthreads();
     return prefix[n];
 }
@@ -365,7 +386,9 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     }
     fence_proxy_async_smem();
     if (warp == Cfg::kMmaWarp) tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
-    const int32_t total = build_unit_prefix(P, prefix);  // ends with __syncthreads
+    uint8_t* unit_ord = reinterpret_cast<uint8_t*>(prefix + Cfg::kMaxUnits + 1);
+    // (the P buffer is free until the first step: scratch for the ordering)
+    const int32_t total = build_unit_prefix(P, prefix, unit_ord, reinterpret_cast<uint32_t*>(p_smem));
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -401,7 +424,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                     cand += gridDim.x;
                 }
                 if (cand >= total) break;
-                I = tile_item(P, prefix, cand);
+                I = tile_item(P, prefix, unit_ord, cand);
                 if (I.nsteps > 0) {
                     it = cand;
                     break;
@@ -532,7 +555,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 const int32_t it = item_q[slot];
                 mbar_arrive(iqempty_u32 + 8 * slot);
                 if (it < 0) return false;
-                const TileItem I = tile_item(P, prefix, it);
+                const TileItem I = tile_item(P, prefix, unit_ord, it);
                 c = Cur{it, 0, I.nsteps, iq, gs};
                 return true;
             };
@@ -617,7 +640,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             const int32_t it = item_q[slot];
             mbar_arrive(iqempty_u32 + 8 * slot);
             if (it < 0) break;
-            const TileItem I = tile_item(P, prefix, it);
+            const TileItem I = tile_item(P, prefix, unit_ord, it);
             const int tok = hh * P.half_tokens + row / g;  // token of the tile (a sequence in prefix mode)
             const bool row_ok = row < half_rows && tok < I.ntok;
             const int32_t ktok = I.tok0 + tok;  // token within the unit
