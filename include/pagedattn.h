@@ -33,8 +33,9 @@
  * default stream) and return once the work is enqueued.
  *
  * Early start of the decode kernels: every decode entry point (pa_decode,
- * pa_decode_partitions, pa_decode_reduce, pa_decode_fp8, pa_decode_multi,
- * pa_decode_shared_prefix, pa_decode_noalloc) launches its kernels with
+ * pa_decode_partitions, pa_decode_reduce, pa_decode_fp8 and its two steps,
+ * pa_decode_multi, pa_decode_shared_prefix and its prompt-group form,
+ * pa_decode_noalloc) launches its kernels with
  * programmatic stream serialization, so they may start before the previous
  * kernel in the stream has finished.  Before waiting for that kernel they
  * already read seq_lens, block_tables, q_start, the prefix groups and q (they never touch the
@@ -156,6 +157,33 @@ PA_API int pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache
                          int32_t num_blocks, int32_t block_size, float scale,
                          int32_t partition_blocks, void* workspace, size_t workspace_bytes,
                          void* out, void* stream);
+
+/*
+ * The two steps of pa_decode_fp8 as separate calls (as pa_decode_partitions
+ * and pa_decode_reduce are for pa_decode), so that each kernel can be timed
+ * on its own; issued back to back on one stream they give pa_decode_fp8's
+ * result bit for bit.  pa_decode_fp8_partitions takes pa_decode_fp8's
+ * arguments and writes out[] for the single-piece (sequence, kv head) units
+ * and the workspace partials for the others.  pa_decode_fp8_reduce takes
+ * pa_decode_reduce's arguments (out is bf16) and merges the partials of an
+ * E4M3 partition step (the warp ranges of the balanced split depend on the
+ * kernel form, so the bf16 reduce must not be used on them).
+ * Interface plumbing: no passage (the pages define no API); the arithmetic
+ * is pa_decode_fp8's and pa_decode_reduce's.  Errors as for those calls.
+ */
+PA_API int pa_decode_fp8_partitions(const void* q, const void* k_cache, const void* v_cache,
+                                    const float* k_scale, const float* v_scale,
+                                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                    const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t num_blocks, int32_t block_size, float scale,
+                                    int32_t partition_blocks, void* workspace, size_t workspace_bytes,
+                                    void* out, void* stream);
+PA_API int pa_decode_fp8_reduce(const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                                int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t max_blocks_per_seq, int32_t block_size,
+                                int32_t partition_blocks, const void* workspace,
+                                size_t workspace_bytes, void* out, void* stream);
 
 /*
  * Several new query tokens per sequence: the check step of speculative

@@ -193,6 +193,30 @@ int encode_pool_map(CUtensorMap* map, const void* base, int64_t rows, int head_d
     return PA_OK;
 }
 
+// The bf16 pool seen as a 3-D tensor [slab][rows][64 columns] (slab stride
+// 128 bytes, row stride head_dim * 2), for head_dim 128: one 64 x 16 x 2 box
+// lands a block-head's whole tile (4 KB) as its two 128-byte-swizzled
+// column slabs one after the other.  head_dim 64 has one slab: the 2-D map.
+int encode_pool_map_blocks(CUtensorMap* map, const void* base, int64_t rows, int head_dim) {
+    if (head_dim != 128) return encode_pool_map(map, base, rows, head_dim);
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    int rc = get_encoder(&enc);
+    if (rc != PA_OK) return rc;
+    cuuint64_t dims[3] = {64u, static_cast<cuuint64_t>(rows), 2u};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2, 128u};
+    cuuint32_t box[3] = {64u, 16u, 2u};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
+                      "cuTensorMapEncodeTiled (block tiles) failed (CUresult %d)", static_cast<int>(r));
+        return PA_ERR_CUDA;
+    }
+    return PA_OK;
+}
+
 // ------------------------------------------------------------ planning
 constexpr int32_t kMinChunk = 16;  // balanced split: fewest blocks in one warp's range
 
@@ -508,9 +532,10 @@ int mma_shape_for(const DecodeParams& P, LaunchShape* L) {
     return rows <= 8 ? mma_shape<64, 8, FP8>(P, L) : mma_shape<64, 16, FP8>(P, L);
 }
 
-int decode_shape(const DecodeParams& P, int32_t dtype, LaunchShape* L) {
+// fp8: the E4M3 form of the decode kernel (caches of 8-bit codes).
+int decode_shape(const DecodeParams& P, int32_t dtype, bool fp8, LaunchShape* L) {
     if (dtype == PA_DTYPE_BF16)
-        return P.k_scale ? mma_shape_for<true>(P, L) : mma_shape_for<false>(P, L);
+        return fp8 ? mma_shape_for<true>(P, L) : mma_shape_for<false>(P, L);
     if (P.head_dim == 128) return P.group <= 4 ? simt_shape<128, 4>(P, L) : simt_shape<128, 16>(P, L);
     return P.group <= 4 ? simt_shape<64, 4>(P, L) : simt_shape<64, 16>(P, L);
 }
@@ -631,7 +656,7 @@ int launch_tiles(const TileParams& base, const void* q, int64_t q_rows, const vo
     const int64_t rows = static_cast<int64_t>(base.num_blocks) * base.num_kv_heads * kBlockTokens;
     alignas(64) CUtensorMap mk, mv, mq;
     if ((rc = encode_pool_map(&mk, k_cache, rows, D)) != PA_OK) return rc;
-    if ((rc = encode_pool_map(&mv, v_cache, rows, D)) != PA_OK) return rc;
+    if ((rc = encode_pool_map_blocks(&mv, v_cache, rows, D)) != PA_OK) return rc;
     if ((rc = encode_q_map(&mq, q, q_rows > 0 ? q_rows : 1, base.num_q_heads, D, base.group)) != PA_OK) return rc;
     DeviceInfo di;
     if ((rc = device_info(&di)) != PA_OK) return rc;
@@ -699,7 +724,7 @@ int launch_prefix_tiles(const DecodeParams& P, Plan* plan, cudaStream_t st) {
 }
 
 template <typename OutT, int D>
-int launch_reduce(const DecodeParams& base, int32_t dtype, cudaStream_t st) {
+int launch_reduce(const DecodeParams& base, int32_t dtype, bool fp8, cudaStream_t st) {
     if (base.q_start && !(base.balanced && base.piece_base == 0)) {
         // row-wise merge over every query-token row at once (rows locate their
         // sequence through q_start)
@@ -722,7 +747,7 @@ int launch_reduce(const DecodeParams& base, int32_t dtype, cudaStream_t st) {
         cudaError_t e;
         if (P.balanced && P.piece_base == 0) {
             LaunchShape L;
-            int r = decode_shape(P, dtype, &L);
+            int r = decode_shape(P, dtype, fp8, &L);
             if (r != PA_OK) return r;
             const int decode_warps = L.grid * (L.threads / 32);
             if (decode_warps < 2) return PA_OK;  // one warp range: nothing was cut
@@ -743,13 +768,16 @@ int launch_reduce(const DecodeParams& base, int32_t dtype, cudaStream_t st) {
     });
 }
 
-int run_reduce(const DecodeParams& P, const Plan& plan, int32_t dtype, cudaStream_t st) {
+// fp8: the partials came from the E4M3 decode kernel (whose launch shape the
+// balanced merge recomputes); by default, when P carries the E4M3 scales.
+int run_reduce(const DecodeParams& P, const Plan& plan, int32_t dtype, cudaStream_t st, int fp8 = -1) {
     if (P.num_seqs == 0 || !plan.split) return PA_OK;
+    const bool f8 = fp8 < 0 ? P.k_scale != nullptr : fp8 != 0;
     if (dtype == PA_DTYPE_BF16)
-        return P.head_dim == 128 ? launch_reduce<__nv_bfloat16, 128>(P, dtype, st)
-                                 : launch_reduce<__nv_bfloat16, 64>(P, dtype, st);
-    return P.head_dim == 128 ? launch_reduce<float, 128>(P, dtype, st)
-                             : launch_reduce<float, 64>(P, dtype, st);
+        return P.head_dim == 128 ? launch_reduce<__nv_bfloat16, 128>(P, dtype, f8, st)
+                                 : launch_reduce<__nv_bfloat16, 64>(P, dtype, f8, st);
+    return P.head_dim == 128 ? launch_reduce<float, 128>(P, dtype, f8, st)
+                             : launch_reduce<float, 64>(P, dtype, f8, st);
 }
 
 // Several query tokens per sequence with group * max_q_len > 16 (prefill
@@ -1027,7 +1055,7 @@ int pa_decode_reduce(const int32_t* seq_lens, int32_t max_seq_len, int32_t num_s
     Plan plan;
     int rc = prepare_decode(a, false, &P, &plan);
     if (rc != PA_OK) return rc;
-    return run_reduce(P, plan, dtype, a.stream);
+    return run_reduce(P, plan, dtype, a.stream, 0);
 }
 
 int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
@@ -1068,6 +1096,42 @@ int pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const
     rc = run_partitions(P, PA_DTYPE_BF16, a.stream);
     if (rc != PA_OK) return rc;
     return run_reduce(P, plan, PA_DTYPE_BF16, a.stream);
+}
+
+int pa_decode_fp8_partitions(const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                             const float* v_scale, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                             const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs,
+                             int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                             int32_t block_size, float scale, int32_t partition_blocks, void* workspace,
+                             size_t workspace_bytes, void* out, void* stream) {
+    if (!k_scale || !v_scale) return PA_ERR_INVALID_ARG;
+    DecodeArgs a = make_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                             max_seq_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                             block_size, scale, partition_blocks, workspace, workspace_bytes, out,
+                             PA_DTYPE_BF16, stream);
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    DecodeParams P;
+    Plan plan;
+    int rc = prepare_decode(a, true, &P, &plan);
+    if (rc != PA_OK) return rc;
+    return run_partitions(P, PA_DTYPE_BF16, a.stream);
+}
+
+int pa_decode_fp8_reduce(const int32_t* seq_lens, int32_t max_seq_len, int32_t num_seqs, int32_t num_q_heads,
+                         int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq, int32_t block_size,
+                         int32_t partition_blocks, const void* workspace, size_t workspace_bytes, void* out,
+                         void* stream) {
+    const DecodeArgs a = make_args(nullptr, nullptr, nullptr, nullptr, max_blocks_per_seq, seq_lens,
+                                   max_seq_len, num_seqs, num_q_heads, num_kv_heads, head_dim, 1,
+                                   block_size, 1.0f, partition_blocks,
+                                   const_cast<void*>(workspace), workspace_bytes, out, PA_DTYPE_BF16,
+                                   stream);
+    DecodeParams P;
+    Plan plan;
+    int rc = prepare_decode(a, false, &P, &plan);
+    if (rc != PA_OK) return rc;
+    return run_reduce(P, plan, PA_DTYPE_BF16, a.stream, 1);
 }
 
 // ------------------------------------------------------------ no-allocation decode

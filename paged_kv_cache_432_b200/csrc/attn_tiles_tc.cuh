@@ -43,8 +43,12 @@
 // half w / 4, TMEM lanes 32 (w mod 4) .. +31), warp 8 TMA producer, warp 9
 // MMA issue (one thread).  Per item, the producer loads the tile's Q rows with
 // one 3-D TMA box per half and 64-column slab (tokens x heads x columns, the
-// 128-byte swizzle), then 64-key steps of K and V (4 blocks, 64 x 16 boxes)
-// into a 3-stage ring.  The MMA thread issues S of step j + 1 (both halves)
+// 128-byte swizzle), then 64-key steps of K and V (4 blocks) into a 4-stage
+// ring: K as 64 x 16 boxes per block and slab (the K-major layout of the
+// scores' B operand keeps a slab's 64 keys together), V as one 3-D box per
+// block (64 columns x 16 rows x 2 slabs, 4 KB), which is exactly one k-step
+// of P V's MN-major B operand.  (Measured on B200: 4 KB boxes move a 32 KB
+// step 20% faster than 2 KB boxes when every SM loads.)  The MMA thread issues S of step j + 1 (both halves)
 // before P V of step j (two S buffers per half in TMEM), so the tensor cores
 // run while the softmax works, also across item boundaries.  A softmax thread
 // reads its row of S straight from TMEM, takes the running max with the scale
@@ -114,7 +118,10 @@ struct TileCfg {
     static constexpr int kQHalfBytes = kSlabs * kHalfRows * 128;
     static constexpr int kQBytes = kTileHalves * kQHalfBytes;
     static constexpr int kKVSlab = kKeys * 128;               // one slab of K (or V) for a step
-    static constexpr int kStageBytes = 2 * kSlabs * kKVSlab;  // K slabs, then V slabs
+    static constexpr int kStageBytes = 2 * kSlabs * kKVSlab;  // K slabs, then V blocks
+    // V of a step: block after block (one TMA box each), a block's slabs after
+    // each other (16 rows of 128 bytes per slab)
+    static constexpr int kVBlockBytes = kSlabs * kBlockTokens * 128;
     static constexpr int kStages = 4;
     static constexpr int kPHalfBytes = kHalfRows * 128;       // P: 64 bf16 keys per row
     static constexpr int kPBytes = kTileHalves * kPHalfBytes;
@@ -494,11 +501,9 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                     for (int c = lane; c < Cfg::kStepBlocks * Cfg::kSlabs * kBlockTokens * 8; c += 32) {
                         const int bb = c / (Cfg::kSlabs * kBlockTokens * 8);
                         if ((present >> bb) & 1u) continue;
-                        const int rem = c % (Cfg::kSlabs * kBlockTokens * 8);
-                        const int sl = rem / (kBlockTokens * 8), rr = rem % (kBlockTokens * 8);
-                        const int t = bb * kBlockTokens + rr / 8;
-                        *reinterpret_cast<uint4*>(ring_smem + st * Cfg::kStageBytes + (Cfg::kSlabs + sl) * Cfg::kKVSlab +
-                                                  t * 128 + (rr % 8) * 16) = make_uint4(0, 0, 0, 0);
+                        const int rem = c % (Cfg::kSlabs * kBlockTokens * 8);  // the block's 16-byte chunks
+                        *reinterpret_cast<uint4*>(ring_smem + st * Cfg::kStageBytes + Cfg::kSlabs * Cfg::kKVSlab +
+                                                  bb * Cfg::kVBlockBytes + rem * 16) = make_uint4(0, 0, 0, 0);
                     }
                     fence_proxy_async_smem();
                 }
@@ -513,12 +518,15 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                     if (lane == 0 && pbb >= 0) {
                         const int32_t row = (pbb * P.num_kv_heads + I.h) * kBlockTokens;
 #pragma unroll
-                        for (int sl = 0; sl < Cfg::kSlabs; ++sl) {
+                        for (int sl = 0; sl < Cfg::kSlabs; ++sl)
                             tma_load_2d(sbase + sl * Cfg::kKVSlab + bb * kBlockTokens * 128, &tmap_k, sl * 64, row,
                                         full_u32 + 8 * st, keep);
-                            tma_load_2d(sbase + (Cfg::kSlabs + sl) * Cfg::kKVSlab + bb * kBlockTokens * 128, &tmap_v,
-                                        sl * 64, row, full_u32 + 8 * st, keep);
-                        }
+                        // V: the block's slabs in one box (the map is 3-D: 64 columns x rows x slabs)
+                        const uint32_t vdst = sbase + Cfg::kSlabs * Cfg::kKVSlab + bb * Cfg::kVBlockBytes;
+                        if constexpr (Cfg::kSlabs > 1)
+                            tma_load_3d(vdst, &tmap_v, 0, row, 0, full_u32 + 8 * st, keep);
+                        else
+                            tma_load_2d(vdst, &tmap_v, 0, row, full_u32 + 8 * st, keep);
                     }
                 }
                 __syncwarp();
@@ -568,10 +576,20 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 }
                 return first_step(c.iq + 1, c.gs + 1, n);
             };
-            auto issue_s = [&](const Cur& c) -> bool {
+            // S of step c waits for its Q (first step of an item) and its K
+            auto wait_s = [&](const Cur& c) -> bool {
                 if (c.j == 0 && !mbar_wait_bounded_thread(qfull_u32, c.iq & 1u)) return false;
+                return mbar_wait_bounded_thread(full_u32 + 8 * (c.gs % S), (c.gs / S) & 1u);
+            };
+            // P V of step c waits for its P; the first step of an item
+            // overwrites O, which the softmax must have read out for the
+            // previous item
+            auto wait_pv = [&](const Cur& c) -> bool {
+                if (c.j == 0 && c.iq > 0 && !mbar_wait_bounded_thread(ofree_u32, (c.iq - 1) & 1u)) return false;
+                return mbar_wait_bounded_thread(pfull_u32, c.gs & 1u);
+            };
+            auto issue_s = [&](const Cur& c) {
                 const int st = c.gs % S;
-                if (!mbar_wait_bounded_thread(full_u32 + 8 * st, (c.gs / S) & 1u)) return false;
                 tc_fence_after();
                 const uint32_t kb = ring_u32 + st * Cfg::kStageBytes;
 #pragma unroll
@@ -587,33 +605,39 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 }
                 umma_commit(sfull_u32 + 8 * (c.gs & 1u));
                 if (c.j + 1 == c.nsteps) umma_commit(qempty_u32);  // the item's last read of Q
-                return true;
             };
-            Cur cur;
-            bool have = first_step(0, 0, cur);
-            if (have) ok = issue_s(cur);
-            while (have && ok) {
-                Cur nxt;
-                const bool more = next_step(cur, nxt);
-                if (more && !(ok = issue_s(nxt))) break;
-                // P V of the current step; the first step of an item overwrites O,
-                // which the softmax must have read out for the previous item
-                if (cur.j == 0 && cur.iq > 0 && !(ok = mbar_wait_bounded_thread(ofree_u32, (cur.iq - 1) & 1u)))
-                    break;
-                if (!(ok = mbar_wait_bounded_thread(pfull_u32, cur.gs & 1u))) break;
+            auto issue_pv = [&](const Cur& c) {
                 tc_fence_after();
-                const uint32_t vb = ring_u32 + (cur.gs % S) * Cfg::kStageBytes + Cfg::kSlabs * Cfg::kKVSlab;
+                const uint32_t vb = ring_u32 + (c.gs % S) * Cfg::kStageBytes + Cfg::kSlabs * Cfg::kKVSlab;
 #pragma unroll
                 for (int hh = 0; hh < kTileHalves; ++hh) {
 #pragma unroll
-                    for (int ks = 0; ks < K / 16; ++ks) {
+                    for (int ks = 0; ks < K / 16; ++ks) {  // k-step ks: the keys of block ks
                         const uint64_t a = umma_desc_sw128(p_u32 + hh * Cfg::kPHalfBytes + ks * 32u, 16, 1024);
-                        const uint64_t bd = umma_desc_sw128(vb + ks * 16 * 128, Cfg::kKVSlab, 1024);
-                        umma_bf16(tmem + hh * Cfg::kHalfCols + Cfg::kColO, a, bd, kIdescO, cur.j > 0 || ks > 0);
+                        const uint64_t bd = umma_desc_sw128(vb + ks * Cfg::kVBlockBytes, 2048, 1024);
+                        umma_bf16(tmem + hh * Cfg::kHalfCols + Cfg::kColO, a, bd, kIdescO, c.j > 0 || ks > 0);
                     }
                 }
                 umma_commit(odone_u32);
-                umma_commit(empty_u32 + 8 * (cur.gs % S));
+                umma_commit(empty_u32 + 8 * (c.gs % S));  // the stage may be refilled
+            };
+            // S(j + 1) goes before P V(j), so that the tensor cores compute the
+            // next scores while the softmax works on this step.  (Measured:
+            // letting P V(j) go first whenever K(j + 1) lands after P(j)
+            // delays the next softmax by a P V and was 27% slower.)
+            Cur cur;
+            bool have = first_step(0, 0, cur);
+            if (have && (ok = wait_s(cur))) issue_s(cur);
+            while (have && ok) {
+                Cur nxt;
+                const bool more = next_step(cur, nxt);
+                if (!ok) break;  // the item queue's wait gave up
+                if (more) {
+                    if (!(ok = wait_s(nxt))) break;
+                    issue_s(nxt);
+                }
+                if (!(ok = wait_pv(cur))) break;
+                issue_pv(cur);
                 if (!more) break;
                 cur = nxt;
             }
@@ -740,8 +764,9 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                         for (int e = threadIdx.x; e < zrows * Cfg::kSlabs * 8; e += Cfg::kSoftmaxThreads) {
                             const int zr = K - zrows + e / (Cfg::kSlabs * 8);
                             const int sl = (e / 8) % Cfg::kSlabs;
-                            *reinterpret_cast<uint4*>(ring_smem + st * Cfg::kStageBytes + (Cfg::kSlabs + sl) * Cfg::kKVSlab +
-                                                      zr * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4*>(ring_smem + st * Cfg::kStageBytes + Cfg::kSlabs * Cfg::kKVSlab +
+                                                      (zr / kBlockTokens) * Cfg::kVBlockBytes + sl * kBlockTokens * 128 +
+                                                      (zr % kBlockTokens) * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
                         }
                     }
                     fence_proxy_async_smem();

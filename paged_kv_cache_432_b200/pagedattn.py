@@ -43,6 +43,9 @@ SIGNATURES = {
     "pa_cache_write_fp8": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _P, _P, _I32, _I32, _P, _P, _P]),
     "pa_decode_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32,
                                      _F, _I32, _P, _SZ, _P, _P]),
+    "pa_decode_fp8_partitions": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
+                                                _I32, _I32, _F, _I32, _P, _SZ, _P, _P]),
+    "pa_decode_fp8_reduce": (ctypes.c_int, [_P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ, _P, _P]),
     "pa_decode_partition_blocks": (_I32, [_I32, _I32, _I32, _I32, _I32]),
     "pa_decode_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "pa_decode": (ctypes.c_int, _DECODE_ARGS),
@@ -160,6 +163,29 @@ def decode_fp8(q, k_cache, v_cache, k_scale, v_scale, block_tables, seq_lens, sc
                              _stream(stream))
     _check("pa_decode_fp8", rc)
     return out
+
+
+def decode_fp8_partitions(q, k_cache, v_cache, k_scale, v_scale, block_tables, seq_lens, scale, out, max_seq_len,
+                          partition_blocks, workspace, stream=None) -> None:
+    """pa_decode_fp8_partitions: the E4M3 block-table walk alone (final rows + partials)."""
+    N, Hq, D = q.shape
+    NB, Hkv, B, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().pa_decode_fp8_partitions(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+                                        _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), max_seq_len, N,
+                                        Hq, Hkv, D, NB, B, float(scale), partition_blocks, _ptr(workspace),
+                                        ws_bytes, _ptr(out), _stream(stream))
+    _check("pa_decode_fp8_partitions", rc)
+
+
+def decode_fp8_reduce(seq_lens, out, num_kv_heads, max_blocks_per_seq, max_seq_len, partition_blocks,
+                      workspace, stream=None) -> None:
+    """pa_decode_fp8_reduce: the log-sum-exp merge of an E4M3 partition step."""
+    N, Hq, D = out.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().pa_decode_fp8_reduce(_ptr(seq_lens), max_seq_len, N, Hq, num_kv_heads, D, max_blocks_per_seq, 16,
+                                    partition_blocks, _ptr(workspace), ws_bytes, _ptr(out), _stream(stream))
+    _check("pa_decode_fp8_reduce", rc)
 
 
 def partition_blocks(num_seqs, num_kv_heads, max_seq_len, partition_blocks=0, block_size=16) -> int:

@@ -212,6 +212,24 @@ def test_fp8_entry_points_reject_bad_arguments_on_the_host(lib):
     assert drc(10, 34) == pa.PA_ERR_UNSUPPORTED      # 34 / 2 = group of 17
     assert drc(15, float("inf")) == pa.PA_ERR_INVALID_ARG
 
+    # the partition step alone validates the same way
+    dp = lib.pa_decode_fp8_partitions
+
+    def prc(i=None, val=None):
+        a = list(base)
+        if i is not None:
+            a[i] = val
+        return dp(*a)
+
+    assert prc(3, None) == pa.PA_ERR_INVALID_ARG
+    assert prc(0, 8) == pa.PA_ERR_INVALID_ARG
+    assert prc(12, 96) == pa.PA_ERR_UNSUPPORTED
+    # the E4M3 merge: sizes as pa_decode_reduce, the workspace checked first
+    r = lib.pa_decode_fp8_reduce
+    assert r(16, 2048, 4, 8, 2, 128, 128, 16, 0, None, 0, 16, None) == pa.PA_ERR_WORKSPACE
+    assert r(16, 2048, 4, 8, 2, 96, 128, 16, 0, 256, 1 << 20, 16, None) == pa.PA_ERR_UNSUPPORTED
+    assert r(16, 2048, 4, 8, 3, 128, 128, 16, 0, 256, 1 << 20, 16, None) == pa.PA_ERR_INVALID_ARG
+
 
 def test_get_device_error_rejects_null(lib):
     assert lib.pa_get_device_error(None, 0, None) == pa.PA_ERR_INVALID_ARG
@@ -226,7 +244,8 @@ def _comment_before(name: str) -> str:
 
 
 @pytest.mark.parametrize("name", ["pa_cache_write", "pa_decode", "pa_decode_workspace_size",
-                                  "pa_get_device_error", "pa_status_string"])
+                                  "pa_get_device_error", "pa_status_string", "pa_decode_fp8_partitions",
+                                  "pa_decode_fp8_reduce"])
 def test_boundary_calls_cite_a_passage_or_say_plumbing(name):
     """Each call of the boundary names the page passage that defines it, or
     says that it is interface plumbing with no passage."""

@@ -131,6 +131,28 @@ def test_fp8_decode_ragged_lengths(Hq, Hkv):
     assert pa.device_error() == 0
 
 
+@pytest.mark.parametrize("Hq,Hkv,pb", [(32, 32, 0), (32, 8, 0), (8, 2, 3), (64, 8, 32)])
+def test_fp8_partitions_then_reduce_equal_the_one_call(Hq, Hkv, pb):
+    """pa_decode_fp8_partitions followed by pa_decode_fp8_reduce is
+    pa_decode_fp8 bit for bit (the same kernels, the merge told the E4M3
+    warp ranges), and both match the oracle."""
+    rng = np.random.default_rng(Hq + Hkv + pb)
+    lens = [int(x) for x in rng.integers(1, 3000, size=20)] + [0, 1, 4097]
+    w = wl.build(lens, Hq, Hkv, 128, torch.bfloat16, seed=23 + pb, device=DEV)
+    kc, vc, ks, vs = _fp8_case(w)
+    one = pa.decode_fp8(w.q, kc, vc, ks, vs, w.block_tables, w.seq_lens, w.scale, max_seq_len=w.max_seq_len,
+                        partition_blocks=pb)
+    ws = pa.alloc_workspace(w.num_seqs, Hq, Hkv, 128, w.max_seq_len, pb, device=DEV)
+    out = torch.full_like(w.q, float("nan"))
+    pa.decode_fp8_partitions(w.q, kc, vc, ks, vs, w.block_tables, w.seq_lens, w.scale, out, w.max_seq_len, pb, ws)
+    if ws is not None:
+        pa.decode_fp8_reduce(w.seq_lens, out, Hkv, w.block_tables.shape[1], w.max_seq_len, pb, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), one.view(torch.int16))
+    assert_close(to_f64(out), _oracle_fp8(w, kc, vc, ks, vs), torch.bfloat16, f"fp8 two steps {Hq}/{Hkv} pb={pb}")
+    assert pa.device_error() == 0
+
+
 def test_fp8_decode_scales_are_per_head():
     """Doubling one kv head's K scale changes only that head's rows; the V
     scale multiplies its rows exactly when the softmax is unchanged."""
