@@ -647,9 +647,12 @@ TileSplit choose_tile_split(int sms, int64_t work_tiles, int32_t nb_max) {
     return TileSplit{(nb_max + ch - 1) / ch, ch};
 }
 
+// counter_zeroed: the caller set the item counter to zero before (the
+// shared-prefix tiles launched after the private-block decode: a memset
+// between the two would keep the tiles from starting early).
 template <int D>
 int launch_tiles(const TileParams& base, const void* q, int64_t q_rows, const void* k_cache,
-                 const void* v_cache, int64_t items_bound, cudaStream_t st) {
+                 const void* v_cache, int64_t items_bound, cudaStream_t st, bool counter_zeroed = false) {
     auto kernel = attn_tiles_tc_kernel<D>;
     int rc = ensure_smem_attr(kernel, TileCfg<D>::kSmem);
     if (rc != PA_OK) return rc;
@@ -670,8 +673,10 @@ int launch_tiles(const TileParams& base, const void* q, int64_t q_rows, const vo
         cudaError_t e;
         if (items_bound > grid) {
             // more items than CTAs: they are claimed from a counter, which starts at zero
-            e = cudaMemsetAsync(P.item_counter, 0, sizeof(int32_t), st);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (tile item counter)");
+            if (!counter_zeroed) {
+                e = cudaMemsetAsync(P.item_counter, 0, sizeof(int32_t), st);
+                if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (tile item counter)");
+            }
         } else {
             P.item_counter = nullptr;  // at most one item per CTA: no counter
         }
@@ -684,8 +689,15 @@ int launch_tiles(const TileParams& base, const void* q, int64_t q_rows, const vo
 
 // The shared prefixes' key chunks through the tile kernel (prefix mode: one
 // group of every sequence, or P.num_groups groups from P.group_start /
-// P.group_blocks); sets plan->prefix_splits / prefix_split_blocks.
-int launch_prefix_tiles(const DecodeParams& P, Plan* plan, cudaStream_t st) {
+// P.group_blocks): the launch's parameters and item count; sets
+// plan->prefix_splits / prefix_split_blocks.
+struct PrefixTiles {
+    TileParams T;
+    int64_t items;
+    int sms;
+};
+
+int plan_prefix_tiles(const DecodeParams& P, Plan* plan, PrefixTiles* pt) {
     DeviceInfo di;
     int rc = device_info(&di);
     if (rc != PA_OK) return rc;
@@ -693,7 +705,7 @@ int launch_prefix_tiles(const DecodeParams& P, Plan* plan, cudaStream_t st) {
                                            plan->shared_blocks);
     plan->prefix_splits = sp.splits;
     plan->prefix_split_blocks = sp.chunk_blocks;
-    TileParams T;
+    TileParams& T = pt->T;
     std::memset(&T, 0, sizeof T);
     T.block_tables = P.block_tables;
     T.seq_lens = P.seq_lens;
@@ -718,9 +730,15 @@ int launch_prefix_tiles(const DecodeParams& P, Plan* plan, cudaStream_t st) {
     T.len_cap = P.len_cap;
     T.shared_blocks = plan->shared_blocks;
     T.scale_log2 = P.scale_log2;
-    const int64_t items = static_cast<int64_t>(plan->prefix_row_tiles) * P.num_kv_heads * sp.splits;
-    return P.head_dim == 128 ? launch_tiles<128>(T, P.q, P.num_seqs, P.k_cache, P.v_cache, items, st)
-                             : launch_tiles<64>(T, P.q, P.num_seqs, P.k_cache, P.v_cache, items, st);
+    pt->items = static_cast<int64_t>(plan->prefix_row_tiles) * P.num_kv_heads * sp.splits;
+    pt->sms = di.sms;
+    return PA_OK;
+}
+
+int launch_prefix_tiles(const DecodeParams& P, const PrefixTiles& pt, cudaStream_t st, bool counter_zeroed) {
+    return P.head_dim == 128
+               ? launch_tiles<128>(pt.T, P.q, P.num_seqs, P.k_cache, P.v_cache, pt.items, st, counter_zeroed)
+               : launch_tiles<64>(pt.T, P.q, P.num_seqs, P.k_cache, P.v_cache, pt.items, st, counter_zeroed);
 }
 
 template <typename OutT, int D>
@@ -778,6 +796,40 @@ int run_reduce(const DecodeParams& P, const Plan& plan, int32_t dtype, cudaStrea
                                  : launch_reduce<__nv_bfloat16, 64>(P, dtype, f8, st);
     return P.head_dim == 128 ? launch_reduce<float, 128>(P, dtype, f8, st)
                              : launch_reduce<float, 64>(P, dtype, f8, st);
+}
+
+// The shared-prefix decode's three steps.  The private blocks' decode goes
+// first and the prefix tiles right after it, marked independent: the tiles'
+// CTAs take each SM the decode leaves (its slowest warps' tail) instead of
+// waiting for the whole grid, and their start-up (cold Q and K/V loads) hides
+// under it.  The merge waits for the tiles, which wait for the decode before
+// they complete.  With more prompt groups than one tile launch holds, the
+// tiles launch in several grids and go first, each waiting as usual.
+int run_shared_prefix(DecodeParams& P, Plan& plan, int32_t dtype, cudaStream_t st) {
+    PrefixTiles pt;
+    int rc = plan_prefix_tiles(P, &plan, &pt);
+    if (rc != PA_OK) return rc;
+    // the private pieces follow the chunks actually used (the most a group has);
+    // a group's own chunk count follows from its shared blocks and the chunk size
+    P.piece_base = plan.prefix_splits;
+    P.group_chunk = plan.prefix_split_blocks;
+    const int32_t max_units = P.head_dim == 128 ? TileCfg<128>::kMaxUnits : TileCfg<64>::kMaxUnits;
+    if (pt.T.num_units <= max_units) {
+        if (pt.items > pt.sms) {  // the tiles claim items from the counter: zero it before the decode
+            cudaError_t e = cudaMemsetAsync(pt.T.item_counter, 0, sizeof(int32_t), st);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (tile item counter)");
+        }
+        rc = run_partitions(P, dtype, st);
+        if (rc != PA_OK) return rc;
+        pt.T.independent = 1;
+        rc = launch_prefix_tiles(P, pt, st, true);
+    } else {
+        rc = launch_prefix_tiles(P, pt, st, false);
+        if (rc != PA_OK) return rc;
+        rc = run_partitions(P, dtype, st);
+    }
+    if (rc != PA_OK) return rc;
+    return run_reduce(P, plan, dtype, st);
 }
 
 // Several query tokens per sequence with group * max_q_len > 16 (prefill
@@ -1211,12 +1263,7 @@ int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_ca
     int rc = prepare_decode(a, true, &P, &plan, shared_blocks);
     if (rc != PA_OK) return rc;
     if (num_seqs == 0) return PA_OK;
-    rc = launch_prefix_tiles(P, &plan, a.stream);
-    if (rc != PA_OK) return rc;
-    P.piece_base = plan.prefix_splits;  // the private pieces follow the chunks actually used
-    rc = run_partitions(P, dtype, a.stream);
-    if (rc != PA_OK) return rc;
-    return run_reduce(P, plan, dtype, a.stream);
+    return run_shared_prefix(P, plan, dtype, a.stream);
 }
 
 int pa_decode_shared_prefix_groups(const void* q, const void* k_cache, const void* v_cache,
@@ -1246,13 +1293,7 @@ int pa_decode_shared_prefix_groups(const void* q, const void* k_cache, const voi
     P.group_start = group_start;
     P.group_blocks = group_shared_blocks;
     P.num_groups = num_groups;
-    rc = launch_prefix_tiles(P, &plan, a.stream);
-    if (rc != PA_OK) return rc;
-    P.piece_base = plan.prefix_splits;  // the private pieces follow the most chunks a group has
-    P.group_chunk = plan.prefix_split_blocks;
-    rc = run_partitions(P, dtype, a.stream);
-    if (rc != PA_OK) return rc;
-    return run_reduce(P, plan, dtype, a.stream);
+    return run_shared_prefix(P, plan, dtype, a.stream);
 }
 
 size_t pa_decode_shared_prefix_groups_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,

@@ -105,6 +105,13 @@ struct TileParams {
     int32_t shared_blocks;   // prefix: blocks of every group when group_blocks is null, else
                              //   the bound on group_blocks
     int32_t direct;          // 1: one chunk per unit, rows written to out as final bf16
+    // 1: the grid launched just before this one in the stream (the decode of
+    // the private blocks) computes something this launch does not read, and
+    // lets it start only after the kernels before it have completed.  Then
+    // no role waits for it at the start; one thread waits at the very end, so
+    // that this grid completes after it (the merge that follows waits for
+    // this grid, and so for both).
+    int32_t independent;
     float scale_log2;        // softmax scale * log2(e)
 };
 
@@ -408,7 +415,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         const uint64_t keep = l2_policy_evict_last();  // K/V and Q are read by several tiles
         bool ok = true;
         uint32_t iq = 0, gs = 0;  // items with work, global steps
-        bool waited = false;       // grid_dependency_wait done
+        bool waited = P.independent != 0;  // grid_dependency_wait done (or not needed)
         bool first = true;         // the CTA's first item is item blockIdx.x
         int32_t cand = blockIdx.x;
         while (ok) {
@@ -656,7 +663,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         const float sl2 = P.scale_log2;
         bool ok = true;  // warp-uniform: a wait that gave up stops TMEM work and arrivals
         uint32_t gs = 0;
-        bool waited = false;  // grid_dependency_wait done (before the first output write)
+        bool waited = P.independent != 0;  // grid_dependency_wait done (before the first output write)
         for (uint32_t iq = 0; ok; ++iq) {
             const uint32_t slot = iq % Cfg::kItemSlots;
             ok = mbar_wait_bounded(iqfull_u32 + 8 * slot, (iq / Cfg::kItemSlots) & 1u);
@@ -849,6 +856,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::kTmemCols);
     }
+    if (P.independent && threadIdx.x == 0) grid_dependency_wait();  // complete after the grid before
 }
 
 }  // namespace pa

@@ -177,7 +177,6 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // schedule, the first table window and, into L2, the first query rows are
     // ready when the wait ends.  The pool (which the cache write fills), the
     // output and the workspace are touched only after it.
-    allow_dependents();  // the reduction may launch and wait for this grid
     const Schedule sched = make_schedule(P, prefix, WARPS);  // ends with __syncthreads
     const int32_t my_warp = blockIdx.x * WARPS + warp;
     Cursor pc;  // producer: the piece whose next block is loaded next
@@ -193,6 +192,11 @@ decode_bf16_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         (static_cast<size_t>(pc.s) * P.num_q_heads + pc.h * P.group) * D + 64 * lane);
     }
     grid_dependency_wait();
+    // Dependents may start only now, once every CTA has passed the wait: the
+    // kernels launched before this one have then completed, so a following
+    // grid that does not depend on this one (the shared-prefix tiles) may
+    // read what they wrote without waiting for this grid.
+    allow_dependents();
     zero_empty_sequences<__nv_bfloat16>(P, lens);
     if (!pc.valid) return;
     Cursor cc = pc;  // consumer: the piece being computed
