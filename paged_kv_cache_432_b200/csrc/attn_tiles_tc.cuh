@@ -48,16 +48,19 @@
 // scores' B operand keeps a slab's 64 keys together), V as one 3-D box per
 // block (64 columns x 16 rows x 2 slabs, 4 KB), which is exactly one k-step
 // of P V's MN-major B operand.  (Measured on B200: 4 KB boxes move a 32 KB
-// step 20% faster than 2 KB boxes when every SM loads.)  The MMA thread issues S of step j + 1 (both halves)
-// before P V of step j (two S buffers per half in TMEM), so the tensor cores
-// run while the softmax works, also across item boundaries.  A softmax thread
-// reads its row of S straight from TMEM, takes the running max with the scale
-// folded into one multiply-add per key (a step that is wholly visible needs
-// no masking), writes P (bf16) to shared memory, rescales its O row in TMEM
-// when the max moved, and at the item's end writes the row: a partial (m, l,
-// acc) at piece c, or the final bf16 row when the units have one chunk
-// (prefill), staged through shared memory so that every store writes whole
-// 128-byte lines.
+// step 20% faster than 2 KB boxes when every SM loads.)  The MMA thread
+// issues S of step j + 1 (both halves) before P V of step j (two S buffers
+// per half in TMEM), so the tensor cores run while the softmax works, also
+// across item boundaries.  A softmax thread reads its row of S straight from
+// TMEM, takes the running max with the scale folded into one multiply-add per
+// key (a step that is wholly visible needs no masking), writes P as bf16
+// pairs back over the first half of the S buffer it read (P V takes its A
+// operand from tensor memory, as FlashAttention-4 does: no shared-memory
+// round trip for P), rescales its O row in TMEM when the max moved (only
+// then does it wait for the previous P V), and at the item's end writes the
+// row: a partial (m, l, acc) at piece c, or the final bf16 row when the units
+// have one chunk (prefill), staged through shared memory so that every store
+// writes whole 128-byte lines.
 // All step counters run on across items, so every mbarrier's phase follows
 // from a per-CTA global step or item count.  Every wait is bounded; a role
 // that gives up flags PA_DEVERR_TIMEOUT and stops issuing, the other roles'
@@ -130,7 +133,7 @@ struct TileCfg {
     // each other (16 rows of 128 bytes per slab)
     static constexpr int kVBlockBytes = kSlabs * kBlockTokens * 128;
     static constexpr int kStages = 4;
-    static constexpr int kPHalfBytes = kHalfRows * 128;       // P: 64 bf16 keys per row
+    static constexpr int kPHalfBytes = kHalfRows * 128;       // epilogue staging: 128 bytes per row
     static constexpr int kPBytes = kTileHalves * kPHalfBytes;
     static constexpr int kSoftmaxWarps = 4 * kTileHalves;
     static constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
@@ -342,7 +345,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
-    // layout: Q[half][slab] | ring[S] | P[half] | unit prefix | barriers | TMEM slot | stage masks
+    // layout: Q[half][slab] | ring[S] | staging[half] | unit prefix | barriers | TMEM slot | stage masks
     const uint32_t q_u32 = smem_u32(smem);
     const uint32_t ring_u32 = q_u32 + Cfg::kQBytes;
     const uint32_t p_u32 = ring_u32 + S * Cfg::kStageBytes;
@@ -401,7 +404,7 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     fence_proxy_async_smem();
     if (warp == Cfg::kMmaWarp) tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
     uint8_t* unit_ord = reinterpret_cast<uint8_t*>(prefix + Cfg::kMaxUnits + 1);
-    // (the P buffer is free until the first step: scratch for the ordering)
+    // (the staging buffer is free until the first epilogue: scratch for the ordering)
     const int32_t total = build_unit_prefix(P, prefix, unit_ord, reinterpret_cast<uint32_t*>(p_smem));
     tc_fence_before();
     __syncthreads();
@@ -620,9 +623,10 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 for (int hh = 0; hh < kTileHalves; ++hh) {
 #pragma unroll
                     for (int ks = 0; ks < K / 16; ++ks) {  // k-step ks: the keys of block ks
-                        const uint64_t a = umma_desc_sw128(p_u32 + hh * Cfg::kPHalfBytes + ks * 32u, 16, 1024);
+                        // P: 16 keys = 8 columns of bf16 pairs in the step's S buffer
+                        const uint32_t a = tmem + hh * Cfg::kHalfCols + Cfg::kColS + (c.gs & 1u) * K + ks * 8u;
                         const uint64_t bd = umma_desc_sw128(vb + ks * Cfg::kVBlockBytes, 2048, 1024);
-                        umma_bf16(tmem + hh * Cfg::kHalfCols + Cfg::kColO, a, bd, kIdescO, c.j > 0 || ks > 0);
+                        umma_bf16_tmem_a(tmem + hh * Cfg::kHalfCols + Cfg::kColO, a, bd, kIdescO, c.j > 0 || ks > 0);
                     }
                 }
                 umma_commit(odone_u32);
@@ -659,7 +663,6 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         const int hh = warp >> 2;                // half of the tile
         const int row = 32 * (warp & 3) + lane;  // TMEM lane = row of the half
         const uint32_t lane_base = tmem + hh * Cfg::kHalfCols + ((static_cast<uint32_t>(warp & 3) * 32u) << 16);
-        uint8_t* p_half = p_smem + hh * Cfg::kPHalfBytes;
         const float sl2 = P.scale_log2;
         bool ok = true;  // warp-uniform: a wait that gave up stops TMEM work and arrivals
         uint32_t gs = 0;
@@ -739,13 +742,16 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                         }
                     }
                     l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-                    if (j > 0) {
-                        // P V of the previous step is done: the P buffer is free, O holds the sum up to it
+                    // P V of the previous step must be done before this step's P is
+                    // announced (the phase tracking of o_done stays within one
+                    // step), and before O is rescaled; the P store itself need not
+                    // wait for it (P goes to the other S buffer)
+                    bool prev_done = j == 0;
+                    if (j > 0 && __any_sync(kFullMask, alpha != 1.f)) {
                         ok = mbar_wait_bounded(odone_u32, (gs - 1) & 1u);
                         tc_fence_after();
-                    }
-                    if (ok) {
-                        if (j > 0 && __any_sync(kFullMask, alpha != 1.f)) {
+                        prev_done = true;
+                        if (ok) {
 #pragma unroll
                             for (int c = 0; c < D / 32; ++c) {
                                 float v[32];
@@ -755,12 +761,12 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                                 tmem_st32(lane_base + Cfg::kColO + 32 * c, v);
                             }
                         }
-                        // the row's 64 keys: its 128-byte P row, K-major, 128-byte swizzle
-#pragma unroll
-                        for (int c = 0; c < K / 8; ++c)
-                            *reinterpret_cast<uint4*>(p_half + row * 128 + ((c ^ (row & 7)) << 4)) =
-                                make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
                     }
+                    // the row's 64 weights (bf16 pairs) over the first 32 columns of
+                    // the S buffer just read: P V takes its A operand from there.  S
+                    // of step j + 2 overwrites them only after P V of this step.
+                    if (ok) tmem_st32(lane_base + Cfg::kColS + (gs & 1u) * K, pw);
+                    if (ok && !prev_done) ok = mbar_wait_bounded(odone_u32, (gs - 1) & 1u);
                 }
                 if (ok) {
                     // key slots at or past the sequence's length hold stale data
@@ -781,8 +787,8 @@ attn_tiles_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                     mbar_arrive(pfull_u32);
                 }
             }
-            // ---- the item's rows (the P buffers are free once the last P V is done,
-            // and serve as staging: each warp's 32 rows, 128 bytes of each at a time)
+            // ---- the item's rows, through the staging buffer: each warp's 32
+            // rows, 128 bytes of each at a time
             if (!waited) {
                 grid_dependency_wait();  // before the first write of out or the workspace
                 waited = true;
