@@ -392,6 +392,43 @@ def test_shared_prefix_groups_four_prompts_full_size():
     assert_close(to_f64(out), oracle_decode_all_rows(w, h), torch.bfloat16, "four prompts, every row")
 
 
+def test_shared_prefix_more_items_than_sms():
+    """1280 sequences (one query head per kv head, 32 kv heads) sharing a
+    64-token prompt: 5 row tiles x 32 kv heads = 160 tile items, more than
+    the SMs, so the tiles claim items from the workspace counter, which the
+    call zeroes before the private blocks' decode that runs first."""
+    lens = [64 + 1 + (i * 37) % 120 for i in range(1280)]
+    w = wl.build(lens, 32, 32, 128, torch.bfloat16, seed=71, device=DEV, prefix_len=64, poison_unused=True)
+    out = _shared_prefix_decode(w)
+    assert pa.device_error() == 0
+    assert_close(to_f64(out), oracle_decode_all_rows(w), torch.bfloat16, "shared prefix, 160 tile items")
+
+
+def test_shared_prefix_decode_in_several_launches():
+    """More sequences (2100) than one decode launch holds (2048): the private
+    blocks' decode runs as two grids, then the prefix tiles (which wait for
+    the last of them only at their end), then the merge."""
+    lens = [32 + 1 + (i * 13) % 60 for i in range(2100)]
+    w = wl.build(lens, 8, 2, 128, torch.bfloat16, seed=72, device=DEV, prefix_len=32, poison_unused=True)
+    out = _shared_prefix_decode(w)
+    assert pa.device_error() == 0
+    assert_close(to_f64(out), oracle_decode_all_rows(w), torch.bfloat16, "shared prefix, two decode launches")
+
+
+def test_shared_prefix_groups_more_than_one_tile_launch_holds():
+    """300 prompt groups, more units than one tile launch holds (256): the
+    tiles run first, in two launches, then the decode and the merge."""
+    groups = [(1 + i % 2, 32 + 16 * (i % 3)) for i in range(300)]
+    lens = [pl + 1 + (7 * len(groups) + 3 * k + i) % 50 for i, (count, pl) in enumerate(groups) for k in range(count)]
+    w = wl.build(lens, 8, 2, 128, torch.bfloat16, seed=73, device=DEV, groups=groups, poison_unused=True)
+    out = pa.decode_shared_prefix_groups(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale,
+                                         w.group_start, w.group_blocks, max(w.group_blocks_host),
+                                         max_seq_len=w.max_seq_len)
+    torch.cuda.synchronize()
+    assert pa.device_error() == 0
+    assert_close(to_f64(out), oracle_decode_all_rows(w), torch.bfloat16, "300 prompt groups")
+
+
 def test_shared_prefix_groups_bad_group_list_is_flagged():
     w = wl.build([600, 700, 300], 8, 2, 128, torch.bfloat16, seed=5, device=DEV, groups=[(2, 512), (1, 0)])
     # a count above the bound
