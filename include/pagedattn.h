@@ -200,8 +200,9 @@ PA_API int pa_decode_fp8_reduce(const int32_t* seq_lens, int32_t max_seq_len, in
  * With group * max_q_len <= 16 the (token, head) rows of a (sequence, kv head)
  * fit one warp-level MMA tile and run in the decode kernel (the check of a few
  * drafted tokens); with more (prefill chunks of any length), tiles of up to
- * 128 rows (floor(128 / group) tokens x group heads) of one sequence run on
- * the tensor-memory kernel, reading each K/V block once per tile, with the
+ * 256 rows (two halves of floor(128 / group) tokens x group heads) of one
+ * sequence run on the tensor-memory kernel, reading each K/V block once per
+ * tile, with the
  * keys cut into at most 16 chunks (merged by a log-sum-exp reduction) only
  * when there are too few tiles to fill the device.  A sequence with more than
  * max_q_len or more than seq_lens[s] query tokens has the excess ignored (its
@@ -343,12 +344,13 @@ PA_API int pa_decode_reduce(const int32_t* seq_lens, int32_t max_seq_len, int32_
  * KV-Speicherzuweisung für LLMs?", slavadubrov.com, §"Gemeinsame Nutzung
  * erfordert mehr als Speicherzuweisung"; "PagedAttention et vLLM",
  * aiunderstanding.org, §"Questions fréquemment posées").  Same result as
- * pa_decode, computed in three launches: the query rows of all sequences
- * attend to the shared blocks together, so those blocks are read once per
- * tile of 128 query rows of a kv head rather than once per sequence
- * (5th-generation tensor cores, accumulators in tensor memory);
- * each sequence's own blocks go through the decode kernel; a log-sum-exp
- * reduction merges the two.  Preconditions: every table starts with the
+ * pa_decode, computed in three launches: each sequence's own blocks go
+ * through the decode kernel; then the query rows of all sequences attend to
+ * the shared blocks together, so those blocks are read once per tile of up
+ * to 256 query rows of a kv head rather than once per sequence
+ * (5th-generation tensor cores, accumulators in tensor memory; this launch
+ * starts on the SMs the decode leaves, without waiting for the decode, and
+ * completes after it); a log-sum-exp reduction merges the two.  Preconditions: every table starts with the
  * prefix blocks of table 0, and every seq_len >= shared_blocks * block_size.
  * A violation is flagged with PA_DEVERR_PREFIX (the result is then
  * meaningless for the offending sequences).  Only PA_DTYPE_BF16.  The
@@ -395,7 +397,7 @@ PA_API size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t n
  * "PagedAttention et vLLM", aiunderstanding.org, §"Mise en œuvre dans le monde
  * réel" and §"Questions fréquemment posées": many requests with a common
  * system prompt).  Each group's shared blocks are read once per tile of up to
- * 128 query rows of its sequences (tensor-memory kernel); each sequence's own
+ * 256 query rows of its sequences (tensor-memory kernel); each sequence's own
  * blocks go through the decode kernel; a log-sum-exp reduction merges both.
  * group_start (int32 [num_groups + 1]) and group_shared_blocks (int32
  * [num_groups]) are device arrays read like the block tables;
