@@ -42,35 +42,62 @@ struct RowPieces {
 };
 
 // One warp merges one row (sequence, query head) from its pieces (partial
-// indices after `base`); lanes hold D/32 consecutive head dims.
+// indices after `base`); lanes hold D/32 consecutive head dims.  The first 32
+// pieces' m and l (one per lane) and the first kPre pieces' acc slices are
+// loaded together, so a row of up to kPre pieces costs one round trip to L2
+// before the arithmetic; the sums run in the same order as a plain loop.
 template <typename OutT, int D>
 __device__ __forceinline__ void merge_row_warp(const DecodeParams& P, size_t base, RowPieces pcs,
                                                OutT* o, int lane) {
     constexpr int DPL = D / 32;
+    constexpr int kPre = 8;
     using Vec = typename std::conditional<DPL == 4, float4, float2>::type;
     const float* wm = P.ws_m + base;
     const float* wl = P.ws_l + base;
     const float* wa = P.ws_acc + base * D + lane * DPL;
     const int parts = pcs.count();
-    float M = -INFINITY;
-    for (int p = lane; p < parts; p += 32) M = fmaxf(M, wm[pcs.index(p)]);
+    float m0 = -INFINITY, l0 = 0.f;  // piece `lane`'s max and sum
+    if (lane < parts) {
+        const int p = pcs.index(lane);
+        m0 = wm[p];
+        l0 = wl[p];
+    }
+    Vec pre[kPre];
+#pragma unroll
+    for (int q = 0; q < kPre; ++q)
+        if (q < parts) pre[q] = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(pcs.index(q)) * D);
+    float M = m0;
+    for (int p = lane + 32; p < parts; p += 32) M = fmaxf(M, wm[pcs.index(p)]);
     M = warp_max(M);
     if (M == -INFINITY) {  // every piece fully masked, or none
 #pragma unroll
         for (int e = 0; e < DPL; ++e) o[lane * DPL + e] = from_float<OutT>(0.f);
         return;
     }
-    float den = 0.f;
-    for (int p = lane; p < parts; p += 32) den += expf(wm[pcs.index(p)] - M) * wl[pcs.index(p)];
+    float den = lane < parts ? expf(m0 - M) * l0 : 0.f;
+    for (int p = lane + 32; p < parts; p += 32) den += expf(wm[pcs.index(p)] - M) * wl[pcs.index(p)];
     den = warp_sum(den);
+    // weight of piece q (warp-uniform q): its max from lane q, or from memory past 32
+    auto weight = [&](int q) {
+        const float mq = q < 32 ? __shfl_sync(kFullMask, m0, q & 31) : wm[pcs.index(q)];
+        return expf(mq - M);
+    };
     float a[DPL];
 #pragma unroll
     for (int e = 0; e < DPL; ++e) a[e] = 0.f;
+#pragma unroll
+    for (int q = 0; q < kPre; ++q) {
+        if (q < parts) {
+            const float w = weight(q);
+            const float* f = reinterpret_cast<const float*>(&pre[q]);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) a[e] = fmaf(w, f[e], a[e]);
+        }
+    }
 #pragma unroll 8
-    for (int q = 0; q < parts; ++q) {
-        const int p = pcs.index(q);
-        const float w = expf(wm[p] - M);
-        const Vec x = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(p) * D);
+    for (int q = kPre; q < parts; ++q) {
+        const float w = weight(q);
+        const Vec x = *reinterpret_cast<const Vec*>(wa + static_cast<size_t>(pcs.index(q)) * D);
         const float* f = reinterpret_cast<const float*>(&x);
 #pragma unroll
         for (int e = 0; e < DPL; ++e) a[e] = fmaf(w, f[e], a[e]);
