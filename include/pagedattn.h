@@ -203,8 +203,10 @@ PA_API int pa_decode_fp8_reduce(const int32_t* seq_lens, int32_t max_seq_len, in
  * 256 rows (two halves of floor(128 / group) tokens x group heads) of one
  * sequence run on the tensor-memory kernel, reading each K/V block once per
  * tile, with the
- * keys cut into at most 16 chunks (merged by a log-sum-exp reduction) only
- * when there are too few tiles to fill the device.  A sequence with more than
+ * keys cut into at most 16 chunks (merged by a log-sum-exp reduction) when
+ * there are too few tiles to fill the device, or when the sequences are long
+ * enough (chunks of at least 256 blocks) that more, shorter items even out
+ * the SMs' work.  A sequence with more than
  * max_q_len or more than seq_lens[s] query tokens has the excess ignored (its
  * rows are not written) and PA_DEVERR_SEQ_LEN set.  Workspace from
  * pa_decode_multi_workspace_size (rows are query-token rows); other arguments

@@ -637,11 +637,24 @@ struct TileSplit {
 // Key chunking for `work_tiles` (tile, kv head) pairs over units of at most
 // nb_max key blocks: as many chunks as fill the device's SMs (one tile-kernel
 // CTA each), at most kMaxTileSplits; one chunk when the tiles alone fill it.
+// Long units are cut further, up to kBalanceItemsPerSm items per SM, as long
+// as every chunk keeps at least kMinBalanceChunk blocks: the heaviest-first
+// claiming then evens out the CTAs' work (a few items of very different
+// lengths per SM would leave the last wave half empty), while an item's start
+// and epilogue (~10 us) stay small next to its steps.
+constexpr int64_t kBalanceItemsPerSm = 16;
+constexpr int64_t kMinBalanceChunk = 256;  // 64 steps of 64 keys
 TileSplit choose_tile_split(int sms, int64_t work_tiles, int32_t nb_max) {
+    if (nb_max < 1) nb_max = 1;
     int64_t want = work_tiles > 0 ? sms / work_tiles : 1;
     if (want < 1) want = 1;
+    if (work_tiles > 0) {
+        const int64_t bal = (kBalanceItemsPerSm * sms + work_tiles - 1) / work_tiles;
+        const int64_t by_len = nb_max / kMinBalanceChunk;
+        const int64_t b = bal < by_len ? bal : by_len;
+        if (b > want) want = b;
+    }
     if (want > kMaxTileSplits) want = kMaxTileSplits;
-    if (nb_max < 1) nb_max = 1;
     int32_t ch = static_cast<int32_t>((nb_max + want - 1) / want);
     ch = (ch + kTileStepBlocks - 1) / kTileStepBlocks * kTileStepBlocks;
     return TileSplit{(nb_max + ch - 1) / ch, ch};

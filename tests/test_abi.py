@@ -104,8 +104,13 @@ def test_shared_prefix_workspace_size(lib):
 
 def _tile_splits(sms, work_tiles, nb_max):
     """The key chunking the tile kernel picks (as documented in the header):
-    as many chunks as fill the SMs, at most 16, in multiples of 4 blocks."""
-    want = max(1, min(16, sms // work_tiles if work_tiles else 1))
+    as many chunks as fill the SMs, or, for long units, up to 16 items per SM
+    with chunks of at least 256 blocks; at most 16, in multiples of 4 blocks."""
+    nb_max = max(1, nb_max)
+    want = max(1, sms // work_tiles if work_tiles else 1)
+    if work_tiles:
+        want = max(want, min(-(-16 * sms // work_tiles), nb_max // 256))
+    want = min(16, want)
     ch = -(-nb_max // want)
     ch = -(-ch // 4) * 4
     return -(-nb_max // ch)
