@@ -110,6 +110,29 @@ def test_prefill_many_sequences_without_key_chunks():
     assert_close(to_f64(out), ref, torch.bfloat16, "prefill, 24 sequences")
 
 
+def test_prefill_long_sequences_cut_into_balancing_chunks():
+    """Long sequences with enough tiles to fill the device: the keys are still
+    cut, into chunks of at least 256 blocks, so that more, shorter items even
+    out the SMs' work; each row merges its chunks."""
+    from test_abi import _tile_splits
+
+    rng = np.random.default_rng(9)
+    lens = [int(x) for x in rng.integers(8300, 9000, size=10)]
+    nq = [128] * 10
+    w = wl.build(lens, 16, 2, 128, torch.bfloat16, seed=79, device=DEV, poison_unused=True)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    work_tiles = (-(-sum(nq) // 32) + len(lens)) * 2  # tiles of 2 x 16 tokens x 8 heads, per kv head
+    assert _tile_splits(sms, work_tiles, -(-w.max_seq_len // 16)) >= 2
+    q, qs = _queries(nq, 16, 128, seed=9)
+    out = pa.decode_multi(q, qs, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, max(nq),
+                          max_seq_len=w.max_seq_len)
+    torch.cuda.synchronize()
+    assert pa.device_error() == 0
+    h = host(w)
+    ref = oracle_decode_multi_all_rows(wl.as_numpy(q), h["kc"], h["vc"], h["bt"], h["sl"], qs.cpu().numpy(), w.scale)
+    assert_close(to_f64(out), ref, torch.bfloat16, "prefill, long sequences in balancing chunks")
+
+
 def test_prefill_more_tokens_than_max_q_len_are_flagged():
     w = wl.build([300, 300], 32, 8, 128, torch.bfloat16, seed=6, device=DEV)
     q, qs = _queries([64, 100], 32, 128, seed=6)  # 100 > max_q_len = 80
