@@ -25,6 +25,14 @@ metric: KV GB/s = algorithmic bytes of a step / step time, where the bytes are
 the KV of every token attended (each distinct physical block counted once:
 shared prefix blocks are read once), q, out, table entries and lengths, plus
 the cache write's reads and writes.  Decode tokens/s = sequences / step time.
+
+Besides value and the dominant kernel's roofline the line carries e2e (the
+same steps through the public API from pinned host buffers, run as a serving
+loop: the next step's inputs copied in and the previous step's result read
+back while a step computes, every step's copies inside the timed region),
+e2e_serial (copy in, compute, read back one after another, L2 flushed before
+each step), warm_l2 for a batch that shares a prompt (the steps without the
+flush), the oracle's cpu_baseline, NVML clocks and the launch count.
 """
 from __future__ import annotations
 
